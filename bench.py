@@ -1,0 +1,517 @@
+"""Benchmark of the strided-view GEMM library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dg|reference]
+
+Headline step (one pass of the hot path over one batch): the decode GEMV
+workload, x[1x4096] * W[4096x14336] and x * K^T with K[128x4096] read in place,
+BF16 in, FP32 accumulate, BF16 out, both through dg_gemm.  The metric for
+M = 1 is HBM GB/s: algorithmic bytes (every operand byte read once, every
+output byte written once) per second.  Weights rotate through three copies
+(352 MB, more than the 126 MB L2) so every step streams W from HBM.
+
+Beside the headline the JSON line carries, per workload of the benchmark
+definition, TFLOPS, GB/s and the fraction of the roofline
+max(FLOPs / tensor peak, bytes / HBM bandwidth) under "per_shape"; the
+dominant kernel's roofline ("roofline"); an end-to-end figure through the
+same API with host buffers ("e2e"); the FP64 CPU oracle timed on the host
+("cpu_baseline"); SM clocks sampled during the timed region ("clocks").
+
+--impl reference times the oracle (the plain CPU implementation the tests
+check against) on the same metric and workload, on a bounded sample per step.
+Under torchrun with N > 1, ranks run independent replicas (weak scaling, no
+collective on the data path); rank 0 prints the line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "GEMM TFLOPS & % of roofline per shape (HBM GB/s for M=1) on 1 B200"
+WORKLOAD = ("decode GEMV: x[1x4096]*W[4096x14336] + x*K^T with K[128x4096] read in place; "
+            "BF16 in, FP32 accumulate, BF16 out")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0, "source": "fallback"}
+ROTATE = 3
+
+
+# ----------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def flops_bytes(p: W.Problem):
+    """Algorithmic FLOPs (2MNK) and bytes: A, B and C written once; C read too
+    when beta != 0; the FP8 scales."""
+    es = W.ELEM_SIZE
+    M, N, K = p.M, p.N, p.K
+    b = M * K * es[p.A.dtype] + K * N * es[p.B.dtype] + M * N * es[p.C.dtype]
+    if p.beta != 0:
+        b += M * N * es[p.C.dtype]
+    if p.scale_a is not None:
+        b += 4 * M
+    if p.scale_b is not None:
+        b += 4 * N
+    return 2.0 * M * N * K, float(b)
+
+
+def tensor_peak_tflops(dtype: str, peaks) -> float:
+    base = peaks["bf16_tflops"]
+    return base * 2.0 if dtype == "e4m3" else base  # FP8 dense = 2x BF16 (nominal ratio 4.5/2.25)
+
+
+def roofline_time_s(p: W.Problem, peaks):
+    fl, by = flops_bytes(p)
+    t_tc = fl / (tensor_peak_tflops(p.A.dtype, peaks) * 1e12)
+    t_mem = by / (peaks["hbm_gbs"] * 1e9)
+    return max(t_tc, t_mem), ("tensor" if t_tc >= t_mem else "hbm")
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 100 ms) of SM clock and throttle reasons."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        self.dev = device_index
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvidia-smi unavailable"}
+        rows = []
+        for ts, line in self.samples:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9], parts[4]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        window = "timed region"
+        if not inside:
+            inside = rows
+            window = "whole run (timed region shorter than the sampling interval)"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "no samples"}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside), "window": window}
+
+
+def kernel_traffic(kernel_file: str, summary_file: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (its sha256 is recorded beside it)."""
+    path = os.path.join(ROOT, "profiles", summary_file)
+    src = os.path.join(ROOT, "tcgen05_tmem_gemm_b200", "csrc", kernel_file)
+    if not os.path.exists(path):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    rec = {}
+    for line in open(path):
+        if ":" in line and line.strip().startswith(("dram_bytes_per_launch", "kernel_source_sha")):
+            k, v = line.split(":", 1)
+            rec[k.strip()] = v.strip()
+    if rec.get("kernel_source_sha") != sha:
+        return None
+    try:
+        return float(rec["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------- the dg arm
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def dg_views(p: W.Problem, dg):
+    def v(op):
+        return dg.make_view(op.base.data_ptr() + op.offset, op.shape, op.stride, op.row_dims, op.dtype)
+
+    return v(p.A), v(p.B), v(p.C)
+
+
+def time_problem(p_gpu_list, dg, reps: int, warm: int):
+    """Average device time per call over `reps` calls, rotating through the
+    given device-resident copies (CUDA events on the current stream)."""
+    views = [dg_views(p, dg) for p in p_gpu_list]
+    s = torch.cuda.current_stream()
+    for i in range(warm):
+        q = p_gpu_list[i % len(views)]
+        A, B, C = views[i % len(views)]
+        assert dg.dg_gemm(A, B, C, q.alpha, q.beta, q.scale_a, q.scale_b, s) == dg.DG_OK
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    for i in range(reps):
+        q = p_gpu_list[i % len(views)]
+        A, B, C = views[i % len(views)]
+        starts[i].record(s)
+        st = dg.dg_gemm(A, B, C, q.alpha, q.beta, q.scale_a, q.scale_b, s)
+        ends[i].record(s)
+        assert st == dg.DG_OK
+    torch.cuda.synchronize()
+    assert dg.dg_sync_status(s) == dg.DG_OK
+    ts = [a.elapsed_time(b) * 1e-3 for a, b in zip(starts, ends)]
+    return statistics.median(ts), float(np.percentile(ts, 10)), float(np.percentile(ts, 90))
+
+
+SHAPES = [("small", "small_f16_128x128x256", W.cfg_small, 1),
+          ("gemv", "gemv_bf16_1x14336x4096", W.cfg_gemv, ROTATE),
+          ("gemv_kt", "gemv_kt_bf16_1x128x4096", W.cfg_gemv_kt, 1),
+          ("thin", "thin_f16_64x4096x4096_beta1", W.cfg_thin, 4),
+          ("square_bf16", "square_bf16_4096^3", W.cfg_square_bf16, 2),
+          ("square_e4m3", "square_e4m3_4096^3", W.cfg_square_e4m3, 2),
+          ("strided", "strided_nchw_bf16_3136x1024x256", W.cfg_strided, 8)]
+
+
+def per_shape(dg, peaks, quick: bool, only=None):
+    """Every workload of the benchmark definition: time, TFLOPS, GB/s and
+    fraction of roofline, with the dispatcher's kernel choice."""
+    out = {}
+    reps = 20 if quick else 100
+    for key, name, fn, copies in SHAPES:
+        if only is not None and key != only:
+            continue
+        base = fn()
+        gpus = [base.to("cuda") for _ in range(copies)]
+        A, B, C = dg_views(gpus[0], dg)
+        pl = dg.dg_plan(A, B, C, base.alpha, base.beta, base.scale_a is not None).as_dict()
+        med, p10, p90 = time_problem(gpus, dg, reps, warm=5)
+        fl, by = flops_bytes(base)
+        t_roof, bound = roofline_time_s(base, peaks)
+        out[name] = {"kernel": pl["kind_name"], "us": med * 1e6, "us_p10": p10 * 1e6, "us_p90": p90 * 1e6,
+                     "tflops": fl / med / 1e12, "gbs": by / med / 1e9, "bound": bound,
+                     "roofline_us": t_roof * 1e6, "frac_of_roofline": t_roof / med,
+                     "tiles": {k: pl[k] for k in ("block_n", "split_k", "swap_ab", "p_gather", "grid")},
+                     "l2": f"{copies} rotating input copies" if copies > 1 else "single copy (L2-resident)"}
+        del gpus
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_one_shape(args):
+    torch.cuda.set_device(0)
+    import tcgen05_tmem_gemm_b200 as dg
+
+    res = per_shape(dg, load_peaks(), True, only=args.shape)
+    print(json.dumps({"shape": args.shape, **res}), flush=True)
+
+
+def run_dg(args):
+    world, rank, local = dist_setup()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    import tcgen05_tmem_gemm_b200 as dg
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    # ---- the step's data: three rotating copies of W and K, one x
+    gv = W.cfg_gemv()
+    gk = W.cfg_gemv_kt()
+    step_bytes = flops_bytes(gv)[1] + flops_bytes(gk)[1]
+    copies = []
+    for _ in range(ROTATE):
+        a = gv.to(dev)
+        b = W.Problem(gk.name, a.A, gk.B.to(dev), gk.C.to(dev))  # x shared by both products
+        copies.append((a, b, dg_views(a, dg), dg_views(b, dg)))
+
+    def step(i, ev=None):
+        a, b, va, vb = copies[i % ROTATE]
+        if ev is not None:
+            ev[0].record(stream)
+        st1 = dg.dg_gemm(*va, 1.0, 0.0, None, None, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        st2 = dg.dg_gemm(*vb, 1.0, 0.0, None, None, stream)
+        return st1 | st2
+
+    for i in range(args.warmup):
+        assert step(i) == 0
+    torch.cuda.synchronize()
+    assert dg.dg_sync_status(stream) == dg.DG_OK
+
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = dg.dg_launch_count()
+    w0 = time.time()
+    t_start.record(stream)
+    for i in range(args.steps):
+        assert step(i, evs[i]) == 0
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    w1 = time.time()
+    barrier(world)
+    launches = dg.dg_launch_count() - n0
+    time.sleep(0.25)
+    sampler.stop()
+    assert dg.dg_sync_status(stream) == dg.DG_OK
+    elapsed = t_start.elapsed_time(t_end) * 1e-3
+    elapsed_max = max_over_ranks(elapsed, world, dev)
+    value = step_bytes * world / elapsed_max / 1e9
+    gemv_times = [a.elapsed_time(b) * 1e-3 for a, b in evs]
+    gemv_avg = sum(gemv_times) / len(gemv_times)
+    gemv_bytes = flops_bytes(gv)[1]
+    achieved = gemv_bytes / gemv_avg / 1e9
+    peak_hbm = peaks["hbm_gbs"]
+    traffic = kernel_traffic("gemv.cu", "gemv_n_decode_4096x14336.txt")
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_max / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "bytes_per_step": step_bytes,
+                   "l2": f"inputs rotate through {ROTATE} copies of W and K (352 MB > 126 MB L2)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "kernel": "gemv_n (x*W, 117 MB of W)", "achieved": achieved,
+                     "peak": peak_hbm, "unit": "GB/s", "frac": achieved / peak_hbm,
+                     "traffic": traffic, "algorithmic_bytes": gemv_bytes, "avg_launch_us": gemv_avg * 1e6,
+                     "peak_source": f"{peaks['source']} hbm_gbs (STREAM-style copy)"},
+        "gpu_launches": int(launches),
+        "clocks": sampler.summary(w0, w1),
+    }
+    if rank == 0:
+        if not args.skip_cpu:
+            result["e2e"] = e2e(dg, gv, gk, dev, stream, max(3, min(args.steps, 20)))
+        if not args.no_per_shape:
+            result["per_shape"] = per_shape(dg, peaks, args.quick)
+        if not args.skip_cpu:
+            result["cpu_baseline"] = cpu_baseline(args.quick)
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        barrier(world)
+        dist.destroy_process_group()
+
+
+def e2e(dg, gv, gk, dev, stream, steps):
+    """Same step through dg_gemm with host buffers: pinned host -> device copies
+    of x, W and K, both products, device -> host copies of both outputs, every
+    step, timed with CUDA events."""
+    hx = gv.A.base.pin_memory()
+    hw = gv.B.base.pin_memory()
+    hk = gk.B.base.pin_memory()
+    hy1 = torch.empty_like(gv.C.base).pin_memory()
+    hy2 = torch.empty_like(gk.C.base).pin_memory()
+    dx = torch.empty_like(hx, device=dev)
+    dw = torch.empty_like(hw, device=dev)
+    dk = torch.empty_like(hk, device=dev)
+    dy1 = torch.empty_like(hy1, device=dev)
+    dy2 = torch.empty_like(hy2, device=dev)
+    vx = dg.make_view(dx.data_ptr(), gv.A.shape, gv.A.stride, 1, "bf16")
+    vw = dg.make_view(dw.data_ptr(), gv.B.shape, gv.B.stride, 1, "bf16")
+    vk = dg.make_view(dk.data_ptr(), gk.B.shape, gk.B.stride, 1, "bf16")
+    vy1 = dg.make_view(dy1.data_ptr(), gv.C.shape, gv.C.stride, 1, "bf16")
+    vy2 = dg.make_view(dy2.data_ptr(), gk.C.shape, gk.C.stride, 1, "bf16")
+
+    def one():
+        dx.copy_(hx, non_blocking=True)
+        dw.copy_(hw, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        assert dg.dg_gemm(vx, vw, vy1, 1.0, 0.0, None, None, stream) == dg.DG_OK
+        assert dg.dg_gemm(vx, vk, vy2, 1.0, 0.0, None, None, stream) == dg.DG_OK
+        hy1.copy_(dy1, non_blocking=True)
+        hy2.copy_(dy2, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    t = a.elapsed_time(b) * 1e-3 / steps
+    step_bytes = flops_bytes(gv)[1] + flops_bytes(gk)[1]
+    h2d = (hx.numel() * hx.element_size() + hw.numel() * hw.element_size() + hk.numel() * hk.element_size())
+    d2h = hy1.numel() * hy1.element_size() + hy2.numel() * hy2.element_size()
+    return {"value": step_bytes / t / 1e9, "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": t * 1e3, "steps": steps}
+
+
+# ---------------------------------------------------------- the CPU oracle
+
+def _oracle_step(orc, gv_s, gk, threads):
+    orc.gemm(gv_s, want_bound=False, nthreads=threads)
+    orc.gemm(gk, want_bound=False, nthreads=threads)
+
+
+def _column_sample(gv: W.Problem, cols: int) -> W.Problem:
+    """x * W[:, :cols] as a view of the same W (no copy)."""
+    B = W.Operand(gv.B.base, (gv.K, cols), gv.B.stride, 1, gv.B.dtype)
+    C = W.row_major(torch.empty(1, cols, dtype=torch.bfloat16), "bf16")
+    return W.Problem(gv.name + f"_cols{cols}", gv.A, B, C)
+
+
+def cpu_baseline(quick: bool, target_s: float = 12.0):
+    """The FP64 oracle, as it stands, on this host's cores: repeated decode
+    steps (x*W and x*K^T) for about `target_s` seconds."""
+    import oracle
+
+    orc = oracle.default()
+    threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    gv, gk = W.cfg_gemv(), W.cfg_gemv_kt()
+    step_bytes = flops_bytes(gv)[1] + flops_bytes(gk)[1]
+    t0 = time.perf_counter()
+    _oracle_step(orc, gv, gk, threads)
+    one = time.perf_counter() - t0
+    reps = 1 if quick else max(1, int(target_s / max(one, 1e-3)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        _oracle_step(orc, gv, gk, threads)
+    t = (time.perf_counter() - t0) / reps
+    return {"value": step_bytes / t / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{reps} full decode steps (x*W 1x4096x14336 and x*K^T 1x4096x128), FP64, "
+                      f"{t:.3f} s per step"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return  # the oracle runs once, on rank 0; the other ranks have no work
+    import oracle
+
+    orc = oracle.default()
+    threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    gv, gk = W.cfg_gemv(), W.cfg_gemv_kt()
+    # size each step's sample so the whole run stays within about two minutes
+    t0 = time.perf_counter()
+    _oracle_step(orc, _column_sample(gv, 1024), gk, threads)
+    per_col = (time.perf_counter() - t0) / 1024
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    cols = int(min(gv.N, max(256, budget / max(per_col, 1e-9))))
+    cols -= cols % 8
+    sample = _column_sample(gv, cols)
+    step_bytes = flops_bytes(sample)[1] + flops_bytes(gk)[1]
+    for _ in range(args.warmup):
+        _oracle_step(orc, sample, gk, threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(orc, sample, gk, threads)
+    t = time.perf_counter() - t0
+    value = step_bytes * args.steps / t / 1e9
+    desc = (f"per step: x*W[:, :{cols}] (of 14336 columns) and x*K^T 1x4096x128, FP64 oracle")
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": desc}, "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["dg", "reference"], default="dg")
+    ap.add_argument("--quick", action="store_true", help="fewer repetitions in the side measurements")
+    ap.add_argument("--no-per-shape", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true", help="no CPU baseline and no e2e leg (profiling runs)")
+    ap.add_argument("--shape", default=None,
+                    help="time only this per-shape workload (small, gemv, gemv_kt, thin, square_bf16, "
+                         "square_e4m3, strided) and print its line")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    elif args.shape:
+        run_one_shape(args)
+    else:
+        run_dg(args)
+
+
+if __name__ == "__main__":
+    main()

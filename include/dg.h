@@ -1,0 +1,213 @@
+/*
+ * libdg — strided-view GEMM for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Every entry point computes (part of) the deep-learning GEMM
+ *
+ *     C[m][n] = alpha * sa[m] * sb[n] * sum_k A[m][k] * B[k][n]  +  beta * C[m][n]
+ *
+ * ("DeepGEMM: a recalibration of the compute paradigm", §2.3 and the problem
+ * template of §4.1; "DeepGEMM deep dive", §1.1 for the operation and §2.4 for
+ * the FP8 rescale), with FP32 accumulation, over operands given as strided
+ * "views" that are read in place (recalibration page, §2.1-§2.2: no reshape or
+ * contiguous() copy).
+ *
+ * Conventions shared by all entry points
+ *  - Memory: the caller owns every buffer.  Data pointers are DEVICE pointers
+ *    (cudaMalloc / torch CUDA tensors / managed memory) on the current device.
+ *    The library keeps no pointer after a call returns.  It owns a small
+ *    per-device workspace (status word, split-K partials) allocated on first
+ *    use; the first call on a device should therefore come before any CUDA
+ *    stream capture.
+ *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *    default stream).  Calls are asynchronous on that stream.
+ *  - Errors: argument errors are returned synchronously, before anything is
+ *    launched, and leave C untouched.  A device-side wait that gives up (see
+ *    dg_sync_status) is reported by dg_sync_status.
+ *  - Thread safety: calls may be made from several host threads.  The
+ *    split-K workspace is one per device: two calls that both take the
+ *    split-K path (dg_plan_info.split_k > 1) must not run concurrently on
+ *    different streams (serialise them, or set DG_OPT_MAX_SPLIT_K to 1).
+ *    dg_set_option is process-global and should not race with running calls.
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element types.  A and B must have the same type (F16, BF16 or E4M3; F32
+ * inputs are accepted on the CUDA-core path only).  C may be F32, F16 or BF16.
+ * E4M3 is OCP FP8 E4M3 ("fn": largest finite 448, no infinities). */
+typedef enum {
+    DG_F32 = 0,
+    DG_F16 = 1,
+    DG_BF16 = 2,
+    DG_E4M3 = 3
+} dg_dtype;
+
+/* Status codes.  The error table of the recalibration page (§5.1) names the
+ * failure classes: stride overflow, pointers not on the device, non-finite
+ * alpha/beta, unsupported combinations. */
+typedef enum {
+    DG_OK = 0,
+    DG_ERR_NULL = 1,        /* a required pointer is NULL                        */
+    DG_ERR_NDIM = 2,        /* ndim not in 1..4 or row_dims not in 0..ndim        */
+    DG_ERR_SHAPE = 3,       /* negative size, or A/B/C sizes disagree (K, M, N)   */
+    DG_ERR_DTYPE = 4,       /* unsupported type or A/B type mismatch              */
+    DG_ERR_STRIDE = 5,      /* negative stride, byte extent overflows int64, or
+                               C has two elements at one address                 */
+    DG_ERR_ALIGN = 6,       /* pointer or stride not a multiple of the element    */
+    DG_ERR_POINTER = 7,     /* pointer is not device-accessible                   */
+    DG_ERR_VALUE = 8,       /* alpha or beta not finite                           */
+    DG_ERR_UNSUPPORTED = 9, /* valid request this build does not implement        */
+    DG_ERR_CUDA = 10,       /* a CUDA runtime call failed                          */
+    DG_ERR_TIMEOUT = 11     /* a device-side wait gave up (see dg_sync_status)    */
+} dg_status;
+
+/*
+ * A strided view ("DeepGEMM: a recalibration of the compute paradigm", §3.2).
+ *  ptr       address of element (0,...,0); device memory.
+ *  ndim      1..4 dims; shape[d] >= 0 elements; stride[d] >= 0 in BYTES
+ *            (not elements: §3.2 fixes byte strides).
+ *  row_dims  the first row_dims dims flatten row-major (last fastest) into the
+ *            matrix row index, the remaining dims into the column index.  So a
+ *            [M,K] row-major matrix is shape {M,K}, stride {K*es, es},
+ *            row_dims 1; its transpose as a [K,M] operand is shape {K,M},
+ *            stride {es, K*es}; an NCHW tensor read as [N*H*W, C] is shape
+ *            {N,H,W,C}, strides {sN,sH,sW,sC}, row_dims 3.
+ *  dtype     a dg_dtype value.
+ * The page's `layout` tag and `align` hint are not fields: strides are
+ * authoritative and alignment is derived from ptr and strides.  A zero stride
+ * broadcasts (allowed for A and B, rejected for C unless the dim has size 1).
+ */
+typedef struct {
+    void *ptr;
+    int32_t ndim;
+    int32_t row_dims;
+    int64_t shape[4];
+    int64_t stride[4];
+    int32_t dtype;
+    int32_t reserved; /* set to 0 */
+} dg_view;
+
+/*
+ * dg_gemm — C = alpha * diag(sa) * (A B) * diag(sb) + beta * C.
+ *  A [M x K], B [K x N], C [M x N]: views as above (C is read when beta != 0
+ *  and written always; it must not overlap A or B).
+ *  alpha, beta: finite.  beta == 0 never reads C (NaN in C does not leak);
+ *  alpha == 0 never reads A or B and yields beta * C.
+ *  scale_a: device float32[M] or NULL (all ones); scale_b: device float32[N]
+ *  or NULL.  They are the per-row (per-token) scale of A and the per-column
+ *  (per-channel) scale of B of the FP8 precision mode ("DeepGEMM deep dive",
+ *  §2.4), applied exactly once in the epilogue; allowed for every input type.
+ * Returns DG_OK once the work is enqueued on `stream`.
+ */
+dg_status dg_gemm(const dg_view *A, const dg_view *B, const dg_view *C,
+                  float alpha, float beta,
+                  const float *scale_a, const float *scale_b,
+                  void *stream);
+
+/*
+ * dg_gemv — y = alpha * x W + beta * y for a single row (or up to 8 rows) of
+ * activations: the decode-time thin GEMM of "DeepGEMM is not a new model: the
+ * inner discipline of GPU matrix multiplication" (§2, [1,4096]x[4096,14336];
+ * §4, [1,4096]x[4096,128]).  x is [R x K] with R <= 8 (a 1-D view of K
+ * elements is one row), W is [K x N], y is [R x N].  It is dg_gemm with no
+ * scales; dg_gemm itself also routes M <= 8 here when W's layout allows.
+ * Returns DG_ERR_UNSUPPORTED if R > 8.
+ */
+dg_status dg_gemv(const dg_view *x, const dg_view *W, const dg_view *y,
+                  float alpha, float beta, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *dg_status_string(dg_status s);
+
+/*
+ * dg_sync_status — synchronise `stream`, then return and clear the device
+ * error word of the current device: DG_ERR_TIMEOUT if a kernel's bounded wait
+ * gave up since the last check (its output is then undefined), DG_ERR_CUDA if
+ * the synchronisation failed, DG_OK otherwise.
+ */
+dg_status dg_sync_status(void *stream);
+
+/* ----------------------------------------------------------- introspection
+ * Host-only helpers: they read no device memory and launch nothing, so they
+ * also work on a machine without a GPU. */
+
+/* Result of view analysis (recalibration page, §2.2: effective span,
+ * contiguous segments).  Size-1 dims are dropped and neighbouring dims merged
+ * when stride[i] == stride[i+1] * shape[i+1], separately for the row group and
+ * the column group. */
+typedef struct {
+    int64_t rows, cols;
+    int32_t n_row, n_col;       /* merged dims in each group (0 = extent 1)     */
+    int64_t row_shape[4], row_stride[4];
+    int64_t col_shape[4], col_stride[4];
+    int32_t unit_dim;           /* 1: columns unit-stride (row-major), 2: rows
+                                   unit-stride (column-major), 0: neither          */
+    int32_t tma_ok;             /* expressible as one 2-D TMA tensor map         */
+    int64_t span_bytes;         /* max byte offset touched + element size         */
+    int32_t vec_bytes;          /* widest aligned contiguous run (1..16 bytes)    */
+    int32_t reserved;
+} dg_view_info;
+
+dg_status dg_analyse_view(const dg_view *v, dg_view_info *out);
+
+/* Kernel families the dispatcher chooses between. */
+typedef enum {
+    DG_KIND_NONE = 0,      /* nothing to do (M == 0 or N == 0)                     */
+    DG_KIND_SCALE_C = 1,   /* alpha == 0 or K == 0: C = beta * C                   */
+    DG_KIND_SIMT = 2,      /* CUDA-core tiled kernel, any view                      */
+    DG_KIND_GEMV_N = 3,    /* M <= 8, W unit-stride along N                         */
+    DG_KIND_GEMV_K = 4,    /* M <= 8, W unit-stride along K                         */
+    DG_KIND_UMMA = 5       /* tcgen05 tensor-core kernel, TMEM accumulators          */
+} dg_kind;
+
+typedef struct {
+    int32_t kind;          /* dg_kind                                               */
+    int32_t swap_ab;       /* UMMA: computes C^T = B^T A^T (tensor-core M runs on N) */
+    int32_t p_gather;      /* UMMA: the M-side operand is loaded by threads, not TMA */
+    int32_t p_mn_major;    /* UMMA: operand layouts in smem (0 K-major, 1 MN-major)  */
+    int32_t q_mn_major;
+    int32_t block_m, block_n, block_k;
+    int32_t stages;
+    int32_t split_k;
+    int32_t grid;          /* CTAs launched                                          */
+    int32_t vec_bytes;     /* gather / GEMV vector width                             */
+    int64_t M, N, K;
+} dg_plan_info;
+
+/* The dispatch decision dg_gemm would take for these views (pointers are only
+ * used for their alignment).  `num_sms` <= 0 means the current device's count
+ * (148 when no device is present). */
+dg_status dg_plan(const dg_view *A, const dg_view *B, const dg_view *C,
+                  float alpha, float beta, int has_scales, int num_sms,
+                  dg_plan_info *out);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t dg_launch_count(void);
+
+/* Process-global options (tests and benchmarks). */
+typedef enum {
+    DG_OPT_FORCE_KIND = 1,        /* 0 = automatic, else a dg_kind to use when it is
+                                     applicable (DG_KIND_SIMT always is)              */
+    DG_OPT_WAIT_TIMEOUT_MS = 2,   /* bound on every device-side wait (default 2000)   */
+    DG_OPT_TEST_STALL = 3,        /* 1: the tensor-core kernel's loader issues no
+                                     copies, so its waits run out and the call
+                                     reports DG_ERR_TIMEOUT (tests of the bound)      */
+    DG_OPT_MAX_SPLIT_K = 4        /* upper bound on split-K (default 16; 1 disables)   */
+} dg_option;
+
+dg_status dg_set_option(int option, int64_t value);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int dg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H_ */

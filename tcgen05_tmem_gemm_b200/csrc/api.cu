@@ -1,0 +1,567 @@
+// C-ABI entry points of libdg: argument validation, the view-analysis
+// dispatcher, per-device state and the launches.
+//
+// Dispatch ("DeepGEMM: a recalibration of the compute paradigm", §2.2: view
+// analysis picks the tiling from the contiguous segments; "DeepGEMM deep
+// dive", §4.1: compare the arithmetic intensity with the machine balance):
+//   M == 0 or N == 0         -> nothing
+//   alpha == 0 or K == 0     -> C = beta * C
+//   M <= 8, W unit-stride    -> GEMV (HBM-bound: 2 flops per weight byte pair)
+//   16-bit / E4M3 operands   -> tcgen05 tensor-core kernel; operands TMA can
+//                               describe are loaded by TMA, one that it cannot
+//                               (non-16-byte strides) by thread gathers; thin
+//                               M (<= 64) swaps A and B so N fills the
+//                               128-row tensor-core tile; few tiles -> split-K
+//   anything else            -> CUDA-core tiled kernel
+#include <atomic>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "dg_internal.h"
+
+namespace dg {
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_force_kind{0};
+std::atomic<int64_t> g_timeout_ms{2000};
+std::atomic<int> g_stall{0};
+std::atomic<int> g_max_split{16};
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kWorkspaceBytes = size_t(24) << 20;   // split-K partial tiles
+constexpr size_t kCounterCount = 1 << 16;              // split-K arrival counters
+
+struct DeviceState {
+    bool ready = false;
+    int num_sms = 0;
+    int *err_word = nullptr;       // device
+    uint32_t *counters = nullptr;  // device, zeroed
+    float *ws = nullptr;           // device
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+dg_status device_state(DeviceState **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DG_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState &d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DG_ERR_CUDA;
+        if (cudaMalloc(&d.err_word, sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
+        if (cudaMalloc(&d.counters, kCounterCount * sizeof(uint32_t)) != cudaSuccess) return DG_ERR_CUDA;
+        if (cudaMalloc(&d.ws, kWorkspaceBytes) != cudaSuccess) return DG_ERR_CUDA;
+        if (cudaMemset(d.err_word, 0, sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
+        if (cudaMemset(d.counters, 0, kCounterCount * sizeof(uint32_t)) != cudaSuccess) return DG_ERR_CUDA;
+        if (cudaDeviceSynchronize() != cudaSuccess) return DG_ERR_CUDA;
+        if (!g_encode) {
+            cudaDriverEntryPointQueryResult q;
+            void *fn = nullptr;
+            if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+                    cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || !fn)
+                return DG_ERR_CUDA;
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        d.ready = true;
+    }
+    *out = &d;
+    return DG_OK;
+}
+
+bool device_accessible(const void *p) {
+    if (!p) return false;
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (a.type == cudaMemoryTypeManaged) return true;
+    if (a.type != cudaMemoryTypeDevice) return false;
+    int dev = -1;
+    cudaGetDevice(&dev);
+    return a.device == dev;
+}
+
+DevView dev_view(const dg_view *v, const ViewInfo &vi) {
+    DevView d{};
+    d.ptr = static_cast<const char *>(v->ptr);
+    d.row = vi.row;
+    d.col = vi.col;
+    d.dtype = v->dtype;
+    return d;
+}
+
+// stride of a group with at most one merged dim (0 when the group is empty)
+int64_t axis_stride(const Axis &a) { return a.n == 1 ? a.stride[0] : 0; }
+
+struct Plan {
+    dg_plan_info info{};
+    // UMMA specifics
+    bool fp8 = false;
+    size_t smem = 0;
+};
+
+struct Views {
+    const dg_view *A, *B, *C;
+    ViewInfo a, b, c;
+};
+
+uint32_t make_idesc(int in_dtype, bool p_mn, bool q_mn, int bn) {
+    uint32_t d = 0;
+    d |= 1u << 4;                                    // D format: F32
+    const uint32_t fmt = (in_dtype == DG_BF16) ? 1u : 0u;  // F16 = 0, BF16 = 1; E4M3 = 0 (kind::f8f6f4)
+    d |= fmt << 7;                                   // A format
+    d |= fmt << 10;                                  // B format
+    d |= (p_mn ? 1u : 0u) << 15;                     // A major (1 = MN)
+    d |= (q_mn ? 1u : 0u) << 16;                     // B major
+    d |= (uint32_t)(bn >> 3) << 17;                  // N >> 3
+    d |= (uint32_t)(128 >> 4) << 24;                 // M >> 4
+    return d;
+}
+
+bool gemv_applicable(const Views &v, int64_t M, int64_t N, int64_t K, int kind) {
+    const int dt = v.A->dtype;
+    if (dt != DG_F16 && dt != DG_BF16) return false;
+    if (M > 8 || K > INT32_MAX || N > INT32_MAX) return false;
+    if (v.c.row.n > 1 || v.c.col.n > 1) return false;
+    const uintptr_t wp = reinterpret_cast<uintptr_t>(v.B->ptr);
+    if (wp % 16) return false;
+    if (kind == DG_KIND_GEMV_N) {
+        // B: columns one unit-stride dim, rows one dim with a 16-byte multiple stride
+        if (!(v.b.col.n == 1 && v.b.col.stride[0] == 2 && v.b.row.n <= 1)) return false;
+        if (N % 8) return false;
+        if (v.b.row.n == 1 && v.b.row.stride[0] % 16) return false;
+        return true;
+    }
+    if (kind == DG_KIND_GEMV_K) {
+        if (!(v.b.row.n == 1 && v.b.row.stride[0] == 2 && v.b.col.n <= 1)) return false;
+        if (K % 8) return false;
+        if (v.b.col.n == 1 && v.b.col.stride[0] % 16) return false;
+        return true;
+    }
+    return false;
+}
+
+// Which UMMA configuration serves these views (false: none).
+bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, int num_sms, Plan *pl) {
+    const int dt = v.A->dtype;
+    if (dt != DG_F16 && dt != DG_BF16 && dt != DG_E4M3) return false;
+    if (v.c.row.n > 1 || v.c.col.n > 1) return false;
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return false;
+    const bool a_tma = v.a.tma_ok, b_tma = v.b.tma_ok;
+    if (!a_tma && !b_tma) return false;
+    const bool thin = (M <= 64 && N >= 2 * M);
+    bool swap;
+    if (!a_tma) swap = false;       // A is loaded by threads as the M-side operand
+    else if (!b_tma) swap = true;   // B is, after the swap
+    else swap = thin;
+    const ViewInfo &pvi = swap ? v.b : v.a;
+    const bool p_tma = swap ? b_tma : a_tma;
+    // unit-stride direction of P(i, k) and Q(k, j)
+    // A: rows = i/m, cols = k.  B: rows = k, cols = j/n.
+    bool p_mn, q_mn;
+    if (!swap) {
+        p_mn = (v.a.unit_dim == 2);
+        q_mn = (v.b.unit_dim == 1);
+    } else {
+        p_mn = (v.b.unit_dim == 1);
+        q_mn = (v.a.unit_dim == 2);
+    }
+    int gather_vec = 1;
+    if (!p_tma) {
+        // innermost unit-stride dim of the gathered operand decides its layout
+        const Axis &ig = swap ? pvi.col : pvi.row;   // i group of P
+        const Axis &kg = swap ? pvi.row : pvi.col;   // k group of P
+        const int es = pvi.es;
+        if (ig.n >= 1 && ig.stride[ig.n - 1] == es) p_mn = true;
+        else if (kg.n >= 1 && kg.stride[kg.n - 1] == es) p_mn = false;
+        else p_mn = false;
+        gather_vec = pvi.vec_bytes / es;
+        if (gather_vec < 1) gather_vec = 1;
+        if (!(ig.n >= 1 && ig.stride[ig.n - 1] == es) && !(kg.n >= 1 && kg.stride[kg.n - 1] == es)) gather_vec = 1;
+    }
+    const int64_t Mi = swap ? N : M, Nj = swap ? M : N;
+    const int es = elem_size(dt);
+    const int bk = 128 / es;
+    int bn;
+    const int64_t tiles_i = (Mi + 127) / 128;
+    if (Nj <= 64 && !q_mn) {
+        bn = (int)((Nj + 15) / 16) * 16;
+    } else if (tiles_i * ((Nj + 255) / 256) >= num_sms) {
+        bn = 256;
+    } else if (Nj > 64) {
+        bn = 128;
+    } else {
+        bn = 64;
+    }
+    if (q_mn) {
+        const int per = 128 / es;  // MN elements per 128-byte box row
+        bn = (int)(((bn + per - 1) / per) * per);
+        if (bn > 256) return false;
+    }
+    const int64_t tiles_j = (Nj + bn - 1) / bn;
+    const int64_t tiles = tiles_i * tiles_j;
+    const int64_t kb_total = (K + bk - 1) / bk;
+    int64_t split = 1;
+    const int max_split = g_max_split.load();
+    if (tiles * 2 <= num_sms && kb_total >= 8 && max_split > 1) {
+        split = std::min<int64_t>(num_sms / tiles, kb_total / 4);
+        split = std::min<int64_t>(split, max_split);
+        if (split < 1) split = 1;
+    }
+    int64_t kb_per = (kb_total + split - 1) / split;
+    split = (kb_total + kb_per - 1) / kb_per;
+    if (split > 1) {
+        const size_t need = (size_t)tiles * split * 128 * bn * sizeof(float);
+        if (need > kWorkspaceBytes || (size_t)tiles * 4 > kCounterCount) { split = 1; kb_per = kb_total; }
+    }
+    const int64_t units = tiles * split;
+    if (units > INT32_MAX) return false;
+    const int stages = umma_max_stages(bn, !p_tma);
+    dg_plan_info &in = pl->info;
+    in.kind = DG_KIND_UMMA;
+    in.swap_ab = swap;
+    in.p_gather = !p_tma;
+    in.p_mn_major = p_mn;
+    in.q_mn_major = q_mn;
+    in.block_m = 128;
+    in.block_n = bn;
+    in.block_k = bk;
+    in.stages = stages;
+    in.split_k = (int32_t)split;
+    in.grid = (int32_t)std::min<int64_t>(units, num_sms);
+    in.vec_bytes = p_tma ? 16 : gather_vec * es;
+    pl->fp8 = (dt == DG_E4M3);
+    pl->smem = umma_smem_bytes(bn, 128, stages, !p_tma);
+    return true;
+}
+
+dg_status make_plan(Views &v, float alpha, float beta, int num_sms, Plan *pl) {
+    (void)beta;
+    dg_status st;
+    if ((st = analyse(v.A, false, &v.a)) != DG_OK) return st;
+    if ((st = analyse(v.B, false, &v.b)) != DG_OK) return st;
+    if ((st = analyse(v.C, true, &v.c)) != DG_OK) return st;
+    const int64_t M = v.a.rows, K = v.a.cols, N = v.b.cols;
+    if (v.b.rows != K || v.c.rows != M || v.c.cols != N) return DG_ERR_SHAPE;
+    if (v.A->dtype != v.B->dtype) return DG_ERR_DTYPE;
+    if (v.C->dtype == DG_E4M3) return DG_ERR_DTYPE;
+    if (!std::isfinite(alpha) || !std::isfinite(beta)) return DG_ERR_VALUE;
+    dg_plan_info &in = pl->info;
+    std::memset(&in, 0, sizeof(in));
+    in.M = M;
+    in.N = N;
+    in.K = K;
+    in.split_k = 1;
+    if (M == 0 || N == 0) { in.kind = DG_KIND_NONE; return DG_OK; }
+    if (alpha == 0.f || K == 0) { in.kind = DG_KIND_SCALE_C; return DG_OK; }
+    const int force = g_force_kind.load();
+    const bool simt_only = (v.A->dtype == DG_F32) || force == DG_KIND_SIMT;
+    if (!simt_only) {
+        if (force == DG_KIND_GEMV_N || force == DG_KIND_GEMV_K) {
+            if (gemv_applicable(v, M, N, K, force)) { in.kind = force; return DG_OK; }
+        } else if (force == DG_KIND_UMMA) {
+            if (umma_plan(v, M, N, K, num_sms, pl)) return DG_OK;
+        } else {
+            if (M <= 8) {
+                if (gemv_applicable(v, M, N, K, DG_KIND_GEMV_N)) { in.kind = DG_KIND_GEMV_N; return DG_OK; }
+                if (gemv_applicable(v, M, N, K, DG_KIND_GEMV_K)) { in.kind = DG_KIND_GEMV_K; return DG_OK; }
+            }
+            if (umma_plan(v, M, N, K, num_sms, pl)) return DG_OK;
+        }
+    }
+    if (M > int64_t(65535) * 64 || N > INT32_MAX || K > INT32_MAX) return DG_ERR_UNSUPPORTED;
+    in.kind = DG_KIND_SIMT;
+    in.block_m = 64;
+    in.block_n = 64;
+    in.block_k = 16;
+    return DG_OK;
+}
+
+CUtensorMapDataType tma_dtype(int dt) {
+    switch (dt) {
+    case DG_F16: return CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    case DG_BF16: return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    default: return CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    }
+}
+
+// 2-D tensor map: `inner` elements along the unit-stride dim, `outer` along
+// the other (byte stride `outer_stride`), box = 128 bytes x box_outer rows,
+// 128-byte swizzle, zero fill out of bounds.
+bool encode_2d(CUtensorMap *m, int dt, const void *ptr, int64_t inner, int64_t outer, int64_t outer_stride,
+               int box_outer) {
+    const int es = elem_size(dt);
+    if (outer <= 1) outer_stride = ((inner * es + 15) / 16) * 16;  // any legal value
+    if (outer_stride == 0) outer_stride = 16;
+    cuuint64_t gdim[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+    cuuint64_t gstride[1] = {(cuuint64_t)outer_stride};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / es), (cuuint32_t)box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, tma_dtype(dt), 2, const_cast<void *>(ptr), gdim, gstride, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+EpiParams epi_params(const Views &v, bool swap, float alpha, float beta, const float *sa, const float *sb) {
+    EpiParams e{};
+    e.c = static_cast<char *>(v.C->ptr);
+    const int64_t crs = axis_stride(v.c.row), ccs = axis_stride(v.c.col);
+    e.ci = swap ? ccs : crs;
+    e.cj = swap ? crs : ccs;
+    e.c_dtype = v.C->dtype;
+    const int ces = elem_size(v.C->dtype);
+    e.vec_ok = (e.cj == ces) && (reinterpret_cast<uintptr_t>(e.c) % 16 == 0) && (e.ci % 16 == 0);
+    e.alpha = alpha;
+    e.beta = beta;
+    e.scale_i = swap ? sb : sa;
+    e.scale_j = swap ? sa : sb;
+    return e;
+}
+
+dg_status launch(const Views &v, const Plan &pl, float alpha, float beta, const float *sa, const float *sb,
+                 cudaStream_t stream, DeviceState *ds) {
+    const dg_plan_info &in = pl.info;
+    cudaError_t err = cudaSuccess;
+    switch (in.kind) {
+    case DG_KIND_NONE: return DG_OK;
+    case DG_KIND_SCALE_C: {
+        err = launch_scale_c(dev_view(v.C, v.c), in.M, in.N, beta, stream);
+        break;
+    }
+    case DG_KIND_SIMT: {
+        SimtParams p{};
+        p.a = dev_view(v.A, v.a);
+        p.b = dev_view(v.B, v.b);
+        p.c = dev_view(v.C, v.c);
+        p.M = (int32_t)in.M;
+        p.N = (int32_t)in.N;
+        p.K = (int32_t)in.K;
+        p.epi = epi_params(v, false, alpha, beta, sa, sb);
+        err = launch_simt(p, stream);
+        break;
+    }
+    case DG_KIND_GEMV_N:
+    case DG_KIND_GEMV_K: {
+        GemvParams p{};
+        p.x = dev_view(v.A, v.a);
+        p.w = static_cast<const char *>(v.B->ptr);
+        p.w_ld = (in.kind == DG_KIND_GEMV_N) ? axis_stride(v.b.row) : axis_stride(v.b.col);
+        p.R = (int32_t)in.M;
+        p.K = (int32_t)in.K;
+        p.N = (int32_t)in.N;
+        p.in_dtype = v.A->dtype;
+        p.epi = epi_params(v, false, alpha, beta, sa, sb);
+        int grid = 0;
+        err = (in.kind == DG_KIND_GEMV_N) ? launch_gemv_n(p, stream, ds->num_sms, &grid)
+                                          : launch_gemv_k(p, stream, ds->num_sms, &grid);
+        break;
+    }
+    case DG_KIND_UMMA: {
+        const bool swap = in.swap_ab != 0;
+        const int dt = v.A->dtype;
+        const int es = elem_size(dt);
+        const int bk = in.block_k, bn = in.block_n;
+        const int64_t Mi = swap ? in.N : in.M, Nj = swap ? in.M : in.N;
+        CUtensorMap tp, tq;
+        std::memset(&tp, 0, sizeof(tp));
+        std::memset(&tq, 0, sizeof(tq));
+        // P(i, k): A (no swap) or B^T; Q(k, j): B (no swap) or A^T
+        const dg_view *Pv = swap ? v.B : v.A;
+        const dg_view *Qv = swap ? v.A : v.B;
+        const ViewInfo &pi = swap ? v.b : v.a;
+        const ViewInfo &qi = swap ? v.a : v.b;
+        const Axis &p_i = swap ? pi.col : pi.row, &p_k = swap ? pi.row : pi.col;
+        const Axis &q_k = swap ? qi.col : qi.row, &q_j = swap ? qi.row : qi.col;
+        if (!in.p_gather) {
+            const bool ok = in.p_mn_major ? encode_2d(&tp, dt, Pv->ptr, Mi, in.K, axis_stride(p_k), bk)
+                                          : encode_2d(&tp, dt, Pv->ptr, in.K, Mi, axis_stride(p_i), 128);
+            if (!ok) return DG_ERR_UNSUPPORTED;
+        }
+        {
+            const bool ok = in.q_mn_major ? encode_2d(&tq, dt, Qv->ptr, Nj, in.K, axis_stride(q_k), bk)
+                                          : encode_2d(&tq, dt, Qv->ptr, in.K, Nj, axis_stride(q_j), bn);
+            if (!ok) return DG_ERR_UNSUPPORTED;
+        }
+        UmmaParams p{};
+        p.Mi = (int32_t)Mi;
+        p.Nj = (int32_t)Nj;
+        p.K = (int32_t)in.K;
+        p.bn = bn;
+        p.bk = bk;
+        p.stages = in.stages;
+        p.tiles_i = (int32_t)((Mi + 127) / 128);
+        p.tiles_j = (int32_t)((Nj + bn - 1) / bn);
+        p.split_k = in.split_k;
+        p.kb_total = (int32_t)((in.K + bk - 1) / bk);
+        p.kb_per_split = (p.kb_total + p.split_k - 1) / p.split_k;
+        p.num_units = p.tiles_i * p.tiles_j * p.split_k;
+        p.p_mn_major = in.p_mn_major;
+        p.q_mn_major = in.q_mn_major;
+        p.idesc = make_idesc(dt, in.p_mn_major, in.q_mn_major, bn);
+        int tc = 32;
+        while (tc < 2 * bn) tc *= 2;
+        p.tmem_cols = tc;
+        p.epi = epi_params(v, swap, alpha, beta, sa, sb);
+        if (in.p_gather) {
+            DevView d{};
+            d.ptr = static_cast<const char *>(Pv->ptr);
+            d.row = p_i;
+            d.col = p_k;
+            d.dtype = dt;
+            p.pv = d;
+            p.gather_vec = in.vec_bytes / es;
+        }
+        p.ws = ds->ws;
+        p.counters = ds->counters;
+        p.err_word = ds->err_word;
+        p.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
+        p.stall_loader = g_stall.load();
+        err = launch_umma(p, &tp, &tq, pl.fp8, in.p_gather != 0, in.grid, pl.smem, stream);
+        break;
+    }
+    default: return DG_ERR_UNSUPPORTED;
+    }
+    if (err != cudaSuccess) return DG_ERR_CUDA;
+    g_launches.fetch_add(1);
+    return DG_OK;
+}
+
+}  // namespace
+}  // namespace dg
+
+using namespace dg;
+
+extern "C" {
+
+dg_status dg_gemm(const dg_view *A, const dg_view *B, const dg_view *C, float alpha, float beta,
+                  const float *scale_a, const float *scale_b, void *stream) {
+    if (!A || !B || !C) return DG_ERR_NULL;
+    Views v{A, B, C, {}, {}, {}};
+    Plan pl;
+    // argument errors are reported before any CUDA call
+    dg_status st = make_plan(v, alpha, beta, 148, &pl);
+    if (st != DG_OK) return st;
+    if (pl.info.kind == DG_KIND_NONE) return DG_OK;
+    DeviceState *ds = nullptr;
+    st = device_state(&ds);
+    if (st != DG_OK) return st;
+    if (ds->num_sms != 148) {
+        st = make_plan(v, alpha, beta, ds->num_sms, &pl);
+        if (st != DG_OK) return st;
+    }
+    const dg_plan_info &in = pl.info;
+    if (in.kind == DG_KIND_NONE) return DG_OK;
+    // every buffer the launch touches must live on this device
+    const bool use_ab = in.kind != DG_KIND_SCALE_C;
+    if (use_ab && (!device_accessible(A->ptr) || !device_accessible(B->ptr))) return DG_ERR_POINTER;
+    if (!device_accessible(C->ptr)) return DG_ERR_POINTER;
+    if (use_ab && scale_a && !device_accessible(scale_a)) return DG_ERR_POINTER;
+    if (use_ab && scale_b && !device_accessible(scale_b)) return DG_ERR_POINTER;
+    return launch(v, pl, alpha, beta, use_ab ? scale_a : nullptr, use_ab ? scale_b : nullptr,
+                  static_cast<cudaStream_t>(stream), ds);
+}
+
+dg_status dg_gemv(const dg_view *x, const dg_view *W, const dg_view *y, float alpha, float beta, void *stream) {
+    if (!x || !W || !y) return DG_ERR_NULL;
+    ViewInfo xi;
+    dg_status st = analyse(x, false, &xi);
+    if (st != DG_OK) return st;
+    if (xi.rows > 8) return DG_ERR_UNSUPPORTED;
+    return dg_gemm(x, W, y, alpha, beta, nullptr, nullptr, stream);
+}
+
+const char *dg_status_string(dg_status s) {
+    switch (s) {
+    case DG_OK: return "ok";
+    case DG_ERR_NULL: return "null pointer";
+    case DG_ERR_NDIM: return "ndim must be 1..4 and row_dims 0..ndim";
+    case DG_ERR_SHAPE: return "shape mismatch or negative size";
+    case DG_ERR_DTYPE: return "unsupported element type combination";
+    case DG_ERR_STRIDE: return "negative/overflowing stride or overlapping output";
+    case DG_ERR_ALIGN: return "pointer or stride not a multiple of the element size";
+    case DG_ERR_POINTER: return "pointer is not device memory of the current device";
+    case DG_ERR_VALUE: return "alpha or beta is not finite";
+    case DG_ERR_UNSUPPORTED: return "request not supported";
+    case DG_ERR_CUDA: return "CUDA runtime error";
+    case DG_ERR_TIMEOUT: return "a device-side wait timed out";
+    default: return "unknown status";
+    }
+}
+
+dg_status dg_sync_status(void *stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DG_ERR_CUDA;
+    DeviceState *ds = nullptr;
+    dg_status st = device_state(&ds);
+    if (st != DG_OK) return st;
+    int word = 0;
+    if (cudaMemcpy(&word, ds->err_word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DG_ERR_CUDA;
+    if (word != 0) {
+        // an aborted split-K reduction may have left arrival counts behind
+        if (cudaMemset(ds->err_word, 0, sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
+        if (cudaMemset(ds->counters, 0, kCounterCount * sizeof(uint32_t)) != cudaSuccess) return DG_ERR_CUDA;
+        if (cudaDeviceSynchronize() != cudaSuccess) return DG_ERR_CUDA;
+        return word == DG_ERR_TIMEOUT ? DG_ERR_TIMEOUT : DG_ERR_CUDA;
+    }
+    return DG_OK;
+}
+
+dg_status dg_analyse_view(const dg_view *v, dg_view_info *out);  // view.cpp
+
+dg_status dg_plan(const dg_view *A, const dg_view *B, const dg_view *C, float alpha, float beta, int has_scales,
+                  int num_sms, dg_plan_info *out) {
+    (void)has_scales;
+    if (!A || !B || !C || !out) return DG_ERR_NULL;
+    if (num_sms <= 0) {
+        int dev = 0, n = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+            num_sms = n;
+        else {
+            cudaGetLastError();
+            num_sms = 148;
+        }
+    }
+    Views v{A, B, C, {}, {}, {}};
+    Plan pl;
+    dg_status st = make_plan(v, alpha, beta, num_sms, &pl);
+    if (st != DG_OK) return st;
+    *out = pl.info;
+    return DG_OK;
+}
+
+uint64_t dg_launch_count(void) { return g_launches.load(); }
+
+dg_status dg_set_option(int option, int64_t value) {
+    switch (option) {
+    case DG_OPT_FORCE_KIND:
+        if (value < 0 || value > DG_KIND_UMMA) return DG_ERR_VALUE;
+        g_force_kind.store((int)value);
+        return DG_OK;
+    case DG_OPT_WAIT_TIMEOUT_MS:
+        if (value < 1 || value > 600000) return DG_ERR_VALUE;
+        g_timeout_ms.store(value);
+        return DG_OK;
+    case DG_OPT_TEST_STALL:
+        g_stall.store(value ? 1 : 0);
+        return DG_OK;
+    case DG_OPT_MAX_SPLIT_K:
+        if (value < 1 || value > 64) return DG_ERR_VALUE;
+        g_max_split.store((int)value);
+        return DG_OK;
+    default: return DG_ERR_VALUE;
+    }
+}
+
+int dg_version(void) { return 100; }
+
+}  // extern "C"

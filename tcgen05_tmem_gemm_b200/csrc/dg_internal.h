@@ -1,0 +1,127 @@
+// Internal interfaces of libdg: the device-side view description, the
+// per-kernel parameter blocks and the launchers each kernel file exports to
+// the dispatcher.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/dg.h"
+
+namespace dg {
+
+constexpr int kMaxDims = 4;
+
+// One group (rows or columns) of a view after size-1 dims are dropped and
+// contiguous neighbours merged; dims are listed outermost first.  An index in
+// [0, prod(size)) is unflattened row-major over the group.
+struct Axis {
+    int32_t n;
+    int32_t pad_;
+    int64_t size[kMaxDims];
+    int64_t stride[kMaxDims];  // bytes
+};
+
+// A view as the kernels see it: element (r, c) lives at ptr + off(row, r) + off(col, c).
+struct DevView {
+    const char *ptr;
+    Axis row, col;
+    int32_t dtype;
+    int32_t pad_;
+};
+
+__host__ __device__ inline int64_t axis_offset(const Axis &a, int64_t idx) {
+    int64_t off = 0;
+    for (int d = a.n - 1; d >= 0; --d) {
+        const int64_t s = a.size[d];
+        const int64_t q = idx / s;
+        off += (idx - q * s) * a.stride[d];
+        idx = q;
+    }
+    return off;
+}
+
+// Host-side analysis of one view (see view.cpp).
+struct ViewInfo {
+    int64_t rows = 0, cols = 0;
+    Axis row{}, col{};
+    int unit_dim = 0;      // 1: col group is one unit-stride dim, 2: row group is
+    bool tma_ok = false;   // one 2-D TMA map covers it
+    int vec_bytes = 1;     // widest aligned run along the unit-stride dim
+    int64_t span = 0;      // bytes touched from ptr
+    int es = 0;            // element size
+};
+
+dg_status analyse(const dg_view *v, bool is_output, ViewInfo *info);
+int elem_size(int dtype);
+
+// ------------------------------------------------------------- kernel params
+
+// Epilogue target: C viewed as (i, j) with byte strides, i on the tensor-core
+// M side, j on the N side (swapped when the kernel computes C^T).
+struct EpiParams {
+    char *c;
+    int64_t ci, cj;          // byte strides of C along i and j
+    int32_t c_dtype;
+    int32_t vec_ok;          // C contiguous along j with 16-byte aligned rows
+    float alpha, beta;
+    const float *scale_i;    // per-i scale or null
+    const float *scale_j;    // per-j scale or null
+};
+
+struct UmmaParams {
+    int32_t Mi, Nj, K;       // tensor-core problem: D[Mi x Nj] = P[Mi x K] Q[K x Nj]
+    int32_t bn;              // tile width along j (64, 128 or 256)
+    int32_t bk;              // tile depth (128 bytes of K)
+    int32_t stages;
+    int32_t tiles_i, tiles_j, split_k, kb_per_split, kb_total;
+    int32_t num_units;       // tiles_i * tiles_j * split_k
+    int32_t p_mn_major, q_mn_major;
+    uint32_t idesc;          // instruction descriptor
+    int32_t tmem_cols;
+    EpiParams epi;
+    // thread-loaded P operand (gather variant)
+    DevView pv;              // rows = i, cols = k
+    int32_t gather_vec;      // elements per load
+    // split-K workspace
+    float *ws;
+    uint32_t *counters;
+    // control
+    int *err_word;
+    uint64_t timeout_ns;
+    int32_t stall_loader;
+};
+
+struct GemvParams {
+    DevView x;               // [R x K]
+    const char *w;           // W base
+    int64_t w_ld;            // bytes between consecutive k (GEMV_N) or n (GEMV_K)
+    int32_t R, K, N;
+    int32_t in_dtype;
+    EpiParams epi;           // i = row of x, j = n
+    int32_t k_split;         // GEMV_K: warps per output column
+};
+
+struct SimtParams {
+    DevView a, b;            // a: rows m, cols k;  b: rows k, cols n
+    DevView c;               // rows m, cols n
+    int32_t M, N, K;
+    EpiParams epi;           // i = m, j = n (c pointer unused; see c view)
+};
+
+// ------------------------------------------------------------------ launchers
+// Each returns cudaSuccess or the launch error; `launches` is incremented by
+// the number of kernels enqueued.
+
+cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq,
+                        bool fp8, bool gather, int grid, size_t smem, cudaStream_t s);
+size_t umma_smem_bytes(int bn, int bk_bytes, int stages, bool gather);
+int umma_max_stages(int bn, bool gather);
+
+cudaError_t launch_gemv_n(const GemvParams &p, cudaStream_t s, int num_sms, int *grid_out);
+cudaError_t launch_gemv_k(const GemvParams &p, cudaStream_t s, int num_sms, int *grid_out);
+cudaError_t launch_simt(const SimtParams &p, cudaStream_t s);
+cudaError_t launch_scale_c(const DevView &c, int64_t M, int64_t N, float beta, cudaStream_t s);
+
+}  // namespace dg

@@ -1,0 +1,514 @@
+// Tensor-core GEMM for sm_100a: tcgen05.mma with TMEM accumulators.
+//
+// Computes D[i][j] = sum_k P[i][k] Q[k][j] tile by tile and applies the
+// epilogue  out = alpha * s_i * s_j * D + beta * C_in  on the way out.  P is A
+// (i = m) and Q is B (j = n), or, when the dispatcher swaps the operands to
+// put a long N on the tensor core's 128-row side, P = B^T and Q = A^T.
+//
+// Structure ("DeepGEMM deep dive" §2.1-§2.3 describe the blocking, register
+// accumulation and the load/compute overlap this re-designs for Blackwell;
+// §3.4 the shared-memory swizzle):
+//  - one CTA per SM, persistent over tiles (i-tile, j-tile, k-split);
+//  - warp 0, one lane: TMA loads of the P and Q tiles into a ring of
+//    `stages` shared-memory buffers in the 128-byte swizzled layout the
+//    tensor core reads, each stage guarded by a full/empty mbarrier pair;
+//  - warp 1: allocates TMEM (two accumulators of bn FP32 columns each), and one
+//    lane issues tcgen05.mma (128 x bn x 16 for 16-bit inputs, x32 for E4M3)
+//    and tcgen05.commit, which frees a stage once its MMAs have read it and
+//    signals a finished accumulator;
+//  - warps 2-5: the epilogue, each owning 32 TMEM lanes (rows): tcgen05.ld,
+//    scale, optional beta * C, convert and store, while the MMA warp already
+//    fills the other accumulator;
+//  - warps 6-9 (gather variant): thread loads of a P operand that TMA cannot
+//    describe (e.g. an NCHW feature map read as [N*H*W, C] with a 392-byte
+//    channel stride), written into the same swizzled layout
+//    ("DeepGEMM: a recalibration of the compute paradigm", §2.2: scatter-gather
+//    loads for the non-contiguous segments of a view).
+//  - split-K: partial tiles go to a workspace; per 32-row quarter the last
+//    arriving split adds the partials in split order (deterministic) and runs
+//    the epilogue ("DeepGEMM deep dive", §5.2).
+// Every wait is bounded (WaitCtl); on expiry the CTA records DG_ERR_TIMEOUT,
+// drains what it has in flight, frees TMEM and exits.
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace dg {
+
+namespace {
+
+constexpr int kBM = 128;             // tensor-core tile rows (TMEM lanes)
+constexpr int kTileBytesK = 128;     // one swizzle row: 64 x 16-bit or 128 x 8-bit
+constexpr int kGatherWarps = 4;
+
+struct SmemLayout {
+    uint32_t stage_bytes, p_bytes, q_bytes;
+    uint32_t bar_off;                // after the stages
+    uint32_t aux_off;                // tmem address, abort flag, gather tables
+    uint32_t total;
+};
+
+__host__ __device__ inline SmemLayout smem_layout(int bn, int stages, bool gather) {
+    SmemLayout L;
+    L.p_bytes = kBM * kTileBytesK;
+    L.q_bytes = (uint32_t)bn * kTileBytesK;
+    L.stage_bytes = L.p_bytes + L.q_bytes;
+    L.bar_off = L.stage_bytes * stages;
+    // full[S], empty[S], tfull[2], tempty[2], drain
+    L.aux_off = L.bar_off + 8 * (2 * stages + 5);
+    uint32_t aux = 16;  // tmem base + abort flag
+    if (gather) aux += 8 * kBM + 8 * 128;  // row offsets of the tile, k offsets of a stage
+    L.total = L.aux_off + aux + 1024;      // + slack to align the base to 1024
+    return L;
+}
+
+struct TileCoord {
+    int ti, tj, split;
+};
+
+__device__ __forceinline__ TileCoord unit_coord(int u, const UmmaParams &p) {
+    TileCoord c;
+    c.split = u % p.split_k;
+    const int t = u / p.split_k;
+    c.ti = t % p.tiles_i;
+    c.tj = t / p.tiles_i;
+    return c;
+}
+
+// Byte offset inside a 128-byte-swizzled tile of an element at (mn, k) for
+// the two layouts the tensor core reads.  `bytek` = k * element size.
+__device__ __forceinline__ uint32_t sw128_kmajor(int mn, int bytek) {
+    return (uint32_t)((mn >> 3) * 1024 + (mn & 7) * 128 + ((((bytek >> 4) ^ (mn & 7)) << 4) | (bytek & 15)));
+}
+__device__ __forceinline__ uint32_t sw128_mnmajor(int bytemn, int k, int chunk_bytes) {
+    const int c = bytemn >> 7, w = bytemn & 127;
+    return (uint32_t)(c * chunk_bytes + (k >> 3) * 1024 + (k & 7) * 128 + ((((w >> 4) ^ (k & 7)) << 4) | (w & 15)));
+}
+
+template <int BYTES>
+__device__ __forceinline__ void gather_copy(uint32_t dst, const char *src, bool valid) {
+    if constexpr (BYTES == 16) {
+        uint4 v = valid ? __ldg(reinterpret_cast<const uint4 *>(src)) : make_uint4(0, 0, 0, 0);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
+    } else if constexpr (BYTES == 8) {
+        uint2 v = valid ? __ldg(reinterpret_cast<const uint2 *>(src)) : make_uint2(0, 0);
+        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst), "r"(v.x), "r"(v.y));
+    } else if constexpr (BYTES == 4) {
+        uint32_t v = valid ? __ldg(reinterpret_cast<const unsigned int *>(src)) : 0u;
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst), "r"(v));
+    } else if constexpr (BYTES == 2) {
+        unsigned short v = valid ? __ldg(reinterpret_cast<const unsigned short *>(src)) : (unsigned short)0;
+        asm volatile("st.shared.u16 [%0], %1;" ::"r"(dst), "h"(v));
+    } else {
+        unsigned char v = valid ? (unsigned char)__ldg(reinterpret_cast<const char *>(src)) : (unsigned char)0;
+        asm volatile("st.shared.u8 [%0], %1;" ::"r"(dst), "r"((uint32_t)v));
+    }
+}
+
+// Fill one stage's P tile (kBM rows of i, bk of k) by thread loads.
+template <int VB>
+__device__ __forceinline__ void gather_stage(const UmmaParams &p, uint32_t p_smem, const int64_t *row_off,
+                                             const int64_t *col_off, int bk, int es, int gtid) {
+    const int vec = VB / es;                       // elements per copy
+    const int nthreads = kGatherWarps * 32;
+    if (p.p_mn_major) {
+        // runs of `vec` consecutive i at one k; consecutive threads take consecutive runs
+        const int runs_i = kBM / vec;
+        const int total = runs_i * bk;
+        const int chunk_bytes = bk * 128;
+        for (int u = gtid; u < total; u += nthreads) {
+            const int k = u / runs_i, i = (u % runs_i) * vec;
+            const int64_t ro = row_off[i], co = col_off[k];
+            const bool ok = ro >= 0 && co >= 0;
+            gather_copy<VB>(p_smem + sw128_mnmajor(i * es, k, chunk_bytes), p.pv.ptr + (ok ? ro + co : 0), ok);
+        }
+    } else {
+        const int runs_k = bk / vec;
+        const int total = kBM * runs_k;
+        for (int u = gtid; u < total; u += nthreads) {
+            const int i = u / runs_k, k = (u % runs_k) * vec;
+            const int64_t ro = row_off[i], co = col_off[k];
+            const bool ok = ro >= 0 && co >= 0;
+            gather_copy<VB>(p_smem + sw128_kmajor(i, k * es), p.pv.ptr + (ok ? ro + co : 0), ok);
+        }
+    }
+}
+
+// OR of `pred` over the gather warps (named barrier 1), returned to all of them.
+__device__ __forceinline__ bool named_bar_or(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "n"(kGatherWarps * 32)
+        : "memory");
+    return r != 0;
+}
+
+template <bool FP8, bool GATHER>
+__global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
+    umma_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
+                     const UmmaParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte alignment for the 128-byte swizzle atoms
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const SmemLayout L = smem_layout(p.bn, p.stages, GATHER);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + L.bar_off;
+    const uint32_t bar_empty = bar_full + 8 * p.stages;
+    const uint32_t bar_tfull = bar_empty + 8 * p.stages;
+    const uint32_t bar_tempty = bar_tfull + 16;
+    const uint32_t bar_drain = bar_tempty + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.aux_off);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.aux_off + 4);
+    int64_t *g_row_off = reinterpret_cast<int64_t *>(smem + L.aux_off + 16);
+    int64_t *g_col_off = g_row_off + kBM;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kEpiWarp0 = 2;
+    const WaitCtl wc{abort_flag, p.err_word, p.timeout_ns};
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(bar_full + 8 * s, GATHER ? 1 + kGatherWarps : 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, 4);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+        tma_prefetch_desc(&tmap_q);
+        if (!GATHER) tma_prefetch_desc(&tmap_p);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int es = FP8 ? 1 : 2;
+    const int bk = p.bk;
+    constexpr int kUmmaK = FP8 ? 32 : 16;           // K per instruction
+    const uint32_t q_box_bytes = (uint32_t)(p.q_mn_major ? bk * 128 : p.bn * 128);
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int it = 0;  // global k-block counter across tiles
+            const uint32_t tx = (GATHER ? 0u : L.p_bytes) + L.q_bytes;
+            for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+                const TileCoord tc = unit_coord(u, p);
+                const int kb0 = tc.split * p.kb_per_split;
+                const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = it % p.stages;
+                    const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
+                    if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) break;
+                    if (p.stall_loader) continue;  // test hook: nothing arrives, consumers time out
+                    const uint32_t full = bar_full + 8 * s;
+                    mbar_arrive_expect_tx(full, tx);
+                    const uint32_t ps = sbase + s * L.stage_bytes;
+                    const uint32_t qs = ps + L.p_bytes;
+                    const int k0 = kb * bk;
+                    if (!GATHER) {
+                        if (p.p_mn_major) {
+                            const int per = 128 / es;  // i per box
+                            for (int c = 0; c < kBM / per; ++c)
+                                tma_load_2d(ps + c * bk * 128, &tmap_p, full, tc.ti * kBM + c * per, k0);
+                        } else {
+                            tma_load_2d(ps, &tmap_p, full, k0, tc.ti * kBM);
+                        }
+                    }
+                    if (p.q_mn_major) {
+                        const int per = 128 / es;
+                        for (int c = 0; c < p.bn / per; ++c)
+                            tma_load_2d(qs + c * q_box_bytes, &tmap_q, full, tc.tj * p.bn + c * per, k0);
+                    } else {
+                        tma_load_2d(qs, &tmap_q, full, k0, tc.tj * p.bn);
+                    }
+                }
+            }
+            // let the copies already issued land before the CTA can exit
+            const int last = it;
+            for (int d = 1; d <= p.stages && last - d >= 0; ++d) {
+                const int j = last - d;
+                if (p.stall_loader) break;
+                mbar_wait_drain(bar_full + 8 * (j % p.stages), (uint32_t)(j / p.stages) & 1u, p.timeout_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int it = 0, local = 0;
+            const uint32_t idesc = p.idesc;
+            // descriptor strides: K-major tiles step 1024 B per 8 rows; MN-major
+            // tiles step 1024 B per 8 k and one 128-byte MN chunk per bk*128 B.
+            const uint32_t p_lbo = p.p_mn_major ? (uint32_t)(bk * 128) : 16u;
+            const uint32_t q_lbo = p.q_mn_major ? (uint32_t)(bk * 128) : 16u;
+            const uint32_t p_kstep = p.p_mn_major ? kUmmaK * 128 : kUmmaK * es;
+            const uint32_t q_kstep = p.q_mn_major ? kUmmaK * 128 : kUmmaK * es;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++local) {
+                const TileCoord tc = unit_coord(u, p);
+                const int kb0 = tc.split * p.kb_per_split;
+                const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+                const int b = local & 1;
+                const uint32_t tph = (uint32_t)(local >> 1) & 1u;
+                if (!mbar_wait(bar_tempty + 8 * b, tph ^ 1u, wc)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * p.bn);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = it % p.stages;
+                    const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
+                    if (!mbar_wait(bar_full + 8 * s, ph, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t ps = sbase + s * L.stage_bytes;
+                    const uint32_t qs = ps + L.p_bytes;
+#pragma unroll
+                    for (int kk = 0; kk < kTileBytesK / (kUmmaK * es); ++kk) {
+                        const uint64_t da = make_sw128_desc(ps + kk * p_kstep, p_lbo, 1024);
+                        const uint64_t db = make_sw128_desc(qs + kk * q_kstep, q_lbo, 1024);
+                        const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
+                        if (FP8) umma_f8(d_tmem, da, db, idesc, acc);
+                        else umma_f16(d_tmem, da, db, idesc, acc);
+                    }
+                    tc_commit(bar_empty + 8 * s);  // stage is free once these MMAs have read it
+                }
+                if (!ok) break;
+                tc_commit(bar_tfull + 8 * b);      // accumulator b is complete
+            }
+            // wait for every MMA this thread issued before TMEM can be freed
+            tc_commit(bar_drain);
+            mbar_wait_drain(bar_drain, 0, p.timeout_ns);
+        }
+    } else if (warp < kEpiWarp0 + 4) {
+        // ---------------------------------------------------------- epilogue
+        const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
+        const int row = quarter * 32 + lane;         // row inside the tile
+        const EpiParams &e = p.epi;
+        int local = 0;
+        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++local) {
+            const TileCoord tc = unit_coord(u, p);
+            const int b = local & 1;
+            const uint32_t tph = (uint32_t)(local >> 1) & 1u;
+            if (!mbar_wait(bar_tfull + 8 * b, tph, wc)) break;
+            tc_fence_after();
+            const int i = tc.ti * kBM + row;
+            const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * p.bn);
+            const int j0 = tc.tj * p.bn;
+
+            if (p.split_k > 1) {
+                // partial tile -> workspace [unit][col][row] (coalesced along rows)
+                float *ws = p.ws + (size_t)u * kBM * p.bn;
+                for (int c0 = 0; c0 < p.bn; c0 += 16) {
+                    uint32_t r[16];
+                    __syncwarp();
+                    tmem_ld16(t_row + c0, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) __stcg(ws + (size_t)(c0 + c) * kBM + row, __uint_as_float(r[c]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_tempty + 8 * b);
+                __threadfence();
+                __syncwarp();
+                const int tile = u / p.split_k;
+                uint32_t prev = 0;
+                if (lane == 0) prev = atomicAdd(p.counters + tile * 4 + quarter, 1u);
+                prev = __shfl_sync(0xffffffffu, prev, 0);
+                if (prev != (uint32_t)(p.split_k - 1)) continue;  // not the last split of this quarter
+                __threadfence();
+                if (i < p.Mi) {
+                    const float asi = e.alpha * (e.scale_i ? e.scale_i[i] : 1.f);
+                    const float *base = p.ws + (size_t)tile * p.split_k * kBM * p.bn;
+                    for (int c = 0; c < p.bn; ++c) {
+                        const int j = j0 + c;
+                        if (j >= p.Nj) break;
+                        float acc = 0.f;
+                        for (int s = 0; s < p.split_k; ++s)
+                            acc += __ldcg(base + ((size_t)s * p.bn + c) * kBM + row);
+                        char *cp = e.c + (int64_t)i * e.ci + (int64_t)j * e.cj;
+                        const float sj = e.scale_j ? e.scale_j[j] : 1.f;
+                        store_elem(cp, e.c_dtype, epi_value(acc, asi, sj, e.beta, cp, e.c_dtype));
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) p.counters[tile * 4 + quarter] = 0u;  // ready for the next call
+                continue;
+            }
+
+            const bool row_ok = i < p.Mi;
+            const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
+            char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
+            for (int c0 = 0; c0 < p.bn; c0 += 16) {
+                uint32_t r[16];
+                __syncwarp();
+                tmem_ld16(t_row + c0, r);
+                tmem_ld_wait();
+                if (!row_ok) continue;
+                const int jb = j0 + c0;
+                if (e.vec_ok && jb + 16 <= p.Nj) {
+                    float v[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const float sj = e.scale_j ? e.scale_j[jb + c] : 1.f;
+                        v[c] = (asi * sj) * __uint_as_float(r[c]);
+                    }
+                    if (e.c_dtype == DG_F32) {
+                        float4 *dst = reinterpret_cast<float4 *>(crow + (int64_t)jb * 4);
+                        if (e.beta != 0.f) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const float4 o = dst[q];
+                                v[4 * q + 0] = fmaf(e.beta, o.x, v[4 * q + 0]);
+                                v[4 * q + 1] = fmaf(e.beta, o.y, v[4 * q + 1]);
+                                v[4 * q + 2] = fmaf(e.beta, o.z, v[4 * q + 2]);
+                                v[4 * q + 3] = fmaf(e.beta, o.w, v[4 * q + 3]);
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    } else {
+                        // 16-bit output: two 16-byte stores
+                        uint4 *dst = reinterpret_cast<uint4 *>(crow + (int64_t)jb * 2);
+                        uint32_t w[8];
+                        if (e.beta != 0.f) {
+                            const uint4 o0 = dst[0], o1 = dst[1];
+                            const uint32_t ow[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                float lo, hi;
+                                if (e.c_dtype == DG_BF16) {
+                                    lo = __uint_as_float(ow[q] << 16);
+                                    hi = __uint_as_float(ow[q] & 0xffff0000u);
+                                } else {
+                                    const float2 t = __half22float2(*reinterpret_cast<const __half2 *>(&ow[q]));
+                                    lo = t.x;
+                                    hi = t.y;
+                                }
+                                v[2 * q] = fmaf(e.beta, lo, v[2 * q]);
+                                v[2 * q + 1] = fmaf(e.beta, hi, v[2 * q + 1]);
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            if (e.c_dtype == DG_BF16) {
+                                __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+                                w[q] = *reinterpret_cast<uint32_t *>(&h);
+                            } else {
+                                __half2 h = __floats2half2_rn(v[2 * q], v[2 * q + 1]);
+                                w[q] = *reinterpret_cast<uint32_t *>(&h);
+                            }
+                        }
+                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int j = jb + c;
+                        if (j < p.Nj) {
+                            char *cp = crow + (int64_t)j * e.cj;
+                            const float sj = e.scale_j ? e.scale_j[j] : 1.f;
+                            store_elem(cp, e.c_dtype, epi_value(__uint_as_float(r[c]), asi, sj, e.beta, cp, e.c_dtype));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tempty + 8 * b);
+        }
+    } else if (GATHER) {
+        // ------------------------------------------------ gather producers
+        // Every exit decision is voted on across the four gather warps
+        // (bar.red), so no warp can be left waiting at their named barrier.
+        const int gtid = threadIdx.x - (kEpiWarp0 + 4) * 32;
+        int it = 0;
+        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+            if (named_bar_or(*abort_flag != 0)) break;
+            const TileCoord tc = unit_coord(u, p);
+            const int kb0 = tc.split * p.kb_per_split;
+            const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+            // row offsets of this tile (-1 past the end); the first barrier of
+            // the k loop orders them before any use
+            for (int r = gtid; r < kBM; r += kGatherWarps * 32) {
+                const int i = tc.ti * kBM + r;
+                g_row_off[r] = i < p.Mi ? axis_offset(p.pv.row, i) : -1;
+            }
+            bool ok = true;
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                const int s = it % p.stages;
+                const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
+                for (int k = gtid; k < bk; k += kGatherWarps * 32) {
+                    const int kg = kb * bk + k;
+                    g_col_off[k] = kg < p.K ? axis_offset(p.pv.col, kg) : -1;
+                }
+                ok = mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc);
+                if (named_bar_or(!ok)) { ok = false; break; }  // also orders the offsets before use
+                if (!p.stall_loader) {
+                    const uint32_t ps = sbase + s * L.stage_bytes;
+                    switch (p.gather_vec * es) {
+                    case 16: gather_stage<16>(p, ps, g_row_off, g_col_off, bk, es, gtid); break;
+                    case 8: gather_stage<8>(p, ps, g_row_off, g_col_off, bk, es, gtid); break;
+                    case 4: gather_stage<4>(p, ps, g_row_off, g_col_off, bk, es, gtid); break;
+                    case 2: gather_stage<2>(p, ps, g_row_off, g_col_off, bk, es, gtid); break;
+                    default: gather_stage<1>(p, ps, g_row_off, g_col_off, bk, es, gtid); break;
+                    }
+                    fence_proxy_async_smem();  // make the stores visible to the tensor core
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_full + 8 * s);
+                }
+                // all offsets consumed before the next stage overwrites them
+                asm volatile("bar.sync 1, %0;" ::"n"(kGatherWarps * 32) : "memory");
+            }
+            if (!ok) break;
+        }
+    }
+
+    // --------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, (uint32_t)p.tmem_cols);
+    }
+}
+
+}  // namespace
+
+size_t umma_smem_bytes(int bn, int bk_bytes, int stages, bool gather) {
+    (void)bk_bytes;
+    return smem_layout(bn, stages, gather).total;
+}
+
+int umma_max_stages(int bn, bool gather) {
+    int s = 2;
+    while (s < 12 && smem_layout(bn, s + 1, gather).total <= 227 * 1024) ++s;
+    return s;
+}
+
+cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq, bool fp8, bool gather,
+                        int grid, size_t smem, cudaStream_t s) {
+    void (*kern)(const CUtensorMap, const CUtensorMap, const UmmaParams);
+    if (fp8) kern = gather ? umma_gemm_kernel<true, true> : umma_gemm_kernel<true, false>;
+    else kern = gather ? umma_gemm_kernel<false, true> : umma_gemm_kernel<false, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int threads = gather ? 320 : 192;
+    kern<<<grid, threads, smem, s>>>(*tp, *tq, p);
+    return cudaGetLastError();
+}
+
+}  // namespace dg

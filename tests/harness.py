@@ -1,0 +1,127 @@
+"""Shared helpers of the GPU parity tests: run a workload through the C ABI
+and compare it with the FP64 oracle element by element.
+
+Tolerances (from the accuracy targets of the benchmark definition; the pages
+themselves only quote a 1e-4 check, "DeepGEMM: a recalibration of the compute
+paradigm", §4.3):
+  with S = |alpha * sa * sb| * sum_k |a b|  (the scale of the rounding error),
+  FP32 output: |got - r| <= 5e-4 * S + 2^-22 * (|r| + |beta c|)
+  BF16 output: |got - r| <= 4e-3 * max(|r|, S)
+  FP16 output: |got - r| <= 2e-3 * max(|r|, S) + 2^-24
+NaN positions must agree exactly; infinities must agree in sign and place.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import tcgen05_tmem_gemm_b200 as dg
+import workloads as W
+
+
+def dg_view_of(op: W.Operand) -> dg.dg_view:
+    return dg.make_view(op.base.data_ptr() + op.offset, op.shape, op.stride, op.row_dims, op.dtype)
+
+
+def run(problem: W.Problem, stream=None, check_status=True) -> W.Problem:
+    """Enqueue dg_gemm for a device-resident problem and wait for it."""
+    A, B, C = dg_view_of(problem.A), dg_view_of(problem.B), dg_view_of(problem.C)
+    st = dg.dg_gemm(A, B, C, problem.alpha, problem.beta, problem.scale_a, problem.scale_b, stream)
+    if check_status:
+        assert st == dg.DG_OK, dg.status_string(st)
+    sst = dg.dg_sync_status(stream)
+    if check_status:
+        assert sst == dg.DG_OK, dg.status_string(sst)
+    return problem
+
+
+def plan(problem: W.Problem) -> dict:
+    A, B, C = dg_view_of(problem.A), dg_view_of(problem.B), dg_view_of(problem.C)
+    return dg.dg_plan(A, B, C, problem.alpha, problem.beta, problem.scale_a is not None).as_dict()
+
+
+def c_matrix(problem: W.Problem) -> np.ndarray:
+    """C as an [M, N] float64 array, read through its view on the host."""
+    op = problem.C
+    base = op.base.detach().cpu()
+    flat = base.reshape(-1).view(torch.uint8)
+    es = W.ELEM_SIZE[op.dtype]
+    M, N = problem.M, problem.N
+    out = np.empty((M, N), dtype=np.float64)
+    # generic gather through the view (C views are small in tests or 2-D)
+    t = torch.as_strided(base.reshape(-1).view(W.TORCH_DTYPE[op.dtype]),
+                         size=op.shape, stride=[s // es for s in op.stride],
+                         storage_offset=op.offset // es)
+    out[:] = t.to(torch.float64).reshape(M, N).numpy()
+    del flat
+    return out
+
+
+def tolerance(out_dtype: str, ref, bound, beta_c):
+    ref = np.abs(ref)
+    if out_dtype == "f32":
+        return 5e-4 * bound + 2.0 ** -22 * (ref + np.abs(beta_c))
+    if out_dtype == "bf16":
+        return 4e-3 * np.maximum(ref, bound)
+    if out_dtype == "f16":
+        return 2e-3 * np.maximum(ref, bound) + 2.0 ** -24
+    raise ValueError(out_dtype)
+
+
+def compare(problem: W.Problem, got, ref, bound, beta_c=None, where=""):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    if beta_c is None:
+        beta_c = np.zeros_like(ref)
+    nan_g, nan_r = np.isnan(got), np.isnan(ref)
+    assert np.array_equal(nan_g, nan_r), f"{where}: NaN positions differ ({nan_g.sum()} vs {nan_r.sum()})"
+    inf_r = np.isinf(ref)
+    assert np.array_equal(np.isinf(got), inf_r), f"{where}: Inf positions differ"
+    assert np.array_equal(got[inf_r], ref[inf_r]), f"{where}: Inf signs differ"
+    fin = ~(nan_r | inf_r)
+    err = np.abs(got[fin] - ref[fin])
+    tol = tolerance(problem.C.dtype, ref[fin], bound[fin], beta_c[fin])
+    bad = err > tol
+    if bad.any():
+        idx = np.argmax(err - tol)
+        raise AssertionError(f"{where}: {bad.sum()} of {err.size} outside tolerance; worst err "
+                             f"{err[idx]:.3e} tol {tol[idx]:.3e} ref {ref[fin][idx]:.6e} got {got[fin][idx]:.6e}")
+    scale = np.maximum(bound[fin], 1e-30)
+    norm = err / scale
+    return {"max": float(norm.max(initial=0)), "mean": float(norm.mean()) if norm.size else 0.0,
+            "rms": float(np.sqrt((norm ** 2).mean())) if norm.size else 0.0}
+
+
+def beta_c_of(problem: W.Problem) -> np.ndarray:
+    if problem.beta == 0:
+        return np.zeros((problem.M, problem.N))
+    return problem.beta * c_matrix(problem)
+
+
+def check_full(problem_cpu: W.Problem, stream=None) -> dict:
+    """Run on the GPU and compare every output with the full oracle."""
+    ref, bound = oracle.gemm(problem_cpu)
+    bc = beta_c_of(problem_cpu)
+    gpu = problem_cpu.to("cuda")
+    run(gpu, stream)
+    got = c_matrix(gpu)
+    return compare(problem_cpu, got, ref, bound, bc, problem_cpu.name)
+
+
+def check_sampled(problem_cpu: W.Problem, npts=2048, seed=0, gpu=None) -> dict:
+    """Run (unless `gpu` already ran) and compare sampled outputs with the
+    one-by-one oracle: random points plus the four corners and the last
+    row and column."""
+    M, N = problem_cpu.M, problem_cpu.N
+    rng = np.random.default_rng(seed)
+    ms = list(rng.integers(0, M, npts)) + [0, 0, M - 1, M - 1] + [M - 1] * 16 + list(rng.integers(0, M, 16))
+    ns = list(rng.integers(0, N, npts)) + [0, N - 1, 0, N - 1] + list(rng.integers(0, N, 16)) + [N - 1] * 16
+    ms, ns = np.array(ms), np.array(ns)
+    ref, bound = oracle.gemm_points(problem_cpu, ms, ns)
+    bc = problem_cpu.beta * c_matrix(problem_cpu)[ms, ns] if problem_cpu.beta != 0 else np.zeros(len(ms))
+    if gpu is None:
+        gpu = problem_cpu.to("cuda")
+        run(gpu)
+    got = c_matrix(gpu)[ms, ns]
+    return compare(problem_cpu, got, ref, bound, bc, problem_cpu.name)

@@ -1,0 +1,310 @@
+"""GPU parity: the CUDA path through the C ABI against the FP64 oracle.
+
+Small problems are compared element by element (they span several tiles and
+end in ragged tails); the benchmark's full-size workloads, in the launch
+configuration the benchmark uses, are compared on sampled outputs computed
+one by one by the oracle.  Index and view handling is checked bit-exactly
+with identity and permutation operands.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tcgen05_tmem_gemm_b200 as dg
+import workloads as W
+from harness import c_matrix, check_full, check_sampled, compare, dg_view_of, plan, run
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _reset_options():
+    yield
+    dg.dg_set_option(dg.DG_OPT_FORCE_KIND, 0)
+    dg.dg_set_option(dg.DG_OPT_TEST_STALL, 0)
+    dg.dg_set_option(dg.DG_OPT_WAIT_TIMEOUT_MS, 2000)
+    dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, 16)
+
+
+def expect_kind(p, kind, **fields):
+    pl = plan(p.to("cuda"))
+    assert pl["kind_name"] == kind, pl
+    for k, v in fields.items():
+        assert pl[k] == v, (k, pl)
+    return pl
+
+
+# ------------------------------------------------------------ small, full compare
+
+def test_small_config_full():
+    p = W.cfg_small()
+    expect_kind(p, "umma")
+    check_full(p)
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 520, 200), (129, 136, 72), (16, 16, 16), (1000, 264, 1000)])
+@pytest.mark.parametrize("dt,out", [("bf16", "bf16"), ("f16", "f32"), ("bf16", "f32")])
+def test_umma_row_major_ragged(M, N, K, dt, out):
+    g = torch.Generator().manual_seed(M * 7 + N + K)
+    A = W.cast(W.normal((M, K), g), dt)
+    B = W.cast(W.normal((K, N), g), dt)
+    p = W.Problem(f"rm_{M}x{N}x{K}_{dt}_{out}", W.row_major(A, dt), W.row_major(B, dt), W.empty_out(M, N, out))
+    expect_kind(p, "umma")
+    check_full(p)
+
+
+@pytest.mark.parametrize("ta,tb", [(True, False), (False, True), (True, True)])
+def test_umma_transposed_operands(ta, tb):
+    # A given as the transpose of an [K, M] tensor (M-major), B as the transpose of [N, K] (K-major)
+    M, N, K = 264, 200, 136
+    g = torch.Generator().manual_seed(17)
+    a = W.cast(W.uniform((K, M) if ta else (M, K), g), "bf16")
+    b = W.cast(W.uniform((N, K) if tb else (K, N), g), "bf16")
+    A = W.transposed(a, "bf16") if ta else W.row_major(a, "bf16")
+    B = W.transposed(b, "bf16") if tb else W.row_major(b, "bf16")
+    p = W.Problem("transposed", A, B, W.empty_out(M, N, "f32"))
+    expect_kind(p, "umma", p_mn_major=int(ta), q_mn_major=int(not tb))
+    check_full(p)
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 384, 272), (128, 128, 128), (77, 256, 512)])
+def test_umma_fp8_scaled(M, N, K):
+    g = torch.Generator().manual_seed(M + N + K)
+    qa, sa = W.quantise_e4m3(W.normal((M, K), g), dim=1)
+    qb, sb = W.quantise_e4m3(W.normal((K, N), g), dim=0)
+    p = W.Problem("fp8", W.row_major(qa, "e4m3"), W.row_major(qb, "e4m3"), W.empty_out(M, N, "bf16"),
+                  1.0, 0.0, sa, sb)
+    expect_kind(p, "umma", block_k=128)
+    check_full(p)
+
+
+def test_fp8_k_major_b():
+    M, N, K = 200, 144, 256
+    g = torch.Generator().manual_seed(5)
+    qa, sa = W.quantise_e4m3(W.normal((M, K), g), dim=1)
+    qbt, sb = W.quantise_e4m3(W.normal((N, K), g), dim=1)  # B^T stored [N, K]
+    p = W.Problem("fp8_kmajor", W.row_major(qa, "e4m3"), W.transposed(qbt, "e4m3"), W.empty_out(M, N, "f32"),
+                  0.5, 0.0, sa, sb)
+    expect_kind(p, "umma", q_mn_major=0)
+    check_full(p)
+
+
+def test_thin_beta_one_split_k():
+    p = W.cfg_thin(M=40, N=1000, K=784)
+    pl = expect_kind(p, "umma", swap_ab=1)
+    assert pl["split_k"] > 1
+    check_full(p)
+
+
+def test_thin_without_split_k_matches():
+    dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, 1)
+    p = W.cfg_thin(M=64, N=512, K=1024)
+    expect_kind(p, "umma", swap_ab=1, split_k=1)
+    check_full(p)
+
+
+@pytest.mark.parametrize("n,c,h,w,N", [(3, 72, 14, 14, 200), (2, 40, 9, 11, 72), (1, 256, 14, 14, 1024)])
+def test_strided_nchw_gather(n, c, h, w, N):
+    p = W.cfg_strided(n=n, c=c, h=h, w=w, N=N)
+    expect_kind(p, "umma", p_gather=1, p_mn_major=1)
+    check_full(p)
+
+
+def test_gemv_shapes():
+    for p in (W.cfg_gemv(K=1000, N=1032), W.cfg_gemv(K=4096, N=4096), W.cfg_gemv(K=8, N=8)):
+        expect_kind(p, "gemv_n")
+        check_full(p)
+    for p in (W.cfg_gemv_kt(K=1032, N=77), W.cfg_gemv_kt(K=4096, N=128)):
+        expect_kind(p, "gemv_k")
+        check_full(p)
+
+
+@pytest.mark.parametrize("R", [2, 3, 8])
+def test_gemv_multi_row(R):
+    g = torch.Generator().manual_seed(R)
+    x = W.cast(W.normal((R, 1536), g), "f16")
+    Wt = W.cast(W.normal((1536, 520), g, 0.05), "f16")
+    C = W.uniform((R, 520), g).contiguous()
+    p = W.Problem("gemv_rows", W.row_major(x, "f16"), W.row_major(Wt, "f16"), W.row_major(C, "f32"), 0.5, -2.0)
+    expect_kind(p, "gemv_n")
+    check_full(p)
+
+
+def test_dg_gemv_entry_point():
+    p = W.cfg_gemv(K=512, N=256).to("cuda")
+    x = dg.make_view(p.A.base.data_ptr(), (512,), (2,), 0, "bf16")  # a 1-D view is one row
+    st = dg.dg_gemv(x, dg_view_of(p.B), dg_view_of(p.C), 1.0, 0.0)
+    assert st == dg.DG_OK and dg.dg_sync_status() == dg.DG_OK
+    ref, bound = oracle.gemm(p.to("cpu"))
+    compare(p, c_matrix(p), ref, bound, where="dg_gemv")
+
+
+@pytest.mark.parametrize("name", ["small", "gemv", "gemv_kt", "thin", "strided"])
+def test_forced_simt_path(name):
+    dg.dg_set_option(dg.DG_OPT_FORCE_KIND, dg.DG_KIND_SIMT)
+    kw = {"small": {}, "gemv": {"K": 512, "N": 264}, "gemv_kt": {"K": 512, "N": 40},
+          "thin": {"M": 40, "N": 264, "K": 300}, "strided": {"n": 2, "c": 40, "h": 9, "w": 11, "N": 72}}[name]
+    p = W.WORKLOADS[name](**kw)
+    expect_kind(p, "simt")
+    check_full(p)
+
+
+def test_f32_inputs_simt():
+    g = torch.Generator().manual_seed(3)
+    q = W.normal((128 * 49,), g)
+    k = W.normal((128 * 49,), g)
+    Q = W.Operand(q, (1, 128, 7, 7), (0, 196, 28, 4), 2, "f32")
+    KT = W.Operand(k, (7, 7, 1, 128), (28, 4, 0, 196), 2, "f32")
+    p = W.Problem("pages_strided_fp32", Q, KT, W.empty_out(128, 128, "f32"))
+    expect_kind(p, "simt")
+    check_full(p)
+
+
+# --------------------------------------------------------------- bit-exact
+
+def test_identity_gathers_strided_a_exactly():
+    # C = A * I with A the NCHW view: products by 1 and sums with 0 are exact,
+    # so the output must equal the gathered A bit for bit.
+    p = W.cfg_strided(n=2, c=64, h=14, w=14, N=64)
+    eye = torch.eye(64, dtype=torch.bfloat16)
+    p = W.Problem("identity", p.A, W.row_major(eye, "bf16"), W.empty_out(p.M, 64, "f32"))
+    expect_kind(p, "umma", p_gather=1)
+    gpu = run(p.to("cuda"))
+    got = c_matrix(gpu)
+    x = p.A.base  # [n, c, h, w]
+    want = x.permute(0, 2, 3, 1).reshape(-1, 64).to(torch.float64).numpy()
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("kind", ["umma", "simt"])
+def test_permutation_exact(kind):
+    if kind == "simt":
+        dg.dg_set_option(dg.DG_OPT_FORCE_KIND, dg.DG_KIND_SIMT)
+    g = torch.Generator().manual_seed(11)
+    M, K = 256, 128
+    a = W.cast(W.uniform((M, K), g), "bf16")
+    perm = torch.randperm(K, generator=g)
+    P = torch.zeros(K, K, dtype=torch.bfloat16)
+    P[perm, torch.arange(K)] = 1
+    p = W.Problem("perm", W.row_major(a, "bf16"), W.row_major(P, "bf16"), W.empty_out(M, K, "f32"))
+    expect_kind(p, kind)
+    got = c_matrix(run(p.to("cuda")))
+    assert np.array_equal(got, a.to(torch.float64).numpy()[:, perm.numpy()])
+
+
+# ----------------------------------------------------------------- edge cases
+
+def test_empty_and_k_zero():
+    for (M, N, K) in ((0, 16, 16), (16, 0, 16)):
+        A = W.row_major(torch.zeros(M, K, dtype=torch.bfloat16), "bf16")
+        B = W.row_major(torch.zeros(K, N, dtype=torch.bfloat16), "bf16")
+        p = W.Problem("empty", A, B, W.empty_out(M, N, "f32")).to("cuda")
+        run(p)
+    c = torch.arange(48, dtype=torch.float32).reshape(6, 8)
+    A = W.Operand(torch.zeros(8, dtype=torch.bfloat16), (6, 0), (0, 2), 1, "bf16")
+    B = W.Operand(torch.zeros(8, dtype=torch.bfloat16), (0, 8), (16, 2), 1, "bf16")
+    p = W.Problem("k0", A, B, W.row_major(c.clone(), "f32"), 1.0, 3.0).to("cuda")
+    run(p)
+    assert np.array_equal(c_matrix(p), 3.0 * c.double().numpy())
+
+
+def test_alpha_zero_never_reads_a():
+    M, N, K = 64, 96, 80
+    a = torch.full((M, K), float("inf")).to(torch.bfloat16)
+    b = torch.ones(K, N, dtype=torch.bfloat16)
+    c = torch.arange(M * N, dtype=torch.float32).reshape(M, N) / 7
+    p = W.Problem("alpha0", W.row_major(a, "bf16"), W.row_major(b, "bf16"), W.row_major(c.clone(), "f32"),
+                  0.0, -0.5).to("cuda")
+    run(p)
+    assert np.array_equal(c_matrix(p), (-0.5 * c).double().numpy())
+
+
+@pytest.mark.parametrize("kind", ["umma", "gemv_n", "simt"])
+def test_beta_zero_ignores_nan_c_and_nan_propagates(kind):
+    M = 4 if kind == "gemv_n" else 200
+    N, K = 136, 96
+    if kind == "simt":
+        dg.dg_set_option(dg.DG_OPT_FORCE_KIND, dg.DG_KIND_SIMT)
+    g = torch.Generator().manual_seed(1)
+    a = W.cast(W.uniform((M, K), g), "bf16")
+    a[1, 5] = float("nan")
+    b = W.cast(W.uniform((K, N), g), "bf16")
+    b[7, 3] = float("inf")
+    p = W.Problem("nan", W.row_major(a, "bf16"), W.row_major(b, "bf16"), W.empty_out(M, N, "f32"))
+    expect_kind(p, kind)
+    check_full(p)
+
+
+def test_scales_applied_once():
+    M, N, K = 256, 256, 128
+    a = torch.ones(M, K).to(torch.float8_e4m3fn)
+    b = torch.ones(K, N).to(torch.float8_e4m3fn)
+    sa = torch.tensor([2.0 ** (j % 5 - 2) for j in range(M)])
+    sb = torch.tensor([2.0 ** (-(j % 3)) for j in range(N)])
+    p = W.Problem("scales", W.row_major(a, "e4m3"), W.row_major(b, "e4m3"), W.empty_out(M, N, "f32"),
+                  1.0, 0.0, sa, sb)
+    got = c_matrix(run(p.to("cuda")))
+    assert np.array_equal(got, K * np.outer(sa.numpy(), sb.numpy()))
+
+
+def test_output_guard_band_untouched():
+    M, N, K = 130, 72, 64
+    g = torch.Generator().manual_seed(8)
+    a = W.cast(W.uniform((M, K), g), "f16")
+    b = W.cast(W.uniform((K, N), g), "f16")
+    ld = N + 24  # C embedded in a wider buffer, canaries on both sides
+    buf = torch.full((M + 2, ld), 12345.0)
+    C = W.Operand(buf, (M, N), (ld * 4, 4), 1, "f32", offset=(ld + 8) * 4)
+    p = W.Problem("guard", W.row_major(a, "f16"), W.row_major(b, "f16"), C)
+    gpu = run(p.to("cuda"))
+    out = gpu.C.base.cpu()
+    mask = torch.ones_like(out, dtype=torch.bool)
+    mask[1:M + 1, 8:8 + N] = False
+    assert torch.all(out[mask] == 12345.0)
+    ref, bound = oracle.gemm(p)
+    compare(p, c_matrix(gpu), ref, bound, where="guard")
+
+
+def test_pointer_and_value_errors():
+    p = W.cfg_small(M=16, N=16, K=16)
+    A, B, C = (dg.make_view(o.base.data_ptr(), o.shape, o.stride, o.row_dims, o.dtype) for o in (p.A, p.B, p.C))
+    assert dg.dg_gemm(A, B, C, 1.0, 0.0) == dg.DG_ERR_POINTER  # host memory
+    gp = p.to("cuda")
+    A, B, C = dg_view_of(gp.A), dg_view_of(gp.B), dg_view_of(gp.C)
+    assert dg.dg_gemm(A, B, C, math.nan, 0.0) == dg.DG_ERR_VALUE
+    assert dg.dg_sync_status() == dg.DG_OK
+
+
+def test_bounded_wait_reports_timeout_and_recovers():
+    # The loader issues no copies, so the MMA issuer's wait runs out after the
+    # bound; the kernel records the timeout, frees TMEM and returns.
+    p = W.cfg_small(M=128, N=128, K=256).to("cuda")
+    dg.dg_set_option(dg.DG_OPT_WAIT_TIMEOUT_MS, 300)
+    dg.dg_set_option(dg.DG_OPT_TEST_STALL, 1)
+    A, B, C = dg_view_of(p.A), dg_view_of(p.B), dg_view_of(p.C)
+    assert dg.dg_gemm(A, B, C, 1.0, 0.0) == dg.DG_OK
+    assert dg.dg_sync_status() == dg.DG_ERR_TIMEOUT
+    dg.dg_set_option(dg.DG_OPT_TEST_STALL, 0)
+    check_full(W.cfg_small())
+
+
+def test_streams_and_launch_count():
+    s = torch.cuda.Stream()
+    n0 = dg.dg_launch_count()
+    with torch.cuda.stream(s):
+        check_full(W.cfg_small(M=256, N=128, K=64), stream=s)
+    assert dg.dg_launch_count() == n0 + 1
+
+
+# ------------------------------------------------------ full-size, sampled
+
+@pytest.mark.parametrize("name", ["gemv", "gemv_kt", "thin", "square_bf16", "square_e4m3", "strided"])
+def test_full_size_sampled(name):
+    p = W.WORKLOADS[name]()
+    pl = expect_kind(p, {"gemv": "gemv_n", "gemv_kt": "gemv_k"}.get(name, "umma"))
+    if name == "thin":
+        assert pl["swap_ab"] == 1 and pl["split_k"] == 4
+    check_sampled(p, npts=3000)
