@@ -14,20 +14,20 @@
  * Conventions shared by all entry points
  *  - Memory: the caller owns every buffer.  Data pointers are DEVICE pointers
  *    (cudaMalloc / torch CUDA tensors / managed memory) on the current device.
- *    The library keeps no pointer after a call returns.  It owns a small
- *    per-device workspace (status word, split-K partials) allocated on first
- *    use; the first call on a device should therefore come before any CUDA
+ *    The library keeps no pointer after a call returns.  It owns one
+ *    4-byte device status word per device, allocated on the first call on
+ *    that device; that first call should therefore come before any CUDA
  *    stream capture.
  *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *    default stream).  Calls are asynchronous on that stream.
  *  - Errors: argument errors are returned synchronously, before anything is
  *    launched, and leave C untouched.  A device-side wait that gives up (see
  *    dg_sync_status) is reported by dg_sync_status.
- *  - Thread safety: calls may be made from several host threads.  The
- *    split-K workspace is one per device: two calls that both take the
- *    split-K path (dg_plan_info.split_k > 1) must not run concurrently on
- *    different streams (serialise them, or set DG_OPT_MAX_SPLIT_K to 1).
- *    dg_set_option is process-global and should not race with running calls.
+ *  - Thread safety: calls may be made from several host threads and their
+ *    kernels may run concurrently on different streams: split-K partial
+ *    sums stay in on-chip (cluster) shared memory, so calls share no scratch
+ *    buffers.  dg_set_option is process-global and should not race with
+ *    running calls.
  */
 #ifndef DG_H_
 #define DG_H_
@@ -198,7 +198,8 @@ typedef enum {
     DG_OPT_TEST_STALL = 3,        /* 1: the tensor-core kernel's loader issues no
                                      copies, so its waits run out and the call
                                      reports DG_ERR_TIMEOUT (tests of the bound)      */
-    DG_OPT_MAX_SPLIT_K = 4        /* upper bound on split-K (default 16; 1 disables)   */
+    DG_OPT_MAX_SPLIT_K = 4        /* upper bound on the tensor-core kernel's split-K
+                                     (default and cluster limit 8; 1 disables)         */
 } dg_option;
 
 dg_status dg_set_option(int option, int64_t value);

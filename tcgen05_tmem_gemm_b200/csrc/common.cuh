@@ -31,6 +31,10 @@ __device__ __forceinline__ void store_elem(char *p, int dtype, float v) {
     }
 }
 
+__host__ __device__ __forceinline__ int elem_bytes(int dtype) {
+    return dtype == DG_F32 ? 4 : dtype == DG_E4M3 ? 1 : 2;
+}
+
 // out = alpha * s_i * s_j * acc + beta * c_in   (c_in read only when beta != 0)
 __device__ __forceinline__ float epi_value(float acc, float alpha_si, float sj, float beta, const char *c,
                                            int c_dtype) {

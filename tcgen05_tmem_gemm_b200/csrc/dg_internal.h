@@ -84,9 +84,6 @@ struct UmmaParams {
     // thread-loaded P operand (gather variant)
     DevView pv;              // rows = i, cols = k
     int32_t gather_vec;      // elements per load
-    // split-K workspace
-    float *ws;
-    uint32_t *counters;
     // control
     int *err_word;
     uint64_t timeout_ns;
@@ -100,7 +97,11 @@ struct GemvParams {
     int32_t R, K, N;
     int32_t in_dtype;
     EpiParams epi;           // i = row of x, j = n
-    int32_t k_split;         // GEMV_K: warps per output column
+    int32_t kper;            // GEMV_N: rows of W per block (multiple of 32)
+    int32_t x_vec16;         // x unit-stride along k, 16-byte aligned rows, K % 8 == 0
+    int64_t x_ld;            // bytes between rows of x (x_vec16 only)
+    int *err_word;
+    uint64_t timeout_ns;
 };
 
 struct SimtParams {
@@ -119,8 +120,9 @@ cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtens
 size_t umma_smem_bytes(int bn, int bk_bytes, int stages, bool gather);
 int umma_max_stages(int bn, bool gather);
 
-cudaError_t launch_gemv_n(const GemvParams &p, cudaStream_t s, int num_sms, int *grid_out);
-cudaError_t launch_gemv_k(const GemvParams &p, cudaStream_t s, int num_sms, int *grid_out);
+cudaError_t launch_gemv_n(const GemvParams &p, const CUtensorMap *tmap_w, cudaStream_t s, int *grid_out);
+size_t gemv_n_smem_bytes(int r_inst, int kper);
+cudaError_t launch_gemv_k(const GemvParams &p, cudaStream_t s, int *grid_out);
 cudaError_t launch_simt(const SimtParams &p, cudaStream_t s);
 cudaError_t launch_scale_c(const DevView &c, int64_t M, int64_t N, float beta, cudaStream_t s);
 

@@ -5,25 +5,37 @@
 // [1,4096]x[4096,128], the single-token Q K^T) stream W once from HBM and do
 // two flops per weight, so they are judged on bytes per second.  Tensor cores
 // would waste 127/128 of every instruction at M = 1; these kernels use CUDA
-// cores with 16-byte coalesced loads, FP32 accumulation and a warp-shuffle
-// plus shared-memory reduction (inner-discipline page §3.2, the shuffle
-// exchange), and no atomics, so results are deterministic.
+// cores with FP32 accumulation, and reductions in a fixed order (warp
+// shuffles and shared memory, the inner-discipline page's §3.2 exchange), so
+// results are deterministic.
 //
-//  gemv_n:  W unit-stride along n (row-major [K, N]).  A thread owns 8
-//           consecutive columns; a warp covers TX threads along n and 32/TX
-//           rows along k; the block's 8 warps split k further.
-//  gemv_k:  W unit-stride along k (e.g. K^T read in place from a row-major
-//           [N, K] key matrix).  A warp walks one column's k range with
-//           16-byte loads; four warps share one column and meet in shared
-//           memory.
+//  gemv_n:  W unit-stride along n (row-major [K, N]).  A block owns a strip of
+//           256 columns and a range of k.  One producer lane streams 32 x 256
+//           tiles of W into a ring of shared-memory stages with TMA (the bytes
+//           in flight per SM are the ring, not registers); eight consumer
+//           warps read them (a lane = 8 columns) and accumulate.  The k ranges
+//           of one strip form a thread-block cluster: each block leaves its
+//           256 partial sums in shared memory and, after a cluster barrier,
+//           block s adds slice s of the strip across the cluster through
+//           distributed shared memory, in rank order ("DeepGEMM deep dive",
+//           §5.2 split-K, reduced here on chip instead of through HBM).
+//  gemv_k:  W unit-stride along k (K^T read in place from a row-major [N, K]
+//           key matrix).  Four warps share one column, each walking a quarter
+//           of k with every 16-byte load of its range in flight at once.
+#include <atomic>
+
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace dg {
 
 namespace {
 
-constexpr int NT = 256;       // threads per block
-constexpr int KC = 1024;      // k rows of x staged in shared memory at a time
+constexpr int kNB = 256;        // columns per gemv_n block
+constexpr int kRows = 32;       // rows of W per TMA stage
+constexpr int kStages = 6;      // ring depth
+constexpr int kCW = 8;          // consumer warps
+constexpr int kNT = 32 * (kCW + 1);
 
 template <typename T>
 __device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8]);
@@ -58,15 +70,33 @@ __device__ __forceinline__ uint4 ldg_stream(const void *p) {
     return r;
 }
 
-// Stage x[r][k0 .. k0+KC) as float (zero beyond K or R).
-template <int R>
-__device__ __forceinline__ void stage_x(float *xs, const GemvParams &p, int k0) {
-    for (int e = threadIdx.x; e < R * KC; e += NT) {
-        const int r = e / KC, kk = e % KC, k = k0 + kk;
-        float v = 0.f;
-        if (r < p.R && k < p.K)
-            v = load_elem(p.x.ptr + axis_offset(p.x.row, r) + axis_offset(p.x.col, k), p.x.dtype);
-        xs[r * KC + kk] = v;
+// x[r][k0 .. k0+len) -> xs[r * pitch + kk] as float, zero beyond K or R.
+// 16-byte loads when x is unit-stride along k and aligned, else element loads.
+template <typename T, int R>
+__device__ __forceinline__ void stage_x(float *xs, int pitch, const GemvParams &p, int k0, int len, int tid,
+                                        int nthreads) {
+    const bool fast = p.x_vec16 && (k0 % 8 == 0);
+    if (fast) {
+        const int nv = (len + 7) / 8;
+        for (int e = tid; e < R * nv; e += nthreads) {
+            const int r = e / nv, v8 = e - r * nv, kk = v8 * 8, k = k0 + kk;
+            float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (r < p.R && k < p.K) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(p.x.ptr + (int64_t)r * p.x_ld + (int64_t)k * 2);
+                unpack8<T>(v, f);
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                if (kk + c < len) xs[r * pitch + kk + c] = (k + c < p.K) ? f[c] : 0.f;
+        }
+    } else {
+        for (int e = tid; e < R * len; e += nthreads) {
+            const int r = e / len, kk = e - r * len, k = k0 + kk;
+            float v = 0.f;
+            if (r < p.R && k < p.K)
+                v = load_elem(p.x.ptr + axis_offset(p.x.row, r) + axis_offset(p.x.col, k), p.x.dtype);
+            xs[r * pitch + kk] = v;
+        }
     }
 }
 
@@ -77,122 +107,203 @@ __device__ __forceinline__ void store_out(const EpiParams &e, int r, int n, floa
     store_elem(cp, e.c_dtype, epi_value(acc, asi, sj, e.beta, cp, e.c_dtype));
 }
 
-template <typename T, int R, int TX>
-__global__ void __launch_bounds__(NT) gemv_n_kernel(const GemvParams p) {
-    constexpr int KY_W = 32 / TX;           // k rows per warp step
-    constexpr int KY = KY_W * (NT / 32);    // k rows per block step
-    constexpr int NB = 8 * TX;              // columns per block
-    extern __shared__ float smem[];
-    float *xs = smem;                       // [R][KC]
-    float *red = smem + R * KC;             // [8 warps][R][NB]
+struct GemvNLayout {
+    uint32_t ring, xs, part, bars, flag, total;
+};
 
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int tx = lane % TX, ky = warp * KY_W + lane / TX;
-    const int n = blockIdx.x * NB + tx * 8;
-    const bool col_ok = n < p.N;            // N % 8 == 0 is guaranteed by the dispatcher
-    float acc[R][8];
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+__host__ __device__ inline GemvNLayout gemv_n_layout(int R, int kper) {
+    GemvNLayout L;
+    L.ring = 0;
+    L.xs = kStages * kRows * kNB * 2;                    // 16-bit W tiles
+    L.part = L.xs + (uint32_t)(R * kper * 4);
+    L.bars = L.part + (uint32_t)(R * kNB * 4);
+    L.flag = L.bars + 8 * 2 * kStages;
+    L.total = L.flag + 16 + 1024;                        // + alignment slack
+    return L;
+}
 
-    const char *wcol = p.w + (int64_t)n * sizeof(T);
-    for (int k0 = 0; k0 < p.K; k0 += KC) {
-        __syncthreads();
-        stage_x<R>(xs, p, k0);
-        __syncthreads();
-        const int kend = min(KC, p.K - k0);
-        if (col_ok) {
-            int kk = ky;
-            constexpr int U = 4;
-            for (; kk + (U - 1) * KY < kend; kk += U * KY) {
-                uint4 v[U];
-#pragma unroll
-                for (int u = 0; u < U; ++u) v[u] = ldg_stream(wcol + (int64_t)(k0 + kk + u * KY) * p.w_ld);
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    float f[8];
-                    unpack8<T>(v[u], f);
-#pragma unroll
-                    for (int r = 0; r < R; ++r) {
-                        const float xv = xs[r * KC + kk + u * KY];
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(xv, f[c], acc[r][c]);
-                    }
-                }
+template <typename T, int R>
+__global__ void __launch_bounds__(kNT) gemv_n_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                                                     const GemvParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const GemvNLayout L = gemv_n_layout(R, p.kper);
+    float *xs = reinterpret_cast<float *>(smem + L.xs);
+    float *part = reinterpret_cast<float *>(smem + L.part);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + L.bars, bar_empty = bar_full + 8 * kStages;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.flag);
+    const WaitCtl wc{abort_flag, p.err_word, p.timeout_ns};
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * kNB;
+    const int kb0 = blockIdx.y * p.kper;
+    const int kn = min(p.K - kb0, p.kper);
+    const int nst = (kn + kRows - 1) / kRows;
+    const int nsplit = gridDim.y;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, kCW);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    stage_x<T, R>(xs, p.kper, p, kb0, kn, threadIdx.x, kNT);
+    __syncthreads();
+
+    if (warp == kCW) {
+        // ----------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int it = 0;
+            for (; it < nst; ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) break;
+                mbar_arrive_expect_tx(bar_full + 8 * s, kRows * kNB * 2);
+                tma_load_2d(sbase + L.ring + s * (kRows * kNB * 2), &tmap_w, bar_full + 8 * s, n0, kb0 + it * kRows);
             }
-            for (; kk < kend; kk += KY) {
-                uint4 v = ldg_stream(wcol + (int64_t)(k0 + kk) * p.w_ld);
+            for (int d = 1; d <= kStages && it - d >= 0; ++d) {
+                const int j = it - d;
+                mbar_wait_drain(bar_full + 8 * (j % kStages), (uint32_t)(j / kStages) & 1u, p.timeout_ns);
+            }
+        }
+    } else {
+        // -------------------------------------------------------- consumers
+        float acc[R][8];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+        for (int it = 0; it < nst; ++it) {
+            const int s = it % kStages;
+            const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+            if (!mbar_wait(bar_full + 8 * s, ph, wc)) break;
+            const uint8_t *tile = smem + L.ring + s * (kRows * kNB * 2);
+            uint4 v[kRows / kCW];
+#pragma unroll
+            for (int j = 0; j < kRows / kCW; ++j)
+                v[j] = *reinterpret_cast<const uint4 *>(tile + (warp + kCW * j) * (kNB * 2) + lane * 16);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+#pragma unroll
+            for (int j = 0; j < kRows / kCW; ++j) {
+                const int kk = it * kRows + warp + kCW * j;
+                if (kk >= kn) continue;  // rows past this block's range (TMA fills past K with zeros)
                 float f[8];
-                unpack8<T>(v, f);
+                unpack8<T>(v[j], f);
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    const float xv = xs[r * KC + kk];
+                    const float xv = xs[r * p.kper + kk];
 #pragma unroll
                     for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(xv, f[c], acc[r][c]);
                 }
             }
         }
+        // the ring is free once every consumer warp is past its loop
+        asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+        float *red = reinterpret_cast<float *>(smem + L.ring);   // [kCW][R][kNB]
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            float4 *dst = reinterpret_cast<float4 *>(red + (warp * R + r) * kNB + lane * 8);
+            dst[0] = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+            dst[1] = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+        for (int e = threadIdx.x; e < R * kNB; e += kCW * 32) {
+            const int r = e / kNB, j = e - r * kNB;
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < kCW; ++w) sum += red[(w * R + r) * kNB + j];
+            if (nsplit == 1) {
+                if (r < p.R && n0 + j < p.N) store_out(p.epi, r, n0 + j, sum);
+            } else {
+                part[r * kNB + j] = sum;
+            }
+        }
     }
-    // reduce the KY_W rows inside the warp (lanes tx, tx+TX, ...)
-#pragma unroll
-    for (int off = TX; off < 32; off <<= 1)
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) acc[r][c] += __shfl_xor_sync(0xffffffffu, acc[r][c], off);
-    if (lane < TX) {
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) red[(warp * R + r) * NB + tx * 8 + c] = acc[r][c];
-    }
+    if (nsplit == 1) return;
+
+    // ---------------------------------------------- cluster reduction of k splits
     __syncthreads();
-    // across the 8 warps, in warp order, then the epilogue
-    for (int e = threadIdx.x; e < R * NB; e += NT) {
-        const int r = e / NB, j = e % NB;
-        const int nn = blockIdx.x * NB + j;
-        if (r >= p.R || nn >= p.N) continue;
-        float s = 0.f;
+    cluster_sync();
+    {
+        const uint32_t rank = cluster_ctarank();
+        const int c0 = (int)(rank * kNB / nsplit), c1 = (int)((rank + 1) * kNB / nsplit);
+        const int width = c1 - c0;
+        const uint32_t part_addr = sbase + L.part;
+        for (int e = threadIdx.x; e < R * width; e += kNT) {
+            const int r = e / width, j = c0 + (e - r * width);
+            if (r >= p.R || n0 + j >= p.N) continue;
+            // all remote loads issued before the sum, which runs in rank order
+            float v[8];
 #pragma unroll
-        for (int w = 0; w < NT / 32; ++w) s += red[(w * R + r) * NB + j];
-        store_out(p.epi, r, nn, s);
+            for (int q = 0; q < 8; ++q)
+                v[q] = q < nsplit ? dsmem_ld_f32(dsmem_map(part_addr + (r * kNB + j) * 4, q)) : 0.f;
+            float sum = 0.f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (q < nsplit) sum += v[q];
+            store_out(p.epi, r, n0 + j, sum);
+        }
     }
+    cluster_sync();  // keep every block's partials alive until all remote reads are done
 }
 
-// Four warps per column; a block covers two columns.
+// Four warps per column; a block covers two columns.  A warp's loads over its
+// quarter of k are all issued before any is used.
 template <typename T, int R>
-__global__ void __launch_bounds__(NT) gemv_k_kernel(const GemvParams p) {
-    constexpr int WPC = 4;                  // warps per column
-    constexpr int CPB = (NT / 32) / WPC;    // columns per block
+__global__ void __launch_bounds__(256) gemv_k_kernel(const GemvParams p) {
+    constexpr int WPC = 4;
+    constexpr int CPB = 8 / WPC;
+    constexpr int MAXV = 8;                 // 16-byte loads per lane kept in flight
     extern __shared__ float smem[];
-    float *xs = smem;                       // [R][KC]
-    float *red = smem + R * KC;             // [8 warps][R]
+    float *xs = smem;                       // [R][K]
+    float *red = smem + R * p.K;            // [8 warps][R]
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int n = blockIdx.x * CPB + warp / WPC;
     const int q = warp % WPC;
     const bool col_ok = n < p.N;
     const char *wrow = p.w + (int64_t)(col_ok ? n : 0) * p.w_ld;
+    // this warp's k range, a multiple of 8 elements
+    const int kq = ((p.K / 8 + WPC - 1) / WPC) * 8;
+    const int ka = q * kq, kb = min(p.K, ka + kq);
+
+    stage_x<T, R>(xs, p.K, p, 0, p.K, threadIdx.x, 256);
+    __syncthreads();
     float acc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r] = 0.f;
-
-    for (int k0 = 0; k0 < p.K; k0 += KC) {
-        __syncthreads();
-        stage_x<R>(xs, p, k0);
-        __syncthreads();
-        const int kend = min(KC, p.K - k0);   // K % 8 == 0 is guaranteed
-        if (col_ok) {
-            // this warp's quarter of the chunk, 8 elements per lane per step
-            for (int kk = (q * 32 + lane) * 8; kk < kend; kk += WPC * 32 * 8) {
-                uint4 v = ldg_stream(wrow + (int64_t)(k0 + kk) * sizeof(T));
+    if (col_ok) {
+        for (int k0 = ka + lane * 8; k0 < kb; k0 += 32 * 8 * MAXV) {
+            uint4 v[MAXV];
+#pragma unroll
+            for (int u = 0; u < MAXV; ++u) {
+                const int k = k0 + u * 256;
+                v[u] = (k < kb) ? ldg_stream(wrow + (int64_t)k * sizeof(T)) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < MAXV; ++u) {
+                const int k = k0 + u * 256;
+                if (k >= kb) break;
                 float f[8];
-                unpack8<T>(v, f);
+                unpack8<T>(v[u], f);
 #pragma unroll
-                for (int r = 0; r < R; ++r)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) acc[r] = fmaf(xs[r * KC + kk + c], f[c], acc[r]);
+                for (int r = 0; r < R; ++r) {
+                    const float4 x0 = *reinterpret_cast<const float4 *>(xs + r * p.K + k);
+                    const float4 x1 = *reinterpret_cast<const float4 *>(xs + r * p.K + k + 4);
+                    acc[r] = fmaf(x0.x, f[0], acc[r]);
+                    acc[r] = fmaf(x0.y, f[1], acc[r]);
+                    acc[r] = fmaf(x0.z, f[2], acc[r]);
+                    acc[r] = fmaf(x0.w, f[3], acc[r]);
+                    acc[r] = fmaf(x1.x, f[4], acc[r]);
+                    acc[r] = fmaf(x1.y, f[5], acc[r]);
+                    acc[r] = fmaf(x1.z, f[6], acc[r]);
+                    acc[r] = fmaf(x1.w, f[7], acc[r]);
+                }
             }
         }
     }
@@ -216,50 +327,61 @@ __global__ void __launch_bounds__(NT) gemv_k_kernel(const GemvParams p) {
     }
 }
 
-template <typename T, int R, int TX>
-cudaError_t run_n(const GemvParams &p, cudaStream_t s, int *grid_out) {
-    constexpr int NB = 8 * TX;
-    const int grid = (p.N + NB - 1) / NB;
-    const size_t smem = sizeof(float) * (R * KC + (NT / 32) * R * NB);
-    auto kern = gemv_n_kernel<T, R, TX>;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    kern<<<grid, NT, smem, s>>>(p);
-    *grid_out = grid;
-    return cudaGetLastError();
+// Raise a kernel's dynamic shared-memory limit once per size, not per call
+// (`Tag` gives each kernel instantiation its own record).
+template <typename Tag, typename K>
+cudaError_t ensure_smem(K kern, size_t smem) {
+    static std::atomic<int> limit{48 * 1024};
+    if ((int)smem <= limit.load()) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) limit.store((int)smem);
+    return e;
 }
 
+template <typename T, int R, int Kind>
+struct KernelTag {};
+
 template <typename T, int R>
-cudaError_t run_n_tx(const GemvParams &p, cudaStream_t s, int num_sms, int *grid_out) {
-    // widest warp footprint along n that still gives every SM a block
-    const int blocks32 = (p.N + 255) / 256, blocks16 = (p.N + 127) / 128, blocks8 = (p.N + 63) / 64;
-    if (blocks32 >= num_sms) return run_n<T, R, 32>(p, s, grid_out);
-    if (blocks16 >= num_sms) return run_n<T, R, 16>(p, s, grid_out);
-    if (blocks8 >= num_sms) return run_n<T, R, 8>(p, s, grid_out);
-    return run_n<T, R, 4>(p, s, grid_out);
+cudaError_t run_n(const GemvParams &p, const CUtensorMap *tmap, cudaStream_t s, int *grid_out) {
+    const int gx = (p.N + kNB - 1) / kNB;
+    const int gy = (p.K + p.kper - 1) / p.kper;
+    const size_t smem = gemv_n_layout(R, p.kper).total;
+    auto kern = gemv_n_kernel<T, R>;
+    cudaError_t e = ensure_smem<KernelTag<T, R, 0>>(kern, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(gx, gy);
+    cfg.blockDim = dim3(kNT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = gy;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = gy > 1 ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, *tmap, p);
+    *grid_out = gx * gy;
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <typename T>
-cudaError_t run_n_r(const GemvParams &p, cudaStream_t s, int num_sms, int *grid_out) {
-    if (p.R <= 1) return run_n_tx<T, 1>(p, s, num_sms, grid_out);
-    if (p.R <= 2) return run_n_tx<T, 2>(p, s, num_sms, grid_out);
-    if (p.R <= 4) return run_n_tx<T, 4>(p, s, num_sms, grid_out);
-    return run_n_tx<T, 8>(p, s, num_sms, grid_out);
+cudaError_t run_n_r(const GemvParams &p, const CUtensorMap *tmap, cudaStream_t s, int *grid_out) {
+    if (p.R <= 1) return run_n<T, 1>(p, tmap, s, grid_out);
+    if (p.R <= 2) return run_n<T, 2>(p, tmap, s, grid_out);
+    if (p.R <= 4) return run_n<T, 4>(p, tmap, s, grid_out);
+    return run_n<T, 8>(p, tmap, s, grid_out);
 }
 
 template <typename T, int R>
 cudaError_t run_k(const GemvParams &p, cudaStream_t s, int *grid_out) {
-    constexpr int CPB = 2;
-    const int grid = (p.N + CPB - 1) / CPB;
-    const size_t smem = sizeof(float) * (R * KC + (NT / 32) * R);
+    const int grid = (p.N + 1) / 2;
+    const size_t smem = sizeof(float) * ((size_t)R * p.K + 8 * R);
     auto kern = gemv_k_kernel<T, R>;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    kern<<<grid, NT, smem, s>>>(p);
+    cudaError_t e = ensure_smem<KernelTag<T, R, 1>>(kern, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, 256, smem, s>>>(p);
     *grid_out = grid;
     return cudaGetLastError();
 }
@@ -274,14 +396,15 @@ cudaError_t run_k_r(const GemvParams &p, cudaStream_t s, int *grid_out) {
 
 }  // namespace
 
-cudaError_t launch_gemv_n(const GemvParams &p, cudaStream_t s, int num_sms, int *grid_out) {
-    if (p.in_dtype == DG_BF16) return run_n_r<__nv_bfloat16>(p, s, num_sms, grid_out);
-    if (p.in_dtype == DG_F16) return run_n_r<__half>(p, s, num_sms, grid_out);
+size_t gemv_n_smem_bytes(int r_inst, int kper) { return gemv_n_layout(r_inst, kper).total; }
+
+cudaError_t launch_gemv_n(const GemvParams &p, const CUtensorMap *tmap, cudaStream_t s, int *grid_out) {
+    if (p.in_dtype == DG_BF16) return run_n_r<__nv_bfloat16>(p, tmap, s, grid_out);
+    if (p.in_dtype == DG_F16) return run_n_r<__half>(p, tmap, s, grid_out);
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_gemv_k(const GemvParams &p, cudaStream_t s, int num_sms, int *grid_out) {
-    (void)num_sms;
+cudaError_t launch_gemv_k(const GemvParams &p, cudaStream_t s, int *grid_out) {
     if (p.in_dtype == DG_BF16) return run_k_r<__nv_bfloat16>(p, s, grid_out);
     if (p.in_dtype == DG_F16) return run_k_r<__half>(p, s, grid_out);
     return cudaErrorInvalidValue;

@@ -70,13 +70,22 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtParams p) {
         if (m >= p.M) continue;
         const float asi = e.alpha * (e.scale_i ? e.scale_i[m] : 1.f);
         const int64_t cro = axis_offset(p.c.row, m);
+        char *cp[4];
+        float cin[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int n = n0 + tx * 4 + j;
-            if (n >= p.N) continue;
-            char *cp = const_cast<char *>(p.c.ptr) + cro + axis_offset(p.c.col, n);
+            cp[j] = n < p.N ? const_cast<char *>(p.c.ptr) + cro + axis_offset(p.c.col, n) : nullptr;
+            cin[j] = (cp[j] && e.beta != 0.f) ? load_elem(cp[j], p.c.dtype) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (!cp[j]) continue;
+            const int n = n0 + tx * 4 + j;
             const float sj = e.scale_j ? e.scale_j[n] : 1.f;
-            store_elem(cp, p.c.dtype, epi_value(acc[i][j], asi, sj, e.beta, cp, p.c.dtype));
+            float v = (asi * sj) * acc[i][j];
+            if (e.beta != 0.f) v = fmaf(e.beta, cin[j], v);
+            store_elem(cp[j], p.c.dtype, v);
         }
     }
 }

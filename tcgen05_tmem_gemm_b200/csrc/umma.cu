@@ -29,6 +29,8 @@
 //    the epilogue ("DeepGEMM deep dive", §5.2).
 // Every wait is bounded (WaitCtl); on expiry the CTA records DG_ERR_TIMEOUT,
 // drains what it has in flight, frees TMEM and exits.
+#include <atomic>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -39,6 +41,7 @@ namespace {
 constexpr int kBM = 128;             // tensor-core tile rows (TMEM lanes)
 constexpr int kTileBytesK = 128;     // one swizzle row: 64 x 16-bit or 128 x 8-bit
 constexpr int kGatherWarps = 4;
+constexpr int kPartPitch = kBM + 1;   // floats per column of a parked split-K partial
 
 struct SmemLayout {
     uint32_t stage_bytes, p_bytes, q_bytes;
@@ -84,52 +87,67 @@ __device__ __forceinline__ uint32_t sw128_mnmajor(int bytemn, int k, int chunk_b
     return (uint32_t)(c * chunk_bytes + (k >> 3) * 1024 + (k & 7) * 128 + ((((w >> 4) ^ (k & 7)) << 4) | (w & 15)));
 }
 
+template <int BYTES> struct VecOf;
+template <> struct VecOf<16> { using T = uint4; };
+template <> struct VecOf<8> { using T = uint2; };
+template <> struct VecOf<4> { using T = uint32_t; };
+template <> struct VecOf<2> { using T = unsigned short; };
+template <> struct VecOf<1> { using T = unsigned char; };
+
 template <int BYTES>
-__device__ __forceinline__ void gather_copy(uint32_t dst, const char *src, bool valid) {
+__device__ __forceinline__ typename VecOf<BYTES>::T gather_load(const char *src, bool valid) {
+    using V = typename VecOf<BYTES>::T;
+    if (!valid) return V{};
+    return __ldg(reinterpret_cast<const V *>(src));
+}
+
+template <int BYTES>
+__device__ __forceinline__ void st_shared_vec(uint32_t dst, const typename VecOf<BYTES>::T &v) {
     if constexpr (BYTES == 16) {
-        uint4 v = valid ? __ldg(reinterpret_cast<const uint4 *>(src)) : make_uint4(0, 0, 0, 0);
         asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
     } else if constexpr (BYTES == 8) {
-        uint2 v = valid ? __ldg(reinterpret_cast<const uint2 *>(src)) : make_uint2(0, 0);
         asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst), "r"(v.x), "r"(v.y));
     } else if constexpr (BYTES == 4) {
-        uint32_t v = valid ? __ldg(reinterpret_cast<const unsigned int *>(src)) : 0u;
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst), "r"(v));
     } else if constexpr (BYTES == 2) {
-        unsigned short v = valid ? __ldg(reinterpret_cast<const unsigned short *>(src)) : (unsigned short)0;
         asm volatile("st.shared.u16 [%0], %1;" ::"r"(dst), "h"(v));
     } else {
-        unsigned char v = valid ? (unsigned char)__ldg(reinterpret_cast<const char *>(src)) : (unsigned char)0;
         asm volatile("st.shared.u8 [%0], %1;" ::"r"(dst), "r"((uint32_t)v));
     }
 }
 
-// Fill one stage's P tile (kBM rows of i, bk of k) by thread loads.
+// Fill one stage's P tile (kBM rows of i, bk of k) by thread loads, kUnroll
+// loads in flight per thread before their shared-memory stores.
 template <int VB>
 __device__ __forceinline__ void gather_stage(const UmmaParams &p, uint32_t p_smem, const int64_t *row_off,
                                              const int64_t *col_off, int bk, int es, int gtid) {
+    using V = typename VecOf<VB>::T;
+    constexpr int kUnroll = 16;
     const int vec = VB / es;                       // elements per copy
     const int nthreads = kGatherWarps * 32;
-    if (p.p_mn_major) {
-        // runs of `vec` consecutive i at one k; consecutive threads take consecutive runs
-        const int runs_i = kBM / vec;
-        const int total = runs_i * bk;
-        const int chunk_bytes = bk * 128;
-        for (int u = gtid; u < total; u += nthreads) {
-            const int k = u / runs_i, i = (u % runs_i) * vec;
-            const int64_t ro = row_off[i], co = col_off[k];
+    const bool mn = p.p_mn_major != 0;
+    const int runs = mn ? kBM / vec : bk / vec;    // runs along the unit-stride dim
+    const int total = mn ? runs * bk : kBM * runs;
+    const int chunk_bytes = bk * 128;
+    for (int base = gtid; base < total; base += nthreads * kUnroll) {
+        V v[kUnroll];
+        uint32_t dst[kUnroll];
+#pragma unroll
+        for (int r = 0; r < kUnroll; ++r) {
+            const int u = base + r * nthreads;
+            int i, k;
+            if (mn) { k = u / runs; i = (u - k * runs) * vec; }
+            else { i = u / runs; k = (u - i * runs) * vec; }
+            const bool in_tile = u < total;
+            const int64_t ro = in_tile ? row_off[i] : -1, co = in_tile ? col_off[k] : -1;
             const bool ok = ro >= 0 && co >= 0;
-            gather_copy<VB>(p_smem + sw128_mnmajor(i * es, k, chunk_bytes), p.pv.ptr + (ok ? ro + co : 0), ok);
+            v[r] = gather_load<VB>(p.pv.ptr + (ok ? ro + co : 0), ok);
+            dst[r] = in_tile ? p_smem + (mn ? sw128_mnmajor(i * es, k, chunk_bytes) : sw128_kmajor(i, k * es))
+                             : 0xffffffffu;
         }
-    } else {
-        const int runs_k = bk / vec;
-        const int total = kBM * runs_k;
-        for (int u = gtid; u < total; u += nthreads) {
-            const int i = u / runs_k, k = (u % runs_k) * vec;
-            const int64_t ro = row_off[i], co = col_off[k];
-            const bool ok = ro >= 0 && co >= 0;
-            gather_copy<VB>(p_smem + sw128_kmajor(i, k * es), p.pv.ptr + (ok ? ro + co : 0), ok);
-        }
+#pragma unroll
+        for (int r = 0; r < kUnroll; ++r)
+            if (dst[r] != 0xffffffffu) st_shared_vec<VB>(dst[r], v[r]);
     }
 }
 
@@ -307,43 +325,20 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             const int j0 = tc.tj * p.bn;
 
             if (p.split_k > 1) {
-                // partial tile -> workspace [unit][col][row] (coalesced along rows)
-                float *ws = p.ws + (size_t)u * kBM * p.bn;
+                // one unit per CTA: park the partial tile in this CTA's shared
+                // memory (the operand ring is idle once the accumulator is
+                // complete), [column][row] with a 129-float pitch; the cluster
+                // reduces it after the role loops.
+                float *part = reinterpret_cast<float *>(smem);
                 for (int c0 = 0; c0 < p.bn; c0 += 16) {
                     uint32_t r[16];
                     __syncwarp();
                     tmem_ld16(t_row + c0, r);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) __stcg(ws + (size_t)(c0 + c) * kBM + row, __uint_as_float(r[c]));
+                    for (int c = 0; c < 16; ++c) part[(c0 + c) * kPartPitch + row] = __uint_as_float(r[c]);
                 }
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_tempty + 8 * b);
-                __threadfence();
-                __syncwarp();
-                const int tile = u / p.split_k;
-                uint32_t prev = 0;
-                if (lane == 0) prev = atomicAdd(p.counters + tile * 4 + quarter, 1u);
-                prev = __shfl_sync(0xffffffffu, prev, 0);
-                if (prev != (uint32_t)(p.split_k - 1)) continue;  // not the last split of this quarter
-                __threadfence();
-                if (i < p.Mi) {
-                    const float asi = e.alpha * (e.scale_i ? e.scale_i[i] : 1.f);
-                    const float *base = p.ws + (size_t)tile * p.split_k * kBM * p.bn;
-                    for (int c = 0; c < p.bn; ++c) {
-                        const int j = j0 + c;
-                        if (j >= p.Nj) break;
-                        float acc = 0.f;
-                        for (int s = 0; s < p.split_k; ++s)
-                            acc += __ldcg(base + ((size_t)s * p.bn + c) * kBM + row);
-                        char *cp = e.c + (int64_t)i * e.ci + (int64_t)j * e.cj;
-                        const float sj = e.scale_j ? e.scale_j[j] : 1.f;
-                        store_elem(cp, e.c_dtype, epi_value(acc, asi, sj, e.beta, cp, e.c_dtype));
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) p.counters[tile * 4 + quarter] = 0u;  // ready for the next call
                 continue;
             }
 
@@ -414,13 +409,22 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                     }
                 } else {
+                    // any C strides: every C load of the chunk is issued before
+                    // the first store, so they overlap instead of queueing
+                    float cin[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int j = jb + c;
+                        cin[c] = (e.beta != 0.f && j < p.Nj) ? load_elem(crow + (int64_t)j * e.cj, e.c_dtype) : 0.f;
+                    }
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
                         const int j = jb + c;
                         if (j < p.Nj) {
-                            char *cp = crow + (int64_t)j * e.cj;
                             const float sj = e.scale_j ? e.scale_j[j] : 1.f;
-                            store_elem(cp, e.c_dtype, epi_value(__uint_as_float(r[c]), asi, sj, e.beta, cp, e.c_dtype));
+                            float val = (asi * sj) * __uint_as_float(r[c]);
+                            if (e.beta != 0.f) val = fmaf(e.beta, cin[c], val);
+                            store_elem(crow + (int64_t)j * e.cj, e.c_dtype, val);
                         }
                     }
                 }
@@ -476,6 +480,64 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
         }
     }
 
+    if (p.split_k > 1) {
+        // ------------------------------------------ cluster reduction of k splits
+        // CTA s of the cluster owns rows [128 s / S, 128 (s+1) / S) of the tile
+        // and adds that slice of every split's partial, in rank order, through
+        // distributed shared memory.
+        tc_fence_before();
+        __syncthreads();
+        cluster_sync();
+        if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+            const EpiParams &e = p.epi;
+            const TileCoord tc = unit_coord(blockIdx.x, p);
+            const int S = p.split_k;
+            const uint32_t rank = cluster_ctarank();
+            const int r0 = (int)(rank * kBM / S), r1 = (int)((rank + 1) * kBM / S), rs = r1 - r0;
+            const int t = threadIdx.x - kEpiWarp0 * 32;
+            const bool along_i = (e.ci == (int64_t)elem_bytes(e.c_dtype));  // C contiguous along i
+            const uint32_t part_addr = sbase;
+            constexpr int kB = 8;  // outputs per thread per batch, all their loads in flight together
+            for (int base = t; base < rs * p.bn; base += 128 * kB) {
+                int ii[kB], jj[kB];
+                float v[kB][8], cin[kB];
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    const int el = base + b * 128;
+                    int r = 0, c = 0;
+                    if (along_i) { r = el % rs; c = el / rs; }
+                    else { c = el % p.bn; r = el / p.bn; }
+                    const int i = tc.ti * kBM + r0 + r, j = tc.tj * p.bn + c;
+                    const bool ok = el < rs * p.bn && i < p.Mi && j < p.Nj;
+                    ii[b] = ok ? i : -1;
+                    jj[b] = j;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        v[b][q] = (ok && q < S)
+                                      ? dsmem_ld_f32(dsmem_map(part_addr + (uint32_t)((c * kPartPitch + r0 + r) * 4), q))
+                                      : 0.f;
+                    cin[b] = (ok && e.beta != 0.f) ? load_elem(e.c + (int64_t)i * e.ci + (int64_t)j * e.cj, e.c_dtype)
+                                                   : 0.f;
+                }
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    if (ii[b] < 0) continue;
+                    const int i = ii[b], j = jj[b];
+                    float acc = 0.f;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        if (q < S) acc += v[b][q];
+                    const float asi = e.alpha * (e.scale_i ? e.scale_i[i] : 1.f);
+                    const float sj = e.scale_j ? e.scale_j[j] : 1.f;
+                    float val = (asi * sj) * acc;
+                    if (e.beta != 0.f) val = fmaf(e.beta, cin[b], val);
+                    store_elem(e.c + (int64_t)i * e.ci + (int64_t)j * e.cj, e.c_dtype, val);
+                }
+            }
+        }
+        cluster_sync();  // partials stay alive until every CTA of the cluster has read them
+    }
+
     // --------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
@@ -504,11 +566,29 @@ cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtens
     void (*kern)(const CUtensorMap, const CUtensorMap, const UmmaParams);
     if (fp8) kern = gather ? umma_gemm_kernel<true, true> : umma_gemm_kernel<true, false>;
     else kern = gather ? umma_gemm_kernel<false, true> : umma_gemm_kernel<false, false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int threads = gather ? 320 : 192;
-    kern<<<grid, threads, smem, s>>>(*tp, *tq, p);
-    return cudaGetLastError();
+    // raise the kernel's dynamic shared-memory limit once per size, not per call
+    static std::atomic<int> s_limit[4];
+    std::atomic<int> &lim = s_limit[(fp8 ? 2 : 0) + (gather ? 1 : 0)];
+    cudaError_t e = cudaSuccess;
+    if ((int)smem > lim.load()) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        lim.store((int)smem);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(gather ? 320 : 192);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.split_k;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.split_k > 1 ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, *tp, *tq, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace dg

@@ -26,7 +26,7 @@ def _reset_options():
     dg.dg_set_option(dg.DG_OPT_FORCE_KIND, 0)
     dg.dg_set_option(dg.DG_OPT_TEST_STALL, 0)
     dg.dg_set_option(dg.DG_OPT_WAIT_TIMEOUT_MS, 2000)
-    dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, 16)
+    dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, 8)
 
 
 def expect_kind(p, kind, **fields):
