@@ -178,6 +178,8 @@ typedef struct {
     int32_t grid;          /* CTAs launched                                          */
     int32_t vec_bytes;     /* gather / GEMV vector width                             */
     int64_t M, N, K;
+    int32_t cta_pair;      /* UMMA: two CTAs of a cluster share each 256-row tile     */
+    int32_t reserved;
 } dg_plan_info;
 
 /* The dispatch decision dg_gemm would take for these views (pointers are only
@@ -198,8 +200,11 @@ typedef enum {
     DG_OPT_TEST_STALL = 3,        /* 1: the tensor-core kernel's loader issues no
                                      copies, so its waits run out and the call
                                      reports DG_ERR_TIMEOUT (tests of the bound)      */
-    DG_OPT_MAX_SPLIT_K = 4        /* upper bound on the tensor-core kernel's split-K
+    DG_OPT_MAX_SPLIT_K = 4,       /* upper bound on the tensor-core kernel's split-K
                                      (default and cluster limit 8; 1 disables)         */
+    DG_OPT_CTA_PAIR = 5           /* paired-CTA (256-row) tensor-core tiles: 0 never,
+                                     1 for large problems (default), 2 whenever the
+                                     operands allow                                    */
 } dg_option;
 
 dg_status dg_set_option(int option, int64_t value);

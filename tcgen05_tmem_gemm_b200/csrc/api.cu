@@ -31,6 +31,7 @@ std::atomic<int> g_force_kind{0};
 std::atomic<int64_t> g_timeout_ms{2000};
 std::atomic<int> g_stall{0};
 std::atomic<int> g_max_split{8};
+std::atomic<int> g_pair{1};
 std::atomic<uint32_t> g_epoch{1};  // bumped by every option change: cached launches go stale
 
 constexpr int kMaxDevices = 64;
@@ -142,7 +143,7 @@ struct Views {
     ViewInfo a, b, c;
 };
 
-uint32_t make_idesc(int in_dtype, bool p_mn, bool q_mn, int bn) {
+uint32_t make_idesc(int in_dtype, bool p_mn, bool q_mn, int bn, int m = 128) {
     uint32_t d = 0;
     d |= 1u << 4;                                    // D format: F32
     const uint32_t fmt = (in_dtype == DG_BF16) ? 1u : 0u;  // F16 = 0, BF16 = 1; E4M3 = 0 (kind::f8f6f4)
@@ -151,7 +152,7 @@ uint32_t make_idesc(int in_dtype, bool p_mn, bool q_mn, int bn) {
     d |= (p_mn ? 1u : 0u) << 15;                     // A major (1 = MN)
     d |= (q_mn ? 1u : 0u) << 16;                     // B major
     d |= (uint32_t)(bn >> 3) << 17;                  // N >> 3
-    d |= (uint32_t)(128 >> 4) << 24;                 // M >> 4
+    d |= (uint32_t)(m >> 4) << 24;                   // M >> 4 (256 for a CTA pair)
     return d;
 }
 
@@ -279,7 +280,16 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, int num_sms, Pla
     split = (kb_total + kb_per - 1) / kb_per;
     const int64_t units = tiles * split;
     if (units > INT32_MAX) return false;
-    const int stages = umma_max_stages(bn, !p_tma);
+    // a CTA pair shares each 256 x bn tile when there are enough tiles to fill
+    // the machine (or when forced); TMA operands only, no split
+    const int pair_mode = g_pair.load();
+    bool pair = false;
+    if (pair_mode > 0 && p_tma && split == 1 && bn >= 128 && num_sms >= 2) {
+        const int per = 128 / es;
+        const bool halves_ok = !q_mn || ((bn / 2) % per == 0);
+        if (halves_ok) pair = (pair_mode == 2) || (Mi >= 256 && tiles >= num_sms);
+    }
+    const int stages = pair ? umma_pair_max_stages(bn) : umma_max_stages(bn, !p_tma);
     dg_plan_info &in = pl->info;
     in.kind = DG_KIND_UMMA;
     in.swap_ab = swap;
@@ -293,8 +303,14 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, int num_sms, Pla
     in.split_k = (int32_t)split;
     in.grid = (int32_t)(split > 1 ? units : std::min<int64_t>(units, num_sms));  // split: one unit per CTA
     in.vec_bytes = p_tma ? 16 : gather_vec * es;
+    in.cta_pair = pair;
+    if (pair) {
+        const int64_t pair_units = ((Mi + 255) / 256) * tiles_j;
+        in.block_m = 256;
+        in.grid = (int32_t)(2 * std::min<int64_t>(pair_units, num_sms / 2));
+    }
     pl->fp8 = (dt == DG_E4M3);
-    pl->smem = umma_smem_bytes(bn, 128, stages, !p_tma);
+    pl->smem = pair ? umma_pair_smem_bytes(bn, stages) : umma_smem_bytes(bn, 128, stages, !p_tma);
     return true;
 }
 
@@ -439,7 +455,7 @@ struct LaunchRec {
     GemvParams gemv{};
     UmmaParams umma{};
     CUtensorMap t0{}, t1{};
-    bool fp8 = false, gather = false;
+    bool fp8 = false, gather = false, pair = false;
     int grid = 0;
     size_t smem = 0;
 };
@@ -515,8 +531,9 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
             if (!ok) return DG_ERR_UNSUPPORTED;
         }
         {
+            const int q_rows = in.cta_pair ? bn / 2 : bn;  // a CTA of a pair loads half of the tile's columns
             const bool ok = in.q_mn_major ? encode_2d(&tq, dt, Qv->ptr, Nj, in.K, axis_stride(q_k), bk)
-                                          : encode_2d(&tq, dt, Qv->ptr, in.K, Nj, axis_stride(q_j), bn);
+                                          : encode_2d(&tq, dt, Qv->ptr, in.K, Nj, axis_stride(q_j), q_rows);
             if (!ok) return DG_ERR_UNSUPPORTED;
         }
         UmmaParams p{};
@@ -526,7 +543,7 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         p.bn = bn;
         p.bk = bk;
         p.stages = in.stages;
-        p.tiles_i = (int32_t)((Mi + 127) / 128);
+        p.tiles_i = (int32_t)((Mi + in.block_m - 1) / in.block_m);
         p.tiles_j = (int32_t)((Nj + bn - 1) / bn);
         p.split_k = in.split_k;
         p.kb_total = (int32_t)((in.K + bk - 1) / bk);
@@ -534,7 +551,7 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         p.num_units = p.tiles_i * p.tiles_j * p.split_k;
         p.p_mn_major = in.p_mn_major;
         p.q_mn_major = in.q_mn_major;
-        p.idesc = make_idesc(dt, in.p_mn_major, in.q_mn_major, bn);
+        p.idesc = make_idesc(dt, in.p_mn_major, in.q_mn_major, bn, in.cta_pair ? 256 : 128);
         int tc = 32;
         while (tc < 2 * bn) tc *= 2;
         p.tmem_cols = tc;
@@ -552,6 +569,7 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         p.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
         p.stall_loader = g_stall.load();
         rec->umma = p;
+        rec->pair = in.cta_pair != 0;
         rec->fp8 = pl.fp8;
         rec->gather = in.p_gather != 0;
         rec->grid = in.grid;
@@ -573,7 +591,10 @@ dg_status fire(const LaunchRec &r, cudaStream_t stream) {
     case DG_KIND_SIMT: err = launch_simt(r.simt, stream); break;
     case DG_KIND_GEMV_N: err = launch_gemv_n(r.gemv, &r.t0, stream, &grid); break;
     case DG_KIND_GEMV_K: err = launch_gemv_k(r.gemv, stream, &grid); break;
-    case DG_KIND_UMMA: err = launch_umma(r.umma, &r.t0, &r.t1, r.fp8, r.gather, r.grid, r.smem, stream); break;
+    case DG_KIND_UMMA:
+        err = r.pair ? launch_umma_pair(r.umma, &r.t0, &r.t1, r.fp8, r.grid, r.smem, stream)
+                     : launch_umma(r.umma, &r.t0, &r.t1, r.fp8, r.gather, r.grid, r.smem, stream);
+        break;
     default: return DG_ERR_UNSUPPORTED;
     }
     if (err != cudaSuccess) return DG_ERR_CUDA;
@@ -743,6 +764,10 @@ dg_status dg_set_option(int option, int64_t value) {
         return DG_OK;
     case DG_OPT_TEST_STALL:
         g_stall.store(value ? 1 : 0);
+        return DG_OK;
+    case DG_OPT_CTA_PAIR:
+        if (value < 0 || value > 2) return DG_ERR_VALUE;
+        g_pair.store((int)value);
         return DG_OK;
     case DG_OPT_MAX_SPLIT_K:
         if (value < 1 || value > 64) return DG_ERR_VALUE;

@@ -9,6 +9,48 @@
 
 namespace dg {
 
+// Programmatic dependent launch.  Every kernel here is launched with
+// programmatic stream serialisation: it may be scheduled while the previous
+// kernel on the stream is still running, so its very first action is to wait
+// for that kernel to complete (and its writes to be visible) before touching
+// global memory.  Short kernels then release their dependents at once; long
+// ones release them at their tail (after the main loop), so waiting
+// dependents do not hold SM slots while the main loop runs.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_then_release() {
+    pdl_wait();
+    pdl_release();
+}
+
+// cudaLaunchKernelEx with programmatic stream serialisation and an optional
+// thread-block cluster shape.
+template <typename Kern, typename... Args>
+cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s, dim3 cluster,
+                      Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster.x * cluster.y * cluster.z > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster.x;
+        attr[n].val.clusterDim.y = cluster.y;
+        attr[n].val.clusterDim.z = cluster.z;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 __device__ __forceinline__ float load_elem(const char *p, int dtype) {
     switch (dtype) {
     case DG_F32: return *reinterpret_cast<const float *>(p);

@@ -119,6 +119,10 @@ cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtens
                         bool fp8, bool gather, int grid, size_t smem, cudaStream_t s);
 size_t umma_smem_bytes(int bn, int bk_bytes, int stages, bool gather);
 int umma_max_stages(int bn, bool gather);
+cudaError_t launch_umma_pair(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq, bool fp8, int grid,
+                             size_t smem, cudaStream_t s);
+size_t umma_pair_smem_bytes(int bn, int stages);
+int umma_pair_max_stages(int bn);
 
 cudaError_t launch_gemv_n(const GemvParams &p, const CUtensorMap *tmap_w, cudaStream_t s, int *grid_out);
 size_t gemv_n_smem_bytes(int r_inst, int kper);

@@ -36,6 +36,7 @@ constexpr int kRows = 32;       // rows of W per TMA stage
 constexpr int kStages = 6;      // ring depth
 constexpr int kCW = 8;          // consumer warps
 constexpr int kNT = 32 * (kCW + 1);
+constexpr int kReleaseStages = 6;  // dependents are released this many stages before the end
 
 template <typename T>
 __device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8]);
@@ -125,6 +126,7 @@ __host__ __device__ inline GemvNLayout gemv_n_layout(int R, int kper) {
 template <typename T, int R>
 __global__ void __launch_bounds__(kNT) gemv_n_kernel(const __grid_constant__ CUtensorMap tmap_w,
                                                      const GemvParams p) {
+    pdl_wait();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const GemvNLayout L = gemv_n_layout(R, p.kper);
@@ -158,9 +160,13 @@ __global__ void __launch_bounds__(kNT) gemv_n_kernel(const __grid_constant__ CUt
         // ----------------------------------------------------- TMA producer
         if (lane == 0) {
             int it = 0;
+            const int release_at = max(0, nst - kReleaseStages);
             for (; it < nst; ++it) {
                 const int s = it % kStages;
                 const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                // a few stages before the end: let the next kernel be scheduled, so its
+                // launch latency overlaps this kernel's last loads and reduction
+                if (it == release_at) pdl_release();
                 if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) break;
                 mbar_arrive_expect_tx(bar_full + 8 * s, kRows * kNB * 2);
                 tma_load_2d(sbase + L.ring + s * (kRows * kNB * 2), &tmap_w, bar_full + 8 * s, n0, kb0 + it * kRows);
@@ -259,6 +265,7 @@ __global__ void __launch_bounds__(256) gemv_k_kernel(const GemvParams p) {
     constexpr int WPC = 4;
     constexpr int CPB = 8 / WPC;
     constexpr int MAXV = 8;                 // 16-byte loads per lane kept in flight
+    pdl_wait_then_release();
     extern __shared__ float smem[];
     float *xs = smem;                       // [R][K]
     float *red = smem + R * p.K;            // [8 warps][R]
@@ -349,21 +356,9 @@ cudaError_t run_n(const GemvParams &p, const CUtensorMap *tmap, cudaStream_t s, 
     auto kern = gemv_n_kernel<T, R>;
     cudaError_t e = ensure_smem<KernelTag<T, R, 0>>(kern, smem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(gx, gy);
-    cfg.blockDim = dim3(kNT);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = gy;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = gy > 1 ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kern, *tmap, p);
+    e = launch_ex(kern, dim3(gx, gy), dim3(kNT), smem, s, dim3(1, gy, 1), *tmap, p);
     *grid_out = gx * gy;
-    return e != cudaSuccess ? e : cudaGetLastError();
+    return e;
 }
 
 template <typename T>
@@ -381,9 +376,8 @@ cudaError_t run_k(const GemvParams &p, cudaStream_t s, int *grid_out) {
     auto kern = gemv_k_kernel<T, R>;
     cudaError_t e = ensure_smem<KernelTag<T, R, 1>>(kern, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 256, smem, s>>>(p);
     *grid_out = grid;
-    return cudaGetLastError();
+    return launch_ex(kern, dim3(grid), dim3(256), smem, s, dim3(1, 1, 1), p);
 }
 
 template <typename T>

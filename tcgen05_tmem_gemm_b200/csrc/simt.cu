@@ -15,6 +15,7 @@ namespace {
 constexpr int TM = 64, TN = 64, TK = 16, NT = 256;
 
 __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtParams p) {
+    pdl_wait_then_release();
     __shared__ float As[TK][TM + 4];
     __shared__ float Bs[TK][TN + 4];
     __shared__ int64_t a_row_off[TM], b_col_off[TN];
@@ -91,6 +92,7 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtParams p) {
 }
 
 __global__ void scale_c_kernel(const DevView c, int64_t M, int64_t N, float beta) {
+    pdl_wait_then_release();
     const int64_t total = M * N;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
@@ -105,16 +107,14 @@ __global__ void scale_c_kernel(const DevView c, int64_t M, int64_t N, float beta
 cudaError_t launch_simt(const SimtParams &p, cudaStream_t s) {
     dim3 grid((p.N + TN - 1) / TN, (p.M + TM - 1) / TM);
     if (grid.y > 65535) return cudaErrorInvalidConfiguration;
-    simt_gemm_kernel<<<grid, NT, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_ex(simt_gemm_kernel, grid, dim3(NT), 0, s, dim3(1, 1, 1), p);
 }
 
 cudaError_t launch_scale_c(const DevView &c, int64_t M, int64_t N, float beta, cudaStream_t s) {
     const int64_t total = M * N;
     int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 16);
     if (blocks < 1) blocks = 1;
-    scale_c_kernel<<<blocks, 256, 0, s>>>(c, M, N, beta);
-    return cudaGetLastError();
+    return launch_ex(scale_c_kernel, dim3(blocks), dim3(256), 0, s, dim3(1, 1, 1), c, M, N, beta);
 }
 
 }  // namespace dg

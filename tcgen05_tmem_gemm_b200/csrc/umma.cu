@@ -33,6 +33,7 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "umma_common.cuh"
 
 namespace dg {
 
@@ -169,6 +170,7 @@ template <bool FP8, bool GATHER>
 __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const UmmaParams p) {
+    pdl_wait();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -304,6 +306,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                 if (!ok) break;
                 tc_commit(bar_tfull + 8 * b);      // accumulator b is complete
             }
+            pdl_release();  // every MMA is issued: the next kernel may be scheduled during the epilogue
             // wait for every MMA this thread issued before TMEM can be freed
             tc_commit(bar_drain);
             mbar_wait_drain(bar_drain, 0, p.timeout_ns);
@@ -351,83 +354,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                 tmem_ld16(t_row + c0, r);
                 tmem_ld_wait();
                 if (!row_ok) continue;
-                const int jb = j0 + c0;
-                if (e.vec_ok && jb + 16 <= p.Nj) {
-                    float v[16];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const float sj = e.scale_j ? e.scale_j[jb + c] : 1.f;
-                        v[c] = (asi * sj) * __uint_as_float(r[c]);
-                    }
-                    if (e.c_dtype == DG_F32) {
-                        float4 *dst = reinterpret_cast<float4 *>(crow + (int64_t)jb * 4);
-                        if (e.beta != 0.f) {
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const float4 o = dst[q];
-                                v[4 * q + 0] = fmaf(e.beta, o.x, v[4 * q + 0]);
-                                v[4 * q + 1] = fmaf(e.beta, o.y, v[4 * q + 1]);
-                                v[4 * q + 2] = fmaf(e.beta, o.z, v[4 * q + 2]);
-                                v[4 * q + 3] = fmaf(e.beta, o.w, v[4 * q + 3]);
-                            }
-                        }
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                    } else {
-                        // 16-bit output: two 16-byte stores
-                        uint4 *dst = reinterpret_cast<uint4 *>(crow + (int64_t)jb * 2);
-                        uint32_t w[8];
-                        if (e.beta != 0.f) {
-                            const uint4 o0 = dst[0], o1 = dst[1];
-                            const uint32_t ow[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                float lo, hi;
-                                if (e.c_dtype == DG_BF16) {
-                                    lo = __uint_as_float(ow[q] << 16);
-                                    hi = __uint_as_float(ow[q] & 0xffff0000u);
-                                } else {
-                                    const float2 t = __half22float2(*reinterpret_cast<const __half2 *>(&ow[q]));
-                                    lo = t.x;
-                                    hi = t.y;
-                                }
-                                v[2 * q] = fmaf(e.beta, lo, v[2 * q]);
-                                v[2 * q + 1] = fmaf(e.beta, hi, v[2 * q + 1]);
-                            }
-                        }
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            if (e.c_dtype == DG_BF16) {
-                                __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
-                                w[q] = *reinterpret_cast<uint32_t *>(&h);
-                            } else {
-                                __half2 h = __floats2half2_rn(v[2 * q], v[2 * q + 1]);
-                                w[q] = *reinterpret_cast<uint32_t *>(&h);
-                            }
-                        }
-                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                    }
-                } else {
-                    // any C strides: every C load of the chunk is issued before
-                    // the first store, so they overlap instead of queueing
-                    float cin[16];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const int j = jb + c;
-                        cin[c] = (e.beta != 0.f && j < p.Nj) ? load_elem(crow + (int64_t)j * e.cj, e.c_dtype) : 0.f;
-                    }
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const int j = jb + c;
-                        if (j < p.Nj) {
-                            const float sj = e.scale_j ? e.scale_j[j] : 1.f;
-                            float val = (asi * sj) * __uint_as_float(r[c]);
-                            if (e.beta != 0.f) val = fmaf(e.beta, cin[c], val);
-                            store_elem(crow + (int64_t)j * e.cj, e.c_dtype, val);
-                        }
-                    }
-                }
+                epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
             }
             tc_fence_before();
             __syncwarp();
@@ -575,20 +502,7 @@ cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtens
         if (e != cudaSuccess) return e;
         lim.store((int)smem);
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(gather ? 320 : 192);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p.split_k;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = p.split_k > 1 ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kern, *tp, *tq, p);
-    return e != cudaSuccess ? e : cudaGetLastError();
+    return launch_ex(kern, dim3(grid), dim3(gather ? 320 : 192), smem, s, dim3(p.split_k, 1, 1), *tp, *tq, p);
 }
 
 }  // namespace dg

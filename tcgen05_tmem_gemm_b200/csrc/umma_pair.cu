@@ -1,0 +1,251 @@
+// Paired-CTA tensor-core GEMM for sm_100a: tcgen05.mma.cta_group::2.
+//
+// Two CTAs of a cluster compute one 256 x bn tile of D = P Q together.  Each
+// CTA loads its own 128 rows of P and its own half (bn/2 columns) of Q into
+// its shared memory, holds its 128 x bn half of the accumulator in its TMEM,
+// and runs its own epilogue; the even CTA of the pair issues the MMAs for
+// both.  Against one CTA per 128 x bn tile this halves each SM's share of the
+// Q tile: 32 KB instead of 48 KB of operands per 64-deep k step at bn = 256,
+// so more stages fit in shared memory and less L2 bandwidth is needed per
+// flop ("DeepGEMM deep dive", §2.1-§2.3: blocking for reuse, and overlapping
+// loads with compute, taken to the pair of SMs that Blackwell's tensor core
+// can drive as one).
+//
+// Barriers: full[s] lives in the even CTA and counts the copy bytes of both
+// CTAs (each CTA's TMA loads signal it across the pair); empty[s] and the
+// accumulator-ready barriers exist in both CTAs and are signalled by one
+// multicast tcgen05.commit; accumulator-drained barriers live in the even CTA
+// and collect the epilogue warps of both.  Every wait is bounded as in the
+// single-CTA kernel.  Loads use no cluster multicast.
+#include <atomic>
+
+#include "common.cuh"
+#include "sm100.cuh"
+#include "umma_common.cuh"
+
+namespace dg {
+
+namespace {
+
+constexpr int kHalfM = 128;   // rows of P (and TMEM lanes) per CTA
+constexpr int kRowBytes = 128;
+
+struct PairLayout {
+    uint32_t a_bytes, b_bytes, stage_bytes, bar_off, aux_off, total;
+};
+
+__host__ __device__ inline PairLayout pair_layout(int bn, int stages) {
+    PairLayout L;
+    L.a_bytes = kHalfM * kRowBytes;
+    L.b_bytes = (uint32_t)(bn / 2) * kRowBytes;
+    L.stage_bytes = L.a_bytes + L.b_bytes;
+    L.bar_off = L.stage_bytes * stages;
+    // full[S], empty[S], tfull[2], tempty[2], drain
+    L.aux_off = L.bar_off + 8 * (2 * stages + 5);
+    L.total = L.aux_off + 16 + 1024;
+    return L;
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(192, 1)
+    umma_pair_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
+                     const UmmaParams p) {
+    pdl_wait();
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const PairLayout L = pair_layout(p.bn, p.stages);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + L.bar_off;
+    const uint32_t bar_empty = bar_full + 8 * p.stages;
+    const uint32_t bar_tfull = bar_empty + 8 * p.stages;
+    const uint32_t bar_tempty = bar_tfull + 16;
+    const uint32_t bar_drain = bar_tempty + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.aux_off);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.aux_off + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cluster_id = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const WaitCtl wc{abort_flag, p.err_word, p.timeout_ns};
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, 8);  // four epilogue warps in each CTA of the pair
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+        tma_prefetch_desc(&tmap_p);
+        tma_prefetch_desc(&tmap_q);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before either signals the other's
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int es = FP8 ? 1 : 2;
+    const int bk = p.bk;
+    const int half_bn = p.bn / 2;
+    constexpr int kUmmaK = FP8 ? 32 : 16;
+    const int per = 128 / es;  // MN elements per 128-byte row of an MN-major box
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            int it = 0;
+            for (int u = cluster_id; u < p.num_units && !*abort_flag; u += nclusters) {
+                const int ti = u % p.tiles_i, tj = u / p.tiles_i;
+                const int i0 = ti * 2 * kHalfM + (int)rank * kHalfM;
+                const int j0 = tj * p.bn + (int)rank * half_bn;
+                for (int kb = 0; kb < p.kb_total; ++kb, ++it) {
+                    const int s = it % p.stages;
+                    const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
+                    if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) break;
+                    if (p.stall_loader) continue;
+                    const uint32_t full_c = dsmem_map(bar_full + 8 * s, 0);
+                    if (leader) mbar_arrive_expect_tx(bar_full + 8 * s, 2 * L.stage_bytes);
+                    const uint32_t as = sbase + s * L.stage_bytes;
+                    const uint32_t bs = as + L.a_bytes;
+                    const int k0 = kb * bk;
+                    if (p.p_mn_major) {
+                        for (int c = 0; c < kHalfM / per; ++c)
+                            tma_load_2d_pair(as + c * bk * 128, &tmap_p, full_c, i0 + c * per, k0);
+                    } else {
+                        tma_load_2d_pair(as, &tmap_p, full_c, k0, i0);
+                    }
+                    if (p.q_mn_major) {
+                        for (int c = 0; c < half_bn / per; ++c)
+                            tma_load_2d_pair(bs + c * bk * 128, &tmap_q, full_c, j0 + c * per, k0);
+                    } else {
+                        tma_load_2d_pair(bs, &tmap_q, full_c, k0, j0);
+                    }
+                }
+            }
+            if (!leader) pdl_release();
+            // full[] of the even CTA counts both CTAs' bytes: once its last
+            // phases complete, every copy of the pair has landed
+            if (leader && !p.stall_loader)
+                for (int d = 1; d <= p.stages && it - d >= 0; ++d) {
+                    const int j = it - d;
+                    mbar_wait_drain(bar_full + 8 * (j % p.stages), (uint32_t)(j / p.stages) & 1u, p.timeout_ns);
+                }
+        }
+    } else if (warp == 1) {
+        // ----------------------------------------- MMA issuer (even CTA only)
+        if (lane == 0 && leader) {
+            int it = 0, local = 0;
+            const uint32_t p_lbo = p.p_mn_major ? (uint32_t)(bk * 128) : 16u;
+            const uint32_t q_lbo = p.q_mn_major ? (uint32_t)(bk * 128) : 16u;
+            const uint32_t p_kstep = p.p_mn_major ? kUmmaK * 128 : kUmmaK * es;
+            const uint32_t q_kstep = p.q_mn_major ? kUmmaK * 128 : kUmmaK * es;
+            bool ok = true;
+            for (int u = cluster_id; u < p.num_units && ok; u += nclusters, ++local) {
+                const int b = local & 1;
+                const uint32_t tph = (uint32_t)(local >> 1) & 1u;
+                if (!mbar_wait(bar_tempty + 8 * b, tph ^ 1u, wc)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * p.bn);
+                for (int kb = 0; kb < p.kb_total; ++kb, ++it) {
+                    const int s = it % p.stages;
+                    const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
+                    if (!mbar_wait(bar_full + 8 * s, ph, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t as = sbase + s * L.stage_bytes;
+                    const uint32_t bs = as + L.a_bytes;
+#pragma unroll
+                    for (int kk = 0; kk < kRowBytes / (kUmmaK * es); ++kk) {
+                        const uint64_t da = make_sw128_desc(as + kk * p_kstep, p_lbo, 1024);
+                        const uint64_t db = make_sw128_desc(bs + kk * q_kstep, q_lbo, 1024);
+                        const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+                        if (FP8) umma_f8_pair(d_tmem, da, db, p.idesc, acc);
+                        else umma_f16_pair(d_tmem, da, db, p.idesc, acc);
+                    }
+                    tc_commit_pair_mc(bar_empty + 8 * s, 0x3);  // the stage is free in both CTAs
+                }
+                if (!ok) break;
+                tc_commit_pair_mc(bar_tfull + 8 * b, 0x3);       // both halves of the accumulator are ready
+            }
+            pdl_release();
+            tc_commit_pair_mc(bar_drain, 0x1);
+            mbar_wait_drain(bar_drain, 0, p.timeout_ns);
+        }
+    } else {
+        // ------------------------------------------- epilogue (both CTAs)
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const EpiParams &e = p.epi;
+        int local = 0;
+        for (int u = cluster_id; u < p.num_units; u += nclusters, ++local) {
+            const int ti = u % p.tiles_i, tj = u / p.tiles_i;
+            const int b = local & 1;
+            const uint32_t tph = (uint32_t)(local >> 1) & 1u;
+            if (!mbar_wait(bar_tfull + 8 * b, tph, wc)) break;
+            tc_fence_after();
+            const int i = ti * 2 * kHalfM + (int)rank * kHalfM + row;
+            const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * p.bn);
+            const int j0 = tj * p.bn;
+            const bool row_ok = i < p.Mi;
+            const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
+            char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
+            for (int c0 = 0; c0 < p.bn; c0 += 16) {
+                uint32_t r[16];
+                __syncwarp();
+                tmem_ld16(t_row + c0, r);
+                tmem_ld_wait();
+                if (!row_ok) continue;
+                epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(dsmem_map(bar_tempty + 8 * b, 0));
+        }
+    }
+
+    // --------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // neither CTA frees TMEM or exits while the pair still uses it
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, (uint32_t)p.tmem_cols);
+    }
+}
+
+}  // namespace
+
+size_t umma_pair_smem_bytes(int bn, int stages) { return pair_layout(bn, stages).total; }
+
+int umma_pair_max_stages(int bn) {
+    int s = 2;
+    while (s < 12 && pair_layout(bn, s + 1).total <= 227 * 1024) ++s;
+    return s;
+}
+
+cudaError_t launch_umma_pair(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq, bool fp8, int grid,
+                             size_t smem, cudaStream_t s) {
+    void (*kern)(const CUtensorMap, const CUtensorMap, const UmmaParams);
+    kern = fp8 ? umma_pair_kernel<true> : umma_pair_kernel<false>;
+    static std::atomic<int> s_limit[2];
+    std::atomic<int> &lim = s_limit[fp8 ? 1 : 0];
+    if ((int)smem > lim.load()) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        lim.store((int)smem);
+    }
+    return launch_ex(kern, dim3(grid), dim3(192), smem, s, dim3(2, 1, 1), *tp, *tq, p);
+}
+
+}  // namespace dg

@@ -127,6 +127,7 @@ def test_plan_small_gemm_umma():
     pl = plan_of("small")
     assert pl["kind_name"] == "umma" and pl["swap_ab"] == 0 and pl["block_n"] == 128
     assert pl["p_mn_major"] == 0 and pl["q_mn_major"] == 1 and pl["split_k"] == 1
+    assert pl["cta_pair"] == 0  # one tile: no pairing
 
 
 def test_plan_thin_swaps_and_splits():
@@ -139,6 +140,7 @@ def test_plan_thin_swaps_and_splits():
 def test_plan_square_bf16_and_fp8():
     pl = plan_of("square_bf16", M=4096, N=4096, K=64)
     assert pl["kind_name"] == "umma" and pl["block_n"] == 256 and pl["grid"] == 148
+    assert pl["cta_pair"] == 1 and pl["block_m"] == 256  # CTA pairs share 256-row tiles
     pl = plan_of("square_e4m3", M=4096, N=4096, K=64)
     assert pl["kind_name"] == "umma" and pl["block_k"] == 128 and pl["q_mn_major"] == 1
 

@@ -27,6 +27,7 @@ def _reset_options():
     dg.dg_set_option(dg.DG_OPT_TEST_STALL, 0)
     dg.dg_set_option(dg.DG_OPT_WAIT_TIMEOUT_MS, 2000)
     dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, 8)
+    dg.dg_set_option(dg.DG_OPT_CTA_PAIR, 1)
 
 
 def expect_kind(p, kind, **fields):
@@ -89,6 +90,39 @@ def test_fp8_k_major_b():
     p = W.Problem("fp8_kmajor", W.row_major(qa, "e4m3"), W.transposed(qbt, "e4m3"), W.empty_out(M, N, "f32"),
                   0.5, 0.0, sa, sb)
     expect_kind(p, "umma", q_mn_major=0)
+    check_full(p)
+
+
+@pytest.mark.parametrize("M,N,K,dt,out,ta,tb", [
+    (300, 520, 200, "bf16", "bf16", False, False),
+    (1000, 264, 1000, "f16", "f32", False, False),
+    (264, 200, 136, "bf16", "f32", True, False),
+    (520, 256, 64, "bf16", "bf16", False, True),
+    (256, 128, 16, "f16", "f16", False, False),
+])
+def test_umma_cta_pair_forced(M, N, K, dt, out, ta, tb):
+    # two CTAs of a cluster share each 256-row tile (tcgen05 cta_group::2)
+    dg.dg_set_option(dg.DG_OPT_CTA_PAIR, 2)
+    g = torch.Generator().manual_seed(M + 3 * N + K)
+    a = W.cast(W.normal((K, M) if ta else (M, K), g), dt)
+    b = W.cast(W.normal((N, K) if tb else (K, N), g), dt)
+    A = W.transposed(a, dt) if ta else W.row_major(a, dt)
+    B = W.transposed(b, dt) if tb else W.row_major(b, dt)
+    c = W.uniform((M, N), g)
+    p = W.Problem("pair", A, B, W.row_major(c.to(W.TORCH_DTYPE[out]).contiguous(), out), 0.75, 0.5)
+    expect_kind(p, "umma", cta_pair=1, block_m=256)
+    check_full(p)
+
+
+def test_umma_cta_pair_fp8():
+    dg.dg_set_option(dg.DG_OPT_CTA_PAIR, 2)
+    M, N, K = 384, 256, 384
+    g = torch.Generator().manual_seed(77)
+    qa, sa = W.quantise_e4m3(W.normal((M, K), g), dim=1)
+    qbt, sb = W.quantise_e4m3(W.normal((N, K), g), dim=1)
+    p = W.Problem("pair_fp8", W.row_major(qa, "e4m3"), W.transposed(qbt, "e4m3"), W.empty_out(M, N, "bf16"),
+                  1.0, 0.0, sa, sb)
+    expect_kind(p, "umma", cta_pair=1)
     check_full(p)
 
 
@@ -307,4 +341,6 @@ def test_full_size_sampled(name):
     pl = expect_kind(p, {"gemv": "gemv_n", "gemv_kt": "gemv_k"}.get(name, "umma"))
     if name == "thin":
         assert pl["swap_ab"] == 1 and pl["split_k"] == 4
+    if name.startswith("square"):
+        assert pl["cta_pair"] == 1
     check_sampled(p, npts=3000)
