@@ -306,9 +306,25 @@ def run_one_shape(args):
 
     if args.max_split:
         dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, args.max_split)
+    if args.early_launch >= 0:
+        dg.dg_set_option(dg.DG_OPT_EARLY_LAUNCH, args.early_launch)
 
     res = per_shape(dg, load_peaks(), True, only=args.shape)
-    print(json.dumps({"shape": args.shape, **res}), flush=True)
+    out = {"shape": args.shape, **res}
+    if args.trace:
+        # one more call with CTA 0's phase timestamps (ns from kernel entry)
+        buf = torch.zeros(64, dtype=torch.int64, device="cuda")
+        key = [k for k in SHAPES if k[0] == args.shape][0]
+        prob = key[2]().to("cuda")
+        dg.dg_set_option(dg.DG_OPT_TRACE, buf.data_ptr())
+        A, B, C = dg_views(prob, dg)
+        assert dg.dg_gemm(A, B, C, prob.alpha, prob.beta, prob.scale_a, prob.scale_b) == dg.DG_OK
+        torch.cuda.synchronize()
+        dg.dg_set_option(dg.DG_OPT_TRACE, 0)
+        t = buf.cpu().tolist()
+        t0 = t[0]
+        out["trace_ns"] = {i: (v - t0) for i, v in enumerate(t) if v}
+    print(json.dumps(out), flush=True)
 
 
 def run_dg(args):
@@ -324,6 +340,8 @@ def run_dg(args):
         torch.cuda.set_device(0)
     import tcgen05_tmem_gemm_b200 as dg
 
+    if args.early_launch >= 0:
+        dg.dg_set_option(dg.DG_OPT_EARLY_LAUNCH, args.early_launch)
     dev = torch.device("cuda", torch.cuda.current_device())
     peaks = load_peaks()
     stream = torch.cuda.Stream()  # graphs are captured on a side stream; every call of the step uses it
@@ -559,6 +577,9 @@ def main():
                     help="time only this per-shape workload (small, gemv, gemv_kt, thin, square_bf16, "
                          "square_e4m3, strided) and print its line")
     ap.add_argument("--max-split", type=int, default=0, help="with --shape: cap the tensor-core split-K")
+    ap.add_argument("--trace", action="store_true", help="with --shape: phase timestamps of CTA 0")
+    ap.add_argument("--early-launch", type=int, default=-1,
+                    help="programmatic dependent launch policy (0 off, 1 at kernel start, 2 near the end)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -202,9 +202,16 @@ typedef enum {
                                      reports DG_ERR_TIMEOUT (tests of the bound)      */
     DG_OPT_MAX_SPLIT_K = 4,       /* upper bound on the tensor-core kernel's split-K
                                      (default and cluster limit 8; 1 disables)         */
-    DG_OPT_CTA_PAIR = 5           /* paired-CTA (256-row) tensor-core tiles: 0 never,
+    DG_OPT_CTA_PAIR = 5,          /* paired-CTA (256-row) tensor-core tiles: 0 never,
                                      1 for large problems (default), 2 whenever the
                                      operands allow                                    */
+    DG_OPT_EARLY_LAUNCH = 6,      /* programmatic dependent launch: 0 off, 1 release the
+                                     next kernel at the start of each kernel, 2 release
+                                     it near the end of long kernels; default 0: it did
+                                     not shorten back-to-back decode steps             */
+    DG_OPT_TRACE = 7              /* device address of 64 uint64 slots (0 = off): the
+                                     single-CTA tensor-core kernel's CTA 0 writes
+                                     %globaltimer at its phase boundaries (analysis)   */
 } dg_option;
 
 dg_status dg_set_option(int option, int64_t value);

@@ -28,7 +28,8 @@ ELEM_SIZE = {DG_F32: 4, DG_F16: 2, DG_BF16: 2, DG_E4M3: 1}
  DG_KIND_UMMA) = range(6)
 KIND_NAME = {0: "none", 1: "scale_c", 2: "simt", 3: "gemv_n", 4: "gemv_k", 5: "umma"}
 
-DG_OPT_FORCE_KIND, DG_OPT_WAIT_TIMEOUT_MS, DG_OPT_TEST_STALL, DG_OPT_MAX_SPLIT_K, DG_OPT_CTA_PAIR = 1, 2, 3, 4, 5
+(DG_OPT_FORCE_KIND, DG_OPT_WAIT_TIMEOUT_MS, DG_OPT_TEST_STALL, DG_OPT_MAX_SPLIT_K, DG_OPT_CTA_PAIR,
+ DG_OPT_EARLY_LAUNCH, DG_OPT_TRACE) = 1, 2, 3, 4, 5, 6, 7
 
 
 class dg_view(ctypes.Structure):

@@ -32,6 +32,8 @@ std::atomic<int64_t> g_timeout_ms{2000};
 std::atomic<int> g_stall{0};
 std::atomic<int> g_max_split{8};
 std::atomic<int> g_pair{1};
+std::atomic<int> g_pdl{0};
+std::atomic<uint64_t> g_trace{0};
 std::atomic<uint32_t> g_epoch{1};  // bumped by every option change: cached launches go stale
 
 constexpr int kMaxDevices = 64;
@@ -451,6 +453,7 @@ struct LaunchRec {
     DevView c{};
     int64_t M = 0, N = 0;
     float beta = 0.f;
+    int pdl = 0;
     SimtParams simt{};
     GemvParams gemv{};
     UmmaParams umma{};
@@ -464,6 +467,7 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
                   DeviceState *ds, LaunchRec *rec) {
     const dg_plan_info &in = pl.info;
     rec->kind = in.kind;
+    rec->pdl = g_pdl.load();
     switch (in.kind) {
     case DG_KIND_NONE: return DG_OK;
     case DG_KIND_SCALE_C: {
@@ -482,6 +486,7 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         p.N = (int32_t)in.N;
         p.K = (int32_t)in.K;
         p.epi = epi_params(v, false, alpha, beta, sa, sb);
+        p.pdl = rec->pdl;
         rec->simt = p;
         break;
     }
@@ -498,6 +503,7 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         p.epi = epi_params(v, false, alpha, beta, sa, sb);
         p.err_word = ds->err_word;
         p.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
+        p.pdl = rec->pdl;
         // x read with 16-byte loads when it is unit-stride along k
         const bool x_unit = v.a.col.n == 1 && v.a.col.stride[0] == 2 && v.A->dtype == v.B->dtype;
         p.x_ld = axis_stride(v.a.row);
@@ -568,6 +574,8 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         p.err_word = ds->err_word;
         p.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
         p.stall_loader = g_stall.load();
+        p.pdl = rec->pdl;
+        p.trace = reinterpret_cast<uint64_t *>(g_trace.load());
         rec->umma = p;
         rec->pair = in.cta_pair != 0;
         rec->fp8 = pl.fp8;
@@ -587,7 +595,7 @@ dg_status fire(const LaunchRec &r, cudaStream_t stream) {
     int grid = 0;
     switch (r.kind) {
     case DG_KIND_NONE: return DG_OK;
-    case DG_KIND_SCALE_C: err = launch_scale_c(r.c, r.M, r.N, r.beta, stream); break;
+    case DG_KIND_SCALE_C: err = launch_scale_c(r.c, r.M, r.N, r.beta, r.pdl, stream); break;
     case DG_KIND_SIMT: err = launch_simt(r.simt, stream); break;
     case DG_KIND_GEMV_N: err = launch_gemv_n(r.gemv, &r.t0, stream, &grid); break;
     case DG_KIND_GEMV_K: err = launch_gemv_k(r.gemv, stream, &grid); break;
@@ -764,6 +772,13 @@ dg_status dg_set_option(int option, int64_t value) {
         return DG_OK;
     case DG_OPT_TEST_STALL:
         g_stall.store(value ? 1 : 0);
+        return DG_OK;
+    case DG_OPT_TRACE:
+        g_trace.store((uint64_t)value);
+        return DG_OK;
+    case DG_OPT_EARLY_LAUNCH:
+        if (value < 0 || value > 2) return DG_ERR_VALUE;
+        g_pdl.store((int)value);
         return DG_OK;
     case DG_OPT_CTA_PAIR:
         if (value < 0 || value > 2) return DG_ERR_VALUE;

@@ -88,6 +88,8 @@ struct UmmaParams {
     int *err_word;
     uint64_t timeout_ns;
     int32_t stall_loader;
+    int32_t pdl;             // 0 off, 1 release dependents at start, 2 near the end
+    uint64_t *trace;         // optional phase timestamps of CTA 0 (%globaltimer, ns)
 };
 
 struct GemvParams {
@@ -102,6 +104,7 @@ struct GemvParams {
     int64_t x_ld;            // bytes between rows of x (x_vec16 only)
     int *err_word;
     uint64_t timeout_ns;
+    int32_t pdl;             // 0 off, 1 release dependents at start, 2 near the end
 };
 
 struct SimtParams {
@@ -109,6 +112,7 @@ struct SimtParams {
     DevView c;               // rows m, cols n
     int32_t M, N, K;
     EpiParams epi;           // i = m, j = n (c pointer unused; see c view)
+    int32_t pdl;
 };
 
 // ------------------------------------------------------------------ launchers
@@ -128,6 +132,6 @@ cudaError_t launch_gemv_n(const GemvParams &p, const CUtensorMap *tmap_w, cudaSt
 size_t gemv_n_smem_bytes(int r_inst, int kper);
 cudaError_t launch_gemv_k(const GemvParams &p, cudaStream_t s, int *grid_out);
 cudaError_t launch_simt(const SimtParams &p, cudaStream_t s);
-cudaError_t launch_scale_c(const DevView &c, int64_t M, int64_t N, float beta, cudaStream_t s);
+cudaError_t launch_scale_c(const DevView &c, int64_t M, int64_t N, float beta, int pdl, cudaStream_t s);
 
 }  // namespace dg

@@ -127,6 +127,7 @@ template <typename T, int R>
 __global__ void __launch_bounds__(kNT) gemv_n_kernel(const __grid_constant__ CUtensorMap tmap_w,
                                                      const GemvParams p) {
     pdl_wait();
+    if (p.pdl == 1) pdl_release();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const GemvNLayout L = gemv_n_layout(R, p.kper);
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(kNT) gemv_n_kernel(const __grid_constant__ CUt
                 const uint32_t ph = (uint32_t)(it / kStages) & 1u;
                 // a few stages before the end: let the next kernel be scheduled, so its
                 // launch latency overlaps this kernel's last loads and reduction
-                if (it == release_at) pdl_release();
+                if (it == release_at && p.pdl == 2) pdl_release();
                 if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) break;
                 mbar_arrive_expect_tx(bar_full + 8 * s, kRows * kNB * 2);
                 tma_load_2d(sbase + L.ring + s * (kRows * kNB * 2), &tmap_w, bar_full + 8 * s, n0, kb0 + it * kRows);
@@ -356,7 +357,7 @@ cudaError_t run_n(const GemvParams &p, const CUtensorMap *tmap, cudaStream_t s, 
     auto kern = gemv_n_kernel<T, R>;
     cudaError_t e = ensure_smem<KernelTag<T, R, 0>>(kern, smem);
     if (e != cudaSuccess) return e;
-    e = launch_ex(kern, dim3(gx, gy), dim3(kNT), smem, s, dim3(1, gy, 1), *tmap, p);
+    e = launch_ex(kern, dim3(gx, gy), dim3(kNT), smem, s, dim3(1, gy, 1), p.pdl, *tmap, p);
     *grid_out = gx * gy;
     return e;
 }
@@ -377,7 +378,7 @@ cudaError_t run_k(const GemvParams &p, cudaStream_t s, int *grid_out) {
     cudaError_t e = ensure_smem<KernelTag<T, R, 1>>(kern, smem);
     if (e != cudaSuccess) return e;
     *grid_out = grid;
-    return launch_ex(kern, dim3(grid), dim3(256), smem, s, dim3(1, 1, 1), p);
+    return launch_ex(kern, dim3(grid), dim3(256), smem, s, dim3(1, 1, 1), p.pdl, p);
 }
 
 template <typename T>

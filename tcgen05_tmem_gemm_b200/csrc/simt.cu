@@ -107,14 +107,14 @@ __global__ void scale_c_kernel(const DevView c, int64_t M, int64_t N, float beta
 cudaError_t launch_simt(const SimtParams &p, cudaStream_t s) {
     dim3 grid((p.N + TN - 1) / TN, (p.M + TM - 1) / TM);
     if (grid.y > 65535) return cudaErrorInvalidConfiguration;
-    return launch_ex(simt_gemm_kernel, grid, dim3(NT), 0, s, dim3(1, 1, 1), p);
+    return launch_ex(simt_gemm_kernel, grid, dim3(NT), 0, s, dim3(1, 1, 1), p.pdl, p);
 }
 
-cudaError_t launch_scale_c(const DevView &c, int64_t M, int64_t N, float beta, cudaStream_t s) {
+cudaError_t launch_scale_c(const DevView &c, int64_t M, int64_t N, float beta, int pdl, cudaStream_t s) {
     const int64_t total = M * N;
     int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 16);
     if (blocks < 1) blocks = 1;
-    return launch_ex(scale_c_kernel, dim3(blocks), dim3(256), 0, s, dim3(1, 1, 1), c, M, N, beta);
+    return launch_ex(scale_c_kernel, dim3(blocks), dim3(256), 0, s, dim3(1, 1, 1), pdl, c, M, N, beta);
 }
 
 }  // namespace dg

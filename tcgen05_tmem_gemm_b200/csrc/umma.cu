@@ -152,6 +152,15 @@ __device__ __forceinline__ void gather_stage(const UmmaParams &p, uint32_t p_sme
     }
 }
 
+// Phase timestamps of CTA 0 for performance analysis (DG_OPT_TRACE): slot 0
+// entry, 1 set-up done, 2+kb first-unit loads issued (k block kb < 16),
+// 18+kb MMAs of k block kb issued, 34 first accumulator complete (seen by the
+// epilogue), 35 first epilogue done, 36 teardown, 37..52 gather k block kb
+// written (first unit).
+__device__ __forceinline__ void trace_at(const UmmaParams &p, int slot) {
+    if (p.trace != nullptr && blockIdx.x == 0) p.trace[slot] = globaltimer_ns();
+}
+
 // OR of `pred` over the gather warps (named barrier 1), returned to all of them.
 __device__ __forceinline__ bool named_bar_or(bool pred) {
     uint32_t r;
@@ -170,7 +179,9 @@ template <bool FP8, bool GATHER>
 __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const UmmaParams p) {
+    if (threadIdx.x == 0) trace_at(p, 0);
     pdl_wait();
+    if (p.pdl == 1) pdl_release();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -214,6 +225,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    if (threadIdx.x == 0) trace_at(p, 1);
 
     const int es = FP8 ? 1 : 2;
     const int bk = p.bk;
@@ -255,6 +267,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                     } else {
                         tma_load_2d(qs, &tmap_q, full, k0, tc.tj * p.bn);
                     }
+                    if (it < 16) trace_at(p, 2 + it);
                 }
             }
             // let the copies already issued land before the CTA can exit
@@ -302,6 +315,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                         else umma_f16(d_tmem, da, db, idesc, acc);
                     }
                     tc_commit(bar_empty + 8 * s);  // stage is free once these MMAs have read it
+                    if (it < 16) trace_at(p, 18 + it);
                 }
                 if (!ok) break;
                 tc_commit(bar_tfull + 8 * b);      // accumulator b is complete
@@ -323,6 +337,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             const uint32_t tph = (uint32_t)(local >> 1) & 1u;
             if (!mbar_wait(bar_tfull + 8 * b, tph, wc)) break;
             tc_fence_after();
+            if (local == 0 && threadIdx.x == kEpiWarp0 * 32) trace_at(p, 34);
             const int i = tc.ti * kBM + row;
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * p.bn);
             const int j0 = tc.tj * p.bn;
@@ -359,6 +374,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_tempty + 8 * b);
+            if (local == 0 && threadIdx.x == kEpiWarp0 * 32) trace_at(p, 35);
         }
     } else if (GATHER) {
         // ------------------------------------------------ gather producers
@@ -399,6 +415,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                     fence_proxy_async_smem();  // make the stores visible to the tensor core
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_full + 8 * s);
+                    if (it < 16 && gtid == 0) trace_at(p, 37 + it);
                 }
                 // all offsets consumed before the next stage overwrites them
                 asm volatile("bar.sync 1, %0;" ::"n"(kGatherWarps * 32) : "memory");
@@ -466,6 +483,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     }
 
     // --------------------------------------------------------------- teardown
+    if (threadIdx.x == 0) trace_at(p, 36);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -502,7 +520,7 @@ cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtens
         if (e != cudaSuccess) return e;
         lim.store((int)smem);
     }
-    return launch_ex(kern, dim3(grid), dim3(gather ? 320 : 192), smem, s, dim3(p.split_k, 1, 1), *tp, *tq, p);
+    return launch_ex(kern, dim3(grid), dim3(gather ? 320 : 192), smem, s, dim3(p.split_k, 1, 1), p.pdl, *tp, *tq, p);
 }
 
 }  // namespace dg

@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(192, 1)
     umma_pair_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const UmmaParams p) {
     pdl_wait();
+    if (p.pdl == 1) pdl_release();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const PairLayout L = pair_layout(p.bn, p.stages);
@@ -245,7 +246,7 @@ cudaError_t launch_umma_pair(const UmmaParams &p, const CUtensorMap *tp, const C
         if (e != cudaSuccess) return e;
         lim.store((int)smem);
     }
-    return launch_ex(kern, dim3(grid), dim3(192), smem, s, dim3(2, 1, 1), *tp, *tq, p);
+    return launch_ex(kern, dim3(grid), dim3(192), smem, s, dim3(2, 1, 1), p.pdl, *tp, *tq, p);
 }
 
 }  // namespace dg

@@ -28,6 +28,7 @@ def _reset_options():
     dg.dg_set_option(dg.DG_OPT_WAIT_TIMEOUT_MS, 2000)
     dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, 8)
     dg.dg_set_option(dg.DG_OPT_CTA_PAIR, 1)
+    dg.dg_set_option(dg.DG_OPT_EARLY_LAUNCH, 0)
 
 
 def expect_kind(p, kind, **fields):
@@ -101,8 +102,10 @@ def test_fp8_k_major_b():
     (256, 128, 16, "f16", "f16", False, False),
 ])
 def test_umma_cta_pair_forced(M, N, K, dt, out, ta, tb):
-    # two CTAs of a cluster share each 256-row tile (tcgen05 cta_group::2)
+    # two CTAs of a cluster share each 256-row tile (tcgen05 cta_group::2); pairs
+    # take no split-K, so split-K is switched off for these shapes
     dg.dg_set_option(dg.DG_OPT_CTA_PAIR, 2)
+    dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, 1)
     g = torch.Generator().manual_seed(M + 3 * N + K)
     a = W.cast(W.normal((K, M) if ta else (M, K), g), dt)
     b = W.cast(W.normal((N, K) if tb else (K, N), g), dt)
@@ -116,6 +119,7 @@ def test_umma_cta_pair_forced(M, N, K, dt, out, ta, tb):
 
 def test_umma_cta_pair_fp8():
     dg.dg_set_option(dg.DG_OPT_CTA_PAIR, 2)
+    dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, 1)
     M, N, K = 384, 256, 384
     g = torch.Generator().manual_seed(77)
     qa, sa = W.quantise_e4m3(W.normal((M, K), g), dim=1)
