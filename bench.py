@@ -160,7 +160,7 @@ def kernel_traffic(kernel_file: str, summary_file: str):
     for line in open(path):
         if ":" in line and line.strip().startswith(("dram_bytes_per_launch", "kernel_source_sha")):
             k, v = line.split(":", 1)
-            rec[k.strip()] = v.strip()
+            rec[k.strip()] = v.split()[0] if v.split() else ""
     if rec.get("kernel_source_sha") != sha:
         return None
     try:

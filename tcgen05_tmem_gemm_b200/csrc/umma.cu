@@ -48,6 +48,7 @@ struct SmemLayout {
     uint32_t stage_bytes, p_bytes, q_bytes;
     uint32_t bar_off;                // after the stages
     uint32_t aux_off;                // tmem address, abort flag, gather tables
+    uint32_t epi_off;                // per-epilogue-warp staging blocks
     uint32_t total;
 };
 
@@ -61,7 +62,8 @@ __host__ __device__ inline SmemLayout smem_layout(int bn, int stages, bool gathe
     L.aux_off = L.bar_off + 8 * (2 * stages + 5);
     uint32_t aux = 16;  // tmem base + abort flag
     if (gather) aux += 8 * kBM + 8 * 128;  // row offsets of the tile, k offsets of a stage
-    L.total = L.aux_off + aux + 1024;      // + slack to align the base to 1024
+    L.epi_off = L.aux_off + aux;
+    L.total = L.epi_off + 4 * kEpiStageBytes + 1024;  // + slack to align the base to 1024
     return L;
 }
 
@@ -156,7 +158,8 @@ __device__ __forceinline__ void gather_stage(const UmmaParams &p, uint32_t p_sme
 // entry, 1 set-up done, 2+kb first-unit loads issued (k block kb < 16),
 // 18+kb MMAs of k block kb issued, 34 first accumulator complete (seen by the
 // epilogue), 35 first epilogue done, 36 teardown, 37..52 gather k block kb
-// written (first unit).
+// written (first unit); split-K: 53 partial parked, 54 first cluster barrier
+// passed, 55 reduction done, 56 second cluster barrier passed.
 __device__ __forceinline__ void trace_at(const UmmaParams &p, int slot) {
     if (p.trace != nullptr && blockIdx.x == 0) p.trace[slot] = globaltimer_ns();
 }
@@ -357,19 +360,26 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                     for (int c = 0; c < 16; ++c) part[(c0 + c) * kPartPitch + row] = __uint_as_float(r[c]);
                 }
                 tc_fence_before();
+                if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 53);
                 continue;
             }
 
-            const bool row_ok = i < p.Mi;
-            const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
-            char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
-            for (int c0 = 0; c0 < p.bn; c0 += 16) {
-                uint32_t r[16];
-                __syncwarp();
-                tmem_ld16(t_row + c0, r);
-                tmem_ld_wait();
-                if (!row_ok) continue;
-                epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
+            if (e.vec_ok && p.bn % 32 == 0) {
+                // C contiguous along j: rows staged through shared memory, coalesced stores
+                float *stage = reinterpret_cast<float *>(smem + L.epi_off) + (warp - kEpiWarp0) * 32 * kStagePitch;
+                epilogue_rows_staged(e, stage, t_row, tc.ti * kBM + quarter * 32, p.Mi, j0, p.bn, p.Nj);
+            } else {
+                const bool row_ok = i < p.Mi;
+                const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
+                char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
+                for (int c0 = 0; c0 < p.bn; c0 += 16) {
+                    uint32_t r[16];
+                    __syncwarp();
+                    tmem_ld16(t_row + c0, r);
+                    tmem_ld_wait();
+                    if (!row_ok) continue;
+                    epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -432,6 +442,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
         tc_fence_before();
         __syncthreads();
         cluster_sync();
+        if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 54);
         if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
             const EpiParams &e = p.epi;
             const TileCoord tc = unit_coord(blockIdx.x, p);
@@ -479,7 +490,9 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                 }
             }
         }
+        if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 55);
         cluster_sync();  // partials stay alive until every CTA of the cluster has read them
+        if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 56);
     }
 
     // --------------------------------------------------------------- teardown
