@@ -292,6 +292,16 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, int num_sms, Pla
         if (halves_ok) pair = (pair_mode == 2) || (Mi >= 256 && tiles >= num_sms);
     }
     const int stages = pair ? umma_pair_max_stages(bn) : umma_max_stages(bn, !p_tma);
+    if (split > 1) {
+        // the owner CTA receives every split's rows in its operand ring
+        const int64_t recv = split * bn * ((128 + split - 1) / split) * 4;
+        const int64_t ring = (int64_t)stages * (128 * 128 + bn * 128);
+        if (recv > ring) {
+            split = 1;
+            kb_per = kb_total;
+        }
+    }
+    const int64_t units2 = tiles * split;
     dg_plan_info &in = pl->info;
     in.kind = DG_KIND_UMMA;
     in.swap_ab = swap;
@@ -303,7 +313,7 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, int num_sms, Pla
     in.block_k = bk;
     in.stages = stages;
     in.split_k = (int32_t)split;
-    in.grid = (int32_t)(split > 1 ? units : std::min<int64_t>(units, num_sms));  // split: one unit per CTA
+    in.grid = (int32_t)(split > 1 ? units2 : std::min<int64_t>(units2, num_sms));  // split: one unit per CTA
     in.vec_bytes = p_tma ? 16 : gather_vec * es;
     in.cta_pair = pair;
     if (pair) {

@@ -32,6 +32,8 @@ struct DevView {
 };
 
 __host__ __device__ inline int64_t axis_offset(const Axis &a, int64_t idx) {
+    if (a.n == 1) return idx * a.stride[0];  // one merged dim: no division
+    if (a.n == 0) return 0;
     int64_t off = 0;
     for (int d = a.n - 1; d >= 0; --d) {
         const int64_t s = a.size[d];

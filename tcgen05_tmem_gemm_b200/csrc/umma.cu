@@ -42,13 +42,11 @@ namespace {
 constexpr int kBM = 128;             // tensor-core tile rows (TMEM lanes)
 constexpr int kTileBytesK = 128;     // one swizzle row: 64 x 16-bit or 128 x 8-bit
 constexpr int kGatherWarps = 4;
-constexpr int kPartPitch = kBM + 1;   // floats per column of a parked split-K partial
 
 struct SmemLayout {
     uint32_t stage_bytes, p_bytes, q_bytes;
     uint32_t bar_off;                // after the stages
     uint32_t aux_off;                // tmem address, abort flag, gather tables
-    uint32_t epi_off;                // per-epilogue-warp staging blocks
     uint32_t total;
 };
 
@@ -61,9 +59,8 @@ __host__ __device__ inline SmemLayout smem_layout(int bn, int stages, bool gathe
     // full[S], empty[S], tfull[2], tempty[2], drain
     L.aux_off = L.bar_off + 8 * (2 * stages + 5);
     uint32_t aux = 16;  // tmem base + abort flag
-    if (gather) aux += 8 * kBM + 8 * 128;  // row offsets of the tile, k offsets of a stage
-    L.epi_off = L.aux_off + aux;
-    L.total = L.epi_off + 4 * kEpiStageBytes + 1024;  // + slack to align the base to 1024
+    if (gather) aux += 8 * kBM;  // row offsets of the tile
+    L.total = L.aux_off + aux + 1024;  // + slack to align the base to 1024
     return L;
 }
 
@@ -98,7 +95,7 @@ template <> struct VecOf<2> { using T = unsigned short; };
 template <> struct VecOf<1> { using T = unsigned char; };
 
 template <int BYTES>
-__device__ __forceinline__ typename VecOf<BYTES>::T gather_load(const char *src, bool valid) {
+__device__ __forceinline__ typename VecOf<BYTES>::T gather_load_one(const char *src, bool valid) {
     using V = typename VecOf<BYTES>::T;
     if (!valid) return V{};
     return __ldg(reinterpret_cast<const V *>(src));
@@ -119,47 +116,12 @@ __device__ __forceinline__ void st_shared_vec(uint32_t dst, const typename VecOf
     }
 }
 
-// Fill one stage's P tile (kBM rows of i, bk of k) by thread loads, kUnroll
-// loads in flight per thread before their shared-memory stores.
-template <int VB>
-__device__ __forceinline__ void gather_stage(const UmmaParams &p, uint32_t p_smem, const int64_t *row_off,
-                                             const int64_t *col_off, int bk, int es, int gtid) {
-    using V = typename VecOf<VB>::T;
-    constexpr int kUnroll = 16;
-    const int vec = VB / es;                       // elements per copy
-    const int nthreads = kGatherWarps * 32;
-    const bool mn = p.p_mn_major != 0;
-    const int runs = mn ? kBM / vec : bk / vec;    // runs along the unit-stride dim
-    const int total = mn ? runs * bk : kBM * runs;
-    const int chunk_bytes = bk * 128;
-    for (int base = gtid; base < total; base += nthreads * kUnroll) {
-        V v[kUnroll];
-        uint32_t dst[kUnroll];
-#pragma unroll
-        for (int r = 0; r < kUnroll; ++r) {
-            const int u = base + r * nthreads;
-            int i, k;
-            if (mn) { k = u / runs; i = (u - k * runs) * vec; }
-            else { i = u / runs; k = (u - i * runs) * vec; }
-            const bool in_tile = u < total;
-            const int64_t ro = in_tile ? row_off[i] : -1, co = in_tile ? col_off[k] : -1;
-            const bool ok = ro >= 0 && co >= 0;
-            v[r] = gather_load<VB>(p.pv.ptr + (ok ? ro + co : 0), ok);
-            dst[r] = in_tile ? p_smem + (mn ? sw128_mnmajor(i * es, k, chunk_bytes) : sw128_kmajor(i, k * es))
-                             : 0xffffffffu;
-        }
-#pragma unroll
-        for (int r = 0; r < kUnroll; ++r)
-            if (dst[r] != 0xffffffffu) st_shared_vec<VB>(dst[r], v[r]);
-    }
-}
-
 // Phase timestamps of CTA 0 for performance analysis (DG_OPT_TRACE): slot 0
 // entry, 1 set-up done, 2+kb first-unit loads issued (k block kb < 16),
 // 18+kb MMAs of k block kb issued, 34 first accumulator complete (seen by the
 // epilogue), 35 first epilogue done, 36 teardown, 37..52 gather k block kb
-// written (first unit); split-K: 53 partial parked, 54 first cluster barrier
-// passed, 55 reduction done, 56 second cluster barrier passed.
+// written (first unit); split-K: 53 accumulator complete, 54 first cluster
+// barrier passed, 55 partials pushed and second barrier passed, 56 reduced.
 __device__ __forceinline__ void trace_at(const UmmaParams &p, int slot) {
     if (p.trace != nullptr && blockIdx.x == 0) p.trace[slot] = globaltimer_ns();
 }
@@ -176,6 +138,189 @@ __device__ __forceinline__ bool named_bar_or(bool pred) {
         : "r"((uint32_t)pred), "n"(kGatherWarps * 32)
         : "memory");
     return r != 0;
+}
+
+// Thread loads of one stage of the P tile (kBM rows of i, bk of k), split in
+// two halves so that a stage's loads can be in flight while the previous
+// stage is stored: gather_load fills registers (at most kGatherUnroll copies
+// per thread), gather_store writes them in the 128-byte-swizzled layout.
+// Copy u of a stage covers `vec` consecutive elements along the unit-stride
+// dimension; consecutive threads take consecutive copies.
+constexpr int kGatherUnroll = 16;
+
+struct GatherGeom {
+    bool mn;
+    int vec, runs, total, chunk_bytes, es;
+};
+
+__device__ __forceinline__ GatherGeom gather_geom(const UmmaParams &p, int VB, int bk, int es) {
+    GatherGeom g;
+    g.mn = p.p_mn_major != 0;
+    g.vec = VB / es;
+    g.runs = g.mn ? kBM / g.vec : bk / g.vec;
+    g.total = g.mn ? g.runs * bk : kBM * g.runs;
+    g.chunk_bytes = bk * 128;
+    g.es = es;
+    return g;
+}
+
+// Copies first, first + 128, first + 256, ... of a stage: along the unit-
+// stride dim their position is fixed and the other index advances by
+// 128 / runs per copy (runs is a power of two dividing 128), so no index is
+// divided inside the loops.
+template <int VB>
+__device__ __forceinline__ void gather_load(const UmmaParams &p, const GatherGeom &g, const int64_t *row_off,
+                                            int kbase, int first, typename VecOf<VB>::T (&v)[kGatherUnroll]) {
+    const int nthreads = kGatherWarps * 32;
+    const int step = nthreads / g.runs;
+    if (g.mn) {
+        // fixed i (a run of vec rows), k advancing by `step`
+        const int i = (first % g.runs) * g.vec;
+        const int64_t ro = row_off[i];
+        const int k0 = first / g.runs;
+#pragma unroll
+        for (int r = 0; r < kGatherUnroll; ++r) {
+            const int u = first + r * nthreads;
+            const int kg = kbase + k0 + r * step;
+            const bool ok = u < g.total && ro >= 0 && kg < p.K;
+            v[r] = gather_load_one<VB>(p.pv.ptr + (ok ? ro + axis_offset(p.pv.col, kg) : 0), ok);
+        }
+    } else {
+        // fixed k (a run of vec columns), i advancing by `step`
+        const int kg = kbase + (first % g.runs) * g.vec;
+        const int64_t co = kg < p.K ? axis_offset(p.pv.col, kg) : -1;
+        const int i0 = first / g.runs;
+#pragma unroll
+        for (int r = 0; r < kGatherUnroll; ++r) {
+            const int u = first + r * nthreads;
+            const int i = i0 + r * step;
+            const int64_t ro = (u < g.total) ? row_off[i] : -1;
+            const bool ok = ro >= 0 && co >= 0;
+            v[r] = gather_load_one<VB>(p.pv.ptr + (ok ? ro + co : 0), ok);
+        }
+    }
+}
+
+template <int VB>
+__device__ __forceinline__ void gather_store(const GatherGeom &g, uint32_t p_smem, int first,
+                                             const typename VecOf<VB>::T (&v)[kGatherUnroll]) {
+    const int nthreads = kGatherWarps * 32;
+    const int step = nthreads / g.runs;
+    const int fixed = (first % g.runs) * g.vec, moving0 = first / g.runs;
+#pragma unroll
+    for (int r = 0; r < kGatherUnroll; ++r) {
+        const int u = first + r * nthreads;
+        if (u >= g.total) continue;
+        const int moving = moving0 + r * step;
+        st_shared_vec<VB>(p_smem + (g.mn ? sw128_mnmajor(fixed * g.es, moving, g.chunk_bytes)
+                                         : sw128_kmajor(moving, fixed * g.es)),
+                          v[r]);
+    }
+}
+
+// cp.async version of a batch: the same copies as gather_load/gather_store,
+// issued as asynchronous global -> shared copies (no register staging).
+template <int VB>
+__device__ __forceinline__ void gather_issue_async(const UmmaParams &p, const GatherGeom &g, const int64_t *row_off,
+                                                   int kbase, int first, uint32_t p_smem) {
+    const int nthreads = kGatherWarps * 32;
+    const int step = nthreads / g.runs;
+    const int fixed = (first % g.runs) * g.vec, moving0 = first / g.runs;
+    if (g.mn) {
+        const int64_t ro = row_off[fixed];
+#pragma unroll
+        for (int r = 0; r < kGatherUnroll; ++r) {
+            const int u = first + r * nthreads;
+            if (u >= g.total) break;
+            const int k = moving0 + r * step, kg = kbase + k;
+            const bool ok = ro >= 0 && kg < p.K;
+            cp_async_zfill<VB>(p_smem + sw128_mnmajor(fixed * g.es, k, g.chunk_bytes),
+                               p.pv.ptr + (ok ? ro + axis_offset(p.pv.col, kg) : 0), ok);
+        }
+    } else {
+        const int kg = kbase + fixed;
+        const int64_t co = kg < p.K ? axis_offset(p.pv.col, kg) : -1;
+#pragma unroll
+        for (int r = 0; r < kGatherUnroll; ++r) {
+            const int u = first + r * nthreads;
+            if (u >= g.total) break;
+            const int i = moving0 + r * step;
+            const int64_t ro = row_off[i];
+            const bool ok = ro >= 0 && co >= 0;
+            cp_async_zfill<VB>(p_smem + sw128_kmajor(i, fixed * g.es), p.pv.ptr + (ok ? ro + co : 0), ok);
+        }
+    }
+}
+
+// The gather role for one vector width.  Per tile: row offsets once.  When
+// a stage is at most one batch per thread (kGatherUnroll copies), the next
+// k block's loads are issued before this block is stored, so two stages of
+// loads are in flight; wider stages are loaded and stored batch by batch.
+// Every exit decision is voted on across the gather warps (bar.red), so no
+// warp is left waiting at their named barrier.
+template <int VB>
+__device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayout &L, uint32_t sbase,
+                                            uint32_t bar_full, uint32_t bar_empty, int64_t *g_row_off,
+                                            volatile int *abort_flag, const WaitCtl &wc, int bk, int es, int gtid,
+                                            int lane) {
+    using V = typename VecOf<VB>::T;
+    const GatherGeom g = gather_geom(p, VB, bk, es);
+    const int nthreads = kGatherWarps * 32;
+    const bool one_batch = VB < 4 && g.total <= nthreads * kGatherUnroll;  // register path look-ahead
+    int it = 0;
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+        if (named_bar_or(*abort_flag != 0)) break;
+        const TileCoord tc = unit_coord(u, p);
+        const int kb0 = tc.split * p.kb_per_split;
+        const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+        for (int r = gtid; r < kBM; r += nthreads) {
+            const int i = tc.ti * kBM + r;
+            g_row_off[r] = i < p.Mi ? axis_offset(p.pv.row, i) : -1;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kGatherWarps * 32) : "memory");
+        bool ok = true;
+        V cur[kGatherUnroll], nxt[kGatherUnroll];
+        if (one_batch && kb0 < kb1) gather_load<VB>(p, g, g_row_off, kb0 * bk, gtid, cur);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            const int s = it % p.stages;
+            const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
+            if (one_batch && kb + 1 < kb1) gather_load<VB>(p, g, g_row_off, (kb + 1) * bk, gtid, nxt);
+            ok = mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc);
+            if (named_bar_or(!ok)) { ok = false; break; }
+            if (!p.stall_loader && VB >= 4) {
+                // asynchronous copies: the stage completes on the full barrier
+                // when they land, and this warp moves on at once
+                const uint32_t ps = sbase + s * L.stage_bytes;
+                for (int f = gtid; f < g.total; f += nthreads * kGatherUnroll)
+                    gather_issue_async<(VB >= 4 ? VB : 4)>(p, g, g_row_off, kb * bk, f, ps);
+                cp_async_arrive_noinc(bar_full + 8 * s);
+                if (it < 16 && gtid == 0) trace_at(p, 37 + it);
+            } else if (!p.stall_loader) {
+                const uint32_t ps = sbase + s * L.stage_bytes;
+                if (one_batch) {
+                    gather_store<VB>(g, ps, gtid, cur);
+                } else {
+                    for (int f = gtid; f < g.total; f += nthreads * kGatherUnroll) {
+                        gather_load<VB>(p, g, g_row_off, kb * bk, f, cur);
+                        gather_store<VB>(g, ps, f, cur);
+                    }
+                }
+                fence_proxy_async_smem();  // make the stores visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_full + 8 * s);
+                if (it < 16 && gtid == 0) trace_at(p, 37 + it);
+            }
+            if (one_batch) {
+#pragma unroll
+                for (int r = 0; r < kGatherUnroll; ++r) cur[r] = nxt[r];
+            }
+        }
+        // row offsets of this tile stay in use until every gather warp is past it
+        asm volatile("bar.sync 1, %0;" ::"n"(kGatherWarps * 32) : "memory");
+        if (!ok) break;
+    }
+    // nothing this thread copied may land after the CTA has gone
+    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 template <bool FP8, bool GATHER>
@@ -198,7 +343,6 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.aux_off);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.aux_off + 4);
     int64_t *g_row_off = reinterpret_cast<int64_t *>(smem + L.aux_off + 16);
-    int64_t *g_col_off = g_row_off + kBM;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int kEpiWarp0 = 2;
@@ -206,7 +350,9 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
-            mbar_init(bar_full + 8 * s, GATHER ? 1 + kGatherWarps : 1);
+            // gather stages: one arrival per gather thread when its cp.async
+            // copies land (4..16-byte copies), else one per gather warp
+            mbar_init(bar_full + 8 * s, GATHER ? 1 + (p.gather_vec * (FP8 ? 1 : 2) >= 4 ? kGatherWarps * 32 : kGatherWarps) : 1);
             mbar_init(bar_empty + 8 * s, 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -307,6 +453,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                     const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
                     if (!mbar_wait(bar_full + 8 * s, ph, wc)) { ok = false; break; }
                     tc_fence_after();
+                    if (GATHER) fence_proxy_async_smem();  // thread-written P stage -> tensor-core reads
                     const uint32_t ps = sbase + s * L.stage_bytes;
                     const uint32_t qs = ps + L.p_bytes;
 #pragma unroll
@@ -346,40 +493,23 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             const int j0 = tc.tj * p.bn;
 
             if (p.split_k > 1) {
-                // one unit per CTA: park the partial tile in this CTA's shared
-                // memory (the operand ring is idle once the accumulator is
-                // complete), [column][row] with a 129-float pitch; the cluster
-                // reduces it after the role loops.
-                float *part = reinterpret_cast<float *>(smem);
-                for (int c0 = 0; c0 < p.bn; c0 += 16) {
-                    uint32_t r[16];
-                    __syncwarp();
-                    tmem_ld16(t_row + c0, r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) part[(c0 + c) * kPartPitch + row] = __uint_as_float(r[c]);
-                }
+                // one unit per CTA: the partial stays in TMEM until the cluster
+                // has finished its main loops (see the reduction below)
                 tc_fence_before();
                 if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 53);
                 continue;
             }
 
-            if (e.vec_ok && p.bn % 32 == 0) {
-                // C contiguous along j: rows staged through shared memory, coalesced stores
-                float *stage = reinterpret_cast<float *>(smem + L.epi_off) + (warp - kEpiWarp0) * 32 * kStagePitch;
-                epilogue_rows_staged(e, stage, t_row, tc.ti * kBM + quarter * 32, p.Mi, j0, p.bn, p.Nj);
-            } else {
-                const bool row_ok = i < p.Mi;
-                const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
-                char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
-                for (int c0 = 0; c0 < p.bn; c0 += 16) {
-                    uint32_t r[16];
-                    __syncwarp();
-                    tmem_ld16(t_row + c0, r);
-                    tmem_ld_wait();
-                    if (!row_ok) continue;
-                    epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
-                }
+            const bool row_ok = i < p.Mi;
+            const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
+            char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
+            for (int c0 = 0; c0 < p.bn; c0 += 16) {
+                uint32_t r[16];
+                __syncwarp();
+                tmem_ld16(t_row + c0, r);
+                tmem_ld_wait();
+                if (!row_ok) continue;
+                epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
             }
             tc_fence_before();
             __syncwarp();
@@ -388,111 +518,108 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
         }
     } else if (GATHER) {
         // ------------------------------------------------ gather producers
-        // Every exit decision is voted on across the four gather warps
-        // (bar.red), so no warp can be left waiting at their named barrier.
         const int gtid = threadIdx.x - (kEpiWarp0 + 4) * 32;
-        int it = 0;
-        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-            if (named_bar_or(*abort_flag != 0)) break;
-            const TileCoord tc = unit_coord(u, p);
-            const int kb0 = tc.split * p.kb_per_split;
-            const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
-            // row offsets of this tile (-1 past the end); the first barrier of
-            // the k loop orders them before any use
-            for (int r = gtid; r < kBM; r += kGatherWarps * 32) {
-                const int i = tc.ti * kBM + r;
-                g_row_off[r] = i < p.Mi ? axis_offset(p.pv.row, i) : -1;
-            }
-            bool ok = true;
-            for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                const int s = it % p.stages;
-                const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
-                for (int k = gtid; k < bk; k += kGatherWarps * 32) {
-                    const int kg = kb * bk + k;
-                    g_col_off[k] = kg < p.K ? axis_offset(p.pv.col, kg) : -1;
-                }
-                ok = mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc);
-                if (named_bar_or(!ok)) { ok = false; break; }  // also orders the offsets before use
-                if (!p.stall_loader) {
-                    const uint32_t ps = sbase + s * L.stage_bytes;
-                    switch (p.gather_vec * es) {
-                    case 16: gather_stage<16>(p, ps, g_row_off, g_col_off, bk, es, gtid); break;
-                    case 8: gather_stage<8>(p, ps, g_row_off, g_col_off, bk, es, gtid); break;
-                    case 4: gather_stage<4>(p, ps, g_row_off, g_col_off, bk, es, gtid); break;
-                    case 2: gather_stage<2>(p, ps, g_row_off, g_col_off, bk, es, gtid); break;
-                    default: gather_stage<1>(p, ps, g_row_off, g_col_off, bk, es, gtid); break;
-                    }
-                    fence_proxy_async_smem();  // make the stores visible to the tensor core
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_full + 8 * s);
-                    if (it < 16 && gtid == 0) trace_at(p, 37 + it);
-                }
-                // all offsets consumed before the next stage overwrites them
-                asm volatile("bar.sync 1, %0;" ::"n"(kGatherWarps * 32) : "memory");
-            }
-            if (!ok) break;
+        switch (p.gather_vec * es) {
+        case 16: gather_role<16>(p, L, sbase, bar_full, bar_empty, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
+        case 8: gather_role<8>(p, L, sbase, bar_full, bar_empty, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
+        case 4: gather_role<4>(p, L, sbase, bar_full, bar_empty, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
+        case 2: gather_role<2>(p, L, sbase, bar_full, bar_empty, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
+        default: gather_role<1>(p, L, sbase, bar_full, bar_empty, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
         }
     }
 
     if (p.split_k > 1) {
         // ------------------------------------------ cluster reduction of k splits
-        // CTA s of the cluster owns rows [128 s / S, 128 (s+1) / S) of the tile
-        // and adds that slice of every split's partial, in rank order, through
-        // distributed shared memory.
+        // CTA s of the cluster owns rows [128 s / S, 128 (s+1) / S) of the tile.
+        // After every CTA's main loop (barrier 1: all operand rings are idle),
+        // each CTA pushes every row of its partial from TMEM into the owner's
+        // ring with remote shared-memory stores (which do not wait), as
+        // recv[source][column][row - first owned row]; after barrier 2 each
+        // owner adds its S slices in rank order from its own shared memory
+        // and runs the epilogue.
+        const int S = p.split_k;
+        const int rs_max = (kBM + S - 1) / S;
+        const uint32_t rank = cluster_ctarank();
         tc_fence_before();
         __syncthreads();
         cluster_sync();
         if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 54);
         if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+            tc_fence_after();
+            const int quarter = warp & 3;
+            const int row = quarter * 32 + lane;
+            int d = 0;
+            while (d + 1 < S && (d + 1) * kBM / S <= row) ++d;
+            const int rl = row - d * kBM / S;
+            const uint32_t dst = dsmem_map(sbase, (uint32_t)d);
+            const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16);
+            for (int c0 = 0; c0 < p.bn; c0 += 16) {
+                uint32_t r[16];
+                __syncwarp();
+                tmem_ld16(t_row + c0, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    dsmem_st_f32(dst + (uint32_t)((((int)rank * p.bn + c0 + c) * rs_max + rl) * 4), __uint_as_float(r[c]));
+            }
+        }
+        __syncthreads();
+        cluster_sync();
+        if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 55);
+        if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
             const EpiParams &e = p.epi;
             const TileCoord tc = unit_coord(blockIdx.x, p);
-            const int S = p.split_k;
-            const uint32_t rank = cluster_ctarank();
             const int r0 = (int)(rank * kBM / S), r1 = (int)((rank + 1) * kBM / S), rs = r1 - r0;
             const int t = threadIdx.x - kEpiWarp0 * 32;
             const bool along_i = (e.ci == (int64_t)elem_bytes(e.c_dtype));  // C contiguous along i
-            const uint32_t part_addr = sbase;
-            constexpr int kB = 8;  // outputs per thread per batch, all their loads in flight together
-            for (int base = t; base < rs * p.bn; base += 128 * kB) {
+            const float *recv = reinterpret_cast<const float *>(smem);
+            // element e of the owned rs x bn slice: r = e % rs, c = e / rs when C
+            // is contiguous along i (consecutive threads, consecutive addresses),
+            // else c = e % bn, r = e / bn; indices advance without division
+            const int total = rs * p.bn;
+            int r = along_i ? t % rs : t / p.bn, c = along_i ? t / rs : t % p.bn;
+            const int dr = along_i ? 128 % rs : 128 / p.bn, dc = along_i ? 128 / rs : 128 % p.bn;
+            constexpr int kB = 8;  // outputs per thread per batch: their C loads are in flight together
+            for (int base = t; base < total; base += 128 * kB) {
                 int ii[kB], jj[kB];
-                float v[kB][8], cin[kB];
+                float acc[kB], cin[kB];
 #pragma unroll
                 for (int b = 0; b < kB; ++b) {
-                    const int el = base + b * 128;
-                    int r = 0, c = 0;
-                    if (along_i) { r = el % rs; c = el / rs; }
-                    else { c = el % p.bn; r = el / p.bn; }
                     const int i = tc.ti * kBM + r0 + r, j = tc.tj * p.bn + c;
-                    const bool ok = el < rs * p.bn && i < p.Mi && j < p.Nj;
+                    const bool ok = base + b * 128 < total && i < p.Mi && j < p.Nj;
                     ii[b] = ok ? i : -1;
                     jj[b] = j;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        v[b][q] = (ok && q < S)
-                                      ? dsmem_ld_f32(dsmem_map(part_addr + (uint32_t)((c * kPartPitch + r0 + r) * 4), q))
-                                      : 0.f;
+                    float a = 0.f;
+                    if (ok)
+                        for (int q = 0; q < S; ++q) a += recv[(q * p.bn + c) * rs_max + r];
+                    acc[b] = a;
                     cin[b] = (ok && e.beta != 0.f) ? load_elem(e.c + (int64_t)i * e.ci + (int64_t)j * e.cj, e.c_dtype)
                                                    : 0.f;
+                    // advance by 128 elements
+                    if (along_i) {
+                        r += dr;
+                        c += dc;
+                        if (r >= rs) { r -= rs; ++c; }
+                    } else {
+                        c += dc;
+                        r += dr;
+                        if (c >= p.bn) { c -= p.bn; ++r; }
+                    }
                 }
 #pragma unroll
                 for (int b = 0; b < kB; ++b) {
                     if (ii[b] < 0) continue;
                     const int i = ii[b], j = jj[b];
-                    float acc = 0.f;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        if (q < S) acc += v[b][q];
                     const float asi = e.alpha * (e.scale_i ? e.scale_i[i] : 1.f);
                     const float sj = e.scale_j ? e.scale_j[j] : 1.f;
-                    float val = (asi * sj) * acc;
+                    float val = (asi * sj) * acc[b];
                     if (e.beta != 0.f) val = fmaf(e.beta, cin[b], val);
                     store_elem(e.c + (int64_t)i * e.ci + (int64_t)j * e.cj, e.c_dtype, val);
                 }
             }
         }
-        if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 55);
-        cluster_sync();  // partials stay alive until every CTA of the cluster has read them
         if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 56);
+        // no CTA touches another's shared memory after the second barrier
     }
 
     // --------------------------------------------------------------- teardown

@@ -31,7 +31,7 @@ constexpr int kHalfM = 128;   // rows of P (and TMEM lanes) per CTA
 constexpr int kRowBytes = 128;
 
 struct PairLayout {
-    uint32_t a_bytes, b_bytes, stage_bytes, bar_off, aux_off, epi_off, total;
+    uint32_t a_bytes, b_bytes, stage_bytes, bar_off, aux_off, total;
 };
 
 __host__ __device__ inline PairLayout pair_layout(int bn, int stages) {
@@ -42,8 +42,7 @@ __host__ __device__ inline PairLayout pair_layout(int bn, int stages) {
     L.bar_off = L.stage_bytes * stages;
     // full[S], empty[S], tfull[2], tempty[2], drain
     L.aux_off = L.bar_off + 8 * (2 * stages + 5);
-    L.epi_off = L.aux_off + 16;
-    L.total = L.epi_off + 4 * kEpiStageBytes + 1024;
+    L.total = L.aux_off + 16 + 1024;
     return L;
 }
 
@@ -198,21 +197,16 @@ __global__ void __launch_bounds__(192, 1)
             const int i = ti * 2 * kHalfM + (int)rank * kHalfM + row;
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * p.bn);
             const int j0 = tj * p.bn;
-            if (e.vec_ok && p.bn % 32 == 0) {
-                float *stage = reinterpret_cast<float *>(smem + L.epi_off) + (warp - 2) * 32 * kStagePitch;
-                epilogue_rows_staged(e, stage, t_row, i - row + quarter * 32, p.Mi, j0, p.bn, p.Nj);
-            } else {
-                const bool row_ok = i < p.Mi;
-                const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
-                char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
-                for (int c0 = 0; c0 < p.bn; c0 += 16) {
-                    uint32_t r[16];
-                    __syncwarp();
-                    tmem_ld16(t_row + c0, r);
-                    tmem_ld_wait();
-                    if (!row_ok) continue;
-                    epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
-                }
+            const bool row_ok = i < p.Mi;
+            const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
+            char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
+            for (int c0 = 0; c0 < p.bn; c0 += 16) {
+                uint32_t r[16];
+                __syncwarp();
+                tmem_ld16(t_row + c0, r);
+                tmem_ld_wait();
+                if (!row_ok) continue;
+                epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
             }
             tc_fence_before();
             __syncwarp();
