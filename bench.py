@@ -357,20 +357,18 @@ def run_dg(args):
         copies.append((a, b, dg_views(a, dg), dg_views(b, dg)))
     torch.cuda.synchronize()
 
-    # A step is the two dg_gemm calls, enqueued back to back on one stream
-    # (their kernels use programmatic dependent launch, so each one's launch
-    # overlaps the previous one's tail).  CUDA events bracket the x*W kernel
-    # on every EVERY-th step to time it; the other steps carry no events,
-    # which would break that overlap.
-    EVERY = 16
+    # A step is the two dg_gemm calls on one stream.  The timed region replays
+    # CUDA graphs of those calls (captured once; the host launch cost of a
+    # call does not reach the device timeline).  Steps run in units of UNIT:
+    # the unit's x*W products as one graph, bracketed by CUDA events (the
+    # roofline's kernel timing covers every x*W launch of the timed region),
+    # then its x*K^T products as another.  UNIT is a multiple of ROTATE, so
+    # every unit starts on copy 0 and the copies keep rotating across units.
+    UNIT = 16 * ROTATE
 
-    def step(i, ev=None):
+    def step(i):
         a, b, va, vb = copies[i % ROTATE]
-        if ev is not None:
-            ev[0].record(stream)
         st1 = dg.dg_gemm(*va, 1.0, 0.0, None, None, stream)
-        if ev is not None:
-            ev[1].record(stream)
         st2 = dg.dg_gemm(*vb, 1.0, 0.0, None, None, stream)
         return st1 | st2
 
@@ -379,33 +377,69 @@ def run_dg(args):
     torch.cuda.synchronize()
     assert dg.dg_sync_status(stream) == dg.DG_OK
 
+    def capture(which, n):
+        """A CUDA graph of n x*W (which=2) or x*K^T (which=3) calls over the
+        rotating copies, and the number of kernels it launches."""
+        g = torch.cuda.CUDAGraph()
+        n0 = dg.dg_launch_count()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+            for i in range(n):
+                assert dg.dg_gemm(*copies[i % ROTATE][which], 1.0, 0.0, None, None, stream) == 0
+        return g, dg.dg_launch_count() - n0
+
+    graphs = {}
+    units = []
+    left = args.steps
+    while left > 0:
+        n = min(UNIT, left)
+        if n not in graphs:
+            graphs[n] = (capture(2, n), capture(3, n))
+        units.append(n)
+        left -= n
+    torch.cuda.synchronize()
+    assert dg.dg_sync_status(stream) == dg.DG_OK
+
+    def run_units(evs):
+        launches = 0
+        for u, n in enumerate(units):
+            (gw, nw), (gk, nk) = graphs[n]
+            if evs is not None:
+                evs[u][0].record(stream)
+            gw.replay()
+            if evs is not None:
+                evs[u][1].record(stream)
+            gk.replay()
+            launches += nw + nk
+        return launches
+
+    with torch.cuda.stream(stream):
+        run_units(None)  # warm replay of every graph (untimed)
+    torch.cuda.synchronize()
+
     sampler = ClockSampler(torch.cuda.current_device())
     sampler.start()
     time.sleep(0.3)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range((args.steps + EVERY - 1) // EVERY)]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in units]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    n0 = dg.dg_launch_count()
     w0 = time.time()
-    t_start.record(stream)
-    for i in range(args.steps):
-        assert step(i, evs[i // EVERY] if i % EVERY == 0 else None) == 0
-    t_end.record(stream)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        launches = run_units(evs)
+        t_end.record(stream)
     torch.cuda.synchronize()
     w1 = time.time()
     barrier(world)
-    launches = dg.dg_launch_count() - n0
     time.sleep(0.25)
     sampler.stop()
     assert dg.dg_sync_status(stream) == dg.DG_OK
     elapsed = t_start.elapsed_time(t_end) * 1e-3
     elapsed_max = max_over_ranks(elapsed, world, dev)
     value = whole_job_value(step_bytes, args.steps, world, elapsed_max)
-    gemv_times = [a.elapsed_time(b) * 1e-3 for a, b in evs]
-    gemv_avg = sum(gemv_times) / len(gemv_times)
+    gemv_total = sum(a.elapsed_time(b) * 1e-3 for a, b in evs)
+    gemv_avg = gemv_total / args.steps  # every x*W launch of the timed region is inside a bracket
     gemv_bytes = flops_bytes(gv)[1]
     achieved = gemv_bytes / gemv_avg / 1e9
     peak_hbm = peaks["hbm_gbs"]
@@ -417,11 +451,11 @@ def run_dg(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "bytes_per_step": step_bytes,
                    "l2": f"inputs rotate through {ROTATE} copies of W and K (352 MB > 126 MB L2)",
-                   "launch": "two dg_gemm calls per step on one stream; the x*W kernel is bracketed by CUDA "
-                             "events on every 16th step",
+                   "launch": f"two dg_gemm calls per step on one stream, replayed from CUDA graphs in units of "
+                             f"{UNIT} steps: the unit's x*W calls, bracketed by CUDA events, then its x*K^T calls",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "kernel": "gemv_n (x*W, 117 MB of W)", "achieved": achieved,
-                     "timed_launches": len(gemv_times),
+                     "timed_launches": args.steps,
                      "peak": peak_hbm, "unit": "GB/s", "frac": achieved / peak_hbm,
                      "traffic": traffic, "algorithmic_bytes": gemv_bytes, "avg_launch_us": gemv_avg * 1e6,
                      "peak_source": f"{peaks['source']} hbm_gbs (STREAM-style copy)"},

@@ -179,7 +179,8 @@ typedef struct {
     int32_t vec_bytes;     /* gather / GEMV vector width                             */
     int64_t M, N, K;
     int32_t cta_pair;      /* UMMA: two CTAs of a cluster share each 256-row tile     */
-    int32_t reserved;
+    int32_t epi_tma_store; /* UMMA: the epilogue writes C in 32-row x 128-byte blocks
+                              through tensor stores (beta == 0, C row-major along N)  */
 } dg_plan_info;
 
 /* The dispatch decision dg_gemm would take for these views (pointers are only
@@ -209,9 +210,12 @@ typedef enum {
                                      next kernel at the start of each kernel, 2 release
                                      it near the end of long kernels; default 0: it did
                                      not shorten back-to-back decode steps             */
-    DG_OPT_TRACE = 7              /* device address of 64 uint64 slots (0 = off): the
+    DG_OPT_TRACE = 7,             /* device address of 64 uint64 slots (0 = off): the
                                      single-CTA tensor-core kernel's CTA 0 writes
                                      %globaltimer at its phase boundaries (analysis)   */
+    DG_OPT_EPI_TMA = 8            /* 1 (default): tensor-core epilogues store C through
+                                     tensor copies where the plan allows; 0: thread
+                                     stores only                                        */
 } dg_option;
 
 dg_status dg_set_option(int option, int64_t value);

@@ -34,6 +34,7 @@ std::atomic<int> g_max_split{8};
 std::atomic<int> g_pair{1};
 std::atomic<int> g_pdl{0};
 std::atomic<uint64_t> g_trace{0};
+std::atomic<int> g_epi_tma{1};
 std::atomic<uint32_t> g_epoch{1};  // bumped by every option change: cached launches go stale
 
 constexpr int kMaxDevices = 64;
@@ -208,7 +209,7 @@ void gemv_n_split(int64_t M, int64_t N, int64_t K, int num_sms, dg_plan_info *in
 }
 
 // Which UMMA configuration serves these views (false: none).
-bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, int num_sms, Plan *pl) {
+bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int num_sms, Plan *pl) {
     const int dt = v.A->dtype;
     if (dt != DG_F16 && dt != DG_BF16 && dt != DG_E4M3) return false;
     if (v.c.row.n > 1 || v.c.col.n > 1) return false;
@@ -291,12 +292,19 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, int num_sms, Pla
         const bool halves_ok = !q_mn || ((bn / 2) % per == 0);
         if (halves_ok) pair = (pair_mode == 2) || (Mi >= 256 && tiles >= num_sms);
     }
-    const int stages = pair ? umma_pair_max_stages(bn) : umma_max_stages(bn, !p_tma);
+    // the epilogue stores C through tensor copies when C is row-major along j
+    // with 16-byte aligned rows, is not read (beta == 0) and each tile is a
+    // whole number of 128-byte blocks; split tiles use the cluster reduction
+    const int ces = elem_size(v.C->dtype);
+    const int blk = 128 / ces;  // columns per 128-byte block
+    const bool epi_tma = g_epi_tma.load() != 0 && !swap && split == 1 && beta == 0.f && v.c.tma_ok &&
+                         v.c.unit_dim == 1 && bn % blk == 0 && Nj >= blk && Mi >= 32;
+    const int stages = pair ? umma_pair_max_stages(bn, epi_tma) : umma_max_stages(bn, !p_tma, epi_tma);
     if (split > 1) {
-        // the owner CTA receives every split's rows in its operand ring
-        const int64_t recv = split * bn * ((128 + split - 1) / split) * 4;
+        // the split-K reduction stages a CTA's partial and the slices it
+        // receives in its operand ring
         const int64_t ring = (int64_t)stages * (128 * 128 + bn * 128);
-        if (recv > ring) {
+        if ((int64_t)umma_split_ring_bytes(bn, (int)split) > ring) {
             split = 1;
             kb_per = kb_total;
         }
@@ -316,13 +324,14 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, int num_sms, Pla
     in.grid = (int32_t)(split > 1 ? units2 : std::min<int64_t>(units2, num_sms));  // split: one unit per CTA
     in.vec_bytes = p_tma ? 16 : gather_vec * es;
     in.cta_pair = pair;
+    in.epi_tma_store = epi_tma && split == 1;
     if (pair) {
         const int64_t pair_units = ((Mi + 255) / 256) * tiles_j;
         in.block_m = 256;
         in.grid = (int32_t)(2 * std::min<int64_t>(pair_units, num_sms / 2));
     }
     pl->fp8 = (dt == DG_E4M3);
-    pl->smem = pair ? umma_pair_smem_bytes(bn, stages) : umma_smem_bytes(bn, 128, stages, !p_tma);
+    pl->smem = pair ? umma_pair_smem_bytes(bn, stages, epi_tma) : umma_smem_bytes(bn, stages, !p_tma, epi_tma);
     return true;
 }
 
@@ -355,7 +364,7 @@ dg_status make_plan(Views &v, float alpha, float beta, int num_sms, Plan *pl) {
                 return DG_OK;
             }
         } else if (force == DG_KIND_UMMA) {
-            if (umma_plan(v, M, N, K, num_sms, pl)) return DG_OK;
+            if (umma_plan(v, M, N, K, beta, num_sms, pl)) return DG_OK;
         } else {
             if (M <= 8) {
                 if (gemv_applicable(v, M, N, K, DG_KIND_GEMV_N)) {
@@ -365,7 +374,7 @@ dg_status make_plan(Views &v, float alpha, float beta, int num_sms, Plan *pl) {
                 }
                 if (gemv_applicable(v, M, N, K, DG_KIND_GEMV_K)) { in.kind = DG_KIND_GEMV_K; return DG_OK; }
             }
-            if (umma_plan(v, M, N, K, num_sms, pl)) return DG_OK;
+            if (umma_plan(v, M, N, K, beta, num_sms, pl)) return DG_OK;
         }
     }
     if (M > int64_t(65535) * 64 || N > INT32_MAX || K > INT32_MAX) return DG_ERR_UNSUPPORTED;
@@ -378,6 +387,7 @@ dg_status make_plan(Views &v, float alpha, float beta, int num_sms, Plan *pl) {
 
 CUtensorMapDataType tma_dtype(int dt) {
     switch (dt) {
+    case DG_F32: return CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     case DG_F16: return CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     case DG_BF16: return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     default: return CU_TENSOR_MAP_DATA_TYPE_UINT8;
@@ -467,7 +477,7 @@ struct LaunchRec {
     SimtParams simt{};
     GemvParams gemv{};
     UmmaParams umma{};
-    CUtensorMap t0{}, t1{};
+    CUtensorMap t0{}, t1{}, t2{};
     bool fp8 = false, gather = false, pair = false;
     int grid = 0;
     size_t smem = 0;
@@ -552,6 +562,12 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
                                           : encode_2d(&tq, dt, Qv->ptr, in.K, Nj, axis_stride(q_j), q_rows);
             if (!ok) return DG_ERR_UNSUPPORTED;
         }
+        if (in.epi_tma_store) {
+            // C(i, j) in blocks of 32 rows x 128 bytes, the epilogue's unit
+            const int ces = elem_size(v.C->dtype);
+            if (!encode_2d_box(&rec->t2, v.C->dtype, v.C->ptr, Nj, Mi, axis_stride(v.c.row), 128 / ces, 32, true))
+                return DG_ERR_UNSUPPORTED;
+        }
         UmmaParams p{};
         p.Mi = (int32_t)Mi;
         p.Nj = (int32_t)Nj;
@@ -584,6 +600,7 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         p.err_word = ds->err_word;
         p.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
         p.stall_loader = g_stall.load();
+        p.epi_tma = in.epi_tma_store;
         p.pdl = rec->pdl;
         p.trace = reinterpret_cast<uint64_t *>(g_trace.load());
         rec->umma = p;
@@ -610,8 +627,8 @@ dg_status fire(const LaunchRec &r, cudaStream_t stream) {
     case DG_KIND_GEMV_N: err = launch_gemv_n(r.gemv, &r.t0, stream, &grid); break;
     case DG_KIND_GEMV_K: err = launch_gemv_k(r.gemv, stream, &grid); break;
     case DG_KIND_UMMA:
-        err = r.pair ? launch_umma_pair(r.umma, &r.t0, &r.t1, r.fp8, r.grid, r.smem, stream)
-                     : launch_umma(r.umma, &r.t0, &r.t1, r.fp8, r.gather, r.grid, r.smem, stream);
+        err = r.pair ? launch_umma_pair(r.umma, &r.t0, &r.t1, &r.t2, r.fp8, r.grid, r.smem, stream)
+                     : launch_umma(r.umma, &r.t0, &r.t1, &r.t2, r.fp8, r.gather, r.grid, r.smem, stream);
         break;
     default: return DG_ERR_UNSUPPORTED;
     }
@@ -797,6 +814,10 @@ dg_status dg_set_option(int option, int64_t value) {
     case DG_OPT_MAX_SPLIT_K:
         if (value < 1 || value > 64) return DG_ERR_VALUE;
         g_max_split.store((int)value);
+        return DG_OK;
+    case DG_OPT_EPI_TMA:
+        if (value < 0 || value > 1) return DG_ERR_VALUE;
+        g_epi_tma.store((int)value);
         return DG_OK;
     default: return DG_ERR_VALUE;
     }

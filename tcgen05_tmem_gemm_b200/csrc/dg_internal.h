@@ -86,6 +86,7 @@ struct UmmaParams {
     // thread-loaded P operand (gather variant)
     DevView pv;              // rows = i, cols = k
     int32_t gather_vec;      // elements per load
+    int32_t epi_tma;         // 1: the epilogue writes C through tensor stores (third map)
     // control
     int *err_word;
     uint64_t timeout_ns;
@@ -121,14 +122,16 @@ struct SimtParams {
 // Each returns cudaSuccess or the launch error; `launches` is incremented by
 // the number of kernels enqueued.
 
-cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq,
+// tc: C's tensor map when p.epi_tma (otherwise not read)
+cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq, const CUtensorMap *tc,
                         bool fp8, bool gather, int grid, size_t smem, cudaStream_t s);
-size_t umma_smem_bytes(int bn, int bk_bytes, int stages, bool gather);
-int umma_max_stages(int bn, bool gather);
-cudaError_t launch_umma_pair(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq, bool fp8, int grid,
-                             size_t smem, cudaStream_t s);
-size_t umma_pair_smem_bytes(int bn, int stages);
-int umma_pair_max_stages(int bn);
+size_t umma_smem_bytes(int bn, int stages, bool gather, bool epi_tma);
+int umma_max_stages(int bn, bool gather, bool epi_tma);
+uint32_t umma_split_ring_bytes(int bn, int split);  // ring bytes the split-K reduction needs
+cudaError_t launch_umma_pair(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq,
+                             const CUtensorMap *tc, bool fp8, int grid, size_t smem, cudaStream_t s);
+size_t umma_pair_smem_bytes(int bn, int stages, bool epi_tma);
+int umma_pair_max_stages(int bn, bool epi_tma);
 
 cudaError_t launch_gemv_n(const GemvParams &p, const CUtensorMap *tmap_w, cudaStream_t s, int *grid_out);
 size_t gemv_n_smem_bytes(int r_inst, int kper);

@@ -40,28 +40,45 @@ namespace dg {
 namespace {
 
 constexpr int kBM = 128;             // tensor-core tile rows (TMEM lanes)
+constexpr int kMaxSplit = 8;         // k splits of a tile: one portable cluster
 constexpr int kTileBytesK = 128;     // one swizzle row: 64 x 16-bit or 128 x 8-bit
 constexpr int kGatherWarps = 4;
 
 struct SmemLayout {
     uint32_t stage_bytes, p_bytes, q_bytes;
-    uint32_t bar_off;                // after the stages
+    uint32_t epi_off;                // TMA-store epilogue blocks (epi_tma), after the stages
+    uint32_t bar_off;
     uint32_t aux_off;                // tmem address, abort flag, gather tables
     uint32_t total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int bn, int stages, bool gather) {
+__host__ __device__ inline SmemLayout smem_layout(int bn, int stages, bool gather, bool epi_tma) {
     SmemLayout L;
     L.p_bytes = kBM * kTileBytesK;
     L.q_bytes = (uint32_t)bn * kTileBytesK;
-    L.stage_bytes = L.p_bytes + L.q_bytes;
-    L.bar_off = L.stage_bytes * stages;
-    // full[S], empty[S], tfull[2], tempty[2], drain
-    L.aux_off = L.bar_off + 8 * (2 * stages + 5);
+    L.stage_bytes = L.p_bytes + L.q_bytes;  // a multiple of 1024: bn is a multiple of 8
+    L.epi_off = L.stage_bytes * stages;
+    L.bar_off = L.epi_off + (epi_tma ? kEpiStoreBytes : 0u);
+    // full[S], empty[S], tfull[2], tempty[2], drain, recv (split-K slices)
+    L.aux_off = L.bar_off + 8 * (2 * stages + 6);
     uint32_t aux = 16;  // tmem base + abort flag
     if (gather) aux += 8 * kBM;  // row offsets of the tile
     L.total = L.aux_off + aux + 1024;  // + slack to align the base to 1024
     return L;
+}
+
+// Split-K reduction inside the operand ring (idle by then): this CTA's
+// partial as S slices of `slice` bytes (slice d = the rows CTA d of the
+// cluster owns, column-major) from offset 0, then the slices received from
+// the other CTAs, by source rank, from split_in_offset.
+__host__ __device__ inline uint32_t split_slice_bytes(int bn, int S) {
+    return (uint32_t)(bn * ((kBM + S - 1) / S) * 4);
+}
+__host__ __device__ inline uint32_t split_in_offset(int bn, int S) {
+    return (S * split_slice_bytes(bn, S) + 1023u) & ~1023u;
+}
+__host__ __device__ inline uint32_t split_ring_bytes(int bn, int S) {
+    return split_in_offset(bn, S) + S * split_slice_bytes(bn, S);
 }
 
 struct TileCoord {
@@ -326,20 +343,21 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
 template <bool FP8, bool GATHER>
 __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
-                     const UmmaParams p) {
+                     const __grid_constant__ CUtensorMap tmap_c, const UmmaParams p) {
     if (threadIdx.x == 0) trace_at(p, 0);
     pdl_wait();
     if (p.pdl == 1) pdl_release();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const SmemLayout L = smem_layout(p.bn, p.stages, GATHER);
+    const SmemLayout L = smem_layout(p.bn, p.stages, GATHER, p.epi_tma != 0);
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_full = sbase + L.bar_off;
     const uint32_t bar_empty = bar_full + 8 * p.stages;
     const uint32_t bar_tfull = bar_empty + 8 * p.stages;
     const uint32_t bar_tempty = bar_tfull + 16;
     const uint32_t bar_drain = bar_tempty + 16;
+    const uint32_t bar_recv = bar_drain + 8;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L.aux_off);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.aux_off + 4);
     int64_t *g_row_off = reinterpret_cast<int64_t *>(smem + L.aux_off + 16);
@@ -360,11 +378,13 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             mbar_init(bar_tempty + 8 * b, 4);
         }
         mbar_init(bar_drain, 1);
+        mbar_init(bar_recv, 1);
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
         tma_prefetch_desc(&tmap_q);
         if (!GATHER) tma_prefetch_desc(&tmap_p);
+        if (p.epi_tma) tma_prefetch_desc(&tmap_c);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
@@ -479,8 +499,37 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
         // ---------------------------------------------------------- epilogue
         const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
         const int row = quarter * 32 + lane;         // row inside the tile
-        const EpiParams &e = p.epi;
+        const EpiParams e = p.epi;  // a local copy: its fields stay in registers
         int local = 0;
+        uint32_t nblk = 0;  // tensor-store blocks this warp has issued
+        if (p.split_k > 1 && e.beta != 0.f) {
+            // the rows this CTA will reduce: pull their C lines into L2 while
+            // the main loops run
+            const TileCoord tc = unit_coord(blockIdx.x, p);
+            const int S = p.split_k, rank = (int)cluster_ctarank();
+            const int r0 = rank * kBM / S, rs = (rank + 1) * kBM / S - r0;
+            const int ces = elem_bytes(e.c_dtype);
+            const int t = threadIdx.x - kEpiWarp0 * 32;
+            const int i0 = tc.ti * kBM + r0, jt = tc.tj * p.bn;
+            const int ni = min(rs, p.Mi - i0), nj = min(p.bn, p.Nj - jt);
+            if (ni > 0 && nj > 0) {
+                // every 128-byte line a run touches: offsets 0, 128, ... clamped
+                // to the run's last byte (never past the run)
+                if (e.ci == ces) {  // a run of ni elements per column
+                    const int len = ni * ces, per = (len + 127) / 128 + 1;
+                    for (int q = t; q < nj * per; q += 128) {
+                        const int c = q / per, l = q % per;
+                        prefetch_l2(e.c + (int64_t)i0 * e.ci + (int64_t)(jt + c) * e.cj + min(l * 128, len - 1));
+                    }
+                } else if (e.cj == ces) {  // a run of nj elements per row
+                    const int len = nj * ces, per = (len + 127) / 128 + 1;
+                    for (int q = t; q < ni * per; q += 128) {
+                        const int r = q / per, l = q % per;
+                        prefetch_l2(e.c + (int64_t)(i0 + r) * e.ci + (int64_t)jt * e.cj + min(l * 128, len - 1));
+                    }
+                }
+            }
+        }
         for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++local) {
             const TileCoord tc = unit_coord(u, p);
             const int b = local & 1;
@@ -500,22 +549,34 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                 continue;
             }
 
-            const bool row_ok = i < p.Mi;
-            const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
-            char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
-            for (int c0 = 0; c0 < p.bn; c0 += 16) {
-                uint32_t r[16];
+            if (p.epi_tma) {
+                const uint32_t blocks = sbase + L.epi_off + (uint32_t)quarter * 2u * kEpiBlockBytes;
+                const int i_base = tc.ti * kBM + quarter * 32;
                 __syncwarp();
-                tmem_ld16(t_row + c0, r);
-                tmem_ld_wait();
-                if (!row_ok) continue;
-                epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
+                if (e.c_dtype == DG_F32)
+                    epilogue_rows_tma<4>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, p.bn, p.Nj, lane, nblk);
+                else
+                    epilogue_rows_tma<2>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, p.bn, p.Nj, lane, nblk);
+            } else {
+                const bool row_ok = i < p.Mi;
+                const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
+                char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
+                for (int c0 = 0; c0 < p.bn; c0 += 16) {
+                    uint32_t r[16];
+                    __syncwarp();
+                    tmem_ld16(t_row + c0, r);
+                    tmem_ld_wait();
+                    if (!row_ok) continue;
+                    epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_tempty + 8 * b);
             if (local == 0 && threadIdx.x == kEpiWarp0 * 32) trace_at(p, 35);
         }
+        // the tensor stores read this warp's blocks and write C after the loop
+        if (p.epi_tma && lane == 0) bulk_wait_all();
     } else if (GATHER) {
         // ------------------------------------------------ gather producers
         const int gtid = threadIdx.x - (kEpiWarp0 + 4) * 32;
@@ -530,28 +591,39 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
 
     if (p.split_k > 1) {
         // ------------------------------------------ cluster reduction of k splits
-        // CTA s of the cluster owns rows [128 s / S, 128 (s+1) / S) of the tile.
-        // After every CTA's main loop (barrier 1: all operand rings are idle),
-        // each CTA pushes every row of its partial from TMEM into the owner's
-        // ring with remote shared-memory stores (which do not wait), as
-        // recv[source][column][row - first owned row]; after barrier 2 each
-        // owner adds its S slices in rank order from its own shared memory
-        // and runs the epilogue.
+        // CTA s of the cluster owns rows [128 s / S, 128 (s+1) / S) of the
+        // tile.  After barrier 1 (every operand ring of the cluster idle) each
+        // CTA writes its partial from TMEM into its own ring as S slices, slice
+        // d holding the rows CTA d owns (column-major), and one thread copies
+        // every other slice into its owner's ring with a bulk shared-memory
+        // copy that completes on the owner's receive barrier.  An owner adds
+        // the S slices of its rows in rank order (its own slice stays local),
+        // so the sum is deterministic, and runs the epilogue.  Barrier 2 is
+        // arrived at once a CTA has received everything and waited on before
+        // exit: no CTA leaves while a copy out of its shared memory may still
+        // be reading.
         const int S = p.split_k;
         const int rs_max = (kBM + S - 1) / S;
+        const uint32_t slice = split_slice_bytes(p.bn, S);
+        const uint32_t out_slices = sbase;
+        const uint32_t in_slices = sbase + split_in_offset(p.bn, S);
         const uint32_t rank = cluster_ctarank();
+        const bool epi_warp = warp >= kEpiWarp0 && warp < kEpiWarp0 + 4;
+        if (threadIdx.x == kEpiWarp0 * 32) mbar_arrive_expect_tx(bar_recv, (uint32_t)(S - 1) * slice);
         tc_fence_before();
         __syncthreads();
-        cluster_sync();
+        cluster_sync();  // barrier 1
         if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 54);
-        if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+        if (!epi_warp) cluster_arrive();  // barrier 2: nothing to receive here
+        if (epi_warp) {
             tc_fence_after();
             const int quarter = warp & 3;
             const int row = quarter * 32 + lane;
             int d = 0;
             while (d + 1 < S && (d + 1) * kBM / S <= row) ++d;
             const int rl = row - d * kBM / S;
-            const uint32_t dst = dsmem_map(sbase, (uint32_t)d);
+            const uint32_t dst = out_slices + (uint32_t)d * slice + (uint32_t)rl * 4u;
+            const uint32_t col_pitch = (uint32_t)rs_max * 4u;
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16);
             for (int c0 = 0; c0 < p.bn; c0 += 16) {
                 uint32_t r[16];
@@ -559,67 +631,163 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                 tmem_ld16(t_row + c0, r);
                 tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    dsmem_st_f32(dst + (uint32_t)((((int)rank * p.bn + c0 + c) * rs_max + rl) * 4), __uint_as_float(r[c]));
+                for (int c = 0; c < 16; ++c) st_shared_f32(dst + (uint32_t)(c0 + c) * col_pitch, __uint_as_float(r[c]));
             }
-        }
-        __syncthreads();
-        cluster_sync();
-        if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 55);
-        if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
-            const EpiParams &e = p.epi;
-            const TileCoord tc = unit_coord(blockIdx.x, p);
-            const int r0 = (int)(rank * kBM / S), r1 = (int)((rank + 1) * kBM / S), rs = r1 - r0;
-            const int t = threadIdx.x - kEpiWarp0 * 32;
-            const bool along_i = (e.ci == (int64_t)elem_bytes(e.c_dtype));  // C contiguous along i
-            const float *recv = reinterpret_cast<const float *>(smem);
-            // element e of the owned rs x bn slice: r = e % rs, c = e / rs when C
-            // is contiguous along i (consecutive threads, consecutive addresses),
-            // else c = e % bn, r = e / bn; indices advance without division
-            const int total = rs * p.bn;
-            int r = along_i ? t % rs : t / p.bn, c = along_i ? t / rs : t % p.bn;
-            const int dr = along_i ? 128 % rs : 128 / p.bn, dc = along_i ? 128 / rs : 128 % p.bn;
-            constexpr int kB = 8;  // outputs per thread per batch: their C loads are in flight together
-            for (int base = t; base < total; base += 128 * kB) {
-                int ii[kB], jj[kB];
-                float acc[kB], cin[kB];
-#pragma unroll
-                for (int b = 0; b < kB; ++b) {
-                    const int i = tc.ti * kBM + r0 + r, j = tc.tj * p.bn + c;
-                    const bool ok = base + b * 128 < total && i < p.Mi && j < p.Nj;
-                    ii[b] = ok ? i : -1;
-                    jj[b] = j;
-                    float a = 0.f;
-                    if (ok)
-                        for (int q = 0; q < S; ++q) a += recv[(q * p.bn + c) * rs_max + r];
-                    acc[b] = a;
-                    cin[b] = (ok && e.beta != 0.f) ? load_elem(e.c + (int64_t)i * e.ci + (int64_t)j * e.cj, e.c_dtype)
-                                                   : 0.f;
-                    // advance by 128 elements
-                    if (along_i) {
-                        r += dr;
-                        c += dc;
-                        if (r >= rs) { r -= rs; ++c; }
-                    } else {
-                        c += dc;
-                        r += dr;
-                        if (c >= p.bn) { c -= p.bn; ++r; }
-                    }
+            if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 57);
+            fence_proxy_async_smem();  // the slices are read by the bulk copies
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            if (threadIdx.x == kEpiWarp0 * 32 && !*abort_flag) {
+                trace_at(p, 58);
+                for (int q = 1; q < S; ++q) {
+                    const uint32_t dr = (rank + (uint32_t)q) % (uint32_t)S;
+                    bulk_copy_to_cluster(dsmem_map(in_slices + rank * slice, dr), out_slices + dr * slice, slice,
+                                         dsmem_map(bar_recv, dr));
                 }
+                trace_at(p, 59);
+            }
+            const bool received = mbar_wait(bar_recv, 0, wc);
+            cluster_arrive();  // barrier 2: every copy into this CTA has landed
+            if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 55);
+            if (received) {
+                const EpiParams e = p.epi;  // a local copy: its fields stay in registers
+                const TileCoord tc = unit_coord(blockIdx.x, p);
+                const int r0 = (int)(rank * kBM / S), r1 = (int)((rank + 1) * kBM / S), rs = r1 - r0;
+                const int t = threadIdx.x - kEpiWarp0 * 32;
+                const int bn = p.bn, Mi = p.Mi, Nj = p.Nj;
+                const int i0 = tc.ti * kBM + r0, jt = tc.tj * bn;
+                const float alpha = e.alpha, beta = e.beta;
+                const float *const scale_i = e.scale_i, *const scale_j = e.scale_j;
+                char *const cbase = e.c;
+                const int64_t ci = e.ci, cj = e.cj;
+                const int cdt = e.c_dtype;
+                // slice of source q: local for this CTA's own rank
+                uint32_t src[kMaxSplit];
 #pragma unroll
-                for (int b = 0; b < kB; ++b) {
-                    if (ii[b] < 0) continue;
-                    const int i = ii[b], j = jj[b];
-                    const float asi = e.alpha * (e.scale_i ? e.scale_i[i] : 1.f);
-                    const float sj = e.scale_j ? e.scale_j[j] : 1.f;
-                    float val = (asi * sj) * acc[b];
-                    if (e.beta != 0.f) val = fmaf(e.beta, cin[b], val);
-                    store_elem(e.c + (int64_t)i * e.ci + (int64_t)j * e.cj, e.c_dtype, val);
+                for (int q = 0; q < kMaxSplit; ++q)
+                    src[q] = q == (int)rank ? out_slices + rank * slice : in_slices + (uint32_t)q * slice;
+                const bool vec4 = cdt == DG_F32 && ci == 4 && rs_max % 4 == 0 && rs % 4 == 0 && i0 % 4 == 0 &&
+                                  cj % 16 == 0 && (reinterpret_cast<uintptr_t>(cbase) & 15) == 0;
+                if (vec4) {
+                    // four consecutive rows (contiguous in C and in a slice) per
+                    // thread and step; consecutive threads take consecutive rows
+                    const int g_rows = rs / 4, total = g_rows * bn;
+                    constexpr int kB = 4;
+                    for (int base = t; base < total; base += 128 * kB) {
+                        float4 cin[kB], acc[kB];
+#pragma unroll
+                        for (int b = 0; b < kB; ++b) {
+                            const int g = base + b * 128;
+                            const int r = (g % g_rows) * 4, c = g / g_rows;
+                            const int i = i0 + r, j = jt + c;
+                            acc[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            cin[b] = acc[b];
+                            if (g < total && j < Nj && i + 3 < Mi) {
+                                if (beta != 0.f)
+                                    cin[b] = *reinterpret_cast<const float4 *>(cbase + (int64_t)i * 4 + (int64_t)j * cj);
+                                const uint32_t off = (uint32_t)(c * rs_max + r) * 4u;
+#pragma unroll
+                                for (int q = 0; q < kMaxSplit; ++q) {
+                                    if (q < S) {
+                                        const float4 v = ld_shared_v4(src[q] + off);
+                                        acc[b].x += v.x;
+                                        acc[b].y += v.y;
+                                        acc[b].z += v.z;
+                                        acc[b].w += v.w;
+                                    }
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int b = 0; b < kB; ++b) {
+                            const int g = base + b * 128;
+                            const int r = (g % g_rows) * 4, c = g / g_rows;
+                            const int i = i0 + r, j = jt + c;
+                            if (!(g < total && j < Nj && i < Mi)) continue;
+                            const float sj = scale_j ? scale_j[j] : 1.f;
+                            const float a4[4] = {acc[b].x, acc[b].y, acc[b].z, acc[b].w};
+                            const float c4[4] = {cin[b].x, cin[b].y, cin[b].z, cin[b].w};
+                            float o[4];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const float asi = alpha * (scale_i && i + k < Mi ? scale_i[i + k] : 1.f);
+                                o[k] = (asi * sj) * a4[k];
+                                if (beta != 0.f) o[k] = fmaf(beta, c4[k], o[k]);
+                            }
+                            char *dstc = cbase + (int64_t)i * 4 + (int64_t)j * cj;
+                            if (i + 3 < Mi) {
+                                *reinterpret_cast<float4 *>(dstc) = make_float4(o[0], o[1], o[2], o[3]);
+                            } else {
+                                // rows past C: element by element (loads too)
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    if (i + k >= Mi) break;
+                                    float a = 0.f;
+                                    const uint32_t off = (uint32_t)(c * rs_max + r + k) * 4u;
+#pragma unroll
+                                    for (int q = 0; q < kMaxSplit; ++q)
+                                        if (q < S) a += ld_shared_f32(src[q] + off);
+                                    const float asi = alpha * (scale_i ? scale_i[i + k] : 1.f);
+                                    float val = (asi * sj) * a;
+                                    if (beta != 0.f) val = fmaf(beta, load_elem(dstc + k * 4, cdt), val);
+                                    store_elem(dstc + k * 4, cdt, val);
+                                }
+                            }
+                        }
+                    }
+                } else {
+                    // any C layout: element by element; consecutive threads take
+                    // consecutive addresses along C's contiguous dim
+                    const bool along_i = (ci == (int64_t)elem_bytes(cdt));
+                    const int total = rs * bn;
+                    int r = along_i ? t % rs : t / bn, c = along_i ? t / rs : t % bn;
+                    const int dr = along_i ? 128 % rs : 128 / bn, dc = along_i ? 128 / rs : 128 % bn;
+                    constexpr int kB = 8;  // outputs per thread per batch: their C loads are in flight together
+                    for (int base = t; base < total; base += 128 * kB) {
+                        int ii[kB], jj[kB];
+                        float acc[kB], cin[kB];
+#pragma unroll
+                        for (int b = 0; b < kB; ++b) {
+                            const int i = i0 + r, j = jt + c;
+                            const bool ok = base + b * 128 < total && i < Mi && j < Nj;
+                            ii[b] = ok ? i : -1;
+                            jj[b] = j;
+                            float a = 0.f;
+                            if (ok) {
+                                const uint32_t off = (uint32_t)(c * rs_max + r) * 4u;
+#pragma unroll
+                                for (int q = 0; q < kMaxSplit; ++q)
+                                    if (q < S) a += ld_shared_f32(src[q] + off);
+                            }
+                            acc[b] = a;
+                            cin[b] = (ok && beta != 0.f) ? load_elem(cbase + (int64_t)i * ci + (int64_t)j * cj, cdt)
+                                                         : 0.f;
+                            // advance by 128 elements
+                            if (along_i) {
+                                r += dr;
+                                c += dc;
+                                if (r >= rs) { r -= rs; ++c; }
+                            } else {
+                                c += dc;
+                                r += dr;
+                                if (c >= bn) { c -= bn; ++r; }
+                            }
+                        }
+#pragma unroll
+                        for (int b = 0; b < kB; ++b) {
+                            if (ii[b] < 0) continue;
+                            const int i = ii[b], j = jj[b];
+                            const float asi = alpha * (scale_i ? scale_i[i] : 1.f);
+                            const float sj = scale_j ? scale_j[j] : 1.f;
+                            float val = (asi * sj) * acc[b];
+                            if (beta != 0.f) val = fmaf(beta, cin[b], val);
+                            store_elem(cbase + (int64_t)i * ci + (int64_t)j * cj, cdt, val);
+                        }
+                    }
                 }
             }
         }
         if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 56);
-        // no CTA touches another's shared memory after the second barrier
+        cluster_wait();  // barrier 2
     }
 
     // --------------------------------------------------------------- teardown
@@ -635,20 +803,21 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
 
 }  // namespace
 
-size_t umma_smem_bytes(int bn, int bk_bytes, int stages, bool gather) {
-    (void)bk_bytes;
-    return smem_layout(bn, stages, gather).total;
+size_t umma_smem_bytes(int bn, int stages, bool gather, bool epi_tma) {
+    return smem_layout(bn, stages, gather, epi_tma).total;
 }
 
-int umma_max_stages(int bn, bool gather) {
+uint32_t umma_split_ring_bytes(int bn, int split) { return split_ring_bytes(bn, split); }
+
+int umma_max_stages(int bn, bool gather, bool epi_tma) {
     int s = 2;
-    while (s < 12 && smem_layout(bn, s + 1, gather).total <= 227 * 1024) ++s;
+    while (s < 12 && smem_layout(bn, s + 1, gather, epi_tma).total <= 227 * 1024) ++s;
     return s;
 }
 
-cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq, bool fp8, bool gather,
-                        int grid, size_t smem, cudaStream_t s) {
-    void (*kern)(const CUtensorMap, const CUtensorMap, const UmmaParams);
+cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq, const CUtensorMap *tc,
+                        bool fp8, bool gather, int grid, size_t smem, cudaStream_t s) {
+    void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const UmmaParams);
     if (fp8) kern = gather ? umma_gemm_kernel<true, true> : umma_gemm_kernel<true, false>;
     else kern = gather ? umma_gemm_kernel<false, true> : umma_gemm_kernel<false, false>;
     // raise the kernel's dynamic shared-memory limit once per size, not per call
@@ -660,7 +829,8 @@ cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtens
         if (e != cudaSuccess) return e;
         lim.store((int)smem);
     }
-    return launch_ex(kern, dim3(grid), dim3(gather ? 320 : 192), smem, s, dim3(p.split_k, 1, 1), p.pdl, *tp, *tq, p);
+    return launch_ex(kern, dim3(grid), dim3(gather ? 320 : 192), smem, s, dim3(p.split_k, 1, 1), p.pdl, *tp, *tq,
+                     *tc, p);
 }
 
 }  // namespace dg

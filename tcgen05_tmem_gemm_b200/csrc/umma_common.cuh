@@ -2,6 +2,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace dg {
 
@@ -85,6 +86,84 @@ __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow,
                 store_elem(crow + (int64_t)j * e.cj, e.c_dtype, val);
             }
         }
+    }
+}
+
+// Shared memory of the TMA-store epilogue: two blocks of 32 rows x 128 bytes
+// for each of the four epilogue warps.
+constexpr uint32_t kEpiBlockBytes = 32 * 128;
+constexpr uint32_t kEpiStoreBytes = 4 * 2 * kEpiBlockBytes;
+
+// Epilogue of one warp's 32 accumulator rows (TMEM lanes) x bn columns through
+// tensor stores, for beta == 0 and C unit-stride along j.  After tcgen05.ld a
+// thread holds one row, so direct stores would touch 32 rows per instruction.
+// Instead the warp writes 32 rows x 128 bytes of output at a time into a
+// shared-memory block in the 128-byte-swizzle layout (row r's 16-byte unit u
+// sits at unit u ^ (r & 7), so the eight lanes of each store phase hit
+// different banks) and one lane stores the block with a tensor copy, which
+// writes whole lines and skips everything outside C.  Two blocks alternate,
+// so packing one overlaps the copy of the other.  `stage` is this warp's
+// 2 x kEpiBlockBytes (1024-byte aligned), `nblk` counts the blocks the warp
+// has issued; the caller waits for its copies (bulk_wait_all) before exit.
+template <int ES>
+__device__ __forceinline__ void epilogue_rows_tma(const EpiParams &e, const CUtensorMap *cmap, uint32_t stage,
+                                                  uint32_t t_row, int i_base, int Mi, int j0, int bn, int Nj,
+                                                  int lane, uint32_t &nblk) {
+    constexpr int W = 128 / ES;  // output columns per block
+    if (i_base >= Mi) return;    // the whole warp is below C (warp-uniform)
+    // parameters in registers: nothing below re-reads the parameter block
+    const float *const scale_j = e.scale_j;
+    const bool bf16_out = e.c_dtype == DG_BF16;
+    const int i = i_base + lane;
+    const float asi = i < Mi ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
+    for (int c0 = 0; c0 < bn && j0 + c0 < Nj; c0 += W) {
+        uint32_t r[W];
+#pragma unroll
+        for (int q = 0; q < W / 16; ++q)
+            tmem_ld16(t_row + (uint32_t)(c0 + 16 * q), *reinterpret_cast<uint32_t(*)[16]>(&r[16 * q]));
+        tmem_ld_wait();
+        float v[W];
+        if (scale_j != nullptr) {  // per-column scales (FP8): read once per block, clamped at the edge
+            const int jb = j0 + c0;
+#pragma unroll
+            for (int c = 0; c < W; ++c) {
+                const float sj = scale_j[jb + c < Nj ? jb + c : Nj - 1];
+                v[c] = (asi * sj) * __uint_as_float(r[c]);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < W; ++c) v[c] = asi * __uint_as_float(r[c]);
+        }
+        uint32_t w[32];
+        if (ES == 4) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(v[c]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                if (bf16_out) {
+                    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * c], v[2 * c + 1]);
+                    w[c] = *reinterpret_cast<uint32_t *>(&h);
+                } else {
+                    __half2 h = __floats2half2_rn(v[2 * c], v[2 * c + 1]);
+                    w[c] = *reinterpret_cast<uint32_t *>(&h);
+                }
+            }
+        }
+        const uint32_t buf = stage + (nblk & 1u) * kEpiBlockBytes;
+        if (lane == 0) bulk_wait_read<1>();  // the copy that last read this block is done with it
+        __syncwarp();
+        const uint32_t rowa = buf + (uint32_t)lane * 128u;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            st_shared_v4(rowa + ((uint32_t)(u ^ (lane & 7)) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(cmap, buf, j0 + c0, i_base);
+            bulk_commit();
+        }
+        ++nblk;
     }
 }
 

@@ -31,15 +31,16 @@ constexpr int kHalfM = 128;   // rows of P (and TMEM lanes) per CTA
 constexpr int kRowBytes = 128;
 
 struct PairLayout {
-    uint32_t a_bytes, b_bytes, stage_bytes, bar_off, aux_off, total;
+    uint32_t a_bytes, b_bytes, stage_bytes, epi_off, bar_off, aux_off, total;
 };
 
-__host__ __device__ inline PairLayout pair_layout(int bn, int stages) {
+__host__ __device__ inline PairLayout pair_layout(int bn, int stages, bool epi_tma) {
     PairLayout L;
     L.a_bytes = kHalfM * kRowBytes;
     L.b_bytes = (uint32_t)(bn / 2) * kRowBytes;
-    L.stage_bytes = L.a_bytes + L.b_bytes;
-    L.bar_off = L.stage_bytes * stages;
+    L.stage_bytes = L.a_bytes + L.b_bytes;  // a multiple of 1024: bn is a multiple of 16
+    L.epi_off = L.stage_bytes * stages;
+    L.bar_off = L.epi_off + (epi_tma ? kEpiStoreBytes : 0u);
     // full[S], empty[S], tfull[2], tempty[2], drain
     L.aux_off = L.bar_off + 8 * (2 * stages + 5);
     L.total = L.aux_off + 16 + 1024;
@@ -49,12 +50,12 @@ __host__ __device__ inline PairLayout pair_layout(int bn, int stages) {
 template <bool FP8>
 __global__ void __launch_bounds__(192, 1)
     umma_pair_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
-                     const UmmaParams p) {
+                     const __grid_constant__ CUtensorMap tmap_c, const UmmaParams p) {
     pdl_wait();
     if (p.pdl == 1) pdl_release();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const PairLayout L = pair_layout(p.bn, p.stages);
+    const PairLayout L = pair_layout(p.bn, p.stages, p.epi_tma != 0);
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_full = sbase + L.bar_off;
     const uint32_t bar_empty = bar_full + 8 * p.stages;
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(192, 1)
         fence_proxy_async_smem();
         tma_prefetch_desc(&tmap_p);
         tma_prefetch_desc(&tmap_q);
+        if (p.epi_tma) tma_prefetch_desc(&tmap_c);
     }
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
@@ -186,8 +188,9 @@ __global__ void __launch_bounds__(192, 1)
         // ------------------------------------------- epilogue (both CTAs)
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        const EpiParams &e = p.epi;
+        const EpiParams e = p.epi;  // a local copy: its fields stay in registers
         int local = 0;
+        uint32_t nblk = 0;  // tensor-store blocks this warp has issued
         for (int u = cluster_id; u < p.num_units; u += nclusters, ++local) {
             const int ti = u % p.tiles_i, tj = u / p.tiles_i;
             const int b = local & 1;
@@ -197,21 +200,33 @@ __global__ void __launch_bounds__(192, 1)
             const int i = ti * 2 * kHalfM + (int)rank * kHalfM + row;
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * p.bn);
             const int j0 = tj * p.bn;
-            const bool row_ok = i < p.Mi;
-            const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
-            char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
-            for (int c0 = 0; c0 < p.bn; c0 += 16) {
-                uint32_t r[16];
+            if (p.epi_tma) {
+                const uint32_t blocks = sbase + L.epi_off + (uint32_t)quarter * 2u * kEpiBlockBytes;
+                const int i_base = i - lane;
                 __syncwarp();
-                tmem_ld16(t_row + c0, r);
-                tmem_ld_wait();
-                if (!row_ok) continue;
-                epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
+                if (e.c_dtype == DG_F32)
+                    epilogue_rows_tma<4>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, p.bn, p.Nj, lane, nblk);
+                else
+                    epilogue_rows_tma<2>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, p.bn, p.Nj, lane, nblk);
+            } else {
+                const bool row_ok = i < p.Mi;
+                const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
+                char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
+                for (int c0 = 0; c0 < p.bn; c0 += 16) {
+                    uint32_t r[16];
+                    __syncwarp();
+                    tmem_ld16(t_row + c0, r);
+                    tmem_ld_wait();
+                    if (!row_ok) continue;
+                    epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(dsmem_map(bar_tempty + 8 * b, 0));
         }
+        // the tensor stores read this warp's blocks and write C after the loop
+        if (p.epi_tma && lane == 0) bulk_wait_all();
     }
 
     // --------------------------------------------------------------- teardown
@@ -227,17 +242,17 @@ __global__ void __launch_bounds__(192, 1)
 
 }  // namespace
 
-size_t umma_pair_smem_bytes(int bn, int stages) { return pair_layout(bn, stages).total; }
+size_t umma_pair_smem_bytes(int bn, int stages, bool epi_tma) { return pair_layout(bn, stages, epi_tma).total; }
 
-int umma_pair_max_stages(int bn) {
+int umma_pair_max_stages(int bn, bool epi_tma) {
     int s = 2;
-    while (s < 12 && pair_layout(bn, s + 1).total <= 227 * 1024) ++s;
+    while (s < 12 && pair_layout(bn, s + 1, epi_tma).total <= 227 * 1024) ++s;
     return s;
 }
 
-cudaError_t launch_umma_pair(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq, bool fp8, int grid,
-                             size_t smem, cudaStream_t s) {
-    void (*kern)(const CUtensorMap, const CUtensorMap, const UmmaParams);
+cudaError_t launch_umma_pair(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq,
+                             const CUtensorMap *tc, bool fp8, int grid, size_t smem, cudaStream_t s) {
+    void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const UmmaParams);
     kern = fp8 ? umma_pair_kernel<true> : umma_pair_kernel<false>;
     static std::atomic<int> s_limit[2];
     std::atomic<int> &lim = s_limit[fp8 ? 1 : 0];
@@ -246,7 +261,7 @@ cudaError_t launch_umma_pair(const UmmaParams &p, const CUtensorMap *tp, const C
         if (e != cudaSuccess) return e;
         lim.store((int)smem);
     }
-    return launch_ex(kern, dim3(grid), dim3(192), smem, s, dim3(2, 1, 1), p.pdl, *tp, *tq, p);
+    return launch_ex(kern, dim3(grid), dim3(192), smem, s, dim3(2, 1, 1), p.pdl, *tp, *tq, *tc, p);
 }
 
 }  // namespace dg

@@ -128,6 +128,7 @@ def test_plan_small_gemm_umma():
     assert pl["kind_name"] == "umma" and pl["swap_ab"] == 0 and pl["block_n"] == 128
     assert pl["p_mn_major"] == 0 and pl["q_mn_major"] == 1 and pl["split_k"] == 1
     assert pl["cta_pair"] == 0  # one tile: no pairing
+    assert pl["epi_tma_store"] == 1  # beta == 0, row-major FP32 C: tensor stores
 
 
 def test_plan_thin_swaps_and_splits():
@@ -135,6 +136,7 @@ def test_plan_thin_swaps_and_splits():
     assert pl["kind_name"] == "umma" and pl["swap_ab"] == 1
     assert pl["block_n"] == 64 and pl["p_mn_major"] == 1 and pl["q_mn_major"] == 0
     assert pl["split_k"] == 4 and pl["grid"] == 128
+    assert pl["epi_tma_store"] == 0  # beta == 1: split tiles reduce in the cluster
 
 
 def test_plan_square_bf16_and_fp8():
@@ -149,6 +151,7 @@ def test_plan_strided_gathers_a():
     pl = plan_of("strided")
     assert pl["kind_name"] == "umma" and pl["p_gather"] == 1 and pl["swap_ab"] == 0
     assert pl["p_mn_major"] == 1 and pl["vec_bytes"] == 8
+    assert pl["epi_tma_store"] == 1
 
 
 def test_plan_edge_kinds():
@@ -212,3 +215,10 @@ def test_options():
     finally:
         dg.dg_set_option(dg.DG_OPT_FORCE_KIND, 0)
     assert plan_of("small")["kind_name"] == "umma"
+    dg.dg_set_option(dg.DG_OPT_EPI_TMA, 0)
+    try:
+        assert plan_of("small")["epi_tma_store"] == 0
+    finally:
+        dg.dg_set_option(dg.DG_OPT_EPI_TMA, 1)
+    with pytest.raises(dg.DgError):
+        dg.dg_set_option(dg.DG_OPT_EPI_TMA, 2)

@@ -29,6 +29,7 @@ def _reset_options():
     dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, 8)
     dg.dg_set_option(dg.DG_OPT_CTA_PAIR, 1)
     dg.dg_set_option(dg.DG_OPT_EARLY_LAUNCH, 0)
+    dg.dg_set_option(dg.DG_OPT_EPI_TMA, 1)
 
 
 def expect_kind(p, kind, **fields):
@@ -134,6 +135,45 @@ def test_thin_beta_one_split_k():
     p = W.cfg_thin(M=40, N=1000, K=784)
     pl = expect_kind(p, "umma", swap_ab=1)
     assert pl["split_k"] > 1
+    check_full(p)
+
+
+@pytest.mark.parametrize("case", ["s8_ragged_rows", "s3_rows_not_multiple_of_4", "s2_bf16_out", "fp8_scales",
+                                  "no_swap_row_major_c"])
+def test_split_k_cluster_reduction(case):
+    # Every path of the on-chip split-K reduction: four-row vector steps with
+    # a ragged last row group, the element-wise path (S = 3, BF16 output, C
+    # row-major along j) and per-row / per-column scales.
+    g = torch.Generator().manual_seed(len(case) * 31)
+    ms, out, beta = 8, "f32", 1.0
+    if case == "s8_ragged_rows":
+        M, N, K = 64, 1001, 4096
+    elif case == "s3_rows_not_multiple_of_4":
+        M, N, K, ms = 48, 1000, 2048, 3
+    elif case == "s2_bf16_out":
+        M, N, K, ms, out, beta = 64, 512, 2048, 2, "bf16", 0.0
+    elif case == "fp8_scales":
+        M, N, K, out, beta = 32, 1024, 4096, "bf16", 0.0
+    else:
+        M, N, K = 256, 128, 8192
+    dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, ms)
+    if case == "fp8_scales":
+        qa, sa = W.quantise_e4m3(W.normal((M, K), g), dim=1)
+        qb, sb = W.quantise_e4m3(W.normal((K, N), g), dim=0)
+        p = W.Problem(case, W.row_major(qa, "e4m3"), W.row_major(qb, "e4m3"), W.empty_out(M, N, out),
+                      1.0, beta, sa, sb)
+    else:
+        A = W.row_major(W.cast(W.normal((M, K), g), "f16"), "f16")
+        # B read K-major from an [N, K] tensor, so N needs no alignment
+        B = W.transposed(W.cast(W.normal((N, K), g, 0.05), "f16"), "f16")
+        C = W.row_major(W.uniform((M, N), g), "f32") if out == "f32" else W.empty_out(M, N, out)
+        p = W.Problem(case, A, B, C, 1.0, beta)
+    pl = expect_kind(p, "umma")
+    assert pl["split_k"] > 1 and pl["epi_tma_store"] == 0, pl
+    if case == "s3_rows_not_multiple_of_4":
+        assert pl["split_k"] == 3
+    if case == "no_swap_row_major_c":
+        assert pl["swap_ab"] == 0
     check_full(p)
 
 
@@ -286,6 +326,47 @@ def test_scales_applied_once():
                   1.0, 0.0, sa, sb)
     got = c_matrix(run(p.to("cuda")))
     assert np.array_equal(got, K * np.outer(sa.numpy(), sb.numpy()))
+
+
+@pytest.mark.parametrize("M,N,K,dt,out,pair", [
+    (300, 520, 200, "bf16", "bf16", 0),   # ragged rows and columns, 16-bit blocks of 64 columns
+    (129, 136, 72, "f16", "f32", 0),      # one row past a tile, FP32 blocks of 32 columns
+    (520, 384, 128, "bf16", "f32", 2),    # CTA pairs
+    (256, 256, 64, "e4m3", "bf16", 0),    # per-row / per-column scales in the block packing
+])
+def test_epilogue_tensor_stores_match_thread_stores(M, N, K, dt, out, pair):
+    # The two epilogues do the same arithmetic in the same order, so their
+    # outputs agree bit for bit; each is also checked against the oracle.
+    g = torch.Generator().manual_seed(M + 3 * N + K)
+    if dt == "e4m3":
+        qa, sa = W.quantise_e4m3(W.normal((M, K), g), dim=1)
+        qb, sb = W.quantise_e4m3(W.normal((K, N), g), dim=0)
+        p = W.Problem("epi_fp8", W.row_major(qa, "e4m3"), W.row_major(qb, "e4m3"), W.empty_out(M, N, out),
+                      1.5, 0.0, sa, sb)
+    else:
+        A = W.cast(W.normal((M, K), g), dt)
+        B = W.cast(W.normal((K, N), g), dt)
+        p = W.Problem("epi", W.row_major(A, dt), W.row_major(B, dt), W.empty_out(M, N, out), 0.75, 0.0)
+    dg.dg_set_option(dg.DG_OPT_CTA_PAIR, pair)
+    outs = []
+    for tma in (1, 0):
+        dg.dg_set_option(dg.DG_OPT_EPI_TMA, tma)
+        expect_kind(p, "umma", epi_tma_store=tma, cta_pair=int(pair == 2))
+        check_full(p)
+        outs.append(c_matrix(run(p.to("cuda"))))
+    assert np.array_equal(outs[0], outs[1])
+
+
+def test_epilogue_tensor_stores_need_beta_zero_and_row_major_c():
+    M, N, K = 256, 256, 64
+    g = torch.Generator().manual_seed(5)
+    A = W.row_major(W.cast(W.uniform((M, K), g), "bf16"), "bf16")
+    B = W.row_major(W.cast(W.uniform((K, N), g), "bf16"), "bf16")
+    c = W.uniform((M, N), g)
+    expect_kind(W.Problem("b0", A, B, W.row_major(c, "f32"), 1.0, 0.0), "umma", epi_tma_store=1)
+    expect_kind(W.Problem("b1", A, B, W.row_major(c, "f32"), 1.0, 1.0), "umma", epi_tma_store=0)
+    expect_kind(W.Problem("ct", A, B, W.transposed(c.t().contiguous(), "f32"), 1.0, 0.0), "umma",
+                epi_tma_store=0)
 
 
 def test_output_guard_band_untouched():
