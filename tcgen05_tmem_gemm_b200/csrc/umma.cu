@@ -19,7 +19,7 @@
 //  - warps 2-5: the epilogue, each owning 32 TMEM lanes (rows): tcgen05.ld,
 //    scale, optional beta * C, convert and store, while the MMA warp already
 //    fills the other accumulator;
-//  - warps 6-9 (gather variant): thread loads of a P operand that TMA cannot
+//  - warps 6-13 (gather variant): thread loads of a P operand that TMA cannot
 //    describe (e.g. an NCHW feature map read as [N*H*W, C] with a 392-byte
 //    channel stride), written into the same swizzled layout
 //    ("DeepGEMM: a recalibration of the compute paradigm", §2.2: scatter-gather
@@ -42,7 +42,7 @@ namespace {
 constexpr int kBM = 128;             // tensor-core tile rows (TMEM lanes)
 constexpr int kMaxSplit = 8;         // k splits of a tile: one portable cluster
 constexpr int kTileBytesK = 128;     // one swizzle row: 64 x 16-bit or 128 x 8-bit
-constexpr int kGatherWarps = 4;
+constexpr int kGatherWarps = 8;     // gather warps: cp.async latency-bound, so more warps keep more copies in flight
 
 struct SmemLayout {
     uint32_t stage_bytes, p_bytes, q_bytes;
@@ -170,6 +170,30 @@ struct GatherGeom {
     int vec, runs, total, chunk_bytes, es;
 };
 
+// The gathered operand's base and k axis, read from the parameter block once:
+// the copy loops then keep them in registers instead of re-reading them after
+// every asynchronous copy.
+struct GatherSrc {
+    const char *ptr;
+    int64_t kstride;     // byte stride of k when k is one merged dim (k1)
+    const Axis *kaxis;   // otherwise the whole axis
+    int K;
+    bool k1;
+    __device__ __forceinline__ int64_t koff(int kg) const {
+        return k1 ? (int64_t)kg * kstride : axis_offset(*kaxis, kg);
+    }
+};
+
+__device__ __forceinline__ GatherSrc gather_src(const UmmaParams &p) {
+    GatherSrc s;
+    s.ptr = p.pv.ptr;
+    s.k1 = p.pv.col.n == 1;
+    s.kstride = p.pv.col.stride[0];
+    s.kaxis = &p.pv.col;
+    s.K = p.K;
+    return s;
+}
+
 __device__ __forceinline__ GatherGeom gather_geom(const UmmaParams &p, int VB, int bk, int es) {
     GatherGeom g;
     g.mn = p.p_mn_major != 0;
@@ -186,7 +210,7 @@ __device__ __forceinline__ GatherGeom gather_geom(const UmmaParams &p, int VB, i
 // 128 / runs per copy (runs is a power of two dividing 128), so no index is
 // divided inside the loops.
 template <int VB>
-__device__ __forceinline__ void gather_load(const UmmaParams &p, const GatherGeom &g, const int64_t *row_off,
+__device__ __forceinline__ void gather_load(const GatherSrc &src, const GatherGeom &g, const int64_t *row_off,
                                             int kbase, int first, typename VecOf<VB>::T (&v)[kGatherUnroll]) {
     const int nthreads = kGatherWarps * 32;
     const int step = nthreads / g.runs;
@@ -199,13 +223,13 @@ __device__ __forceinline__ void gather_load(const UmmaParams &p, const GatherGeo
         for (int r = 0; r < kGatherUnroll; ++r) {
             const int u = first + r * nthreads;
             const int kg = kbase + k0 + r * step;
-            const bool ok = u < g.total && ro >= 0 && kg < p.K;
-            v[r] = gather_load_one<VB>(p.pv.ptr + (ok ? ro + axis_offset(p.pv.col, kg) : 0), ok);
+            const bool ok = u < g.total && ro >= 0 && kg < src.K;
+            v[r] = gather_load_one<VB>(src.ptr + (ok ? ro + src.koff(kg) : 0), ok);
         }
     } else {
         // fixed k (a run of vec columns), i advancing by `step`
         const int kg = kbase + (first % g.runs) * g.vec;
-        const int64_t co = kg < p.K ? axis_offset(p.pv.col, kg) : -1;
+        const int64_t co = kg < src.K ? src.koff(kg) : -1;
         const int i0 = first / g.runs;
 #pragma unroll
         for (int r = 0; r < kGatherUnroll; ++r) {
@@ -213,7 +237,7 @@ __device__ __forceinline__ void gather_load(const UmmaParams &p, const GatherGeo
             const int i = i0 + r * step;
             const int64_t ro = (u < g.total) ? row_off[i] : -1;
             const bool ok = ro >= 0 && co >= 0;
-            v[r] = gather_load_one<VB>(p.pv.ptr + (ok ? ro + co : 0), ok);
+            v[r] = gather_load_one<VB>(src.ptr + (ok ? ro + co : 0), ok);
         }
     }
 }
@@ -238,8 +262,8 @@ __device__ __forceinline__ void gather_store(const GatherGeom &g, uint32_t p_sme
 // cp.async version of a batch: the same copies as gather_load/gather_store,
 // issued as asynchronous global -> shared copies (no register staging).
 template <int VB>
-__device__ __forceinline__ void gather_issue_async(const UmmaParams &p, const GatherGeom &g, const int64_t *row_off,
-                                                   int kbase, int first, uint32_t p_smem) {
+__device__ __forceinline__ void gather_issue_async(const GatherSrc &src, const GatherGeom &g,
+                                                   const int64_t *row_off, int kbase, int first, uint32_t p_smem) {
     const int nthreads = kGatherWarps * 32;
     const int step = nthreads / g.runs;
     const int fixed = (first % g.runs) * g.vec, moving0 = first / g.runs;
@@ -250,13 +274,13 @@ __device__ __forceinline__ void gather_issue_async(const UmmaParams &p, const Ga
             const int u = first + r * nthreads;
             if (u >= g.total) break;
             const int k = moving0 + r * step, kg = kbase + k;
-            const bool ok = ro >= 0 && kg < p.K;
+            const bool ok = ro >= 0 && kg < src.K;
             cp_async_zfill<VB>(p_smem + sw128_mnmajor(fixed * g.es, k, g.chunk_bytes),
-                               p.pv.ptr + (ok ? ro + axis_offset(p.pv.col, kg) : 0), ok);
+                               src.ptr + (ok ? ro + src.koff(kg) : 0), ok);
         }
     } else {
         const int kg = kbase + fixed;
-        const int64_t co = kg < p.K ? axis_offset(p.pv.col, kg) : -1;
+        const int64_t co = kg < src.K ? src.koff(kg) : -1;
 #pragma unroll
         for (int r = 0; r < kGatherUnroll; ++r) {
             const int u = first + r * nthreads;
@@ -264,7 +288,7 @@ __device__ __forceinline__ void gather_issue_async(const UmmaParams &p, const Ga
             const int i = moving0 + r * step;
             const int64_t ro = row_off[i];
             const bool ok = ro >= 0 && co >= 0;
-            cp_async_zfill<VB>(p_smem + sw128_kmajor(i, fixed * g.es), p.pv.ptr + (ok ? ro + co : 0), ok);
+            cp_async_zfill<VB>(p_smem + sw128_kmajor(i, fixed * g.es), src.ptr + (ok ? ro + co : 0), ok);
         }
     }
 }
@@ -282,6 +306,9 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
                                             int lane) {
     using V = typename VecOf<VB>::T;
     const GatherGeom g = gather_geom(p, VB, bk, es);
+    const GatherSrc src = gather_src(p);
+    const int stages = p.stages;
+    const bool stall = p.stall_loader != 0;
     const int nthreads = kGatherWarps * 32;
     const bool one_batch = VB < 4 && g.total <= nthreads * kGatherUnroll;  // register path look-ahead
     int it = 0;
@@ -297,28 +324,28 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
         asm volatile("bar.sync 1, %0;" ::"n"(kGatherWarps * 32) : "memory");
         bool ok = true;
         V cur[kGatherUnroll], nxt[kGatherUnroll];
-        if (one_batch && kb0 < kb1) gather_load<VB>(p, g, g_row_off, kb0 * bk, gtid, cur);
+        if (one_batch && kb0 < kb1) gather_load<VB>(src, g, g_row_off, kb0 * bk, gtid, cur);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-            const int s = it % p.stages;
-            const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
-            if (one_batch && kb + 1 < kb1) gather_load<VB>(p, g, g_row_off, (kb + 1) * bk, gtid, nxt);
+            const int s = it % stages;
+            const uint32_t ph = (uint32_t)(it / stages) & 1u;
+            if (one_batch && kb + 1 < kb1) gather_load<VB>(src, g, g_row_off, (kb + 1) * bk, gtid, nxt);
             ok = mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc);
             if (named_bar_or(!ok)) { ok = false; break; }
-            if (!p.stall_loader && VB >= 4) {
+            if (!stall && VB >= 4) {
                 // asynchronous copies: the stage completes on the full barrier
                 // when they land, and this warp moves on at once
                 const uint32_t ps = sbase + s * L.stage_bytes;
                 for (int f = gtid; f < g.total; f += nthreads * kGatherUnroll)
-                    gather_issue_async<(VB >= 4 ? VB : 4)>(p, g, g_row_off, kb * bk, f, ps);
+                    gather_issue_async<(VB >= 4 ? VB : 4)>(src, g, g_row_off, kb * bk, f, ps);
                 cp_async_arrive_noinc(bar_full + 8 * s);
                 if (it < 16 && gtid == 0) trace_at(p, 37 + it);
-            } else if (!p.stall_loader) {
+            } else if (!stall) {
                 const uint32_t ps = sbase + s * L.stage_bytes;
                 if (one_batch) {
                     gather_store<VB>(g, ps, gtid, cur);
                 } else {
                     for (int f = gtid; f < g.total; f += nthreads * kGatherUnroll) {
-                        gather_load<VB>(p, g, g_row_off, kb * bk, f, cur);
+                        gather_load<VB>(src, g, g_row_off, kb * bk, f, cur);
                         gather_store<VB>(g, ps, f, cur);
                     }
                 }
@@ -341,7 +368,7 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
 }
 
 template <bool FP8, bool GATHER>
-__global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
+__global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_c, const UmmaParams p) {
     if (threadIdx.x == 0) trace_at(p, 0);
@@ -829,7 +856,7 @@ cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtens
         if (e != cudaSuccess) return e;
         lim.store((int)smem);
     }
-    return launch_ex(kern, dim3(grid), dim3(gather ? 320 : 192), smem, s, dim3(p.split_k, 1, 1), p.pdl, *tp, *tq,
+    return launch_ex(kern, dim3(grid), dim3(gather ? 448 : 192), smem, s, dim3(p.split_k, 1, 1), p.pdl, *tp, *tq,
                      *tc, p);
 }
 
