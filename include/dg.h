@@ -181,6 +181,10 @@ typedef struct {
     int32_t cta_pair;      /* UMMA: two CTAs of a cluster share each 256-row tile     */
     int32_t epi_tma_store; /* UMMA: the epilogue writes C in 32-row x 128-byte blocks
                               through tensor stores (beta == 0, C row-major along N)  */
+    int32_t gather_cluster;/* UMMA, gathered operand: CTAs per cluster that share each
+                              gathered tile, each loading 1/gather_cluster of it and
+                              copying it to the others (1 = no sharing)             */
+    int32_t reserved;
 } dg_plan_info;
 
 /* The dispatch decision dg_gemm would take for these views (pointers are only
@@ -213,9 +217,12 @@ typedef enum {
     DG_OPT_TRACE = 7,             /* device address of 64 uint64 slots (0 = off): the
                                      single-CTA tensor-core kernel's CTA 0 writes
                                      %globaltimer at its phase boundaries (analysis)   */
-    DG_OPT_EPI_TMA = 8            /* 1 (default): tensor-core epilogues store C through
+    DG_OPT_EPI_TMA = 8,           /* 1 (default): tensor-core epilogues store C through
                                      tensor copies where the plan allows; 0: thread
                                      stores only                                        */
+    DG_OPT_GATHER_CLUSTER = 9     /* 1 (default): CTAs that need the same gathered
+                                     operand tile share the loads through distributed
+                                     shared memory; 0: each gathers the whole tile      */
 } dg_option;
 
 dg_status dg_set_option(int option, int64_t value);

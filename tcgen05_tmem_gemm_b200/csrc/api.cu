@@ -35,6 +35,7 @@ std::atomic<int> g_pair{1};
 std::atomic<int> g_pdl{0};
 std::atomic<uint64_t> g_trace{0};
 std::atomic<int> g_epi_tma{1};
+std::atomic<int> g_gather_cluster{1};
 std::atomic<uint32_t> g_epoch{1};  // bumped by every option change: cached launches go stale
 
 constexpr int kMaxDevices = 64;
@@ -310,6 +311,16 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
         }
     }
     const int64_t units2 = tiles * split;
+    // a gathered P tile is shared by the CTAs of its row of tiles: 2 or 4 of
+    // them form a cluster and each gathers its share of every stage
+    int gcl = 1;
+    if (!p_tma && split == 1 && !pair && gather_vec * pvi.es >= 4 && g_gather_cluster.load() != 0) {
+        for (int c : {4, 2})
+            if (tiles_j % c == 0 && num_sms >= c) {
+                gcl = c;
+                break;
+            }
+    }
     dg_plan_info &in = pl->info;
     in.kind = DG_KIND_UMMA;
     in.swap_ab = swap;
@@ -325,6 +336,8 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     in.vec_bytes = p_tma ? 16 : gather_vec * es;
     in.cta_pair = pair;
     in.epi_tma_store = epi_tma && split == 1;
+    in.gather_cluster = gcl;
+    if (gcl > 1) in.grid = (int32_t)std::min<int64_t>(units2, (num_sms / gcl) * gcl);
     if (pair) {
         const int64_t pair_units = ((Mi + 255) / 256) * tiles_j;
         in.block_m = 256;
@@ -601,6 +614,7 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         p.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
         p.stall_loader = g_stall.load();
         p.epi_tma = in.epi_tma_store;
+        p.gather_cluster = in.gather_cluster;
         p.pdl = rec->pdl;
         p.trace = reinterpret_cast<uint64_t *>(g_trace.load());
         rec->umma = p;
@@ -818,6 +832,10 @@ dg_status dg_set_option(int option, int64_t value) {
     case DG_OPT_EPI_TMA:
         if (value < 0 || value > 1) return DG_ERR_VALUE;
         g_epi_tma.store((int)value);
+        return DG_OK;
+    case DG_OPT_GATHER_CLUSTER:
+        if (value < 0 || value > 1) return DG_ERR_VALUE;
+        g_gather_cluster.store((int)value);
         return DG_OK;
     default: return DG_ERR_VALUE;
     }

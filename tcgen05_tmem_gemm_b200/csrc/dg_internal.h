@@ -87,6 +87,8 @@ struct UmmaParams {
     DevView pv;              // rows = i, cols = k
     int32_t gather_vec;      // elements per load
     int32_t epi_tma;         // 1: the epilogue writes C through tensor stores (third map)
+    int32_t gather_cluster;  // > 1: CTAs of a cluster (same i tile) each gather 1/gather_cluster of
+                             // every P stage and copy it into the others' stages
     // control
     int *err_word;
     uint64_t timeout_ns;

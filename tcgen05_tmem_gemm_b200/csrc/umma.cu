@@ -59,8 +59,9 @@ __host__ __device__ inline SmemLayout smem_layout(int bn, int stages, bool gathe
     L.stage_bytes = L.p_bytes + L.q_bytes;  // a multiple of 1024: bn is a multiple of 8
     L.epi_off = L.stage_bytes * stages;
     L.bar_off = L.epi_off + (epi_tma ? kEpiStoreBytes : 0u);
-    // full[S], empty[S], tfull[2], tempty[2], drain, recv (split-K slices)
-    L.aux_off = L.bar_off + 8 * (2 * stages + 6);
+    // full[S], empty[S], part[S] (gather cluster), tfull[2], tempty[2], drain,
+    // recv (split-K slices)
+    L.aux_off = L.bar_off + 8 * (3 * stages + 6);
     uint32_t aux = 16;  // tmem base + abort flag
     if (gather) aux += 8 * kBM;  // row offsets of the tile
     L.total = L.aux_off + aux + 1024;  // + slack to align the base to 1024
@@ -85,8 +86,19 @@ struct TileCoord {
     int ti, tj, split;
 };
 
+// Unit u of the persistent schedule.  With split-K, the splits of a tile are
+// consecutive (one cluster).  With a gather cluster of G CTAs, u = g * G + r:
+// the G CTAs of a cluster take tiles (ti, jg * G + r) of group g, the same
+// rows of P.
 __device__ __forceinline__ TileCoord unit_coord(int u, const UmmaParams &p) {
     TileCoord c;
+    if (p.gather_cluster > 1) {
+        const int G = p.gather_cluster, g = u / G;
+        c.split = 0;
+        c.ti = g % p.tiles_i;
+        c.tj = (g / p.tiles_i) * G + u % G;
+        return c;
+    }
     c.split = u % p.split_k;
     const int t = u / p.split_k;
     c.ti = t % p.tiles_i;
@@ -263,7 +275,8 @@ __device__ __forceinline__ void gather_store(const GatherGeom &g, uint32_t p_sme
 // issued as asynchronous global -> shared copies (no register staging).
 template <int VB>
 __device__ __forceinline__ void gather_issue_async(const GatherSrc &src, const GatherGeom &g,
-                                                   const int64_t *row_off, int kbase, int first, uint32_t p_smem) {
+                                                   const int64_t *row_off, int kbase, int first, int uend,
+                                                   uint32_t p_smem) {
     const int nthreads = kGatherWarps * 32;
     const int step = nthreads / g.runs;
     const int fixed = (first % g.runs) * g.vec, moving0 = first / g.runs;
@@ -272,7 +285,7 @@ __device__ __forceinline__ void gather_issue_async(const GatherSrc &src, const G
 #pragma unroll
         for (int r = 0; r < kGatherUnroll; ++r) {
             const int u = first + r * nthreads;
-            if (u >= g.total) break;
+            if (u >= uend) break;
             const int k = moving0 + r * step, kg = kbase + k;
             const bool ok = ro >= 0 && kg < src.K;
             cp_async_zfill<VB>(p_smem + sw128_mnmajor(fixed * g.es, k, g.chunk_bytes),
@@ -284,7 +297,7 @@ __device__ __forceinline__ void gather_issue_async(const GatherSrc &src, const G
 #pragma unroll
         for (int r = 0; r < kGatherUnroll; ++r) {
             const int u = first + r * nthreads;
-            if (u >= g.total) break;
+            if (u >= uend) break;
             const int i = moving0 + r * step;
             const int64_t ro = row_off[i];
             const bool ok = ro >= 0 && co >= 0;
@@ -301,7 +314,8 @@ __device__ __forceinline__ void gather_issue_async(const GatherSrc &src, const G
 // warp is left waiting at their named barrier.
 template <int VB>
 __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayout &L, uint32_t sbase,
-                                            uint32_t bar_full, uint32_t bar_empty, int64_t *g_row_off,
+                                            uint32_t bar_full, uint32_t bar_empty, uint32_t bar_part,
+                                            int64_t *g_row_off,
                                             volatile int *abort_flag, const WaitCtl &wc, int bk, int es, int gtid,
                                             int lane) {
     using V = typename VecOf<VB>::T;
@@ -311,6 +325,12 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
     const bool stall = p.stall_loader != 0;
     const int nthreads = kGatherWarps * 32;
     const bool one_batch = VB < 4 && g.total <= nthreads * kGatherUnroll;  // register path look-ahead
+    // a gather cluster splits every stage's copies among its CTAs (cp.async
+    // path only); this CTA's copies complete on its part barrier
+    const int G = p.gather_cluster > 1 ? p.gather_cluster : 1;
+    const int grank = G > 1 ? (int)cluster_ctarank() : 0;
+    const int ubeg = grank * (g.total / G), uend = (grank + 1) * (g.total / G);
+    const uint32_t bar_done = G > 1 ? bar_part : bar_full;
     int it = 0;
     for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
         if (named_bar_or(*abort_flag != 0)) break;
@@ -335,9 +355,9 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
                 // asynchronous copies: the stage completes on the full barrier
                 // when they land, and this warp moves on at once
                 const uint32_t ps = sbase + s * L.stage_bytes;
-                for (int f = gtid; f < g.total; f += nthreads * kGatherUnroll)
-                    gather_issue_async<(VB >= 4 ? VB : 4)>(src, g, g_row_off, kb * bk, f, ps);
-                cp_async_arrive_noinc(bar_full + 8 * s);
+                for (int f = ubeg + gtid; f < uend; f += nthreads * kGatherUnroll)
+                    gather_issue_async<(VB >= 4 ? VB : 4)>(src, g, g_row_off, kb * bk, f, uend, ps);
+                cp_async_arrive_noinc(bar_done + 8 * s);
                 if (it < 16 && gtid == 0) trace_at(p, 37 + it);
             } else if (!stall) {
                 const uint32_t ps = sbase + s * L.stage_bytes;
@@ -381,7 +401,8 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_full = sbase + L.bar_off;
     const uint32_t bar_empty = bar_full + 8 * p.stages;
-    const uint32_t bar_tfull = bar_empty + 8 * p.stages;
+    const uint32_t bar_part = bar_empty + 8 * p.stages;
+    const uint32_t bar_tfull = bar_part + 8 * p.stages;
     const uint32_t bar_tempty = bar_tfull + 16;
     const uint32_t bar_drain = bar_tempty + 16;
     const uint32_t bar_recv = bar_drain + 8;
@@ -393,12 +414,18 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     constexpr int kEpiWarp0 = 2;
     const WaitCtl wc{abort_flag, p.err_word, p.timeout_ns};
 
+    const int G = GATHER && p.gather_cluster > 1 ? p.gather_cluster : 1;  // gather cluster size
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             // gather stages: one arrival per gather thread when its cp.async
-            // copies land (4..16-byte copies), else one per gather warp
-            mbar_init(bar_full + 8 * s, GATHER ? 1 + (p.gather_vec * (FP8 ? 1 : 2) >= 4 ? kGatherWarps * 32 : kGatherWarps) : 1);
-            mbar_init(bar_empty + 8 * s, 1);
+            // copies land (4..16-byte copies), else one per gather warp; with
+            // a gather cluster those land on the part barrier and the
+            // forwarding thread arrives once on the stage's full barrier
+            const int gather_arrivals = p.gather_vec * (FP8 ? 1 : 2) >= 4 ? kGatherWarps * 32 : kGatherWarps;
+            mbar_init(bar_full + 8 * s, GATHER ? 1 + (G > 1 ? 1 : gather_arrivals) : 1);
+            // a stage is free once every CTA of a gather cluster has consumed it
+            mbar_init(bar_empty + 8 * s, (uint32_t)G);
+            mbar_init(bar_part + 8 * s, (uint32_t)gather_arrivals);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_tfull + 8 * b, 1);
@@ -432,7 +459,8 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             int it = 0;  // global k-block counter across tiles
-            const uint32_t tx = (GATHER ? 0u : L.p_bytes) + L.q_bytes;
+            // gathered P: the parts of the other CTAs of a gather cluster arrive as bytes
+            const uint32_t tx = (GATHER ? (uint32_t)(G - 1) * (L.p_bytes / G) : L.p_bytes) + L.q_bytes;
             for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
                 const TileCoord tc = unit_coord(u, p);
                 const int kb0 = tc.split * p.kb_per_split;
@@ -473,6 +501,42 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                 if (p.stall_loader) break;
                 mbar_wait_drain(bar_full + 8 * (j % p.stages), (uint32_t)(j / p.stages) & 1u, p.timeout_ns);
             }
+        } else if (GATHER && G > 1 && lane == 1) {
+            // ---------------------------------------- gather-cluster forwarder
+            // Once this CTA's part of a stage has landed, copy it into the same
+            // stage of every other CTA of the cluster (their full barriers count
+            // the bytes), then count the part as arrived here.  The part: a k
+            // range in each 128-byte MN chunk (MN-major), or a row range.
+            const uint32_t grank = cluster_ctarank();
+            const bool mn = p.p_mn_major != 0;
+            const uint32_t part = L.p_bytes / (uint32_t)G;
+            const int nchunk = mn ? (kBM * es) / 128 : 1;
+            const uint32_t piece = part / (uint32_t)nchunk;
+            const uint32_t chunk_bytes = (uint32_t)bk * 128u;
+            const uint32_t first_off = mn ? grank * (uint32_t)(bk / G) * 128u : grank * part;
+            int it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                const TileCoord tc = unit_coord(u, p);
+                const int kb0 = tc.split * p.kb_per_split;
+                const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = it % p.stages;
+                    const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
+                    if (!mbar_wait(bar_part + 8 * s, ph, wc)) { ok = false; break; }
+                    fence_proxy_async_smem();  // cp.async writes -> bulk-copy reads
+                    const uint32_t ps = sbase + s * L.stage_bytes;
+                    for (int q = 1; q < G; ++q) {
+                        const uint32_t d = (grank + (uint32_t)q) % (uint32_t)G;
+                        const uint32_t rbar = dsmem_map(bar_full + 8 * s, d);
+                        for (int c = 0; c < nchunk; ++c) {
+                            const uint32_t off = (uint32_t)c * chunk_bytes + first_off;
+                            bulk_copy_to_cluster(dsmem_map(ps + off, d), ps + off, piece, rbar);
+                        }
+                    }
+                    mbar_arrive(bar_full + 8 * s);
+                }
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer
@@ -511,7 +575,10 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                         if (FP8) umma_f8(d_tmem, da, db, idesc, acc);
                         else umma_f16(d_tmem, da, db, idesc, acc);
                     }
-                    tc_commit(bar_empty + 8 * s);  // stage is free once these MMAs have read it
+                    // the stage is free once these MMAs have read it (in every
+                    // CTA of a gather cluster: they all write into it)
+                    if (G > 1) tc_commit_mc(bar_empty + 8 * s, (uint16_t)((1u << G) - 1u));
+                    else tc_commit(bar_empty + 8 * s);
                     if (it < 16) trace_at(p, 18 + it);
                 }
                 if (!ok) break;
@@ -608,11 +675,11 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         // ------------------------------------------------ gather producers
         const int gtid = threadIdx.x - (kEpiWarp0 + 4) * 32;
         switch (p.gather_vec * es) {
-        case 16: gather_role<16>(p, L, sbase, bar_full, bar_empty, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
-        case 8: gather_role<8>(p, L, sbase, bar_full, bar_empty, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
-        case 4: gather_role<4>(p, L, sbase, bar_full, bar_empty, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
-        case 2: gather_role<2>(p, L, sbase, bar_full, bar_empty, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
-        default: gather_role<1>(p, L, sbase, bar_full, bar_empty, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
+        case 16: gather_role<16>(p, L, sbase, bar_full, bar_empty, bar_part, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
+        case 8: gather_role<8>(p, L, sbase, bar_full, bar_empty, bar_part, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
+        case 4: gather_role<4>(p, L, sbase, bar_full, bar_empty, bar_part, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
+        case 2: gather_role<2>(p, L, sbase, bar_full, bar_empty, bar_part, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
+        default: gather_role<1>(p, L, sbase, bar_full, bar_empty, bar_part, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
         }
     }
 
@@ -821,6 +888,8 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     if (threadIdx.x == 0) trace_at(p, 36);
     tc_fence_before();
     __syncthreads();
+    // a gather cluster's CTAs copy into each other's shared memory: none leaves first
+    if (G > 1) cluster_sync();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
@@ -856,8 +925,9 @@ cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtens
         if (e != cudaSuccess) return e;
         lim.store((int)smem);
     }
-    return launch_ex(kern, dim3(grid), dim3(gather ? 448 : 192), smem, s, dim3(p.split_k, 1, 1), p.pdl, *tp, *tq,
-                     *tc, p);
+    const int cluster = p.split_k > 1 ? p.split_k : (gather && p.gather_cluster > 1 ? p.gather_cluster : 1);
+    return launch_ex(kern, dim3(grid), dim3(gather ? 448 : 192), smem, s, dim3(cluster, 1, 1), p.pdl, *tp, *tq, *tc,
+                     p);
 }
 
 }  // namespace dg

@@ -152,6 +152,13 @@ def test_plan_strided_gathers_a():
     assert pl["kind_name"] == "umma" and pl["p_gather"] == 1 and pl["swap_ab"] == 0
     assert pl["p_mn_major"] == 1 and pl["vec_bytes"] == 8
     assert pl["epi_tma_store"] == 1
+    # the four CTAs along N that need the same A tile share its gather
+    assert pl["block_n"] == 256 and pl["gather_cluster"] == 4 and pl["grid"] == 100
+    dg.dg_set_option(dg.DG_OPT_GATHER_CLUSTER, 0)
+    try:
+        assert plan_of("strided")["gather_cluster"] == 1
+    finally:
+        dg.dg_set_option(dg.DG_OPT_GATHER_CLUSTER, 1)
 
 
 def test_plan_edge_kinds():

@@ -30,6 +30,7 @@ def _reset_options():
     dg.dg_set_option(dg.DG_OPT_CTA_PAIR, 1)
     dg.dg_set_option(dg.DG_OPT_EARLY_LAUNCH, 0)
     dg.dg_set_option(dg.DG_OPT_EPI_TMA, 1)
+    dg.dg_set_option(dg.DG_OPT_GATHER_CLUSTER, 1)
 
 
 def expect_kind(p, kind, **fields):
@@ -189,6 +190,26 @@ def test_strided_nchw_gather(n, c, h, w, N):
     p = W.cfg_strided(n=n, c=c, h=h, w=w, N=N)
     expect_kind(p, "umma", p_gather=1, p_mn_major=1)
     check_full(p)
+
+
+@pytest.mark.parametrize("n,c,h,w,N,cluster", [(3, 72, 14, 14, 200, 2), (1, 256, 14, 14, 1024, 4),
+                                                (2, 40, 10, 10, 1024, 4), (4, 128, 6, 6, 512, 4),
+                                                (2, 64, 7, 2, 512, 4)])
+def test_strided_gather_cluster_matches_single_cta_gather(n, c, h, w, N, cluster):
+    # CTAs sharing an A tile each gather a k-slice of every stage and copy it
+    # to the others; the tensor core then reads the same bytes as when every
+    # CTA gathers the whole tile, so the outputs agree bit for bit.
+    g = torch.Generator().manual_seed(n * c + N)
+    x = W.cast(W.uniform((n, c, h, w), g), "bf16")
+    B = W.cast(W.uniform((c, N), g), "bf16")
+    p = W.Problem("nchw", W.nchw_as_rows(x, "bf16"), W.row_major(B, "bf16"), W.empty_out(n * h * w, N, "f32"))
+    outs = []
+    for on in (1, 0):
+        dg.dg_set_option(dg.DG_OPT_GATHER_CLUSTER, on)
+        expect_kind(p, "umma", p_gather=1, gather_cluster=cluster if on else 1)
+        check_full(p)
+        outs.append(c_matrix(run(p.to("cuda"))))
+    assert np.array_equal(outs[0], outs[1])
 
 
 def test_gemv_shapes():
