@@ -300,12 +300,12 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     const int blk = 128 / ces;  // columns per 128-byte block
     const bool epi_tma = g_epi_tma.load() != 0 && !swap && split == 1 && beta == 0.f && v.c.tma_ok &&
                          v.c.unit_dim == 1 && bn % blk == 0 && Nj >= blk && Mi >= 32;
-    const int stages = pair ? umma_pair_max_stages(bn, epi_tma) : umma_max_stages(bn, !p_tma, epi_tma);
+    int stages = pair ? umma_pair_max_stages(bn, epi_tma) : umma_max_stages(bn, !p_tma, epi_tma, (int)split);
     if (split > 1) {
-        // the split-K reduction stages a CTA's partial and the slices it
-        // receives in its operand ring
+        // the split-K reduction stages a CTA's partial in its operand ring
         const int64_t ring = (int64_t)stages * (128 * 128 + bn * 128);
-        if ((int64_t)umma_split_ring_bytes(bn, (int)split) > ring) {
+        if (stages < 3 || (int64_t)umma_split_out_bytes(bn, (int)split) > ring) {
+            stages = umma_max_stages(bn, !p_tma, epi_tma, 1);
             split = 1;
             kb_per = kb_total;
         }
@@ -344,7 +344,8 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
         in.grid = (int32_t)(2 * std::min<int64_t>(pair_units, num_sms / 2));
     }
     pl->fp8 = (dt == DG_E4M3);
-    pl->smem = pair ? umma_pair_smem_bytes(bn, stages, epi_tma) : umma_smem_bytes(bn, stages, !p_tma, epi_tma);
+    pl->smem = pair ? umma_pair_smem_bytes(bn, stages, epi_tma)
+                    : umma_smem_bytes(bn, stages, !p_tma, epi_tma, (int)split);
     return true;
 }
 

@@ -127,9 +127,9 @@ struct SimtParams {
 // tc: C's tensor map when p.epi_tma (otherwise not read)
 cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq, const CUtensorMap *tc,
                         bool fp8, bool gather, int grid, size_t smem, cudaStream_t s);
-size_t umma_smem_bytes(int bn, int stages, bool gather, bool epi_tma);
-int umma_max_stages(int bn, bool gather, bool epi_tma);
-uint32_t umma_split_ring_bytes(int bn, int split);  // ring bytes the split-K reduction needs
+size_t umma_smem_bytes(int bn, int stages, bool gather, bool epi_tma, int split);
+int umma_max_stages(int bn, bool gather, bool epi_tma, int split);
+uint32_t umma_split_out_bytes(int bn, int split);  // ring bytes a split-K partial is staged in
 cudaError_t launch_umma_pair(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq,
                              const CUtensorMap *tc, bool fp8, int grid, size_t smem, cudaStream_t s);
 size_t umma_pair_smem_bytes(int bn, int stages, bool epi_tma);

@@ -44,21 +44,36 @@ constexpr int kMaxSplit = 8;         // k splits of a tile: one portable cluster
 constexpr int kTileBytesK = 128;     // one swizzle row: 64 x 16-bit or 128 x 8-bit
 constexpr int kGatherWarps = 8;     // gather warps: cp.async latency-bound, so more warps keep more copies in flight
 
+// Split-K reduction: a CTA's partial is staged in its own operand ring (idle
+// once its main loop is done) as S slices of `slice` bytes from offset 0,
+// slice d holding the rows CTA d of the cluster owns (column-major); the
+// slices the other CTAs send it land in a region of its own (S slots, by
+// source rank), so they can arrive while its main loop still runs.
+__host__ __device__ inline uint32_t split_slice_bytes(int bn, int S) {
+    return (uint32_t)(bn * ((kBM + S - 1) / S) * 4);
+}
+__host__ __device__ inline uint32_t split_out_bytes(int bn, int S) { return S * split_slice_bytes(bn, S); }
+__host__ __device__ inline uint32_t split_in_bytes(int bn, int S) {
+    return S > 1 ? (S * split_slice_bytes(bn, S) + 1023u) & ~1023u : 0u;
+}
+
 struct SmemLayout {
     uint32_t stage_bytes, p_bytes, q_bytes;
     uint32_t epi_off;                // TMA-store epilogue blocks (epi_tma), after the stages
+    uint32_t recv_off;               // split-K slices received from the other CTAs
     uint32_t bar_off;
     uint32_t aux_off;                // tmem address, abort flag, gather tables
     uint32_t total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int bn, int stages, bool gather, bool epi_tma) {
+__host__ __device__ inline SmemLayout smem_layout(int bn, int stages, bool gather, bool epi_tma, int split) {
     SmemLayout L;
     L.p_bytes = kBM * kTileBytesK;
     L.q_bytes = (uint32_t)bn * kTileBytesK;
     L.stage_bytes = L.p_bytes + L.q_bytes;  // a multiple of 1024: bn is a multiple of 8
     L.epi_off = L.stage_bytes * stages;
-    L.bar_off = L.epi_off + (epi_tma ? kEpiStoreBytes : 0u);
+    L.recv_off = L.epi_off + (epi_tma ? kEpiStoreBytes : 0u);
+    L.bar_off = L.recv_off + split_in_bytes(bn, split);
     // full[S], empty[S], part[S] (gather cluster), tfull[2], tempty[2], drain,
     // recv (split-K slices)
     L.aux_off = L.bar_off + 8 * (3 * stages + 6);
@@ -66,20 +81,6 @@ __host__ __device__ inline SmemLayout smem_layout(int bn, int stages, bool gathe
     if (gather) aux += 8 * kBM;  // row offsets of the tile
     L.total = L.aux_off + aux + 1024;  // + slack to align the base to 1024
     return L;
-}
-
-// Split-K reduction inside the operand ring (idle by then): this CTA's
-// partial as S slices of `slice` bytes (slice d = the rows CTA d of the
-// cluster owns, column-major) from offset 0, then the slices received from
-// the other CTAs, by source rank, from split_in_offset.
-__host__ __device__ inline uint32_t split_slice_bytes(int bn, int S) {
-    return (uint32_t)(bn * ((kBM + S - 1) / S) * 4);
-}
-__host__ __device__ inline uint32_t split_in_offset(int bn, int S) {
-    return (S * split_slice_bytes(bn, S) + 1023u) & ~1023u;
-}
-__host__ __device__ inline uint32_t split_ring_bytes(int bn, int S) {
-    return split_in_offset(bn, S) + S * split_slice_bytes(bn, S);
 }
 
 struct TileCoord {
@@ -397,7 +398,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const SmemLayout L = smem_layout(p.bn, p.stages, GATHER, p.epi_tma != 0);
+    const SmemLayout L = smem_layout(p.bn, p.stages, GATHER, p.epi_tma != 0, p.split_k);
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_full = sbase + L.bar_off;
     const uint32_t bar_empty = bar_full + 8 * p.stages;
@@ -433,6 +434,9 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         }
         mbar_init(bar_drain, 1);
         mbar_init(bar_recv, 1);
+        // split-K: the slices of this CTA's rows from the other CTAs of the cluster
+        if (p.split_k > 1)
+            mbar_arrive_expect_tx(bar_recv, (uint32_t)(p.split_k - 1) * split_slice_bytes(p.bn, p.split_k));
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -446,6 +450,18 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     }
     tc_fence_before();
     __syncthreads();
+    // CTAs of a cluster write into each other's shared memory and barriers
+    // (split-K slices, gather-cluster parts and stage releases).  Every thread
+    // arrives on the cluster barrier once this CTA's barriers are initialised;
+    // a thread waits for it before its first access to another CTA, and at the
+    // latest before the next cluster barrier, so the start is not delayed.
+    // Cluster barrier operations are always issued by whole, converged warps.
+    const bool clustered = p.split_k > 1 || G > 1;
+    bool cluster_ready = !clustered;  // warp-uniform
+    if (clustered) {
+        __syncwarp();
+        cluster_arrive();
+    }
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     if (threadIdx.x == 0) trace_at(p, 1);
@@ -501,45 +517,16 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                 if (p.stall_loader) break;
                 mbar_wait_drain(bar_full + 8 * (j % p.stages), (uint32_t)(j / p.stages) & 1u, p.timeout_ns);
             }
-        } else if (GATHER && G > 1 && lane == 1) {
-            // ---------------------------------------- gather-cluster forwarder
-            // Once this CTA's part of a stage has landed, copy it into the same
-            // stage of every other CTA of the cluster (their full barriers count
-            // the bytes), then count the part as arrived here.  The part: a k
-            // range in each 128-byte MN chunk (MN-major), or a row range.
-            const uint32_t grank = cluster_ctarank();
-            const bool mn = p.p_mn_major != 0;
-            const uint32_t part = L.p_bytes / (uint32_t)G;
-            const int nchunk = mn ? (kBM * es) / 128 : 1;
-            const uint32_t piece = part / (uint32_t)nchunk;
-            const uint32_t chunk_bytes = (uint32_t)bk * 128u;
-            const uint32_t first_off = mn ? grank * (uint32_t)(bk / G) * 128u : grank * part;
-            int it = 0;
-            bool ok = true;
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-                const TileCoord tc = unit_coord(u, p);
-                const int kb0 = tc.split * p.kb_per_split;
-                const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
-                for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                    const int s = it % p.stages;
-                    const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
-                    if (!mbar_wait(bar_part + 8 * s, ph, wc)) { ok = false; break; }
-                    fence_proxy_async_smem();  // cp.async writes -> bulk-copy reads
-                    const uint32_t ps = sbase + s * L.stage_bytes;
-                    for (int q = 1; q < G; ++q) {
-                        const uint32_t d = (grank + (uint32_t)q) % (uint32_t)G;
-                        const uint32_t rbar = dsmem_map(bar_full + 8 * s, d);
-                        for (int c = 0; c < nchunk; ++c) {
-                            const uint32_t off = (uint32_t)c * chunk_bytes + first_off;
-                            bulk_copy_to_cluster(dsmem_map(ps + off, d), ps + off, piece, rbar);
-                        }
-                    }
-                    mbar_arrive(bar_full + 8 * s);
-                }
-            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer
+        if (G > 1) {
+            // the whole warp, converged: its stage releases and the forwarder's
+            // copies reach the other CTAs, whose barriers must be initialised
+            __syncwarp();
+            cluster_wait();
+            cluster_ready = true;
+        }
         if (lane == 0) {
             int it = 0, local = 0;
             const uint32_t idesc = p.idesc;
@@ -588,6 +575,42 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             // wait for every MMA this thread issued before TMEM can be freed
             tc_commit(bar_drain);
             mbar_wait_drain(bar_drain, 0, p.timeout_ns);
+        } else if (GATHER && G > 1 && lane == 1) {
+            // ---------------------------------------- gather-cluster forwarder
+            // Once this CTA's part of a stage has landed, copy it into the same
+            // stage of every other CTA of the cluster (their full barriers count
+            // the bytes), then count the part as arrived here.  The part: a k
+            // range in each 128-byte MN chunk (MN-major), or a row range.
+            const uint32_t grank = cluster_ctarank();
+            const bool mn = p.p_mn_major != 0;
+            const uint32_t part = L.p_bytes / (uint32_t)G;
+            const int nchunk = mn ? (kBM * es) / 128 : 1;
+            const uint32_t piece = part / (uint32_t)nchunk;
+            const uint32_t chunk_bytes = (uint32_t)bk * 128u;
+            const uint32_t first_off = mn ? grank * (uint32_t)(bk / G) * 128u : grank * part;
+            int it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                const TileCoord tc = unit_coord(u, p);
+                const int kb0 = tc.split * p.kb_per_split;
+                const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = it % p.stages;
+                    const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
+                    if (!mbar_wait(bar_part + 8 * s, ph, wc)) { ok = false; break; }
+                    fence_proxy_async_smem();  // cp.async writes -> bulk-copy reads
+                    const uint32_t ps = sbase + s * L.stage_bytes;
+                    for (int q = 1; q < G; ++q) {
+                        const uint32_t d = (grank + (uint32_t)q) % (uint32_t)G;
+                        const uint32_t rbar = dsmem_map(bar_full + 8 * s, d);
+                        for (int c = 0; c < nchunk; ++c) {
+                            const uint32_t off = (uint32_t)c * chunk_bytes + first_off;
+                            bulk_copy_to_cluster(dsmem_map(ps + off, d), ps + off, piece, rbar);
+                        }
+                    }
+                    mbar_arrive(bar_full + 8 * s);
+                }
+            }
         }
     } else if (warp < kEpiWarp0 + 4) {
         // ---------------------------------------------------------- epilogue
@@ -686,29 +709,31 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     if (p.split_k > 1) {
         // ------------------------------------------ cluster reduction of k splits
         // CTA s of the cluster owns rows [128 s / S, 128 (s+1) / S) of the
-        // tile.  After barrier 1 (every operand ring of the cluster idle) each
-        // CTA writes its partial from TMEM into its own ring as S slices, slice
-        // d holding the rows CTA d owns (column-major), and one thread copies
-        // every other slice into its owner's ring with a bulk shared-memory
-        // copy that completes on the owner's receive barrier.  An owner adds
-        // the S slices of its rows in rank order (its own slice stays local),
-        // so the sum is deterministic, and runs the epilogue.  Barrier 2 is
-        // arrived at once a CTA has received everything and waited on before
-        // exit: no CTA leaves while a copy out of its shared memory may still
-        // be reading.
+        // tile.  Once its own main loop is done (its ring is then idle), each
+        // CTA writes its partial from TMEM into its ring as S slices, slice d
+        // holding the rows CTA d owns (column-major), and one thread copies
+        // every other slice into its owner's receive region with a bulk
+        // shared-memory copy that completes on the owner's receive barrier.
+        // An owner adds the S slices of its rows in rank order (its own slice
+        // stays local), so the sum is deterministic, and runs the epilogue.  A
+        // cluster barrier, arrived at once a CTA has received everything and
+        // waited on before exit, keeps every CTA alive until all copies out of
+        // its shared memory have landed.
         const int S = p.split_k;
         const int rs_max = (kBM + S - 1) / S;
         const uint32_t slice = split_slice_bytes(p.bn, S);
         const uint32_t out_slices = sbase;
-        const uint32_t in_slices = sbase + split_in_offset(p.bn, S);
+        const uint32_t in_slices = sbase + L.recv_off;
         const uint32_t rank = cluster_ctarank();
         const bool epi_warp = warp >= kEpiWarp0 && warp < kEpiWarp0 + 4;
-        if (threadIdx.x == kEpiWarp0 * 32) mbar_arrive_expect_tx(bar_recv, (uint32_t)(S - 1) * slice);
-        tc_fence_before();
-        __syncthreads();
-        cluster_sync();  // barrier 1
         if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 54);
-        if (!epi_warp) cluster_arrive();  // barrier 2: nothing to receive here
+        // cluster barrier operations are issued by whole, converged warps
+        __syncwarp();
+        if (!cluster_ready) {
+            cluster_wait();  // every CTA of the cluster is initialised
+            cluster_ready = true;
+        }
+        if (!epi_warp) cluster_arrive();  // nothing to receive here
         if (epi_warp) {
             tc_fence_after();
             const int quarter = warp & 3;
@@ -740,6 +765,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                 trace_at(p, 59);
             }
             const bool received = mbar_wait(bar_recv, 0, wc);
+            __syncwarp();
             cluster_arrive();  // barrier 2: every copy into this CTA has landed
             if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 55);
             if (received) {
@@ -881,6 +907,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             }
         }
         if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 56);
+        __syncwarp();
         cluster_wait();  // barrier 2
     }
 
@@ -889,7 +916,11 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     tc_fence_before();
     __syncthreads();
     // a gather cluster's CTAs copy into each other's shared memory: none leaves first
-    if (G > 1) cluster_sync();
+    if (G > 1) {
+        __syncwarp();
+        if (!cluster_ready) cluster_wait();  // warp-uniform: warp 1 waited at its start
+        cluster_sync();
+    }
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
@@ -899,15 +930,15 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
 
 }  // namespace
 
-size_t umma_smem_bytes(int bn, int stages, bool gather, bool epi_tma) {
-    return smem_layout(bn, stages, gather, epi_tma).total;
+size_t umma_smem_bytes(int bn, int stages, bool gather, bool epi_tma, int split) {
+    return smem_layout(bn, stages, gather, epi_tma, split).total;
 }
 
-uint32_t umma_split_ring_bytes(int bn, int split) { return split_ring_bytes(bn, split); }
+uint32_t umma_split_out_bytes(int bn, int split) { return split_out_bytes(bn, split); }
 
-int umma_max_stages(int bn, bool gather, bool epi_tma) {
+int umma_max_stages(int bn, bool gather, bool epi_tma, int split) {
     int s = 2;
-    while (s < 12 && smem_layout(bn, s + 1, gather, epi_tma).total <= 227 * 1024) ++s;
+    while (s < 12 && smem_layout(bn, s + 1, gather, epi_tma, split).total <= 227 * 1024) ++s;
     return s;
 }
 
