@@ -738,8 +738,13 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             tc_fence_after();
             const int quarter = warp & 3;
             const int row = quarter * 32 + lane;
-            int d = 0;
-            while (d + 1 < S && (d + 1) * kBM / S <= row) ++d;
+            int d;  // owner of this row
+            if (kBM % S == 0) {
+                d = row / (kBM / S);
+            } else {
+                d = 0;
+                while (d + 1 < S && (d + 1) * kBM / S <= row) ++d;
+            }
             const int rl = row - d * kBM / S;
             const uint32_t dst = out_slices + (uint32_t)d * slice + (uint32_t)rl * 4u;
             const uint32_t col_pitch = (uint32_t)rs_max * 4u;
@@ -764,46 +769,78 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                 }
                 trace_at(p, 59);
             }
+            // the owner's rows: everything below except the slice sums needs
+            // nothing from the other CTAs
+            const EpiParams e = p.epi;  // a local copy: its fields stay in registers
+            const TileCoord tc = unit_coord(blockIdx.x, p);
+            const int r0 = (int)(rank * kBM / S), r1 = (int)((rank + 1) * kBM / S), rs = r1 - r0;
+            const int t = threadIdx.x - kEpiWarp0 * 32;
+            const int bn = p.bn, Mi = p.Mi, Nj = p.Nj;
+            const int i0 = tc.ti * kBM + r0, jt = tc.tj * bn;
+            const float alpha = e.alpha, beta = e.beta;
+            const float *const scale_i = e.scale_i, *const scale_j = e.scale_j;
+            char *const cbase = e.c;
+            const int64_t ci = e.ci, cj = e.cj;
+            const int cdt = e.c_dtype;
+            const bool vec4 = cdt == DG_F32 && ci == 4 && rs_max % 4 == 0 && rs % 4 == 0 && i0 % 4 == 0 &&
+                              cj % 16 == 0 && (reinterpret_cast<uintptr_t>(cbase) & 15) == 0;
+            constexpr int kB4 = 4;  // four-row groups per thread per batch (vector path)
+            const int g_rows = vec4 ? rs / 4 : 1;
+            // vector path: C of the first batch is loaded while the slices travel
+            float4 cfirst[kB4];
+#pragma unroll
+            for (int b = 0; b < kB4; ++b) cfirst[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (vec4 && beta != 0.f) {
+#pragma unroll
+                for (int b = 0; b < kB4; ++b) {
+                    const int g = t + b * 128;
+                    const int i = i0 + (g % g_rows) * 4, j = jt + g / g_rows;
+                    if (g < g_rows * bn && j < Nj && i + 3 < Mi)
+                        cfirst[b] = *reinterpret_cast<const float4 *>(cbase + (int64_t)i * 4 + (int64_t)j * cj);
+                }
+            }
             const bool received = mbar_wait(bar_recv, 0, wc);
             __syncwarp();
             cluster_arrive();  // barrier 2: every copy into this CTA has landed
             if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 55);
             if (received) {
-                const EpiParams e = p.epi;  // a local copy: its fields stay in registers
-                const TileCoord tc = unit_coord(blockIdx.x, p);
-                const int r0 = (int)(rank * kBM / S), r1 = (int)((rank + 1) * kBM / S), rs = r1 - r0;
-                const int t = threadIdx.x - kEpiWarp0 * 32;
-                const int bn = p.bn, Mi = p.Mi, Nj = p.Nj;
-                const int i0 = tc.ti * kBM + r0, jt = tc.tj * bn;
-                const float alpha = e.alpha, beta = e.beta;
-                const float *const scale_i = e.scale_i, *const scale_j = e.scale_j;
-                char *const cbase = e.c;
-                const int64_t ci = e.ci, cj = e.cj;
-                const int cdt = e.c_dtype;
                 // slice of source q: local for this CTA's own rank
                 uint32_t src[kMaxSplit];
 #pragma unroll
                 for (int q = 0; q < kMaxSplit; ++q)
                     src[q] = q == (int)rank ? out_slices + rank * slice : in_slices + (uint32_t)q * slice;
-                const bool vec4 = cdt == DG_F32 && ci == 4 && rs_max % 4 == 0 && rs % 4 == 0 && i0 % 4 == 0 &&
-                                  cj % 16 == 0 && (reinterpret_cast<uintptr_t>(cbase) & 15) == 0;
                 if (vec4) {
                     // four consecutive rows (contiguous in C and in a slice) per
                     // thread and step; consecutive threads take consecutive rows
-                    const int g_rows = rs / 4, total = g_rows * bn;
-                    constexpr int kB = 4;
+                    const int total = g_rows * bn;
+                    constexpr int kB = kB4;
+                    // group g = t + 128 n: row group g % g_rows, column g / g_rows,
+                    // advanced without division
+                    const int dgr = 128 % g_rows, dgc = 128 / g_rows;
+                    int gr = t % g_rows, gc = t / g_rows;
                     for (int base = t; base < total; base += 128 * kB) {
                         float4 cin[kB], acc[kB];
+                        int rr[kB], cc[kB];
 #pragma unroll
                         for (int b = 0; b < kB; ++b) {
                             const int g = base + b * 128;
-                            const int r = (g % g_rows) * 4, c = g / g_rows;
+                            const int r = gr * 4, c = gc;
+                            rr[b] = r;
+                            cc[b] = c;
+                            gr += dgr;
+                            gc += dgc;
+                            if (gr >= g_rows) {
+                                gr -= g_rows;
+                                ++gc;
+                            }
                             const int i = i0 + r, j = jt + c;
                             acc[b] = make_float4(0.f, 0.f, 0.f, 0.f);
                             cin[b] = acc[b];
                             if (g < total && j < Nj && i + 3 < Mi) {
                                 if (beta != 0.f)
-                                    cin[b] = *reinterpret_cast<const float4 *>(cbase + (int64_t)i * 4 + (int64_t)j * cj);
+                                    cin[b] = base == t ? cfirst[b]
+                                                       : *reinterpret_cast<const float4 *>(cbase + (int64_t)i * 4 +
+                                                                                          (int64_t)j * cj);
                                 const uint32_t off = (uint32_t)(c * rs_max + r) * 4u;
 #pragma unroll
                                 for (int q = 0; q < kMaxSplit; ++q) {
@@ -820,7 +857,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
 #pragma unroll
                         for (int b = 0; b < kB; ++b) {
                             const int g = base + b * 128;
-                            const int r = (g % g_rows) * 4, c = g / g_rows;
+                            const int r = rr[b], c = cc[b];
                             const int i = i0 + r, j = jt + c;
                             if (!(g < total && j < Nj && i < Mi)) continue;
                             const float sj = scale_j ? scale_j[j] : 1.f;
