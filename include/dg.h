@@ -184,7 +184,8 @@ typedef struct {
     int32_t gather_cluster;/* UMMA, gathered operand: CTAs per cluster that share each
                               gathered tile, each loading 1/gather_cluster of it and
                               copying it to the others (1 = no sharing)             */
-    int32_t reserved;
+    int32_t pair_half_tiles;/* UMMA, CTA pairs: tiles of the last, partial wave that run
+                              as two half-width tiles each                          */
 } dg_plan_info;
 
 /* The dispatch decision dg_gemm would take for these views (pointers are only
@@ -220,9 +221,11 @@ typedef enum {
     DG_OPT_EPI_TMA = 8,           /* 1 (default): tensor-core epilogues store C through
                                      tensor copies where the plan allows; 0: thread
                                      stores only                                        */
-    DG_OPT_GATHER_CLUSTER = 9     /* 1 (default): CTAs that need the same gathered
+    DG_OPT_GATHER_CLUSTER = 9,    /* 1 (default): CTAs that need the same gathered
                                      operand tile share the loads through distributed
                                      shared memory; 0: each gathers the whole tile      */
+    DG_OPT_PAIR_TAIL = 10         /* 1 (default): CTA pairs run the last, partial wave
+                                     of tiles as half-width tiles; 0: whole tiles only  */
 } dg_option;
 
 dg_status dg_set_option(int option, int64_t value);

@@ -29,7 +29,8 @@ ELEM_SIZE = {DG_F32: 4, DG_F16: 2, DG_BF16: 2, DG_E4M3: 1}
 KIND_NAME = {0: "none", 1: "scale_c", 2: "simt", 3: "gemv_n", 4: "gemv_k", 5: "umma"}
 
 (DG_OPT_FORCE_KIND, DG_OPT_WAIT_TIMEOUT_MS, DG_OPT_TEST_STALL, DG_OPT_MAX_SPLIT_K, DG_OPT_CTA_PAIR,
- DG_OPT_EARLY_LAUNCH, DG_OPT_TRACE, DG_OPT_EPI_TMA, DG_OPT_GATHER_CLUSTER) = 1, 2, 3, 4, 5, 6, 7, 8, 9
+ DG_OPT_EARLY_LAUNCH, DG_OPT_TRACE, DG_OPT_EPI_TMA, DG_OPT_GATHER_CLUSTER,
+ DG_OPT_PAIR_TAIL) = 1, 2, 3, 4, 5, 6, 7, 8, 9, 10
 
 
 class dg_view(ctypes.Structure):
@@ -65,7 +66,7 @@ class dg_plan_info(ctypes.Structure):
         ("vec_bytes", ctypes.c_int32),
         ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
         ("cta_pair", ctypes.c_int32), ("epi_tma_store", ctypes.c_int32),
-        ("gather_cluster", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("gather_cluster", ctypes.c_int32), ("pair_half_tiles", ctypes.c_int32),
     ]
 
     def as_dict(self) -> dict:

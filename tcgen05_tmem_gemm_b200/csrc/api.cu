@@ -36,6 +36,7 @@ std::atomic<int> g_pdl{0};
 std::atomic<uint64_t> g_trace{0};
 std::atomic<int> g_epi_tma{1};
 std::atomic<int> g_gather_cluster{1};
+std::atomic<int> g_pair_tail{1};
 std::atomic<uint32_t> g_epoch{1};  // bumped by every option change: cached launches go stale
 
 constexpr int kMaxDevices = 64;
@@ -290,7 +291,9 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     bool pair = false;
     if (pair_mode > 0 && p_tma && split == 1 && bn >= 128 && num_sms >= 2) {
         const int per = 128 / es;
-        const bool halves_ok = !q_mn || ((bn / 2) % per == 0);
+        // a CTA loads bn/2 columns of Q: whole 128-byte boxes (MN-major) or
+        // two boxes of bn/4 rows (K-major)
+        const bool halves_ok = q_mn ? ((bn / 2) % per == 0) : ((bn / 4) % 8 == 0);
         if (halves_ok) pair = (pair_mode == 2) || (Mi >= 256 && tiles >= num_sms);
     }
     // the epilogue stores C through tensor copies when C is row-major along j
@@ -341,7 +344,15 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     if (pair) {
         const int64_t pair_units = ((Mi + 255) / 256) * tiles_j;
         in.block_m = 256;
-        in.grid = (int32_t)(2 * std::min<int64_t>(pair_units, num_sms / 2));
+        const int64_t ncl = std::min<int64_t>(pair_units, num_sms / 2);
+        in.grid = (int32_t)(2 * ncl);
+        // the last, partial wave of tiles runs as half-width tiles (two per
+        // tile), so it takes half as long; a CTA then loads bn/4 columns of Q
+        const int per = 128 / es;
+        const bool quarter_ok = q_mn ? ((bn / 4) % per == 0) : ((bn / 4) % 8 == 0);
+        const int64_t tail = pair_units % ncl;
+        if (g_pair_tail.load() != 0 && quarter_ok && pair_units > ncl && tail > 0 && 2 * tail <= ncl)
+            in.pair_half_tiles = (int32_t)tail;
     }
     pl->fp8 = (dt == DG_E4M3);
     pl->smem = pair ? umma_pair_smem_bytes(bn, stages, epi_tma)
@@ -571,7 +582,8 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
             if (!ok) return DG_ERR_UNSUPPORTED;
         }
         {
-            const int q_rows = in.cta_pair ? bn / 2 : bn;  // a CTA of a pair loads half of the tile's columns
+            // a CTA of a pair loads half of a tile's columns, as boxes of bn/4 rows when K-major
+            const int q_rows = in.cta_pair ? bn / 4 : bn;
             const bool ok = in.q_mn_major ? encode_2d(&tq, dt, Qv->ptr, Nj, in.K, axis_stride(q_k), bk)
                                           : encode_2d(&tq, dt, Qv->ptr, in.K, Nj, axis_stride(q_j), q_rows);
             if (!ok) return DG_ERR_UNSUPPORTED;
@@ -598,6 +610,14 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         p.p_mn_major = in.p_mn_major;
         p.q_mn_major = in.q_mn_major;
         p.idesc = make_idesc(dt, in.p_mn_major, in.q_mn_major, bn, in.cta_pair ? 256 : 128);
+        p.full_units = p.num_units;
+        if (in.cta_pair) {
+            // whole 256-row tiles; the last in.pair_half_tiles of them as two halves each
+            const int32_t tiles = (int32_t)(((Mi + 255) / 256) * p.tiles_j);
+            p.full_units = tiles - in.pair_half_tiles;
+            p.num_units = p.full_units + 2 * in.pair_half_tiles;
+            p.idesc_half = make_idesc(dt, in.p_mn_major, in.q_mn_major, bn / 2, 256);
+        }
         int tc = 32;
         while (tc < 2 * bn) tc *= 2;
         p.tmem_cols = tc;
@@ -837,6 +857,10 @@ dg_status dg_set_option(int option, int64_t value) {
     case DG_OPT_GATHER_CLUSTER:
         if (value < 0 || value > 1) return DG_ERR_VALUE;
         g_gather_cluster.store((int)value);
+        return DG_OK;
+    case DG_OPT_PAIR_TAIL:
+        if (value < 0 || value > 1) return DG_ERR_VALUE;
+        g_pair_tail.store((int)value);
         return DG_OK;
     default: return DG_ERR_VALUE;
     }

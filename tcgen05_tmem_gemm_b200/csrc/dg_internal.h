@@ -89,6 +89,11 @@ struct UmmaParams {
     int32_t epi_tma;         // 1: the epilogue writes C through tensor stores (third map)
     int32_t gather_cluster;  // > 1: CTAs of a cluster (same i tile) each gather 1/gather_cluster of
                              // every P stage and copy it into the others' stages
+    // CTA pairs: units [0, full_units) are whole 256 x bn tiles; the tiles after
+    // them (the last, partial wave) run as two 256 x bn/2 units each, with
+    // instruction descriptor idesc_half
+    int32_t full_units;
+    uint32_t idesc_half;
     // control
     int *err_word;
     uint64_t timeout_ns;

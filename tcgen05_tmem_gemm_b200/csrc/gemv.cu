@@ -126,6 +126,7 @@ __host__ __device__ inline GemvNLayout gemv_n_layout(int R, int kper) {
 template <typename T, int R>
 __global__ void __launch_bounds__(kNT) gemv_n_kernel(const __grid_constant__ CUtensorMap tmap_w,
                                                      const GemvParams p) {
+    if (threadIdx.x == 0) tma_prefetch_desc(&tmap_w);  // the descriptor fetch overlaps the set-up
     pdl_wait();
     if (p.pdl == 1) pdl_release();
     extern __shared__ __align__(1024) uint8_t smem_raw[];

@@ -393,6 +393,12 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_c, const UmmaParams p) {
     if (threadIdx.x == 0) trace_at(p, 0);
+    if (threadIdx.x == 64) {
+        // descriptor fetches start at once, while thread 0 sets up the barriers
+        tma_prefetch_desc(&tmap_q);
+        if (!GATHER) tma_prefetch_desc(&tmap_p);
+        if (p.epi_tma) tma_prefetch_desc(&tmap_c);
+    }
     pdl_wait();
     if (p.pdl == 1) pdl_release();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -440,9 +446,6 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
-        tma_prefetch_desc(&tmap_q);
-        if (!GATHER) tma_prefetch_desc(&tmap_p);
-        if (p.epi_tma) tma_prefetch_desc(&tmap_c);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);

@@ -47,10 +47,37 @@ __host__ __device__ inline PairLayout pair_layout(int bn, int stages, bool epi_t
     return L;
 }
 
+// Unit u of the pair schedule: whole tiles first (column-major), then each
+// tile of the last, partial wave as two half-width units, so that the last
+// wave takes half as long.
+struct PairUnit {
+    int ti, j0, w;  // tile row, first column, columns
+};
+
+__device__ __forceinline__ PairUnit pair_unit(int u, const UmmaParams &p) {
+    PairUnit r;
+    int t = u, half = -1;
+    if (u >= p.full_units) {
+        t = p.full_units + (u - p.full_units) / 2;
+        half = (u - p.full_units) & 1;
+    }
+    r.ti = t % p.tiles_i;
+    const int tj = t / p.tiles_i;
+    r.w = half < 0 ? p.bn : p.bn / 2;
+    r.j0 = tj * p.bn + (half > 0 ? p.bn / 2 : 0);
+    return r;
+}
+
 template <bool FP8>
 __global__ void __launch_bounds__(192, 1)
     umma_pair_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_c, const UmmaParams p) {
+    if (threadIdx.x == 64) {
+        // descriptor fetches start at once, while thread 0 sets up the barriers
+        tma_prefetch_desc(&tmap_p);
+        tma_prefetch_desc(&tmap_q);
+        if (p.epi_tma) tma_prefetch_desc(&tmap_c);
+    }
     pdl_wait();
     if (p.pdl == 1) pdl_release();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -84,9 +111,6 @@ __global__ void __launch_bounds__(192, 1)
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
-        tma_prefetch_desc(&tmap_p);
-        tma_prefetch_desc(&tmap_q);
-        if (p.epi_tma) tma_prefetch_desc(&tmap_c);
     }
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
@@ -109,16 +133,18 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) {
             int it = 0;
             for (int u = cluster_id; u < p.num_units && !*abort_flag; u += nclusters) {
-                const int ti = u % p.tiles_i, tj = u / p.tiles_i;
-                const int i0 = ti * 2 * kHalfM + (int)rank * kHalfM;
-                const int j0 = tj * p.bn + (int)rank * half_bn;
+                const PairUnit pu = pair_unit(u, p);
+                const int i0 = pu.ti * 2 * kHalfM + (int)rank * kHalfM;
+                const int cw = pu.w / 2;  // this CTA's columns of the unit
+                const int j0 = pu.j0 + (int)rank * cw;
+                const uint32_t tx = 2u * (L.a_bytes + (uint32_t)cw * kRowBytes);  // both CTAs' bytes
                 for (int kb = 0; kb < p.kb_total; ++kb, ++it) {
                     const int s = it % p.stages;
                     const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
                     if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) break;
                     if (p.stall_loader) continue;
                     const uint32_t full_c = dsmem_map(bar_full + 8 * s, 0);
-                    if (leader) mbar_arrive_expect_tx(bar_full + 8 * s, 2 * L.stage_bytes);
+                    if (leader) mbar_arrive_expect_tx(bar_full + 8 * s, tx);
                     const uint32_t as = sbase + s * L.stage_bytes;
                     const uint32_t bs = as + L.a_bytes;
                     const int k0 = kb * bk;
@@ -129,10 +155,13 @@ __global__ void __launch_bounds__(192, 1)
                         tma_load_2d_pair(as, &tmap_p, full_c, k0, i0);
                     }
                     if (p.q_mn_major) {
-                        for (int c = 0; c < half_bn / per; ++c)
+                        for (int c = 0; c < cw / per; ++c)
                             tma_load_2d_pair(bs + c * bk * 128, &tmap_q, full_c, j0 + c * per, k0);
                     } else {
-                        tma_load_2d_pair(bs, &tmap_q, full_c, k0, j0);
+                        // boxes of bn/4 rows: two per CTA for a whole tile, one for a half
+                        for (int c = 0; c < cw / (half_bn / 2); ++c)
+                            tma_load_2d_pair(bs + c * (half_bn / 2) * kRowBytes, &tmap_q, full_c, k0,
+                                             j0 + c * (half_bn / 2));
                     }
                 }
             }
@@ -155,6 +184,7 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t q_kstep = p.q_mn_major ? kUmmaK * 128 : kUmmaK * es;
             bool ok = true;
             for (int u = cluster_id; u < p.num_units && ok; u += nclusters, ++local) {
+                const uint32_t idesc = u < p.full_units ? p.idesc : p.idesc_half;
                 const int b = local & 1;
                 const uint32_t tph = (uint32_t)(local >> 1) & 1u;
                 if (!mbar_wait(bar_tempty + 8 * b, tph ^ 1u, wc)) break;
@@ -172,8 +202,8 @@ __global__ void __launch_bounds__(192, 1)
                         const uint64_t da = make_sw128_desc(as + kk * p_kstep, p_lbo, 1024);
                         const uint64_t db = make_sw128_desc(bs + kk * q_kstep, q_lbo, 1024);
                         const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-                        if (FP8) umma_f8_pair(d_tmem, da, db, p.idesc, acc);
-                        else umma_f16_pair(d_tmem, da, db, p.idesc, acc);
+                        if (FP8) umma_f8_pair(d_tmem, da, db, idesc, acc);
+                        else umma_f16_pair(d_tmem, da, db, idesc, acc);
                     }
                     tc_commit_pair_mc(bar_empty + 8 * s, 0x3);  // the stage is free in both CTAs
                 }
@@ -192,27 +222,27 @@ __global__ void __launch_bounds__(192, 1)
         int local = 0;
         uint32_t nblk = 0;  // tensor-store blocks this warp has issued
         for (int u = cluster_id; u < p.num_units; u += nclusters, ++local) {
-            const int ti = u % p.tiles_i, tj = u / p.tiles_i;
+            const PairUnit pu = pair_unit(u, p);
             const int b = local & 1;
             const uint32_t tph = (uint32_t)(local >> 1) & 1u;
             if (!mbar_wait(bar_tfull + 8 * b, tph, wc)) break;
             tc_fence_after();
-            const int i = ti * 2 * kHalfM + (int)rank * kHalfM + row;
+            const int i = pu.ti * 2 * kHalfM + (int)rank * kHalfM + row;
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * p.bn);
-            const int j0 = tj * p.bn;
+            const int j0 = pu.j0;
             if (p.epi_tma) {
                 const uint32_t blocks = sbase + L.epi_off + (uint32_t)quarter * 2u * kEpiBlockBytes;
                 const int i_base = i - lane;
                 __syncwarp();
                 if (e.c_dtype == DG_F32)
-                    epilogue_rows_tma<4>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, p.bn, p.Nj, lane, nblk);
+                    epilogue_rows_tma<4>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, pu.w, p.Nj, lane, nblk);
                 else
-                    epilogue_rows_tma<2>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, p.bn, p.Nj, lane, nblk);
+                    epilogue_rows_tma<2>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, pu.w, p.Nj, lane, nblk);
             } else {
                 const bool row_ok = i < p.Mi;
                 const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
                 char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
-                for (int c0 = 0; c0 < p.bn; c0 += 16) {
+                for (int c0 = 0; c0 < pu.w; c0 += 16) {
                     uint32_t r[16];
                     __syncwarp();
                     tmem_ld16(t_row + c0, r);

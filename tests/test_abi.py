@@ -143,6 +143,8 @@ def test_plan_square_bf16_and_fp8():
     pl = plan_of("square_bf16", M=4096, N=4096, K=64)
     assert pl["kind_name"] == "umma" and pl["block_n"] == 256 and pl["grid"] == 148
     assert pl["cta_pair"] == 1 and pl["block_m"] == 256  # CTA pairs share 256-row tiles
+    # 256 tiles on 74 pairs: the last 34 run as half-width tiles
+    assert pl["pair_half_tiles"] == 34
     pl = plan_of("square_e4m3", M=4096, N=4096, K=64)
     assert pl["kind_name"] == "umma" and pl["block_k"] == 128 and pl["q_mn_major"] == 1
 
