@@ -422,6 +422,10 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     const WaitCtl wc{abort_flag, p.err_word, p.timeout_ns};
 
     const int G = GATHER && p.gather_cluster > 1 ? p.gather_cluster : 1;  // gather cluster size
+    // gather warps help the epilogue when every CTA has exactly one tile (their
+    // tensor-store blocks then live in the idle operand ring)
+    const bool helpers = GATHER && p.epi_tma && p.split_k == 1 && p.num_units == (int)gridDim.x &&
+                         L.stage_bytes * (uint32_t)p.stages >= (uint32_t)kGatherWarps * 2u * kEpiBlockBytes;
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             // gather stages: one arrival per gather thread when its cp.async
@@ -672,11 +676,13 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             if (p.epi_tma) {
                 const uint32_t blocks = sbase + L.epi_off + (uint32_t)quarter * 2u * kEpiBlockBytes;
                 const int i_base = tc.ti * kBM + quarter * 32;
+                // one tile per CTA with a gather: the gather warps share the strip
+                const int step = helpers ? 3 : 1;
                 __syncwarp();
                 if (e.c_dtype == DG_F32)
-                    epilogue_rows_tma<4>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, p.bn, p.Nj, lane, nblk);
+                    epilogue_rows_tma<4>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, p.bn, p.Nj, lane, nblk, 0, step);
                 else
-                    epilogue_rows_tma<2>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, p.bn, p.Nj, lane, nblk);
+                    epilogue_rows_tma<2>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, p.bn, p.Nj, lane, nblk, 0, step);
             } else {
                 const bool row_ok = i < p.Mi;
                 const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
@@ -706,6 +712,40 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         case 4: gather_role<4>(p, L, sbase, bar_full, bar_empty, bar_part, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
         case 2: gather_role<2>(p, L, sbase, bar_full, bar_empty, bar_part, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
         default: gather_role<1>(p, L, sbase, bar_full, bar_empty, bar_part, g_row_off, abort_flag, wc, bk, es, gtid, lane); break;
+        }
+        if (helpers) {
+            // ------------------------------ gather warps as epilogue helpers
+            // One tile per CTA: once its accumulator is ready, the operand ring
+            // is idle, so each gather warp takes a third of the column blocks
+            // of its TMEM lane quarter, staging its tensor stores in the ring.
+            const int hw = warp - (kEpiWarp0 + 4);  // 0..7
+            const int quarter = warp & 3;
+            const EpiParams e = p.epi;  // a local copy: its fields stay in registers
+            uint32_t nblk = 0;
+            // the ring is idle once every CTA that reads or writes it is done
+            // with its last use of each stage: the empty barriers count every
+            // MMA of a gather cluster, whose completion also means this CTA's
+            // parts have reached the other CTAs
+            bool ready = true;
+            const int kbn = p.kb_total;
+            for (int it = kbn > p.stages ? kbn - p.stages : 0; it < kbn && ready; ++it)
+                ready = mbar_wait(bar_empty + 8 * (it % p.stages), (uint32_t)(it / p.stages) & 1u, wc);
+            if (ready && mbar_wait(bar_tfull, 0u, wc)) {
+                tc_fence_after();
+                const TileCoord tc = unit_coord(blockIdx.x, p);
+                const uint32_t blocks = sbase + (uint32_t)hw * 2u * kEpiBlockBytes;
+                const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16);
+                const int i_base = tc.ti * kBM + quarter * 32, j0 = tc.tj * p.bn;
+                __syncwarp();
+                if (e.c_dtype == DG_F32)
+                    epilogue_rows_tma<4>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, p.bn, p.Nj, lane, nblk,
+                                         1 + hw / 4, 3);
+                else
+                    epilogue_rows_tma<2>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, p.bn, p.Nj, lane, nblk,
+                                         1 + hw / 4, 3);
+                tc_fence_before();
+            }
+            if (lane == 0) bulk_wait_all();
         }
     }
 

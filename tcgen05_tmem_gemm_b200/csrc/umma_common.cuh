@@ -105,10 +105,11 @@ constexpr uint32_t kEpiStoreBytes = 4 * 2 * kEpiBlockBytes;
 // so packing one overlaps the copy of the other.  `stage` is this warp's
 // 2 x kEpiBlockBytes (1024-byte aligned), `nblk` counts the blocks the warp
 // has issued; the caller waits for its copies (bulk_wait_all) before exit.
+// The warp stores 128-byte column blocks blk_first, blk_first + blk_step, ...
 template <int ES>
 __device__ __forceinline__ void epilogue_rows_tma(const EpiParams &e, const CUtensorMap *cmap, uint32_t stage,
                                                   uint32_t t_row, int i_base, int Mi, int j0, int bn, int Nj,
-                                                  int lane, uint32_t &nblk) {
+                                                  int lane, uint32_t &nblk, int blk_first = 0, int blk_step = 1) {
     constexpr int W = 128 / ES;  // output columns per block
     if (i_base >= Mi) return;    // the whole warp is below C (warp-uniform)
     // parameters in registers: nothing below re-reads the parameter block
@@ -116,7 +117,9 @@ __device__ __forceinline__ void epilogue_rows_tma(const EpiParams &e, const CUte
     const bool bf16_out = e.c_dtype == DG_BF16;
     const int i = i_base + lane;
     const float asi = i < Mi ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
-    for (int c0 = 0; c0 < bn && j0 + c0 < Nj; c0 += W) {
+    // blocks blk_first, blk_first + blk_step, ... of the row strip (warps that
+    // share TMEM lanes split a strip this way)
+    for (int c0 = blk_first * W; c0 < bn && j0 + c0 < Nj; c0 += blk_step * W) {
         uint32_t r[W];
 #pragma unroll
         for (int q = 0; q < W / 16; ++q)
