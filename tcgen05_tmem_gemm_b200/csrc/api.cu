@@ -270,6 +270,14 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
         bn = (int)(((bn + per - 1) / per) * per);
         if (bn > 256) return false;
     }
+    if (g_pair.load() != 2) {
+        // very few tiles: narrower ones put more SMs to work, each loading
+        // less of Q and storing less of C (not when CTA pairs are forced:
+        // they need tiles of 128 columns or more)
+        const int bn_min = q_mn ? 128 / es : 32;
+        while (bn / 2 >= bn_min && bn % 2 == 0 && tiles_i * ((Nj + bn / 2 - 1) / (bn / 2)) <= num_sms / 8)
+            bn /= 2;
+    }
     const int64_t tiles_j = (Nj + bn - 1) / bn;
     const int64_t tiles = tiles_i * tiles_j;
     const int64_t kb_total = (K + bk - 1) / bk;

@@ -125,9 +125,9 @@ def test_plan_decode_gemv():
 
 def test_plan_small_gemm_umma():
     pl = plan_of("small")
-    assert pl["kind_name"] == "umma" and pl["swap_ab"] == 0 and pl["block_n"] == 128
+    assert pl["kind_name"] == "umma" and pl["swap_ab"] == 0 and pl["block_n"] == 64  # two CTAs, not one
     assert pl["p_mn_major"] == 0 and pl["q_mn_major"] == 1 and pl["split_k"] == 1
-    assert pl["cta_pair"] == 0  # one tile: no pairing
+    assert pl["cta_pair"] == 0 and pl["grid"] == 2  # few tiles: no pairing
     assert pl["epi_tma_store"] == 1  # beta == 0, row-major FP32 C: tensor stores
 
 
