@@ -75,6 +75,21 @@ def test_umma_transposed_operands(ta, tb):
     check_full(p)
 
 
+@pytest.mark.parametrize("ta,pair", [(True, 0), (False, 0), (True, 2)])
+def test_umma_mn_major_chunk_boxes(ta, pair):
+    # MN-major operands in 128-byte chunk boxes whose last tiles run past M
+    # and N: the trailing boxes are partly or wholly outside the tensor (zero fill).
+    M, N, K = (1280, 320, 200) if pair == 0 else (320, 192, 200)
+    g = torch.Generator().manual_seed(320 + int(ta) + pair)
+    a = W.cast(W.uniform((K, M) if ta else (M, K), g), "bf16")
+    b = W.cast(W.uniform((K, N), g), "bf16")
+    A = W.transposed(a, "bf16") if ta else W.row_major(a, "bf16")
+    p = W.Problem("chunks3d", A, W.row_major(b, "bf16"), W.empty_out(M, N, "f32"))
+    dg.dg_set_option(dg.DG_OPT_CTA_PAIR, pair)
+    expect_kind(p, "umma", p_mn_major=int(ta), q_mn_major=1, cta_pair=int(pair == 2))
+    check_full(p)
+
+
 @pytest.mark.parametrize("M,N,K", [(300, 384, 272), (128, 128, 128), (77, 256, 512)])
 def test_umma_fp8_scaled(M, N, K):
     g = torch.Generator().manual_seed(M + N + K)
