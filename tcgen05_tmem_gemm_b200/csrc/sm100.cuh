@@ -215,10 +215,6 @@ __device__ __forceinline__ uint32_t dsmem_map(uint32_t smem_addr, uint32_t rank)
     return r;
 }
 
-__device__ __forceinline__ void dsmem_st_f32(uint32_t addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-
 __device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
     float v;
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");

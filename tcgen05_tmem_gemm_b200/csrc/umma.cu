@@ -15,18 +15,24 @@
 //  - warp 1: allocates TMEM (two accumulators of bn FP32 columns each), and one
 //    lane issues tcgen05.mma (128 x bn x 16 for 16-bit inputs, x32 for E4M3)
 //    and tcgen05.commit, which frees a stage once its MMAs have read it and
-//    signals a finished accumulator;
+//    signals a finished accumulator; with a gather cluster a second lane
+//    forwards this CTA's gathered parts to the other CTAs;
 //  - warps 2-5: the epilogue, each owning 32 TMEM lanes (rows): tcgen05.ld,
-//    scale, optional beta * C, convert and store, while the MMA warp already
-//    fills the other accumulator;
-//  - warps 6-13 (gather variant): thread loads of a P operand that TMA cannot
-//    describe (e.g. an NCHW feature map read as [N*H*W, C] with a 392-byte
-//    channel stride), written into the same swizzled layout
+//    scale, optional beta * C, convert, and tensor stores of 32-row x 128-byte
+//    blocks (or thread stores), while the MMA warp already fills the other
+//    accumulator;
+//  - warps 6-13 (gather variant): cp.async loads of a P operand that TMA
+//    cannot describe (e.g. an NCHW feature map read as [N*H*W, C] with a
+//    392-byte channel stride), written into the same swizzled layout
 //    ("DeepGEMM: a recalibration of the compute paradigm", §2.2: scatter-gather
-//    loads for the non-contiguous segments of a view).
-//  - split-K: partial tiles go to a workspace; per 32-row quarter the last
-//    arriving split adds the partials in split order (deterministic) and runs
-//    the epilogue ("DeepGEMM deep dive", §5.2).
+//    loads for the non-contiguous segments of a view).  The CTAs that need the
+//    same rows of P form a cluster and each gathers one k-slice of every stage,
+//    copied to the others through distributed shared memory.  With one tile
+//    per CTA these warps then take part of the epilogue;
+//  - split-K: the splits of a tile form a cluster; each CTA sends the rows
+//    other CTAs own from its partial into their shared memory, and each owner
+//    adds the slices in split order (deterministic) and runs the epilogue
+//    ("DeepGEMM deep dive", §5.2).  No global workspace.
 // Every wait is bounded (WaitCtl); on expiry the CTA records DG_ERR_TIMEOUT,
 // drains what it has in flight, frees TMEM and exits.
 #include <atomic>
