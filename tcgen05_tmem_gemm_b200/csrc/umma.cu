@@ -338,7 +338,8 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
     const int grank = G > 1 ? (int)cluster_ctarank() : 0;
     const int ubeg = grank * (g.total / G), uend = (grank + 1) * (g.total / G);
     const uint32_t bar_done = G > 1 ? bar_part : bar_full;
-    int it = 0;
+    int it = 0, gs = 0;
+    uint32_t gph = 0;
     for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
         if (named_bar_or(*abort_flag != 0)) break;
         const TileCoord tc = unit_coord(u, p);
@@ -353,8 +354,12 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
         V cur[kGatherUnroll], nxt[kGatherUnroll];
         if (one_batch && kb0 < kb1) gather_load<VB>(src, g, g_row_off, kb0 * bk, gtid, cur);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-            const int s = it % stages;
-            const uint32_t ph = (uint32_t)(it / stages) & 1u;
+            const int s = gs;
+            const uint32_t ph = gph;
+            if (++gs == stages) {  // stage and phase of the next k block, without division
+                gs = 0;
+                gph ^= 1u;
+            }
             if (one_batch && kb + 1 < kb1) gather_load<VB>(src, g, g_row_off, (kb + 1) * bk, gtid, nxt);
             ok = mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc);
             if (named_bar_or(!ok)) { ok = false; break; }
@@ -487,41 +492,54 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
-            int it = 0;  // global k-block counter across tiles
+            // everything the loop needs in registers (the copies' memory
+            // clobbers would otherwise make it re-read the parameters); stage
+            // and phase advance without division
+            const int stages = p.stages, num_units = p.num_units, kb_total = p.kb_total;
+            const int kb_per_split = p.kb_per_split, bn = p.bn;
+            const bool stall = p.stall_loader != 0, p_mn = p.p_mn_major != 0, q_mn = p.q_mn_major != 0;
+            const uint32_t stage_bytes = L.stage_bytes, p_bytes = L.p_bytes;
+            int it = 0, s = 0;  // global k-block counter across tiles, its stage
+            uint32_t ph = 0;
             // gathered P: the parts of the other CTAs of a gather cluster arrive as bytes
-            const uint32_t tx = (GATHER ? (uint32_t)(G - 1) * (L.p_bytes / G) : L.p_bytes) + L.q_bytes;
-            for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+            const uint32_t tx = (GATHER ? (uint32_t)(G - 1) * (p_bytes / G) : p_bytes) + L.q_bytes;
+            for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
                 const TileCoord tc = unit_coord(u, p);
-                const int kb0 = tc.split * p.kb_per_split;
-                const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+                const int kb0 = tc.split * kb_per_split;
+                const int kb1 = min(kb_total, kb0 + kb_per_split);
+                bool ok = true;
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                    const int s = it % p.stages;
-                    const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
-                    if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) break;
-                    if (p.stall_loader) continue;  // test hook: nothing arrives, consumers time out
-                    const uint32_t full = bar_full + 8 * s;
-                    mbar_arrive_expect_tx(full, tx);
-                    const uint32_t ps = sbase + s * L.stage_bytes;
-                    const uint32_t qs = ps + L.p_bytes;
-                    const int k0 = kb * bk;
-                    if (!GATHER) {
-                        if (p.p_mn_major) {
-                            const int per = 128 / es;  // i per box
-                            for (int c = 0; c < kBM / per; ++c)
-                                tma_load_2d(ps + c * bk * 128, &tmap_p, full, tc.ti * kBM + c * per, k0);
-                        } else {
-                            tma_load_2d(ps, &tmap_p, full, k0, tc.ti * kBM);
+                    if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) { ok = false; break; }
+                    if (!stall) {  // test hook: with stall nothing arrives, consumers time out
+                        const uint32_t full = bar_full + 8 * s;
+                        mbar_arrive_expect_tx(full, tx);
+                        const uint32_t ps = sbase + s * stage_bytes;
+                        const uint32_t qs = ps + p_bytes;
+                        const int k0 = kb * bk;
+                        if (!GATHER) {
+                            if (p_mn) {
+                                const int per = 128 / es;  // i per box
+                                for (int c = 0; c < kBM / per; ++c)
+                                    tma_load_2d(ps + c * bk * 128, &tmap_p, full, tc.ti * kBM + c * per, k0);
+                            } else {
+                                tma_load_2d(ps, &tmap_p, full, k0, tc.ti * kBM);
+                            }
                         }
+                        if (q_mn) {
+                            const int per = 128 / es;
+                            for (int c = 0; c < bn / per; ++c)
+                                tma_load_2d(qs + c * q_box_bytes, &tmap_q, full, tc.tj * bn + c * per, k0);
+                        } else {
+                            tma_load_2d(qs, &tmap_q, full, k0, tc.tj * bn);
+                        }
+                        if (it < 16) trace_at(p, 2 + it);
                     }
-                    if (p.q_mn_major) {
-                        const int per = 128 / es;
-                        for (int c = 0; c < p.bn / per; ++c)
-                            tma_load_2d(qs + c * q_box_bytes, &tmap_q, full, tc.tj * p.bn + c * per, k0);
-                    } else {
-                        tma_load_2d(qs, &tmap_q, full, k0, tc.tj * p.bn);
+                    if (++s == stages) {
+                        s = 0;
+                        ph ^= 1u;
                     }
-                    if (it < 16) trace_at(p, 2 + it);
                 }
+                if (!ok) break;
             }
             // let the copies already issued land before the CTA can exit
             const int last = it;
@@ -541,45 +559,54 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             cluster_ready = true;
         }
         if (lane == 0) {
-            int it = 0, local = 0;
-            const uint32_t idesc = p.idesc;
+            const int stages = p.stages, num_units = p.num_units, kb_total = p.kb_total;
+            const int kb_per_split = p.kb_per_split, bn = p.bn;
+            const uint32_t idesc = p.idesc, stage_bytes = L.stage_bytes;
             // descriptor strides: K-major tiles step 1024 B per 8 rows; MN-major
             // tiles step 1024 B per 8 k and one 128-byte MN chunk per bk*128 B.
             const uint32_t p_lbo = p.p_mn_major ? (uint32_t)(bk * 128) : 16u;
             const uint32_t q_lbo = p.q_mn_major ? (uint32_t)(bk * 128) : 16u;
             const uint32_t p_kstep = p.p_mn_major ? kUmmaK * 128 : kUmmaK * es;
             const uint32_t q_kstep = p.q_mn_major ? kUmmaK * 128 : kUmmaK * es;
+            // descriptors of stage 0; a stage's differ only in the start address
+            // field (address >> 4, below 2^14 for any shared-memory address)
+            const uint64_t da0 = make_sw128_desc(sbase, p_lbo, 1024);
+            const uint64_t db0 = make_sw128_desc(sbase + L.p_bytes, q_lbo, 1024);
+            const uint16_t cl_mask = (uint16_t)((1u << G) - 1u);
+            int it = 0, local = 0, s = 0;
+            uint32_t ph = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++local) {
+            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++local) {
                 const TileCoord tc = unit_coord(u, p);
-                const int kb0 = tc.split * p.kb_per_split;
-                const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+                const int kb0 = tc.split * kb_per_split;
+                const int kb1 = min(kb_total, kb0 + kb_per_split);
                 const int b = local & 1;
                 const uint32_t tph = (uint32_t)(local >> 1) & 1u;
                 if (!mbar_wait(bar_tempty + 8 * b, tph ^ 1u, wc)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(b * p.bn);
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * bn);
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                    const int s = it % p.stages;
-                    const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
                     if (!mbar_wait(bar_full + 8 * s, ph, wc)) { ok = false; break; }
                     tc_fence_after();
                     if (GATHER) fence_proxy_async_smem();  // thread-written P stage -> tensor-core reads
-                    const uint32_t ps = sbase + s * L.stage_bytes;
-                    const uint32_t qs = ps + L.p_bytes;
+                    const uint64_t soff = (uint64_t)((s * stage_bytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < kTileBytesK / (kUmmaK * es); ++kk) {
-                        const uint64_t da = make_sw128_desc(ps + kk * p_kstep, p_lbo, 1024);
-                        const uint64_t db = make_sw128_desc(qs + kk * q_kstep, q_lbo, 1024);
+                        const uint64_t da = da0 + soff + (uint64_t)((kk * p_kstep) >> 4);
+                        const uint64_t db = db0 + soff + (uint64_t)((kk * q_kstep) >> 4);
                         const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
                         if (FP8) umma_f8(d_tmem, da, db, idesc, acc);
                         else umma_f16(d_tmem, da, db, idesc, acc);
                     }
                     // the stage is free once these MMAs have read it (in every
                     // CTA of a gather cluster: they all write into it)
-                    if (G > 1) tc_commit_mc(bar_empty + 8 * s, (uint16_t)((1u << G) - 1u));
+                    if (G > 1) tc_commit_mc(bar_empty + 8 * s, cl_mask);
                     else tc_commit(bar_empty + 8 * s);
                     if (it < 16) trace_at(p, 18 + it);
+                    if (++s == stages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (!ok) break;
                 tc_commit(bar_tfull + 8 * b);      // accumulator b is complete
@@ -601,15 +628,21 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             const uint32_t piece = part / (uint32_t)nchunk;
             const uint32_t chunk_bytes = (uint32_t)bk * 128u;
             const uint32_t first_off = mn ? grank * (uint32_t)(bk / G) * 128u : grank * part;
-            int it = 0;
+            const int stages = p.stages;
+            int fs = 0;  // stage and phase, advanced without division
+            uint32_t fph = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
                 const TileCoord tc = unit_coord(u, p);
                 const int kb0 = tc.split * p.kb_per_split;
                 const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
-                for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                    const int s = it % p.stages;
-                    const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    const int s = fs;
+                    const uint32_t ph = fph;
+                    if (++fs == stages) {
+                        fs = 0;
+                        fph ^= 1u;
+                    }
                     if (!mbar_wait(bar_part + 8 * s, ph, wc)) { ok = false; break; }
                     fence_proxy_async_smem();  // cp.async writes -> bulk-copy reads
                     const uint32_t ps = sbase + s * L.stage_bytes;

@@ -131,39 +131,51 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
-            int it = 0;
-            for (int u = cluster_id; u < p.num_units && !*abort_flag; u += nclusters) {
+            // everything the loop needs in registers: the asynchronous copies
+            // (memory clobbers) would otherwise make it re-read the parameters,
+            // and stage and phase advance without division
+            const int stages = p.stages, kb_total = p.kb_total, num_units = p.num_units;
+            const bool stall = p.stall_loader != 0, p_mn = p.p_mn_major != 0, q_mn = p.q_mn_major != 0;
+            const uint32_t stage_bytes = L.stage_bytes, a_bytes = L.a_bytes;
+            int it = 0, s = 0;
+            uint32_t ph = 0;
+            for (int u = cluster_id; u < num_units && !*abort_flag; u += nclusters) {
                 const PairUnit pu = pair_unit(u, p);
                 const int i0 = pu.ti * 2 * kHalfM + (int)rank * kHalfM;
                 const int cw = pu.w / 2;  // this CTA's columns of the unit
                 const int j0 = pu.j0 + (int)rank * cw;
-                const uint32_t tx = 2u * (L.a_bytes + (uint32_t)cw * kRowBytes);  // both CTAs' bytes
-                for (int kb = 0; kb < p.kb_total; ++kb, ++it) {
-                    const int s = it % p.stages;
-                    const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
-                    if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) break;
-                    if (p.stall_loader) continue;
-                    const uint32_t full_c = dsmem_map(bar_full + 8 * s, 0);
-                    if (leader) mbar_arrive_expect_tx(bar_full + 8 * s, tx);
-                    const uint32_t as = sbase + s * L.stage_bytes;
-                    const uint32_t bs = as + L.a_bytes;
-                    const int k0 = kb * bk;
-                    if (p.p_mn_major) {
-                        for (int c = 0; c < kHalfM / per; ++c)
-                            tma_load_2d_pair(as + c * bk * 128, &tmap_p, full_c, i0 + c * per, k0);
-                    } else {
-                        tma_load_2d_pair(as, &tmap_p, full_c, k0, i0);
+                const uint32_t tx = 2u * (a_bytes + (uint32_t)cw * kRowBytes);  // both CTAs' bytes
+                bool ok = true;
+                for (int kb = 0; kb < kb_total; ++kb, ++it) {
+                    if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) { ok = false; break; }
+                    if (!stall) {
+                        const uint32_t full_c = dsmem_map(bar_full + 8 * s, 0);
+                        if (leader) mbar_arrive_expect_tx(bar_full + 8 * s, tx);
+                        const uint32_t as = sbase + s * stage_bytes;
+                        const uint32_t bs = as + a_bytes;
+                        const int k0 = kb * bk;
+                        if (p_mn) {
+                            for (int c = 0; c < kHalfM / per; ++c)
+                                tma_load_2d_pair(as + c * bk * 128, &tmap_p, full_c, i0 + c * per, k0);
+                        } else {
+                            tma_load_2d_pair(as, &tmap_p, full_c, k0, i0);
+                        }
+                        if (q_mn) {
+                            for (int c = 0; c < cw / per; ++c)
+                                tma_load_2d_pair(bs + c * bk * 128, &tmap_q, full_c, j0 + c * per, k0);
+                        } else {
+                            // boxes of bn/4 rows: two per CTA for a whole tile, one for a half
+                            for (int c = 0; c < cw / (half_bn / 2); ++c)
+                                tma_load_2d_pair(bs + c * (half_bn / 2) * kRowBytes, &tmap_q, full_c, k0,
+                                                 j0 + c * (half_bn / 2));
+                        }
                     }
-                    if (p.q_mn_major) {
-                        for (int c = 0; c < cw / per; ++c)
-                            tma_load_2d_pair(bs + c * bk * 128, &tmap_q, full_c, j0 + c * per, k0);
-                    } else {
-                        // boxes of bn/4 rows: two per CTA for a whole tile, one for a half
-                        for (int c = 0; c < cw / (half_bn / 2); ++c)
-                            tma_load_2d_pair(bs + c * (half_bn / 2) * kRowBytes, &tmap_q, full_c, k0,
-                                             j0 + c * (half_bn / 2));
+                    if (++s == stages) {
+                        s = 0;
+                        ph ^= 1u;
                     }
                 }
+                if (!ok) break;
             }
             if (!leader) pdl_release();
             // full[] of the even CTA counts both CTAs' bytes: once its last
@@ -177,35 +189,44 @@ __global__ void __launch_bounds__(192, 1)
     } else if (warp == 1) {
         // ----------------------------------------- MMA issuer (even CTA only)
         if (lane == 0 && leader) {
-            int it = 0, local = 0;
+            const int stages = p.stages, kb_total = p.kb_total, num_units = p.num_units;
+            const int full_units = p.full_units, bn = p.bn;
+            const uint32_t idesc_full = p.idesc, idesc_half = p.idesc_half, stage_bytes = L.stage_bytes;
             const uint32_t p_lbo = p.p_mn_major ? (uint32_t)(bk * 128) : 16u;
             const uint32_t q_lbo = p.q_mn_major ? (uint32_t)(bk * 128) : 16u;
             const uint32_t p_kstep = p.p_mn_major ? kUmmaK * 128 : kUmmaK * es;
             const uint32_t q_kstep = p.q_mn_major ? kUmmaK * 128 : kUmmaK * es;
+            // descriptors of stage 0; a stage's differ only in the start address
+            // field (address >> 4, below 2^14 for any shared-memory address)
+            const uint64_t da0 = make_sw128_desc(sbase, p_lbo, 1024);
+            const uint64_t db0 = make_sw128_desc(sbase + L.a_bytes, q_lbo, 1024);
+            int local = 0, s = 0;
+            uint32_t ph = 0;
             bool ok = true;
-            for (int u = cluster_id; u < p.num_units && ok; u += nclusters, ++local) {
-                const uint32_t idesc = u < p.full_units ? p.idesc : p.idesc_half;
+            for (int u = cluster_id; u < num_units && ok; u += nclusters, ++local) {
+                const uint32_t idesc = u < full_units ? idesc_full : idesc_half;
                 const int b = local & 1;
                 const uint32_t tph = (uint32_t)(local >> 1) & 1u;
                 if (!mbar_wait(bar_tempty + 8 * b, tph ^ 1u, wc)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(b * p.bn);
-                for (int kb = 0; kb < p.kb_total; ++kb, ++it) {
-                    const int s = it % p.stages;
-                    const uint32_t ph = (uint32_t)(it / p.stages) & 1u;
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * bn);
+                for (int kb = 0; kb < kb_total; ++kb) {
                     if (!mbar_wait(bar_full + 8 * s, ph, wc)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t as = sbase + s * L.stage_bytes;
-                    const uint32_t bs = as + L.a_bytes;
+                    const uint64_t soff = (uint64_t)((s * stage_bytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < kRowBytes / (kUmmaK * es); ++kk) {
-                        const uint64_t da = make_sw128_desc(as + kk * p_kstep, p_lbo, 1024);
-                        const uint64_t db = make_sw128_desc(bs + kk * q_kstep, q_lbo, 1024);
+                        const uint64_t da = da0 + soff + (uint64_t)((kk * p_kstep) >> 4);
+                        const uint64_t db = db0 + soff + (uint64_t)((kk * q_kstep) >> 4);
                         const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
                         if (FP8) umma_f8_pair(d_tmem, da, db, idesc, acc);
                         else umma_f16_pair(d_tmem, da, db, idesc, acc);
                     }
                     tc_commit_pair_mc(bar_empty + 8 * s, 0x3);  // the stage is free in both CTAs
+                    if (++s == stages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (!ok) break;
                 tc_commit_pair_mc(bar_tfull + 8 * b, 0x3);       // both halves of the accumulator are ready
