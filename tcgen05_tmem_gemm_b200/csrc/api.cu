@@ -197,10 +197,10 @@ void gemv_n_split(int64_t M, int64_t N, int64_t K, int num_sms, dg_plan_info *in
     int64_t S = (2 * num_sms + gx / 2) / gx;
     S = std::max<int64_t>(1, std::min<int64_t>(S, kMaxCluster));
     S = std::min<int64_t>(S, std::max<int64_t>(1, K / 64));
-    int64_t kper = ((K + S - 1) / S + 31) / 32 * 32;
+    int64_t kper = ((K + S - 1) / S + 63) / 64 * 64;
     while (kper * r_inst > 16384 && S < kMaxCluster) {
         ++S;
-        kper = ((K + S - 1) / S + 31) / 32 * 32;
+        kper = ((K + S - 1) / S + 63) / 64 * 64;
     }
     S = (K + kper - 1) / kper;
     in->block_n = 256;
@@ -564,7 +564,7 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
                     (v.a.row.n == 0 || p.x_ld % 16 == 0);
         if (in.kind == DG_KIND_GEMV_N) {
             p.kper = in.block_k;
-            if (!encode_2d_box(&rec->t0, v.B->dtype, v.B->ptr, in.N, in.K, p.w_ld, 256, 32, false))
+            if (!encode_2d_box(&rec->t0, v.B->dtype, v.B->ptr, in.N, in.K, p.w_ld, 256, 64, false))
                 return DG_ERR_UNSUPPORTED;
         }
         rec->gemv = p;

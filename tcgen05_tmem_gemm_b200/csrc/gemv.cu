@@ -32,11 +32,11 @@ namespace dg {
 namespace {
 
 constexpr int kNB = 256;        // columns per gemv_n block
-constexpr int kRows = 32;       // rows of W per TMA stage
-constexpr int kStages = 6;      // ring depth
+constexpr int kRows = 64;       // rows of W per TMA stage (one 32 KB box: a TMA unit's byte rate grows with box size)
+constexpr int kStages = 3;      // ring depth
 constexpr int kCW = 8;          // consumer warps
 constexpr int kNT = 32 * (kCW + 1);
-constexpr int kReleaseStages = 6;  // dependents are released this many stages before the end
+constexpr int kReleaseStages = 3;  // dependents are released this many stages before the end
 
 template <typename T>
 __device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8]);
