@@ -281,39 +281,53 @@ __global__ void __launch_bounds__(256) gemv_k_kernel(const GemvParams p) {
     const int kq = ((p.K / 8 + WPC - 1) / WPC) * 8;
     const int ka = q * kq, kb = min(p.K, ka + kq);
 
+    // the first batch of this warp's W loads goes out before x is staged, so
+    // the two round trips to memory overlap
+    const int kfirst = ka + lane * 8;
+    uint4 vfirst[MAXV];
+#pragma unroll
+    for (int u = 0; u < MAXV; ++u) {
+        const int k = kfirst + u * 256;
+        vfirst[u] = (col_ok && k < kb) ? ldg_stream(wrow + (int64_t)k * sizeof(T)) : make_uint4(0, 0, 0, 0);
+    }
     stage_x<T, R>(xs, p.K, p, 0, p.K, threadIdx.x, 256);
     __syncthreads();
     float acc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r] = 0.f;
+    // one batch of MAXV 16-byte loads per lane: the first was issued above
+    auto consume = [&](int k0, const uint4 (&v)[MAXV]) {
+#pragma unroll
+        for (int u = 0; u < MAXV; ++u) {
+            const int k = k0 + u * 256;
+            if (k >= kb) break;
+            float f[8];
+            unpack8<T>(v[u], f);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float4 x0 = *reinterpret_cast<const float4 *>(xs + r * p.K + k);
+                const float4 x1 = *reinterpret_cast<const float4 *>(xs + r * p.K + k + 4);
+                acc[r] = fmaf(x0.x, f[0], acc[r]);
+                acc[r] = fmaf(x0.y, f[1], acc[r]);
+                acc[r] = fmaf(x0.z, f[2], acc[r]);
+                acc[r] = fmaf(x0.w, f[3], acc[r]);
+                acc[r] = fmaf(x1.x, f[4], acc[r]);
+                acc[r] = fmaf(x1.y, f[5], acc[r]);
+                acc[r] = fmaf(x1.z, f[6], acc[r]);
+                acc[r] = fmaf(x1.w, f[7], acc[r]);
+            }
+        }
+    };
     if (col_ok) {
-        for (int k0 = ka + lane * 8; k0 < kb; k0 += 32 * 8 * MAXV) {
+        consume(kfirst, vfirst);
+        for (int k0 = kfirst + 32 * 8 * MAXV; k0 < kb; k0 += 32 * 8 * MAXV) {
             uint4 v[MAXV];
 #pragma unroll
             for (int u = 0; u < MAXV; ++u) {
                 const int k = k0 + u * 256;
                 v[u] = (k < kb) ? ldg_stream(wrow + (int64_t)k * sizeof(T)) : make_uint4(0, 0, 0, 0);
             }
-#pragma unroll
-            for (int u = 0; u < MAXV; ++u) {
-                const int k = k0 + u * 256;
-                if (k >= kb) break;
-                float f[8];
-                unpack8<T>(v[u], f);
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const float4 x0 = *reinterpret_cast<const float4 *>(xs + r * p.K + k);
-                    const float4 x1 = *reinterpret_cast<const float4 *>(xs + r * p.K + k + 4);
-                    acc[r] = fmaf(x0.x, f[0], acc[r]);
-                    acc[r] = fmaf(x0.y, f[1], acc[r]);
-                    acc[r] = fmaf(x0.z, f[2], acc[r]);
-                    acc[r] = fmaf(x0.w, f[3], acc[r]);
-                    acc[r] = fmaf(x1.x, f[4], acc[r]);
-                    acc[r] = fmaf(x1.y, f[5], acc[r]);
-                    acc[r] = fmaf(x1.z, f[6], acc[r]);
-                    acc[r] = fmaf(x1.w, f[7], acc[r]);
-                }
-            }
+            consume(k0, v);
         }
     }
 #pragma unroll
