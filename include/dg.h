@@ -213,8 +213,10 @@ typedef enum {
                                      operands allow                                    */
     DG_OPT_EARLY_LAUNCH = 6,      /* programmatic dependent launch: 0 off, 1 release the
                                      next kernel at the start of each kernel, 2 release
-                                     it near the end of long kernels; default 0: it did
-                                     not shorten back-to-back decode steps             */
+                                     it near the end of long kernels, 3 (default) only
+                                     for the K-contiguous GEMV, whose 64 blocks leave
+                                     room for the next launch (1 and 2 slowed the
+                                     decode step: two W-streaming blocks fill an SM)   */
     DG_OPT_TRACE = 7,             /* device address of 64 uint64 slots (0 = off): the
                                      single-CTA tensor-core kernel's CTA 0 writes
                                      %globaltimer at its phase boundaries (analysis)   */

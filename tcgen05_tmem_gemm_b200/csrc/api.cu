@@ -32,7 +32,7 @@ std::atomic<int64_t> g_timeout_ms{2000};
 std::atomic<int> g_stall{0};
 std::atomic<int> g_max_split{8};
 std::atomic<int> g_pair{1};
-std::atomic<int> g_pdl{0};
+std::atomic<int> g_pdl{3};
 std::atomic<uint64_t> g_trace{0};
 std::atomic<int> g_epi_tma{1};
 std::atomic<int> g_gather_cluster{1};
@@ -520,7 +520,10 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
                   DeviceState *ds, LaunchRec *rec) {
     const dg_plan_info &in = pl.info;
     rec->kind = in.kind;
-    rec->pdl = g_pdl.load();
+    // early launch: mode 3 uses it for the launch-bound K-contiguous GEMV only
+    // (64 blocks: the next launch finds free SMs while it runs)
+    const int pdl_mode = g_pdl.load();
+    rec->pdl = pdl_mode == 3 ? (in.kind == DG_KIND_GEMV_K ? 1 : 0) : pdl_mode;
     switch (in.kind) {
     case DG_KIND_NONE: return DG_OK;
     case DG_KIND_SCALE_C: {
@@ -847,7 +850,7 @@ dg_status dg_set_option(int option, int64_t value) {
         g_trace.store((uint64_t)value);
         return DG_OK;
     case DG_OPT_EARLY_LAUNCH:
-        if (value < 0 || value > 2) return DG_ERR_VALUE;
+        if (value < 0 || value > 3) return DG_ERR_VALUE;
         g_pdl.store((int)value);
         return DG_OK;
     case DG_OPT_CTA_PAIR:

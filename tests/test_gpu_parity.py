@@ -28,7 +28,7 @@ def _reset_options():
     dg.dg_set_option(dg.DG_OPT_WAIT_TIMEOUT_MS, 2000)
     dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, 8)
     dg.dg_set_option(dg.DG_OPT_CTA_PAIR, 1)
-    dg.dg_set_option(dg.DG_OPT_EARLY_LAUNCH, 0)
+    dg.dg_set_option(dg.DG_OPT_EARLY_LAUNCH, 3)
     dg.dg_set_option(dg.DG_OPT_EPI_TMA, 1)
     dg.dg_set_option(dg.DG_OPT_GATHER_CLUSTER, 1)
     dg.dg_set_option(dg.DG_OPT_PAIR_TAIL, 1)
