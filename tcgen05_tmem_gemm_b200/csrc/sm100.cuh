@@ -176,6 +176,11 @@ __device__ __forceinline__ void cluster_sync() {
 // The two halves of cluster_sync, for a barrier whose wait comes later.
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+// An arrival that orders nothing: for barriers that only say "this CTA is done
+// with something" when that fact was already observed through an mbarrier.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
 
 // Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
 // from this CTA's shared memory into the shared memory of a CTA of the

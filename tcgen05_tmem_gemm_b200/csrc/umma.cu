@@ -815,7 +815,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             cluster_wait();  // every CTA of the cluster is initialised
             cluster_ready = true;
         }
-        if (!epi_warp) cluster_arrive();  // nothing to receive here
+        if (!epi_warp) cluster_arrive_relaxed();  // nothing to receive here
         if (epi_warp) {
             tc_fence_after();
             const int quarter = warp & 3;
@@ -883,7 +883,9 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             }
             const bool received = mbar_wait(bar_recv, 0, wc);
             __syncwarp();
-            cluster_arrive();  // barrier 2: every copy into this CTA has landed
+            // barrier 2: every copy into this CTA has landed (seen on bar_recv;
+            // the arrival needs to order nothing else)
+            cluster_arrive_relaxed();
             if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 55);
             if (received) {
                 // slice of source q: local for this CTA's own rank
