@@ -317,8 +317,8 @@ __device__ __forceinline__ void gather_issue_async(const GatherSrc &src, const G
 // a stage is at most one batch per thread (kGatherUnroll copies), the next
 // k block's loads are issued before this block is stored, so two stages of
 // loads are in flight; wider stages are loaded and stored batch by batch.
-// Every exit decision is voted on across the gather warps (bar.red), so no
-// warp is left waiting at their named barrier.
+// Every exit decision is voted on across the gather warps (bar.red) at tile
+// boundaries, so no warp is left waiting at their named barrier.
 template <int VB>
 __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayout &L, uint32_t sbase,
                                             uint32_t bar_full, uint32_t bar_empty, uint32_t bar_part,
@@ -362,7 +362,7 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
             }
             if (one_batch && kb + 1 < kb1) gather_load<VB>(src, g, g_row_off, (kb + 1) * bk, gtid, nxt);
             ok = mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc);
-            if (named_bar_or(!ok)) { ok = false; break; }
+            if (!ok) break;  // the other warps see the abort flag; the vote below makes the exit uniform
             if (!stall && VB >= 4) {
                 // asynchronous copies: the stage completes on the full barrier
                 // when they land, and this warp moves on at once
@@ -391,9 +391,9 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
                 for (int r = 0; r < kGatherUnroll; ++r) cur[r] = nxt[r];
             }
         }
-        // row offsets of this tile stay in use until every gather warp is past it
-        asm volatile("bar.sync 1, %0;" ::"n"(kGatherWarps * 32) : "memory");
-        if (!ok) break;
+        // row offsets of this tile stay in use until every gather warp is past
+        // it; the vote is that barrier, and every warp leaves together
+        if (named_bar_or(!ok)) break;
     }
     // nothing this thread copied may land after the CTA has gone
     asm volatile("cp.async.wait_all;" ::: "memory");
@@ -647,7 +647,8 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                     fence_proxy_async_smem();  // cp.async writes -> bulk-copy reads
                     const uint32_t ps = sbase + s * L.stage_bytes;
                     for (int q = 1; q < G; ++q) {
-                        const uint32_t d = (grank + (uint32_t)q) % (uint32_t)G;
+                        uint32_t d = grank + (uint32_t)q;  // the other CTAs, without division
+                        if (d >= (uint32_t)G) d -= (uint32_t)G;
                         const uint32_t rbar = dsmem_map(bar_full + 8 * s, d);
                         for (int c = 0; c < nchunk; ++c) {
                             const uint32_t off = (uint32_t)c * chunk_bytes + first_off;
