@@ -187,6 +187,7 @@ constexpr int kGatherUnroll = 16;
 struct GatherGeom {
     bool mn;
     int vec, runs, total, chunk_bytes, es;
+    int runs_log2;  // runs is a power of two: indices split with shifts and masks
 };
 
 // The gathered operand's base and k axis, read from the parameter block once:
@@ -219,6 +220,7 @@ __device__ __forceinline__ GatherGeom gather_geom(const UmmaParams &p, int VB, i
     g.vec = VB / es;
     g.runs = g.mn ? kBM / g.vec : bk / g.vec;
     g.total = g.mn ? g.runs * bk : kBM * g.runs;
+    g.runs_log2 = __ffs(g.runs) - 1;
     g.chunk_bytes = bk * 128;
     g.es = es;
     return g;
@@ -232,12 +234,12 @@ template <int VB>
 __device__ __forceinline__ void gather_load(const GatherSrc &src, const GatherGeom &g, const int64_t *row_off,
                                             int kbase, int first, typename VecOf<VB>::T (&v)[kGatherUnroll]) {
     const int nthreads = kGatherWarps * 32;
-    const int step = nthreads / g.runs;
+    const int step = nthreads >> g.runs_log2;
     if (g.mn) {
         // fixed i (a run of vec rows), k advancing by `step`
-        const int i = (first % g.runs) * g.vec;
+        const int i = (first & (g.runs - 1)) * g.vec;
         const int64_t ro = row_off[i];
-        const int k0 = first / g.runs;
+        const int k0 = first >> g.runs_log2;
 #pragma unroll
         for (int r = 0; r < kGatherUnroll; ++r) {
             const int u = first + r * nthreads;
@@ -247,9 +249,9 @@ __device__ __forceinline__ void gather_load(const GatherSrc &src, const GatherGe
         }
     } else {
         // fixed k (a run of vec columns), i advancing by `step`
-        const int kg = kbase + (first % g.runs) * g.vec;
+        const int kg = kbase + (first & (g.runs - 1)) * g.vec;
         const int64_t co = kg < src.K ? src.koff(kg) : -1;
-        const int i0 = first / g.runs;
+        const int i0 = first >> g.runs_log2;
 #pragma unroll
         for (int r = 0; r < kGatherUnroll; ++r) {
             const int u = first + r * nthreads;
@@ -265,8 +267,8 @@ template <int VB>
 __device__ __forceinline__ void gather_store(const GatherGeom &g, uint32_t p_smem, int first,
                                              const typename VecOf<VB>::T (&v)[kGatherUnroll]) {
     const int nthreads = kGatherWarps * 32;
-    const int step = nthreads / g.runs;
-    const int fixed = (first % g.runs) * g.vec, moving0 = first / g.runs;
+    const int step = nthreads >> g.runs_log2;
+    const int fixed = (first & (g.runs - 1)) * g.vec, moving0 = first >> g.runs_log2;
 #pragma unroll
     for (int r = 0; r < kGatherUnroll; ++r) {
         const int u = first + r * nthreads;
@@ -285,8 +287,8 @@ __device__ __forceinline__ void gather_issue_async(const GatherSrc &src, const G
                                                    const int64_t *row_off, int kbase, int first, int uend,
                                                    uint32_t p_smem) {
     const int nthreads = kGatherWarps * 32;
-    const int step = nthreads / g.runs;
-    const int fixed = (first % g.runs) * g.vec, moving0 = first / g.runs;
+    const int step = nthreads >> g.runs_log2;
+    const int fixed = (first & (g.runs - 1)) * g.vec, moving0 = first >> g.runs_log2;
     if (g.mn) {
         const int64_t ro = row_off[fixed];
 #pragma unroll
