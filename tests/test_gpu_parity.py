@@ -469,6 +469,33 @@ def test_bounded_wait_reports_timeout_and_recovers():
     check_full(W.cfg_small())
 
 
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_early_launch_modes_back_to_back(mode):
+    # Programmatic dependent launch lets a kernel start before the previous one
+    # in the stream has finished; every kernel waits for it before touching
+    # memory.  Chained calls where each reads the previous one's output must
+    # still see it: y1 = x W1, then C = A(y1 rows) B, then y2 = x W2 on y1's
+    # buffer again, all queued back to back.
+    dg.dg_set_option(dg.DG_OPT_EARLY_LAUNCH, mode)
+    g = torch.Generator().manual_seed(77 + mode)
+    K, N = 512, 256
+    x = W.cast(W.normal((1, K), g), "bf16").cuda()
+    w1 = W.cast(W.normal((K, N), g, 0.05), "bf16").cuda()
+    y1 = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+    b = W.cast(W.normal((N, 64), g, 0.05), "bf16").cuda()
+    c = torch.empty((1, 64), dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        dg.gemm(x, w1, y1)           # gemv_n
+        dg.gemm(y1, b, c)            # reads y1 right away (gemv_n again, N = 64)
+    torch.cuda.synchronize()
+    assert dg.dg_sync_status() == dg.DG_OK
+    ref1 = x.double().cpu() @ w1.double().cpu()
+    got1 = y1.double().cpu()
+    assert torch.allclose(got1, ref1, rtol=1e-2, atol=1e-2)
+    ref2 = got1 @ b.double().cpu()   # from the y1 the GPU produced (its BF16 rounding included)
+    assert torch.allclose(c.double().cpu(), ref2, rtol=1e-3, atol=1e-3)
+
+
 def test_streams_and_launch_count():
     s = torch.cuda.Stream()
     n0 = dg.dg_launch_count()
