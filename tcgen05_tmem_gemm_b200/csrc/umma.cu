@@ -113,14 +113,22 @@ __device__ __forceinline__ TileCoord unit_coord(int u, const UmmaParams &p) {
     return c;
 }
 
-// Byte offset inside a 128-byte-swizzled tile of an element at (mn, k) for
-// the two layouts the tensor core reads.  `bytek` = k * element size.
+// Byte offset inside a 128-byte-swizzled K-major tile of the element at
+// (mn, k); `bytek` = k * element size.
 __device__ __forceinline__ uint32_t sw128_kmajor(int mn, int bytek) {
     return (uint32_t)((mn >> 3) * 1024 + (mn & 7) * 128 + ((((bytek >> 4) ^ (mn & 7)) << 4) | (bytek & 15)));
 }
-__device__ __forceinline__ uint32_t sw128_mnmajor(int bytemn, int k, int chunk_bytes) {
+// Gathered MN-major tiles are laid out k-slice by k-slice: the 2^ks_log2 rows
+// of k that one MMA instruction consumes (every 128-byte MN chunk of them)
+// are kGatherSliceBytes contiguous bytes, so the k range one CTA of a gather
+// cluster loads is a single block of shared memory.  Within a slice, chunk c
+// starts at c * 2^ks_log2 * 128 bytes; 8-row swizzle atoms of 1024 bytes.
+constexpr int kGatherSliceBytes = 4096;  // 128 rows x 16 (16-bit) or 32 (8-bit) k
+__device__ __forceinline__ uint32_t sw128_mnmajor_ks(int bytemn, int k, int ks_log2) {
     const int c = bytemn >> 7, w = bytemn & 127;
-    return (uint32_t)(c * chunk_bytes + (k >> 3) * 1024 + (k & 7) * 128 + ((((w >> 4) ^ (k & 7)) << 4) | (w & 15)));
+    const int kk = k & ((1 << ks_log2) - 1);
+    return (uint32_t)((k >> ks_log2) * kGatherSliceBytes + (c << ks_log2) * 128 + (kk >> 3) * 1024 + (k & 7) * 128 +
+                      ((((w >> 4) ^ (k & 7)) << 4) | (w & 15)));
 }
 
 template <int BYTES> struct VecOf;
@@ -186,8 +194,9 @@ constexpr int kGatherUnroll = 16;
 
 struct GatherGeom {
     bool mn;
-    int vec, runs, total, chunk_bytes, es;
+    int vec, runs, total, es;
     int runs_log2;  // runs is a power of two: indices split with shifts and masks
+    int ks_log2;    // MN-major: log2 of the k rows per slice (one MMA instruction's K)
 };
 
 // The gathered operand's base and k axis, read from the parameter block once:
@@ -221,7 +230,7 @@ __device__ __forceinline__ GatherGeom gather_geom(const UmmaParams &p, int VB, i
     g.runs = g.mn ? kBM / g.vec : bk / g.vec;
     g.total = g.mn ? g.runs * bk : kBM * g.runs;
     g.runs_log2 = __ffs(g.runs) - 1;
-    g.chunk_bytes = bk * 128;
+    g.ks_log2 = es == 1 ? 5 : 4;  // 32 E4M3 or 16 F16/BF16 k per MMA instruction
     g.es = es;
     return g;
 }
@@ -274,7 +283,7 @@ __device__ __forceinline__ void gather_store(const GatherGeom &g, uint32_t p_sme
         const int u = first + r * nthreads;
         if (u >= g.total) continue;
         const int moving = moving0 + r * step;
-        st_shared_vec<VB>(p_smem + (g.mn ? sw128_mnmajor(fixed * g.es, moving, g.chunk_bytes)
+        st_shared_vec<VB>(p_smem + (g.mn ? sw128_mnmajor_ks(fixed * g.es, moving, g.ks_log2)
                                          : sw128_kmajor(moving, fixed * g.es)),
                           v[r]);
     }
@@ -297,7 +306,7 @@ __device__ __forceinline__ void gather_issue_async(const GatherSrc &src, const G
             if (u >= uend) break;
             const int k = moving0 + r * step, kg = kbase + k;
             const bool ok = ro >= 0 && kg < src.K;
-            cp_async_zfill<VB>(p_smem + sw128_mnmajor(fixed * g.es, k, g.chunk_bytes),
+            cp_async_zfill<VB>(p_smem + sw128_mnmajor_ks(fixed * g.es, k, g.ks_log2),
                                src.ptr + (ok ? ro + src.koff(kg) : 0), ok);
         }
     } else {
@@ -566,9 +575,12 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             const uint32_t idesc = p.idesc, stage_bytes = L.stage_bytes;
             // descriptor strides: K-major tiles step 1024 B per 8 rows; MN-major
             // tiles step 1024 B per 8 k and one 128-byte MN chunk per bk*128 B.
-            const uint32_t p_lbo = p.p_mn_major ? (uint32_t)(bk * 128) : 16u;
+            // gathered MN-major P is laid out k-slice by k-slice (one slice per
+            // MMA step, its MN chunks kUmmaK * 128 bytes apart)
+            const bool p_ks = GATHER && p.p_mn_major;
+            const uint32_t p_lbo = p_ks ? (uint32_t)(kUmmaK * 128) : p.p_mn_major ? (uint32_t)(bk * 128) : 16u;
             const uint32_t q_lbo = p.q_mn_major ? (uint32_t)(bk * 128) : 16u;
-            const uint32_t p_kstep = p.p_mn_major ? kUmmaK * 128 : kUmmaK * es;
+            const uint32_t p_kstep = p_ks ? (uint32_t)kGatherSliceBytes : p.p_mn_major ? kUmmaK * 128 : kUmmaK * es;
             const uint32_t q_kstep = p.q_mn_major ? kUmmaK * 128 : kUmmaK * es;
             // descriptors of stage 0; a stage's differ only in the start address
             // field (address >> 4, below 2^14 for any shared-memory address)
@@ -621,15 +633,11 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             // ---------------------------------------- gather-cluster forwarder
             // Once this CTA's part of a stage has landed, copy it into the same
             // stage of every other CTA of the cluster (their full barriers count
-            // the bytes), then count the part as arrived here.  The part: a k
-            // range in each 128-byte MN chunk (MN-major), or a row range.
+            // the bytes), then count the part as arrived here.  The part is one
+            // contiguous block: whole k-slices (MN-major) or a row range.
             const uint32_t grank = cluster_ctarank();
-            const bool mn = p.p_mn_major != 0;
             const uint32_t part = L.p_bytes / (uint32_t)G;
-            const int nchunk = mn ? (kBM * es) / 128 : 1;
-            const uint32_t piece = part / (uint32_t)nchunk;
-            const uint32_t chunk_bytes = (uint32_t)bk * 128u;
-            const uint32_t first_off = mn ? grank * (uint32_t)(bk / G) * 128u : grank * part;
+            const uint32_t first_off = grank * part;
             const int stages = p.stages;
             int fs = 0;  // stage and phase, advanced without division
             uint32_t fph = 0;
@@ -651,11 +659,8 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                     for (int q = 1; q < G; ++q) {
                         uint32_t d = grank + (uint32_t)q;  // the other CTAs, without division
                         if (d >= (uint32_t)G) d -= (uint32_t)G;
-                        const uint32_t rbar = dsmem_map(bar_full + 8 * s, d);
-                        for (int c = 0; c < nchunk; ++c) {
-                            const uint32_t off = (uint32_t)c * chunk_bytes + first_off;
-                            bulk_copy_to_cluster(dsmem_map(ps + off, d), ps + off, piece, rbar);
-                        }
+                        bulk_copy_to_cluster(dsmem_map(ps + first_off, d), ps + first_off, part,
+                                             dsmem_map(bar_full + 8 * s, d));
                     }
                     mbar_arrive(bar_full + 8 * s);
                 }
