@@ -146,7 +146,12 @@ __global__ void __launch_bounds__(kNT) gemv_n_kernel(const __grid_constant__ CUt
     const int nst = (kn + kRows - 1) / kRows;
     const int nsplit = gridDim.y;
 
-    if (threadIdx.x == 0) {
+    // The producer lane sets up the barriers and puts the first round of W
+    // stages in flight (every stage is free) before x is staged, so the two
+    // trips to memory overlap; the consumers see the barriers after the
+    // block-wide barrier below.
+    const int first_round = min(kStages, nst);
+    if (warp == kCW && lane == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, kCW);
@@ -154,6 +159,10 @@ __global__ void __launch_bounds__(kNT) gemv_n_kernel(const __grid_constant__ CUt
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
+        for (int it = 0; it < first_round; ++it) {
+            mbar_arrive_expect_tx(bar_full + 8 * it, kRows * kNB * 2);
+            tma_load_2d(sbase + L.ring + it * (kRows * kNB * 2), &tmap_w, bar_full + 8 * it, n0, kb0 + it * kRows);
+        }
     }
     stage_x<T, R>(xs, p.kper, p, kb0, kn, threadIdx.x, kNT);
     __syncthreads();
@@ -161,8 +170,9 @@ __global__ void __launch_bounds__(kNT) gemv_n_kernel(const __grid_constant__ CUt
     if (warp == kCW) {
         // ----------------------------------------------------- TMA producer
         if (lane == 0) {
-            int it = 0;
+            int it = first_round;
             const int release_at = max(0, nst - kReleaseStages);
+            if (release_at < first_round && p.pdl == 2) pdl_release();
             for (; it < nst; ++it) {
                 const int s = it % kStages;
                 const uint32_t ph = (uint32_t)(it / kStages) & 1u;
