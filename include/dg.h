@@ -213,10 +213,15 @@ typedef enum {
                                      operands allow                                    */
     DG_OPT_EARLY_LAUNCH = 6,      /* programmatic dependent launch: 0 off, 1 release the
                                      next kernel at the start of each kernel, 2 release
-                                     it near the end of long kernels, 3 (default) only
-                                     for the K-contiguous GEMV, whose 64 blocks leave
-                                     room for the next launch (1 and 2 slowed the
-                                     decode step: two W-streaming blocks fill an SM)   */
+                                     it near the end of long kernels, 3 (default) for
+                                     the K-contiguous GEMV (its 64 blocks leave room
+                                     for the next launch) and the tensor-core kernels
+                                     (released once their MMAs are issued), not for
+                                     the N-contiguous GEMV (1 and 2 slowed the decode
+                                     step: two W-streaming blocks fill an SM).  Every
+                                     kernel waits for the previous one before it
+                                     touches memory, so all modes give the same
+                                     results.                                          */
     DG_OPT_TRACE = 7,             /* device address of 64 uint64 slots (0 = off): the
                                      single-CTA tensor-core kernel's CTA 0 writes
                                      %globaltimer at its phase boundaries (analysis)   */

@@ -520,10 +520,12 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
                   DeviceState *ds, LaunchRec *rec) {
     const dg_plan_info &in = pl.info;
     rec->kind = in.kind;
-    // early launch: mode 3 uses it for the launch-bound K-contiguous GEMV only
-    // (64 blocks: the next launch finds free SMs while it runs)
+    // early launch, mode 3: the launch-bound K-contiguous GEMV (64 blocks: the
+    // next launch finds free SMs while it runs) and the tensor-core kernels
+    // (released once their MMAs are issued; they wait before any memory access),
+    // not the N-contiguous GEMV, whose blocks fill every SM's shared memory
     const int pdl_mode = g_pdl.load();
-    rec->pdl = pdl_mode == 3 ? (in.kind == DG_KIND_GEMV_K ? 1 : 0) : pdl_mode;
+    rec->pdl = pdl_mode == 3 ? (in.kind == DG_KIND_GEMV_K ? 1 : in.kind == DG_KIND_UMMA ? 2 : 0) : pdl_mode;
     switch (in.kind) {
     case DG_KIND_NONE: return DG_OK;
     case DG_KIND_SCALE_C: {

@@ -15,7 +15,7 @@ import torch
 import oracle
 import tcgen05_tmem_gemm_b200 as dg
 import workloads as W
-from harness import c_matrix, check_full, check_sampled, compare, dg_view_of, plan, run
+from harness import c_matrix, check_full, check_sampled, compare, dg_view_of, plan, run, tolerance
 
 pytestmark = pytest.mark.gpu
 
@@ -469,7 +469,7 @@ def test_bounded_wait_reports_timeout_and_recovers():
     check_full(W.cfg_small())
 
 
-@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
 def test_early_launch_modes_back_to_back(mode):
     # Programmatic dependent launch lets a kernel start before the previous one
     # in the stream has finished; every kernel waits for it before touching
@@ -494,6 +494,59 @@ def test_early_launch_modes_back_to_back(mode):
     assert torch.allclose(got1, ref1, rtol=1e-2, atol=1e-2)
     ref2 = got1 @ b.double().cpu()   # from the y1 the GPU produced (its BF16 rounding included)
     assert torch.allclose(c.double().cpu(), ref2, rtol=1e-3, atol=1e-3)
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+def test_early_launch_tensor_core_chain(mode):
+    # The same for the tensor-core kernels: a CTA-pair GEMM, split-K clusters
+    # and a single-CTA GEMM, each reading an output of the calls just before
+    # it, and the first operand written by a torch kernel right before the
+    # first call.  The buffers are rewritten every round while the calls of
+    # the round before may still be in flight; the rounds scale A by 1, 2 and
+    # 4 (exact in BF16), so a stale operand is off by a factor of two.
+    dg.dg_set_option(dg.DG_OPT_EARLY_LAUNCH, mode)
+    g = torch.Generator().manual_seed(123 + mode)
+    bf = torch.bfloat16
+    a = W.cast(W.normal((2048, 1024), g), "bf16").cuda()
+    b1 = W.cast(W.normal((1024, 4096), g, 0.05), "bf16").cuda()
+    b2 = W.cast(W.normal((4096, 2048), g, 0.05), "bf16").cuda()
+    b3 = W.cast(W.normal((256, 512), g, 0.05), "bf16").cuda()
+    b4 = W.cast(W.normal((2048, 256), g, 0.05), "bf16").cuda()
+    a_r = torch.empty_like(a)
+    c1 = torch.empty((2048, 4096), dtype=bf, device="cuda")
+    c2 = torch.empty((64, 2048), dtype=bf, device="cuda")
+    plans = [dg.dg_plan(dg.view(x), dg.view(y), dg.view(z)).as_dict() for x, y, z in
+             [(a_r, b1, c1), (c1[:64], b2, c2), (c1[:512, :256], b3, torch.empty((512, 512), device="cuda")),
+              (c2, b4, torch.empty((64, 256), device="cuda"))]]
+    assert plans[0]["cta_pair"] == 1 and plans[1]["split_k"] > 1 and plans[3]["split_k"] > 1
+    assert plans[2]["cta_pair"] == 0 and plans[2]["split_k"] == 1
+    outs = []
+    for r in range(3):
+        torch.mul(a, float(2 ** r), out=a_r)
+        dg.gemm(a_r, b1, c1)                     # CTA pair, reads a_r at once
+        dg.gemm(c1[:64], b2, c2)                 # split-K cluster, reads c1 at once
+        c3 = torch.empty((512, 512), dtype=torch.float32, device="cuda")
+        dg.gemm(c1[:512, :256], b3, c3)          # single CTA, reads c1 in place
+        c4 = torch.empty((64, 256), dtype=torch.float32, device="cuda")
+        dg.gemm(c2, b4, c4)                      # split-K cluster, reads c2 at once
+        outs.append((float(2 ** r), c1.clone(), c2.clone(), c3, c4))
+    torch.cuda.synchronize()
+    assert dg.dg_sync_status() == dg.DG_OK
+
+    def check(got, x, y, out):
+        # the parity suite's bound: S = |x| |y| summed over k
+        ref, bound = (x @ y).numpy(), (x.abs() @ y.abs()).numpy()
+        err = np.abs(got.double().cpu().numpy() - ref)
+        assert (err <= tolerance(out, ref, bound, np.zeros_like(ref))).all(), float(err.max())
+
+    a_d, b1_d, b2_d, b3_d, b4_d = (t.double().cpu() for t in (a, b1, b2, b3, b4))
+    for f, g1, g2, g3, g4 in outs:
+        g1d, g2d = g1.double().cpu(), g2.double().cpu()
+        check(g1, a_d * f, b1_d, "bf16")
+        # each later product from the values the GPU produced (their BF16 rounding included)
+        check(g2, g1d[:64], b2_d, "bf16")
+        check(g3, g1d[:512, :256], b3_d, "f32")
+        check(g4, g2d, b4_d, "f32")
 
 
 def test_streams_and_launch_count():
