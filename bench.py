@@ -613,7 +613,8 @@ def main():
     ap.add_argument("--max-split", type=int, default=0, help="with --shape: cap the tensor-core split-K")
     ap.add_argument("--trace", action="store_true", help="with --shape: phase timestamps of CTA 0")
     ap.add_argument("--early-launch", type=int, default=-1,
-                    help="programmatic dependent launch policy (0 off, 1 at kernel start, 2 near the end)")
+                    help="programmatic dependent launch policy (0 off, 1 at kernel start, 2 near the end, "
+                         "3 the library's per-kernel default)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
