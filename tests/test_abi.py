@@ -231,3 +231,175 @@ def test_options():
         dg.dg_set_option(dg.DG_OPT_EPI_TMA, 1)
     with pytest.raises(dg.DgError):
         dg.dg_set_option(dg.DG_OPT_EPI_TMA, 2)
+
+
+# ------------------------------------------------------- plan invariants
+#
+# Random views (layouts, paddings, 4-D feature maps, misaligned pointers) through
+# dg_plan, and the launch invariants the kernels are built on: tile shapes the
+# tensor core accepts, cluster sizes within the portable limit, every split
+# owning some k, co-resident split-K and gather clusters, CTA pairs on whole
+# pairs of SMs.
+
+ES = {"f32": 4, "f16": 2, "bf16": 2, "e4m3": 1}
+SMS = 148
+
+
+def _rand_dim(rng, small=False):
+    if rng.random() < 0.5:
+        pool = [1, 2, 3, 4, 5, 7, 8, 9, 16, 31, 32, 63, 64, 65, 96, 127, 128, 129, 200, 255, 256,
+                257, 384, 512, 1000, 1024, 2048, 3136, 4096, 8192]
+        if small:
+            pool = [p for p in pool if p <= 1024]
+        return rng.choice(pool)
+    return rng.randint(1, 1200 if small else 5000)
+
+
+def _matrix_view(rng, base, rows, cols, dt, allow_t=True):
+    """A [rows x cols] view: row-major or transposed storage, padded leading
+    dimension, sometimes an offset start."""
+    es = ES[dt]
+    pad = rng.choice([0, 0, 0, 0, 8, 3, 64])
+    off = rng.choice([0, 0, 0, 0, 0, 1, 8]) * es
+    if allow_t and rng.random() < 0.35:       # stored [cols x rows], viewed transposed
+        ld = rows + pad
+        return dg.make_view(base + off, (rows, cols), (es, ld * es), 1, dt)
+    ld = cols + pad
+    return dg.make_view(base + off, (rows, cols), (ld * es, es), 1, dt)
+
+
+def _random_problem(rng):
+    dt = rng.choice(["f16", "bf16", "bf16", "e4m3", "e4m3", "f32"])
+    cdt = rng.choice(["f32", "bf16", "f16"])
+    if rng.random() < 0.15:
+        # an NCHW feature map read in place as [N*H*W, C]
+        n, hw, c = rng.randint(1, 16), rng.choice([7, 14, 28]), rng.choice([3, 64, 96, 256])
+        K, N = c, _rand_dim(rng, small=True)
+        M = n * hw * hw
+        es = ES[dt]
+        A = dg.make_view(FAKE, (n, hw, hw, c), (c * hw * hw * es, hw * es, es, hw * hw * es), 3, dt)
+    else:
+        M, K, N = _rand_dim(rng), _rand_dim(rng), _rand_dim(rng)
+        if rng.random() < 0.3:
+            M = rng.randint(1, 8)             # decode-sized
+        A = _matrix_view(rng, FAKE, M, K, dt)
+    B = _matrix_view(rng, FAKE * 2, K, N, dt)
+    C = _matrix_view(rng, FAKE * 3, M, N, cdt, allow_t=rng.random() < 0.2)
+    alpha = rng.choice([1.0, 1.0, 2.0, 0.0]) if rng.random() < 0.1 else 1.0
+    beta = rng.choice([0.0, 0.0, 1.0, 0.5])
+    return dt, cdt, M, N, K, A, B, C, alpha, beta
+
+
+def _check_plan(p, dt, M, N, K, alpha):
+    kind = p["kind_name"]
+    assert (p["M"], p["N"], p["K"]) == (M, N, K)
+    if M == 0 or N == 0:
+        assert kind == "none"
+        return
+    if alpha == 0.0 or K == 0:
+        assert kind == "scale_c"
+        return
+    if dt == "f32":
+        assert kind == "simt"
+    if kind == "gemv_n":
+        assert dt in ("f16", "bf16") and M <= 8
+        r_inst = 1 if M <= 1 else 2 if M <= 2 else 4 if M <= 4 else 8
+        S, kper = p["split_k"], p["block_k"]
+        assert p["block_n"] == 256 and kper % 64 == 0 and 1 <= S <= 8
+        assert (S - 1) * kper < K <= S * kper          # every k split owns some k
+        assert kper * r_inst <= 16384                   # its slice of x fits in shared memory
+        assert p["grid"] == -(-N // 256) * S
+    elif kind == "gemv_k":
+        r_inst = 1 if M <= 1 else 2 if M <= 2 else 4 if M <= 4 else 8
+        assert dt in ("f16", "bf16") and M <= 8 and K % 8 == 0 and K * r_inst <= 32768
+    elif kind == "umma":
+        es = ES[dt]
+        assert dt in ("f16", "bf16", "e4m3")
+        bn, split, grid = p["block_n"], p["split_k"], p["grid"]
+        assert p["block_k"] == 128 // es
+        assert 16 <= bn <= 256 and bn % 16 == 0         # N of a 128-row tcgen05.mma
+        if p["q_mn_major"]:
+            assert bn % (128 // es) == 0                 # whole 128-byte boxes
+        assert 1 <= split <= 8 and p["stages"] >= 2
+        Mi, Nj = (N, M) if p["swap_ab"] else (M, N)
+        tiles_j = -(-Nj // bn)
+        tiles = -(-Mi // 128) * tiles_j
+        assert 1 <= grid <= SMS
+        if split > 1:
+            assert p["stages"] >= 3 and not p["cta_pair"] and p["gather_cluster"] == 1
+            assert not p["epi_tma_store"]
+            assert grid == tiles * split                 # one unit per CTA, all resident
+            kb_total = -(-K // p["block_k"])
+            kb_per = -(-kb_total // split)
+            assert (split - 1) * kb_per < kb_total       # every k split owns some k
+        if p["epi_tma_store"]:
+            assert split == 1 and not p["swap_ab"]
+        g = p["gather_cluster"]
+        assert g in (1, 2, 4)
+        if g > 1:
+            assert p["p_gather"] and grid % g == 0 and tiles_j % g == 0
+        if p["cta_pair"]:
+            assert p["block_m"] == 256 and grid % 2 == 0 and bn >= 128 and split == 1
+            assert 0 <= 2 * p["pair_half_tiles"] <= grid // 2
+        else:
+            assert p["block_m"] == 128 and p["pair_half_tiles"] == 0
+        assert p["vec_bytes"] in (1, 2, 4, 8, 16)
+        if not p["p_gather"]:
+            assert p["vec_bytes"] == 16
+    else:
+        assert kind == "simt", kind
+
+
+def test_plan_invariants_random_views():
+    import random
+
+    rng = random.Random(20261203)
+    kinds = {}
+    for _ in range(3000):
+        dt, cdt, M, N, K, A, B, C, alpha, beta = _random_problem(rng)
+        try:
+            info = dg.dg_plan(A, B, C, alpha, beta, rng.random() < 0.3, SMS)
+        except dg.DgError:
+            continue                                     # a view the library rejects up front
+        p = info.as_dict()
+        tags = [p["kind_name"]]
+        if p["kind_name"] == "umma":
+            tags += ["umma/pair"] * p["cta_pair"] + ["umma/split"] * (p["split_k"] > 1)
+            tags += ["umma/gather_cluster"] * (p["gather_cluster"] > 1)
+        for t in tags:
+            kinds[t] = kinds.get(t, 0) + 1
+        _check_plan(p, dt, M, N, K, alpha)
+    # the draw reaches every kernel family and the tensor-core variants
+    for k in ("gemv_n", "gemv_k", "umma", "simt", "umma/pair", "umma/split", "umma/gather_cluster"):
+        assert kinds.get(k, 0) >= 5, kinds
+
+
+def test_plan_invariant_checks_reject_broken_plans():
+    # the checks above are not vacuous: valid plans with one field broken fail them
+    import random
+
+    rng = random.Random(7)
+    found = {}
+    for _ in range(3000):
+        dt, cdt, M, N, K, A, B, C, alpha, beta = _random_problem(rng)
+        try:
+            p = dg.dg_plan(A, B, C, alpha, beta, False, SMS).as_dict()
+        except dg.DgError:
+            continue
+        key = "pair" if p["cta_pair"] else "split" if p["split_k"] > 1 else p["kind_name"]
+        found.setdefault(key, (p, dt, M, N, K, alpha))
+    breaks = {
+        "pair": [("grid", lambda v: v - 1), ("block_n", lambda v: 64)],
+        "split": [("split_k", lambda v: 9), ("grid", lambda v: v + 1), ("stages", lambda v: 2)],
+        "gemv_n": [("block_k", lambda v: v - 64 if v > 64 else v + 1), ("split_k", lambda v: v + 1)],
+        "umma": [("block_n", lambda v: v + 8), ("block_k", lambda v: 32)],
+    }
+    for key, muts in breaks.items():
+        assert key in found, key
+        p, dt, M, N, K, alpha = found[key]
+        _check_plan(p, dt, M, N, K, alpha)
+        for field, f in muts:
+            q = dict(p)
+            q[field] = f(p[field])
+            with pytest.raises(AssertionError):
+                _check_plan(q, dt, M, N, K, alpha)
