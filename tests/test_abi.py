@@ -403,3 +403,78 @@ def test_plan_invariant_checks_reject_broken_plans():
             q[field] = f(p[field])
             with pytest.raises(AssertionError):
                 _check_plan(q, dt, M, N, K, alpha)
+
+
+def _offsets_by_dims(shape, stride, idx_dims):
+    """Byte offset of a flat index unflattened row-major over the given dims."""
+    def off(flat):
+        o = 0
+        for d in reversed(idx_dims):
+            o += (flat % shape[d]) * stride[d]
+            flat //= shape[d]
+        return o
+    return off
+
+
+def test_analyse_random_views_address_the_same_elements():
+    # Size-1 dims dropped and neighbours merged: the merged row and column
+    # groups must reach exactly the bytes the original dims do (checked by
+    # brute force on sampled (row, col) pairs), and the derived facts (extent,
+    # span, unit-stride direction, TMA legality) must agree with the view.
+    import random
+
+    rng = random.Random(99)
+    checked = 0
+    for _ in range(600):
+        dt = rng.choice(["f32", "f16", "bf16", "e4m3"])
+        es = ES[dt]
+        nd = rng.randint(1, 4)
+        shape = [rng.choice([1, 1, 2, 3, 7, 14, 16, 64, 196]) for _ in range(nd)]
+        # strides: mostly packed in some dim order (so that merges happen), at
+        # times padded, broadcast (0) on size-1 dims
+        order = list(range(nd))
+        rng.shuffle(order)
+        stride = [0] * nd
+        run = es
+        for d in reversed(order):
+            stride[d] = run if shape[d] > 1 or rng.random() < 0.5 else 0
+            run *= shape[d] + (rng.choice([0, 0, 0, 1, 8]) if rng.random() < 0.3 else 0)
+        row_dims = rng.randint(0, nd) if nd > 1 else rng.randint(0, 1)
+        ptr = FAKE + rng.choice([0, 0, 0, es, 8, 16])
+        v = dg.make_view(ptr, shape, stride, row_dims, dt)
+        try:
+            info = dg.dg_analyse_view(v)
+        except dg.DgError:
+            continue
+        rows = math_prod(shape[:row_dims])
+        cols = math_prod(shape[row_dims:])
+        assert (info.rows, info.cols) == (rows, cols)
+        orig_r = _offsets_by_dims(shape, stride, list(range(row_dims)))
+        orig_c = _offsets_by_dims(shape, stride, list(range(row_dims, nd)))
+        m_r = _offsets_by_dims(list(info.row_shape), list(info.row_stride), list(range(info.n_row)))
+        m_c = _offsets_by_dims(list(info.col_shape), list(info.col_stride), list(range(info.n_col)))
+        assert math_prod(list(info.row_shape[:info.n_row])) == rows
+        assert math_prod(list(info.col_shape[:info.n_col])) == cols
+        for _ in range(40):
+            r, c = rng.randrange(rows), rng.randrange(cols)
+            assert m_r(r) + m_c(c) == orig_r(r) + orig_c(c), (shape, stride, row_dims, r, c)
+        top = sum((s - 1) * st for s, st in zip(shape, stride))
+        assert info.span_bytes == top + es
+        if info.unit_dim == 1:
+            assert info.n_col == 1 and info.col_stride[0] == es
+        if info.unit_dim == 2:
+            assert info.n_row == 1 and info.row_stride[0] == es
+        if info.tma_ok:
+            assert ptr % 16 == 0 and info.n_row <= 1 and info.n_col <= 1 and info.unit_dim in (1, 2)
+            other = info.row_stride[0] if info.unit_dim == 1 else info.col_stride[0]
+            assert info.n_row == 0 or info.n_col == 0 or other % 16 == 0
+        assert info.vec_bytes in (1, 2, 4, 8, 16)
+        checked += 1
+    assert checked > 400
+
+
+def math_prod(xs):
+    p = 1
+    for x in xs:
+        p *= int(x)
+    return p
