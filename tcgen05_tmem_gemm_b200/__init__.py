@@ -6,7 +6,7 @@ entry points (dg_gemm, dg_gemv, dg_sync_status, ...).  PyTorch is used by
 callers for device memory and streams; a torch tensor can be turned into a
 view with `view()`.
 
-The library must have been built (``python -m tcgen05_tmem_gemm_b200.build``
+The library must have been built (``python tcgen05_tmem_gemm_b200/build.py``
 or ``__graft_entry__.build()``); importing this package without it raises.
 """
 from __future__ import annotations
@@ -83,7 +83,7 @@ class DgError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libdg.so is not built ({LIB_PATH}); run python -m tcgen05_tmem_gemm_b200.build")
+        raise ImportError(f"libdg.so is not built ({LIB_PATH}); run python tcgen05_tmem_gemm_b200/build.py")
     L = ctypes.CDLL(LIB_PATH)
     P = ctypes.POINTER
     V = P(dg_view)

@@ -1,6 +1,6 @@
 """Builds libdg.so in-tree with nvcc for sm_100a.
 
-    python -m tcgen05_tmem_gemm_b200.build [--force]
+    python tcgen05_tmem_gemm_b200/build.py [--force]
 
 Objects go to _build/ at the repository root; the shared library is written
 next to this file so that it travels with the source tree.
