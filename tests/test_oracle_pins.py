@@ -13,7 +13,12 @@ oracle's own code:
     casts and the E4M3 landmarks (448, 2^-9, NaN codes);
   * the pages' strided example (1,128,7,7), strides (0,196,28,4) FP32, against
     numpy's matmul of the reshaped arrays;
-  * linearity in alpha/beta, the alpha = 0 and beta = 0 cases, scales applied once.
+  * linearity in alpha/beta, the alpha = 0 and beta = 0 cases, scales applied once;
+  * the rounding scale S = |alpha sa sb| sum_k |a b| (the oracle's second output,
+    which every GPU tolerance multiplies): worked by hand on a mixed-sign case
+    with a negative alpha and scales (tests/golden/hand_gemm_bound_signed.json),
+    exact rationals in the brute-force pin, E4M3 powers of two, and the
+    one-by-one evaluation equal to the full one.
 The last test plants mistakes in a copy of the oracle source and checks that
 some pin catches every one of them.
 """
@@ -49,8 +54,23 @@ def _f32(x):
 def pin_hand_example(orc):
     g = json.load(open(os.path.join(GOLDEN, "hand_gemm_2x3x2.json")))
     p = _problem(_f32(g["A"]), _f32(g["B"]), _f32(g["C"]), g["alpha"], g["beta"])
-    out = orc.gemm(p, want_bound=False)
+    out, bound = orc.gemm(p, want_bound=True)
     assert np.array_equal(out, np.array(g["expected"]))
+    assert np.array_equal(bound, np.array(g["expected_bound"]))
+
+
+def pin_hand_bound_signed(orc):
+    # mixed-sign products, a negative alpha and per-row / per-column scales:
+    # the rounding scale S = |alpha sa sb| sum_k |a b| worked by hand
+    g = json.load(open(os.path.join(GOLDEN, "hand_gemm_bound_signed.json")))
+    p = _problem(_f32(g["A"]), _f32(g["B"]), _f32(g["C"]), g["alpha"], g["beta"],
+                 torch.tensor(g["scale_a"]), torch.tensor(g["scale_b"]))
+    out, bound = orc.gemm(p, want_bound=True)
+    assert np.array_equal(out, np.array(g["expected"]))
+    assert np.array_equal(bound, np.array(g["expected_bound"]))
+    pts, pbound = orc.gemm_points(p, [0, 0, 1, 1], [0, 1, 0, 1])
+    assert np.array_equal(pts, np.array(g["expected"]).reshape(-1))
+    assert np.array_equal(pbound, np.array(g["expected_bound"]).reshape(-1))
 
 
 def pin_view_address(orc):
@@ -151,10 +171,10 @@ def pin_brute_force(orc):
             b = b32.to(W.TORCH_DTYPE[dt])
             sa = torch.rand(M, generator=g) + 0.5
             sb = torch.rand(N, generator=g) + 0.5
-            alpha, beta = 0.75, -1.25
+            alpha, beta = (0.75 if M % 2 else -0.75), -1.25
             p = _problem(W.row_major(a, dt), W.row_major(b, dt), W.row_major(c32.contiguous(), "f32"),
                          alpha, beta, sa, sb)
-            out = orc.gemm(p, want_bound=False)
+            out, bound = orc.gemm(p, want_bound=True)
             A = _exact_values(a, dt)
             B = _exact_values(b, dt)
             for i in range(M):
@@ -166,6 +186,9 @@ def pin_brute_force(orc):
                     # FP64 rounding of a K-term sum plus the scale and beta steps
                     tol = (K + 4) * 2.0 ** -52 * float(abs(s) * mag + abs(Fraction(beta) * Fraction(float(c32[i, j]))))
                     assert abs(out[i, j] - float(r)) <= tol, (dt, M, N, K, i, j)
+                    # the rounding scale S = |alpha sa sb| sum_k |a b|, exact up to FP64 rounding
+                    S = abs(s) * mag
+                    assert abs(bound[i, j] - float(S)) <= (K + 4) * 2.0 ** -52 * float(S), (dt, M, N, K, i, j)
 
 
 def pin_f16_bf16_tables(orc):
@@ -266,6 +289,17 @@ def pin_scales_once(orc):
                             1.0, 0.0, sa, sb), want_bound=False)
     want = K * np.outer(sa.numpy(), sb.numpy())
     assert np.array_equal(out, want)
+    # E4M3 codes of +-1 and -2 with alpha = -2: the output and its rounding
+    # scale both carry |alpha sa sb| exactly once (powers of two: exact)
+    a = torch.ones(M, K)
+    a[:, ::2] = -2.0
+    a = a.to(torch.float8_e4m3fn)
+    out, bound = orc.gemm(_problem(W.row_major(a, "e4m3"), W.row_major(b, "e4m3"), W.empty_out(M, N, "f32"),
+                                   -2.0, 0.0, sa, sb), want_bound=True)
+    row_sum = (K // 2) * (-2.0) + (K // 2) * 1.0       # sum_k a b
+    row_mag = (K // 2) * 2.0 + (K // 2) * 1.0          # sum_k |a b|
+    assert np.array_equal(out, -2.0 * row_sum * np.outer(sa.numpy(), sb.numpy()))
+    assert np.array_equal(bound, 2.0 * row_mag * np.outer(sa.numpy(), sb.numpy()))
 
 
 def pin_points_match_full(orc):
@@ -275,9 +309,23 @@ def pin_points_match_full(orc):
     ns = [0, 39, 7, 20, 1]
     pts, _ = orc.gemm_points(p, ms, ns)
     assert np.array_equal(pts, full[ms, ns])
+    # the one-by-one evaluation gives the same output and rounding scale as
+    # the full oracle on a scaled E4M3 problem with a negative alpha and beta != 0
+    g = torch.Generator().manual_seed(21)
+    M, N, K = 7, 9, 40
+    qa, sa = W.quantise_e4m3(W.normal((M, K), g), dim=1)
+    qb, sb = W.quantise_e4m3(W.normal((K, N), g), dim=0)
+    q = _problem(W.row_major(qa, "e4m3"), W.row_major(qb, "e4m3"), W.row_major(W.uniform((M, N), g), "f32"),
+                 -1.5, 0.5, sa, sb)
+    full, fbound = orc.gemm(q, want_bound=True)
+    ms = np.repeat(np.arange(M), N)
+    ns = np.tile(np.arange(N), M)
+    pts, pbound = orc.gemm_points(q, ms, ns)
+    assert np.array_equal(pts, full.reshape(-1))
+    assert np.array_equal(pbound, fbound.reshape(-1))
 
 
-PINS = [pin_hand_example, pin_view_address, pin_all_ones, pin_row_sums, pin_index_series,
+PINS = [pin_hand_example, pin_hand_bound_signed, pin_view_address, pin_all_ones, pin_row_sums, pin_index_series,
         pin_rank_one, pin_identity_and_permutation, pin_brute_force, pin_f16_bf16_tables,
         pin_e4m3_table, pin_pages_strided_example, pin_strided_equals_contiguous,
         pin_linearity_alpha_beta, pin_alpha_zero_beta_zero, pin_scales_once, pin_points_match_full]
@@ -303,6 +351,14 @@ MUTANTS = {
                        "for (int64_t k = 0; k + 1 < K; ++k) {\n                    double p"),
     "f16_bias_14": ("v = ldexp(1.0 + (double)f / 1024.0, e - 15);", "v = ldexp(1.0 + (double)f / 1024.0, e - 14);"),
     "beta_zero_reads_c": ("if (beta != 0.0) r += beta * elem(C, m, n);", "r += beta * elem(C, m, n);"),
+    # the rounding scale S = |alpha sa sb| sum_k |a b| that every GPU tolerance multiplies
+    "bound_is_mag": ("bound[m * N + n] = (a ? fabs(s) * mag : 0.0);", "bound[m * N + n] = (a ? mag : 0.0);"),
+    "bound_no_alpha": ("bound[m * N + n] = (a ? fabs(s) * mag : 0.0);",
+                       "bound[m * N + n] = (a ? fabs(s_m * s_n) * mag : 0.0);"),
+    "bound_signed_scale": ("bound[m * N + n] = (a ? fabs(s) * mag : 0.0);", "bound[m * N + n] = (a ? s * mag : 0.0);"),
+    "mag_signed_products": ("acc += p;\n                    mag += fabs(p);", "acc += p;\n                    mag += p;"),
+    "points_bound_is_mag": ("bound[i] = use_ab ? fabs(s) * mag : 0.0;", "bound[i] = use_ab ? mag : 0.0;"),
+    "points_mag_signed": ("acc += p;\n                mag += fabs(p);", "acc += p;\n                mag += p;"),
 }
 
 
