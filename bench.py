@@ -27,6 +27,7 @@ import argparse
 import hashlib
 import json
 import os
+import shutil
 import statistics
 import subprocess
 import sys
@@ -263,23 +264,29 @@ def time_problem(p_gpu_list, dg, reps: int, warm: int):
     return t_graph, t_stream, host
 
 
+# (key, name, workload, rotating copies).  The HBM-bound workloads rotate
+# through enough copies that every call reads at least twice the 126 MB L2
+# worth of other inputs between two uses of the same copy: gemv 3 x 117 MB,
+# gemv_kt 256 x 1 MB, thin 8 x 36 MB, strided 17 x 15 MB.  The square GEMMs are
+# compute-bound (2 copies); the small GEMM is launch-bound and L2-resident.
 SHAPES = [("small", "small_f16_128x128x256", W.cfg_small, 1),
           ("gemv", "gemv_bf16_1x14336x4096", W.cfg_gemv, ROTATE),
-          ("gemv_kt", "gemv_kt_bf16_1x128x4096", W.cfg_gemv_kt, 1),
-          ("thin", "thin_f16_64x4096x4096_beta1", W.cfg_thin, 4),
+          ("gemv_kt", "gemv_kt_bf16_1x128x4096", W.cfg_gemv_kt, 256),
+          ("thin", "thin_f16_64x4096x4096_beta1", W.cfg_thin, 8),
           ("square_bf16", "square_bf16_4096^3", W.cfg_square_bf16, 2),
           ("square_e4m3", "square_e4m3_4096^3", W.cfg_square_e4m3, 2),
-          ("strided", "strided_nchw_bf16_3136x1024x256", W.cfg_strided, 8)]
+          ("strided", "strided_nchw_bf16_3136x1024x256", W.cfg_strided, 17)]
 
 
 def per_shape(dg, peaks, quick: bool, only=None):
     """Every workload of the benchmark definition: time, TFLOPS, GB/s and
     fraction of roofline, with the dispatcher's kernel choice."""
     out = {}
-    reps = 20 if quick else 100
     for key, name, fn, copies in SHAPES:
         if only is not None and key != only:
             continue
+        # every copy is used at least once per graph, so the rotation is real
+        reps = max(20 if quick else 100, copies)
         base = fn()
         gpus = [base.to("cuda") for _ in range(copies)]
         A, B, C = dg_views(gpus[0], dg)
@@ -294,7 +301,8 @@ def per_shape(dg, peaks, quick: bool, only=None):
                      "roofline_us": t_roof * 1e6, "frac_of_roofline": t_roof / med,
                      "tiles": {k: pl[k] for k in ("block_n", "block_k", "split_k", "swap_ab", "p_gather", "grid")},
                      "timing": "CUDA-graph replay of the calls (device time); us_stream: back-to-back stream calls",
-                     "l2": f"{copies} rotating input copies" if copies > 1 else "single copy (L2-resident)"}
+                     "l2": (f"{copies} rotating input copies, {copies * by / 1e6:.0f} MB"
+                            if copies > 1 else "single copy (L2-resident)")}
         del gpus
         torch.cuda.empty_cache()
     return out
@@ -344,7 +352,9 @@ def run_dg(args):
         dg.dg_set_option(dg.DG_OPT_EARLY_LAUNCH, args.early_launch)
     dev = torch.device("cuda", torch.cuda.current_device())
     peaks = load_peaks()
-    stream = torch.cuda.Stream()  # graphs are captured on a side stream; every call of the step uses it
+    # graphs are captured on side streams; every call of the step uses them
+    stream = torch.cuda.Stream()   # x*W
+    side = torch.cuda.Stream()     # x*K^T, concurrent with x*W
 
     # ---- the step's data: three rotating copies of W and K, one x
     gv = W.cfg_gemv()
@@ -357,13 +367,16 @@ def run_dg(args):
         copies.append((a, b, dg_views(a, dg), dg_views(b, dg)))
     torch.cuda.synchronize()
 
-    # A step is the two dg_gemm calls on one stream.  The timed region replays
-    # CUDA graphs of those calls (captured once; the host launch cost of a
-    # call does not reach the device timeline).  Steps run in units of UNIT:
-    # the unit's x*W products as one graph, bracketed by CUDA events (the
-    # roofline's kernel timing covers every x*W launch of the timed region),
-    # then its x*K^T products as another.  UNIT is a multiple of ROTATE, so
-    # every unit starts on copy 0 and the copies keep rotating across units.
+    # A step is the two dg_gemm calls.  They are independent (both read x,
+    # each writes its own output), so x*K^T runs on a second stream beside
+    # x*W: the 1 MB x*K^T is launch-bound and fits on the SMs next to the two
+    # x*W blocks each SM holds.  The timed region replays CUDA graphs of the
+    # calls (captured once; the host launch cost of a call does not reach the
+    # device timeline) in units of UNIT steps: the unit's x*K^T calls on the
+    # side stream, forked from and joined back into the main stream, and its
+    # x*W calls on the main stream, bracketed by CUDA events (the roofline's
+    # kernel timing covers every x*W launch of the timed region).  UNIT is a
+    # multiple of ROTATE, so every unit starts on copy 0.
     UNIT = 16 * ROTATE
 
     def step(i):
@@ -377,14 +390,14 @@ def run_dg(args):
     torch.cuda.synchronize()
     assert dg.dg_sync_status(stream) == dg.DG_OK
 
-    def capture(which, n):
+    def capture(which, n, s):
         """A CUDA graph of n x*W (which=2) or x*K^T (which=3) calls over the
-        rotating copies, and the number of kernels it launches."""
+        rotating copies, captured on stream s, and the number of kernels it launches."""
         g = torch.cuda.CUDAGraph()
         n0 = dg.dg_launch_count()
-        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        with torch.cuda.graph(g, stream=s, capture_error_mode="relaxed"):
             for i in range(n):
-                assert dg.dg_gemm(*copies[i % ROTATE][which], 1.0, 0.0, None, None, stream) == 0
+                assert dg.dg_gemm(*copies[i % ROTATE][which], 1.0, 0.0, None, None, s) == 0
         return g, dg.dg_launch_count() - n0
 
     graphs = {}
@@ -393,7 +406,7 @@ def run_dg(args):
     while left > 0:
         n = min(UNIT, left)
         if n not in graphs:
-            graphs[n] = (capture(2, n), capture(3, n))
+            graphs[n] = (capture(2, n, stream), capture(3, n, side))
         units.append(n)
         left -= n
     torch.cuda.synchronize()
@@ -403,12 +416,19 @@ def run_dg(args):
         launches = 0
         for u, n in enumerate(units):
             (gw, nw), (gk, nk) = graphs[n]
+            fork = torch.cuda.Event()
+            join = torch.cuda.Event()
+            fork.record(stream)
+            side.wait_event(fork)
+            with torch.cuda.stream(side):
+                gk.replay()
+            join.record(side)
             if evs is not None:
                 evs[u][0].record(stream)
             gw.replay()
             if evs is not None:
                 evs[u][1].record(stream)
-            gk.replay()
+            stream.wait_event(join)
             launches += nw + nk
         return launches
 
@@ -433,7 +453,6 @@ def run_dg(args):
     w1 = time.time()
     barrier(world)
     time.sleep(0.25)
-    sampler.stop()
     assert dg.dg_sync_status(stream) == dg.DG_OK
     elapsed = t_start.elapsed_time(t_end) * 1e-3
     elapsed_max = max_over_ranks(elapsed, world, dev)
@@ -443,6 +462,32 @@ def run_dg(args):
     gemv_bytes = flops_bytes(gv)[1]
     achieved = gemv_bytes / gemv_avg / 1e9
     peak_hbm = peaks["hbm_gbs"]
+    clocks = sampler.summary(w0, w1)
+
+    # ---- the same kernel over a long window: at least 1000 back-to-back x*W
+    # launches (graph replays of UNIT calls), bracketed by CUDA events on its
+    # stream, with its own clock samples.  A short timed region weighs its
+    # first launch heavily; this one does not.
+    (gw_long, nw_long), _ = graphs.get(UNIT) or (capture(2, UNIT, stream), None)
+    reps_long = -(-1000 // UNIT)
+    with torch.cuda.stream(stream):
+        gw_long.replay()
+    torch.cuda.synchronize()
+    la, lb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0 = time.time()
+    with torch.cuda.stream(stream):
+        la.record(stream)
+        for _ in range(reps_long):
+            gw_long.replay()
+        lb.record(stream)
+    torch.cuda.synchronize()
+    l1 = time.time()
+    time.sleep(0.25)
+    sampler.stop()
+    assert dg.dg_sync_status(stream) == dg.DG_OK
+    long_launches = reps_long * UNIT
+    long_avg = la.elapsed_time(lb) * 1e-3 / long_launches
+    long_achieved = gemv_bytes / long_avg / 1e9
     traffic = kernel_traffic("gemv.cu", "gemv_n_decode_4096x14336.txt")
 
     result = {
@@ -451,16 +496,20 @@ def run_dg(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "bytes_per_step": step_bytes,
                    "l2": f"inputs rotate through {ROTATE} copies of W and K (352 MB > 126 MB L2)",
-                   "launch": f"two dg_gemm calls per step on one stream, replayed from CUDA graphs in units of "
-                             f"{UNIT} steps: the unit's x*W calls, bracketed by CUDA events, then its x*K^T calls",
+                   "launch": f"two dg_gemm calls per step, replayed from CUDA graphs in units of {UNIT} steps: "
+                             f"the unit's x*K^T calls on a second stream forked from the first, its x*W "
+                             f"calls on the first, bracketed by CUDA events",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "kernel": "gemv_n (x*W, 117 MB of W)", "achieved": achieved,
                      "timed_launches": args.steps,
                      "peak": peak_hbm, "unit": "GB/s", "frac": achieved / peak_hbm,
                      "traffic": traffic, "algorithmic_bytes": gemv_bytes, "avg_launch_us": gemv_avg * 1e6,
-                     "peak_source": f"{peaks['source']} hbm_gbs (STREAM-style copy)"},
+                     "peak_source": f"{peaks['source']} hbm_gbs (STREAM-style copy)",
+                     "long_window": {"launches": long_launches, "avg_launch_us": long_avg * 1e6,
+                                     "achieved": long_achieved, "frac": long_achieved / peak_hbm,
+                                     "clocks": sampler.summary(l0, l1)}},
         "gpu_launches": int(launches),
-        "clocks": sampler.summary(w0, w1),
+        "clocks": clocks,
     }
     if rank == 0:
         if not args.skip_cpu:
@@ -540,13 +589,18 @@ def _column_sample(gv: W.Problem, cols: int) -> W.Problem:
     return W.Problem(gv.name + f"_cols{cols}", gv.A, B, C)
 
 
-def cpu_baseline(quick: bool, target_s: float = 12.0):
-    """The FP64 oracle, as it stands, on this host's cores: repeated decode
-    steps (x*W and x*K^T) for about `target_s` seconds."""
+def _affinity_cores():
+    return sorted(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else list(range(os.cpu_count()))
+
+
+def cpu_baseline_worker(quick: bool, threads: int, target_s: float = 12.0):
+    """The FP64 oracle, as it stands, timed in this process: repeated decode
+    steps (x*W and x*K^T) on every core of the affinity set for about
+    `target_s` seconds, and the small 128x128x256 GEMM on one core.  Run under
+    taskset by cpu_baseline(); touches no GPU."""
     import oracle
 
     orc = oracle.default()
-    threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     gv, gk = W.cfg_gemv(), W.cfg_gemv_kt()
     step_bytes = flops_bytes(gv)[1] + flops_bytes(gk)[1]
     t0 = time.perf_counter()
@@ -557,9 +611,40 @@ def cpu_baseline(quick: bool, target_s: float = 12.0):
     for _ in range(reps):
         _oracle_step(orc, gv, gk, threads)
     t = (time.perf_counter() - t0) / reps
+    small = W.cfg_small()
+    fl_small = flops_bytes(small)[0]
+    orc.gemm(small, want_bound=False, nthreads=1)
+    n_small = 20
+    t0 = time.perf_counter()
+    for _ in range(n_small):
+        orc.gemm(small, want_bound=False, nthreads=1)
+    t_small = (time.perf_counter() - t0) / n_small
     return {"value": step_bytes / t / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"{reps} full decode steps (x*W 1x4096x14336 and x*K^T 1x4096x128), FP64, "
-                      f"{t:.3f} s per step"}
+                      f"{t:.3f} s per step, OpenMP threads bound to the affinity cores",
+            "small_1core": {"workload": "small F16 128x128x256 -> FP32", "s_per_call": t_small,
+                            "gflops": fl_small / t_small / 1e9, "cores": 1}}
+
+
+def cpu_baseline(quick: bool):
+    """cpu_baseline_worker in a child process pinned with taskset to the cores
+    this process may run on (OpenMP threads bound one per core)."""
+    cores = _affinity_cores()
+    env = dict(os.environ, OMP_PROC_BIND="close", OMP_PLACES="cores", CUDA_VISIBLE_DEVICES="")
+    # the parent counts the cores: in the child, the OpenMP runtime binds the
+    # initial thread to one core as soon as it is loaded
+    cmd = [sys.executable, os.path.abspath(__file__), "--cpu-baseline-worker", str(len(cores))] + \
+        (["--quick"] if quick else [])
+    if shutil.which("taskset"):
+        cmd = ["taskset", "-c", ",".join(str(c) for c in cores)] + cmd
+    r = subprocess.run(cmd, capture_output=True, text=True, env=env, timeout=600)
+    if r.returncode != 0:
+        return {"value": None, "unit": "GB/s", "cores": len(cores), "kind": "oracle",
+                "sample": "failed: " + (r.stderr.strip().splitlines() or ["?"])[-1]}
+    out = json.loads(r.stdout.strip().splitlines()[-1])
+    out["pinning"] = f"taskset -c {cores[0]}-{cores[-1]} ({len(cores)} cores)" if shutil.which("taskset") \
+        else "no taskset on this host"
+    return out
 
 
 def run_reference(args):
@@ -612,13 +697,16 @@ def main():
                          "square_e4m3, strided) and print its line")
     ap.add_argument("--max-split", type=int, default=0, help="with --shape: cap the tensor-core split-K")
     ap.add_argument("--trace", action="store_true", help="with --shape: phase timestamps of CTA 0")
+    ap.add_argument("--cpu-baseline-worker", type=int, default=0, help=argparse.SUPPRESS)
     ap.add_argument("--early-launch", type=int, default=-1,
                     help="programmatic dependent launch policy (0 off, 1 at kernel start, 2 near the end, "
                          "3 the library's per-kernel default)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.cpu_baseline_worker:
+        print(json.dumps(cpu_baseline_worker(args.quick, args.cpu_baseline_worker)), flush=True)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.shape:
         run_one_shape(args)

@@ -59,7 +59,11 @@ dg_status device_state(DeviceState **out) {
     DeviceState &d = g_dev[dev];
     if (!d.ready) {
         if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DG_ERR_CUDA;
-        if (cudaMalloc(&d.err_word, sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
+        // a word allocated by an earlier attempt whose later steps failed is reused, not leaked
+        if (!d.err_word && cudaMalloc(&d.err_word, sizeof(int)) != cudaSuccess) {
+            d.err_word = nullptr;
+            return DG_ERR_CUDA;
+        }
         if (cudaMemset(d.err_word, 0, sizeof(int)) != cudaSuccess) return DG_ERR_CUDA;
         if (cudaDeviceSynchronize() != cudaSuccess) return DG_ERR_CUDA;
         if (!g_encode) {
@@ -189,8 +193,9 @@ bool gemv_applicable(const Views &v, int64_t M, int64_t N, int64_t K, int kind) 
 }
 
 // GEMV_N grid: 256-column strips times k splits (one cluster per strip, at
-// most 8), about two blocks per SM, k ranges in whole 32-row TMA stages and
-// each block's slice of x within 64 KB of shared memory.
+// most 8), about two blocks per SM, k ranges in whole 64-row TMA stages (so
+// one split's last stage never reads the next split's rows) and each block's
+// slice of x within 64 KB of shared memory.
 void gemv_n_split(int64_t M, int64_t N, int64_t K, int num_sms, dg_plan_info *in) {
     const int64_t r_inst = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
     const int64_t gx = (N + 255) / 256;

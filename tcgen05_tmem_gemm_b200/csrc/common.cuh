@@ -1,6 +1,9 @@
 // Element load/store helpers and the shared epilogue arithmetic.
 #pragma once
 
+#include <atomic>
+#include <mutex>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -8,6 +11,32 @@
 #include "dg_internal.h"
 
 namespace dg {
+
+// The dynamic shared-memory limit of one kernel, raised per device: the
+// attribute set by cudaFuncSetAttribute belongs to the current device, so a
+// record per process would skip the call on a second device.  The limit only
+// ever grows (under a lock), so a launch that needs less never lowers it
+// beneath a concurrent launch that needs more.
+struct SmemLimit {
+    static constexpr int kDevices = 64;
+    std::atomic<int> bytes[kDevices] = {};
+    std::mutex mu;
+
+    template <typename Kern>
+    cudaError_t ensure(Kern kern, size_t need) {
+        if (need <= 48 * 1024) return cudaSuccess;  // the default limit
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kDevices) return cudaErrorInvalidDevice;
+        if (bytes[dev].load(std::memory_order_acquire) >= (int)need) return cudaSuccess;
+        std::lock_guard<std::mutex> lk(mu);
+        if (bytes[dev].load(std::memory_order_relaxed) >= (int)need) return cudaSuccess;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)need);
+        if (e == cudaSuccess) bytes[dev].store((int)need, std::memory_order_release);
+        return e;
+    }
+};
 
 // Programmatic dependent launch.  Every kernel here is launched with
 // programmatic stream serialisation: it may be scheduled while the previous

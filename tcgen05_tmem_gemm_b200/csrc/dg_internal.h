@@ -109,7 +109,7 @@ struct GemvParams {
     int32_t R, K, N;
     int32_t in_dtype;
     EpiParams epi;           // i = row of x, j = n
-    int32_t kper;            // GEMV_N: rows of W per block (multiple of 32)
+    int32_t kper;            // GEMV_N: rows of W per block (a multiple of the 64-row TMA stage)
     int32_t x_vec16;         // x unit-stride along k, 16-byte aligned rows, K % 8 == 0
     int64_t x_ld;            // bytes between rows of x (x_vec16 only)
     int *err_word;

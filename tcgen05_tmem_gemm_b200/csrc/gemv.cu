@@ -10,7 +10,7 @@
 // results are deterministic.
 //
 //  gemv_n:  W unit-stride along n (row-major [K, N]).  A block owns a strip of
-//           256 columns and a range of k.  One producer lane streams 32 x 256
+//           256 columns and a range of k.  One producer lane streams 64 x 256
 //           tiles of W into a ring of shared-memory stages with TMA (the bytes
 //           in flight per SM are the ring, not registers); eight consumer
 //           warps read them (a lane = 8 columns) and accumulate.  The k ranges
@@ -32,7 +32,9 @@ namespace dg {
 namespace {
 
 constexpr int kNB = 256;        // columns per gemv_n block
-constexpr int kRows = 64;       // rows of W per TMA stage (one 32 KB box: a TMA unit's byte rate grows with box size)
+constexpr int kRows = 64;       // rows of W per TMA stage (one 32 KB box: a TMA unit's byte rate grows with box size).
+                                // A block's k range (kper) is a whole number of stages, so no stage of one
+                                // k split reads rows of the next split.
 constexpr int kStages = 3;      // ring depth
 constexpr int kCW = 8;          // consumer warps
 constexpr int kNT = 32 * (kCW + 1);
@@ -360,15 +362,12 @@ __global__ void __launch_bounds__(256) gemv_k_kernel(const GemvParams p) {
     }
 }
 
-// Raise a kernel's dynamic shared-memory limit once per size, not per call
-// (`Tag` gives each kernel instantiation its own record).
+// Raise a kernel's dynamic shared-memory limit once per device and size, not
+// per call (`Tag` gives each kernel instantiation its own record).
 template <typename Tag, typename K>
 cudaError_t ensure_smem(K kern, size_t smem) {
-    static std::atomic<int> limit{48 * 1024};
-    if ((int)smem <= limit.load()) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess) limit.store((int)smem);
-    return e;
+    static SmemLimit limit;
+    return limit.ensure(kern, smem);
 }
 
 template <typename T, int R, int Kind>
@@ -376,6 +375,7 @@ struct KernelTag {};
 
 template <typename T, int R>
 cudaError_t run_n(const GemvParams &p, const CUtensorMap *tmap, cudaStream_t s, int *grid_out) {
+    if (p.kper <= 0 || p.kper % kRows != 0) return cudaErrorInvalidValue;  // whole stages per k split
     const int gx = (p.N + kNB - 1) / kNB;
     const int gy = (p.K + p.kper - 1) / p.kper;
     const size_t smem = gemv_n_layout(R, p.kper).total;

@@ -1076,15 +1076,10 @@ cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtens
     void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const UmmaParams);
     if (fp8) kern = gather ? umma_gemm_kernel<true, true> : umma_gemm_kernel<true, false>;
     else kern = gather ? umma_gemm_kernel<false, true> : umma_gemm_kernel<false, false>;
-    // raise the kernel's dynamic shared-memory limit once per size, not per call
-    static std::atomic<int> s_limit[4];
-    std::atomic<int> &lim = s_limit[(fp8 ? 2 : 0) + (gather ? 1 : 0)];
-    cudaError_t e = cudaSuccess;
-    if ((int)smem > lim.load()) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        lim.store((int)smem);
-    }
+    // raise the kernel's dynamic shared-memory limit once per device and size, not per call
+    static SmemLimit s_limit[4];
+    const cudaError_t e = s_limit[(fp8 ? 2 : 0) + (gather ? 1 : 0)].ensure(kern, smem);
+    if (e != cudaSuccess) return e;
     const int cluster = p.split_k > 1 ? p.split_k : (gather && p.gather_cluster > 1 ? p.gather_cluster : 1);
     return launch_ex(kern, dim3(grid), dim3(gather ? 448 : 192), smem, s, dim3(cluster, 1, 1), p.pdl, *tp, *tq, *tc,
                      p);

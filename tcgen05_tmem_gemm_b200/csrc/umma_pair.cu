@@ -305,13 +305,9 @@ cudaError_t launch_umma_pair(const UmmaParams &p, const CUtensorMap *tp, const C
                              const CUtensorMap *tc, bool fp8, int grid, size_t smem, cudaStream_t s) {
     void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const UmmaParams);
     kern = fp8 ? umma_pair_kernel<true> : umma_pair_kernel<false>;
-    static std::atomic<int> s_limit[2];
-    std::atomic<int> &lim = s_limit[fp8 ? 1 : 0];
-    if ((int)smem > lim.load()) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        lim.store((int)smem);
-    }
+    static SmemLimit s_limit[2];
+    const cudaError_t e = s_limit[fp8 ? 1 : 0].ensure(kern, smem);
+    if (e != cudaSuccess) return e;
     return launch_ex(kern, dim3(grid), dim3(192), smem, s, dim3(2, 1, 1), p.pdl, *tp, *tq, *tc, p);
 }
 

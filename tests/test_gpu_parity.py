@@ -1,8 +1,9 @@
 """GPU parity: the CUDA path through the C ABI against the FP64 oracle.
 
 Small problems are compared element by element (they span several tiles and
-end in ragged tails); the benchmark's full-size workloads, in the launch
-configuration the benchmark uses, are compared on sampled outputs computed
+end in ragged tails).  The benchmark's full-size workloads, in the launch
+configuration the benchmark uses, are compared element by element too, except
+the two 4096^3 products, whose tile corners and random outputs are computed
 one by one by the oracle.  Index and view handling is checked bit-exactly
 with identity and permutation operands.
 """
@@ -15,7 +16,7 @@ import torch
 import oracle
 import tcgen05_tmem_gemm_b200 as dg
 import workloads as W
-from harness import c_matrix, check_full, check_sampled, compare, dg_view_of, plan, run, tolerance
+from harness import c_matrix, check_full, check_sampled, compare, dg_view_of, plan, run, tile_corners, tolerance
 
 pytestmark = pytest.mark.gpu
 
@@ -557,14 +558,34 @@ def test_streams_and_launch_count():
     assert dg.dg_launch_count() == n0 + 1
 
 
-# ------------------------------------------------------ full-size, sampled
+# ------------------------------------------------------------- full size
+# The benchmark's workloads at their full sizes, in the launch configuration
+# the benchmark times (the plans are asserted).  Every output is compared with
+# the oracle where the oracle finishes in seconds (the decode GEMVs, the thin
+# projection and the strided view); the 4096^3 products are compared on the
+# four corners of every 128 x 128 block (each tile of either kernel shape has
+# its corners among them) plus 3000 random outputs.
 
-@pytest.mark.parametrize("name", ["gemv", "gemv_kt", "thin", "square_bf16", "square_e4m3", "strided"])
-def test_full_size_sampled(name):
+def _assert_bench_plan(name, pl):
+    if name == "thin":
+        assert pl["swap_ab"] == 1 and pl["split_k"] == 4, pl
+    if name == "strided":
+        assert pl["p_gather"] == 1 and pl["gather_cluster"] == 4, pl
+    if name.startswith("square"):
+        assert pl["cta_pair"] == 1, pl
+
+
+@pytest.mark.parametrize("name", ["gemv", "gemv_kt", "thin", "strided"])
+def test_full_size_every_output(name):
     p = W.WORKLOADS[name]()
     pl = expect_kind(p, {"gemv": "gemv_n", "gemv_kt": "gemv_k"}.get(name, "umma"))
-    if name == "thin":
-        assert pl["swap_ab"] == 1 and pl["split_k"] == 4
-    if name.startswith("square"):
-        assert pl["cta_pair"] == 1
-    check_sampled(p, npts=3000)
+    _assert_bench_plan(name, pl)
+    check_full(p)
+
+
+@pytest.mark.parametrize("name", ["square_bf16", "square_e4m3"])
+def test_full_size_square_tile_corners(name):
+    p = W.WORKLOADS[name]()
+    pl = expect_kind(p, "umma")
+    _assert_bench_plan(name, pl)
+    check_sampled(p, npts=3000, extra=tile_corners(p.M, p.N, 128, 128))
