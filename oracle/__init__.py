@@ -6,10 +6,13 @@ It shares no code with the CUDA path; both sides only share the seeded input
 generators in ``workloads.py``.
 
 The oracle computes, in FP64,
-    r[m, n] = alpha * sa[m] * sb[n] * sum_k a(m, k) b(k, n) + beta * c(m, n)
+    z[m, n] = alpha * sa[m] * sb[n] * sum_k a(m, k) b(k, n) + beta * c(m, n) + bias[n]
+    r[m, n] = act(z[m, n])      (identity, ReLU or GeLU in its tanh form)
 over byte-strided views ("DeepGEMM: a recalibration of the compute paradigm",
 §2.3 address formula and §3.2 view struct), decoding FP8 E4M3 from its bits
-("DeepGEMM deep dive", §2.4). See ``dg_oracle.c`` for the readings it takes
+("DeepGEMM deep dive", §2.4), with the fused bias and activation of "DeepGEMM is
+not a new model: the inner discipline of GPU matrix multiplication", §3.3.
+See ``dg_oracle.c`` for the readings it takes
 where the pages are silent.
 """
 from __future__ import annotations
@@ -26,6 +29,7 @@ _SRC = os.path.join(_HERE, "dg_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 DTYPE_CODE = {"f32": 0, "f16": 1, "bf16": 2, "e4m3": 3}
+ACT_CODE = {"none": 0, "relu": 1, "gelu_tanh": 2}
 
 
 class OView(ctypes.Structure):
@@ -57,14 +61,17 @@ class Oracle:
         L = ctypes.CDLL(path)
         P = ctypes.POINTER
         L.dgo_gemm.argtypes = [P(OView), P(OView), P(OView), ctypes.c_double, ctypes.c_double,
-                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-                               ctypes.c_int]
+                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
         L.dgo_gemm.restype = ctypes.c_int
         L.dgo_gemm_points.argtypes = [P(OView), P(OView), P(OView), ctypes.c_double,
                                       ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_void_p, ctypes.c_int,
                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
-                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
         L.dgo_gemm_points.restype = ctypes.c_int
+        L.dgo_activation.argtypes = [ctypes.c_int, ctypes.c_double]
+        L.dgo_activation.restype = ctypes.c_double
         L.dgo_decode_e4m3.argtypes = [ctypes.c_uint]
         L.dgo_decode_e4m3.restype = ctypes.c_double
         L.dgo_decode.argtypes = [ctypes.c_int, ctypes.c_void_p]
@@ -74,8 +81,9 @@ class Oracle:
         L.dgo_max_threads.restype = ctypes.c_int
         self.L = L
 
-    def gemm(self, problem, want_bound: bool = True, nthreads: int = 0):
-        """Full FP64 result (and the rounding scale S) as [M, N] float64 arrays."""
+    def gemm(self, problem, want_bound: bool = True, nthreads: int = 0, want_pre: bool = False):
+        """Full FP64 result as an [M, N] float64 array; with want_bound also the
+        rounding scale S, with want_pre also the value before the activation."""
         keep = []
         ops = (problem.A, problem.B, problem.C)
         bufs = [_Bytes(o) for o in ops]
@@ -83,17 +91,22 @@ class Oracle:
         M, N = problem.M, problem.N
         out = np.empty((M, N), dtype=np.float64)
         bound = np.empty((M, N), dtype=np.float64) if want_bound else None
+        pre = np.empty((M, N), dtype=np.float64) if want_pre else None
         st = self.L.dgo_gemm(ctypes.byref(va), ctypes.byref(vb), ctypes.byref(vc),
                              float(problem.alpha), float(problem.beta),
                              _scale_ptr(problem.scale_a, keep), _scale_ptr(problem.scale_b, keep),
+                             _scale_ptr(getattr(problem, "bias", None), keep),
+                             ACT_CODE[getattr(problem, "act", "none")],
                              out.ctypes.data, None if bound is None else bound.ctypes.data,
-                             nthreads)
+                             None if pre is None else pre.ctypes.data, nthreads)
         if st != 0:
             raise ValueError(f"oracle rejected the problem (status {st})")
-        return (out, bound) if want_bound else out
+        res = (out,) + ((bound,) if want_bound else ()) + ((pre,) if want_pre else ())
+        return res if len(res) > 1 else out
 
-    def gemm_points(self, problem, ms, ns, nthreads: int = 0):
-        """The definition evaluated at the sampled outputs (ms[i], ns[i])."""
+    def gemm_points(self, problem, ms, ns, nthreads: int = 0, want_pre: bool = False):
+        """The definition evaluated at the sampled outputs (ms[i], ns[i]):
+        (out, bound) or, with want_pre, (out, bound, pre)."""
         keep = []
         ops = (problem.A, problem.B, problem.C)
         bufs = [_Bytes(o) for o in ops]
@@ -102,15 +115,22 @@ class Oracle:
         ns = np.ascontiguousarray(np.asarray(ns, dtype=np.int64))
         out = np.empty(len(ms), dtype=np.float64)
         bound = np.empty(len(ms), dtype=np.float64)
+        pre = np.empty(len(ms), dtype=np.float64)
         st = self.L.dgo_gemm_points(ctypes.byref(va), ctypes.byref(vb), ctypes.byref(vc),
                                     float(problem.alpha), float(problem.beta),
                                     _scale_ptr(problem.scale_a, keep),
                                     _scale_ptr(problem.scale_b, keep),
+                                    _scale_ptr(getattr(problem, "bias", None), keep),
+                                    ACT_CODE[getattr(problem, "act", "none")],
                                     ms.ctypes.data, ns.ctypes.data, len(ms),
-                                    out.ctypes.data, bound.ctypes.data, nthreads)
+                                    out.ctypes.data, bound.ctypes.data, pre.ctypes.data, nthreads)
         if st != 0:
             raise ValueError(f"oracle rejected the problem (status {st})")
-        return out, bound
+        return (out, bound, pre) if want_pre else (out, bound)
+
+    def activation(self, act: str, z: float) -> float:
+        """The epilogue's activation applied to one FP64 value."""
+        return self.L.dgo_activation(ACT_CODE[act], float(z))
 
     def decode_e4m3(self, code: int) -> float:
         return self.L.dgo_decode_e4m3(code)
@@ -171,12 +191,16 @@ def _scale_ptr(s, keep):
     return a.ctypes.data
 
 
-def gemm(problem, want_bound: bool = True, nthreads: int = 0):
-    return default().gemm(problem, want_bound, nthreads)
+def gemm(problem, want_bound: bool = True, nthreads: int = 0, want_pre: bool = False):
+    return default().gemm(problem, want_bound, nthreads, want_pre)
 
 
-def gemm_points(problem, ms, ns, nthreads: int = 0):
-    return default().gemm_points(problem, ms, ns, nthreads)
+def gemm_points(problem, ms, ns, nthreads: int = 0, want_pre: bool = False):
+    return default().gemm_points(problem, ms, ns, nthreads, want_pre)
+
+
+def activation(act: str, z: float) -> float:
+    return default().activation(act, z)
 
 
 def decode_e4m3(code: int) -> float:

@@ -18,12 +18,26 @@
  *    rescale step ("DeepGEMM deep dive", §2.4 precision modes; §4.2 warns about
  *    a scale applied twice).
  *
+ *  - The fused epilogue: a bias vector broadcast over rows and an
+ *    element-wise activation applied to the result before it is stored
+ *    ("DeepGEMM is not a new model: the inner discipline of GPU matrix
+ *    multiplication", §3.3, GEMM + BiasAdd + GeLU with GeLU in its tanh
+ *    form; "DeepGEMM deep dive", §5.1 epilogue fusion):
+ *      out[m][n] = act( alpha * sa[m] * sb[n] * sum_k A[m][k] B[k][n]
+ *                       + beta * C[m][n] + bias[n] )
+ *    act is the identity, ReLU, or GeLU in the tanh form
+ *      gelu(z) = z/2 * (1 + tanh( sqrt(2/pi) * (z + 0.044715 z^3) )).
+ *
  * Readings where the pages are silent (each is listed in the design notes):
  *  - beta == 0: C is not read (BLAS convention), so NaN in C does not leak.
  *  - alpha == 0: the product is not formed; the result is beta * C, as the
  *    recalibration page's troubleshooting note (§4.3) requires beta to be
  *    applied even when the A-load is skipped.
  *  - scale pointers may be NULL, meaning all-ones scales.
+ *  - the bias is indexed by the output column n (one value per output
+ *    feature, the same for every row m) and may be NULL (no bias); the
+ *    activation is the last step before the store, after beta * C.
+ *  - ReLU keeps NaN (z < 0 ? 0 : z), so a NaN of the sum still reaches C.
  *  - Accumulation is FP64 in ascending k; no blocking or reordering.
  *
  * Decoders are written from the format definitions: IEEE binary16, bfloat16
@@ -40,6 +54,8 @@
 #endif
 
 enum { DGO_F32 = 0, DGO_F16 = 1, DGO_BF16 = 2, DGO_E4M3 = 3 };
+
+enum { DGO_ACT_NONE = 0, DGO_ACT_RELU = 1, DGO_ACT_GELU_TANH = 2 };
 
 enum {
     DGO_OK = 0,
@@ -173,14 +189,30 @@ static int check_views(const dgo_view *A, const dgo_view *B, const dgo_view *C,
     return DGO_OK;
 }
 
+/* ------------------------------------------------------------ activation */
+
+/* The element-wise activation of the fused epilogue, in FP64. */
+double dgo_activation(int act, double z) {
+    switch (act) {
+    case DGO_ACT_RELU: return z < 0.0 ? 0.0 : z;
+    case DGO_ACT_GELU_TANH: {
+        const double c = sqrt(2.0 / acos(-1.0)); /* sqrt(2 / pi) */
+        return 0.5 * z * (1.0 + tanh(c * (z + 0.044715 * z * z * z)));
+    }
+    default: return z;
+    }
+}
+
 /* -------------------------------------------------------------- the GEMM */
 
 /*
  * Full oracle.  out[m*N + n] receives
- *     r = alpha * sa[m] * sb[n] * sum_k a(m,k) b(k,n)  +  beta * c(m,n)
- * in FP64 (c read only when beta != 0; the sum skipped when alpha == 0), and
- * bound[m*N + n] (if non-NULL) receives |alpha * sa[m] * sb[n]| * sum_k |a b|,
- * the scale against which rounding of the sum is judged.
+ *     z = alpha * sa[m] * sb[n] * sum_k a(m,k) b(k,n)  +  beta * c(m,n)  +  bias[n]
+ *     out = act(z)
+ * in FP64 (c read only when beta != 0; the sum skipped when alpha == 0; the
+ * bias term 0 when bias is NULL), bound[m*N + n] (if non-NULL) receives
+ * |alpha * sa[m] * sb[n]| * sum_k |a b|, the scale against which rounding of
+ * the sum is judged, and pre[m*N + n] (if non-NULL) receives z.
  *
  * A and B are first decoded into FP64 matrices through the view addressing
  * (B stored transposed so the k loop walks memory in order); the triple loop
@@ -188,7 +220,8 @@ static int check_views(const dgo_view *A, const dgo_view *B, const dgo_view *C,
  */
 int dgo_gemm(const dgo_view *A, const dgo_view *B, const dgo_view *C,
              double alpha, double beta, const float *sa, const float *sb,
-             double *out, double *bound, int nthreads) {
+             const float *bias, int act,
+             double *out, double *bound, double *pre, int nthreads) {
     int64_t M, N, K;
     int st = check_views(A, B, C, &M, &N, &K);
     if (st) return st;
@@ -237,7 +270,9 @@ int dgo_gemm(const dgo_view *A, const dgo_view *B, const dgo_view *C,
             double s = alpha * s_m * s_n;
             double r = (a ? s * acc : 0.0);
             if (beta != 0.0) r += beta * elem(C, m, n);
-            out[m * N + n] = r;
+            if (bias) r += (double)bias[n];
+            out[m * N + n] = dgo_activation(act, r);
+            if (pre) pre[m * N + n] = r;
             if (bound) bound[m * N + n] = (a ? fabs(s) * mag : 0.0);
         }
     }
@@ -249,12 +284,14 @@ int dgo_gemm(const dgo_view *A, const dgo_view *B, const dgo_view *C,
 /*
  * The same definition evaluated one output at a time, straight from the
  * views (no pre-decoded copies): used to check sampled outputs of problems
- * too large for the full oracle.
+ * too large for the full oracle.  out, bound and pre as in dgo_gemm, one
+ * entry per point (ms[i], ns[i]).
  */
 int dgo_gemm_points(const dgo_view *A, const dgo_view *B, const dgo_view *C,
                     double alpha, double beta, const float *sa, const float *sb,
+                    const float *bias, int act,
                     const int64_t *ms, const int64_t *ns, int64_t npts,
-                    double *out, double *bound, int nthreads) {
+                    double *out, double *bound, double *pre, int nthreads) {
     int64_t M, N, K;
     int st = check_views(A, B, C, &M, &N, &K);
     if (st) return st;
@@ -280,7 +317,9 @@ int dgo_gemm_points(const dgo_view *A, const dgo_view *B, const dgo_view *C,
         double s = alpha * (sa ? (double)sa[m] : 1.0) * (sb ? (double)sb[n] : 1.0);
         double r = use_ab ? s * acc : 0.0;
         if (beta != 0.0) r += beta * elem(C, m, n);
-        out[i] = r;
+        if (bias) r += (double)bias[n];
+        out[i] = dgo_activation(act, r);
+        if (pre) pre[i] = r;
         if (bound) bound[i] = use_ab ? fabs(s) * mag : 0.0;
     }
     return DGO_OK;

@@ -18,7 +18,12 @@ oracle's own code:
     which every GPU tolerance multiplies): worked by hand on a mixed-sign case
     with a negative alpha and scales (tests/golden/hand_gemm_bound_signed.json),
     exact rationals in the brute-force pin, E4M3 powers of two, and the
-    one-by-one evaluation equal to the full one.
+    one-by-one evaluation equal to the full one;
+  * the fused epilogue (Inner discipline page, §3.3): a hand-worked bias + ReLU
+    case that fixes the bias to the output column and the activation after
+    beta*C (tests/golden/hand_gemm_bias_relu.json); GeLU's tanh form within its
+    4.73e-4 approximation error of z*Phi(z) (Phi from libm's erf), its odd-part
+    identity g(z) - g(-z) = z, slope 1/2 at 0 and limits; ReLU's closed forms.
 The last test plants mistakes in a copy of the oracle source and checks that
 some pin catches every one of them.
 """
@@ -39,8 +44,8 @@ import workloads as W
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
-def _problem(A, B, C, alpha=1.0, beta=0.0, sa=None, sb=None):
-    return W.Problem("pin", A, B, C, alpha, beta, sa, sb)
+def _problem(A, B, C, alpha=1.0, beta=0.0, sa=None, sb=None, bias=None, act="none"):
+    return W.Problem("pin", A, B, C, alpha, beta, sa, sb, bias=bias, act=act)
 
 
 def _f32(x):
@@ -325,10 +330,85 @@ def pin_points_match_full(orc):
     assert np.array_equal(pbound, fbound.reshape(-1))
 
 
+# ------------------------------------------------------ the fused epilogue
+
+def pin_epilogue_hand(orc):
+    g = json.load(open(os.path.join(GOLDEN, "hand_gemm_bias_relu.json")))
+    p = _problem(_f32(g["A"]), _f32(g["B"]), _f32(g["C"]), g["alpha"], g["beta"],
+                 bias=torch.tensor(g["bias"]), act=g["act"])
+    out, bound, pre = orc.gemm(p, want_bound=True, want_pre=True)
+    assert np.array_equal(pre, np.array(g["expected_pre"]))
+    assert np.array_equal(out, np.array(g["expected"]))
+    assert np.array_equal(bound, np.array([[58.0, 64.0], [139.0, 154.0]]))  # S has no bias or C term
+
+
+def _phi(z):
+    return 0.5 * (1.0 + math.erf(z / math.sqrt(2.0)))
+
+
+def pin_gelu_closed_forms(orc):
+    # GeLU(z) = z Phi(z); the tanh form (Inner discipline page, §3.3) is within
+    # 4.73e-4 of it everywhere (the approximation's published maximum error);
+    # Phi comes from libm's erf, an independent special function.
+    g = lambda z: orc.activation("gelu_tanh", z)  # noqa: E731
+    assert g(0.0) == 0.0
+    for i in range(-800, 801):
+        z = i / 100.0
+        assert abs(g(z) - z * _phi(z)) <= 5e-4, z
+        # z Phi(z) - (-z) Phi(-z) = z since Phi(z) + Phi(-z) = 1; the tanh form keeps it (tanh is odd)
+        assert abs((g(z) - g(-z)) - z) <= 4e-16 * max(1.0, abs(z)), z
+    assert g(20.0) == 20.0 and abs(g(-20.0)) <= 1e-300
+    h = 1e-6  # slope 1/2 at 0: Phi(0) = 1/2
+    assert abs((g(h) - g(-h)) / (2 * h) - 0.5) <= 1e-9
+    assert math.isnan(g(float("nan")))
+
+
+def pin_relu_closed_forms(orc):
+    r = lambda z: orc.activation("relu", z)  # noqa: E731
+    for z in (-3.5, -1e-30, 0.0, 2.5, 1e30):
+        assert r(z) - r(-z) == z and r(z) >= 0.0
+    assert r(-2.0) == 0.0 and r(7.25) == 7.25
+    assert math.isnan(r(float("nan")))  # a NaN of the sum still reaches C
+    assert orc.activation("none", -4.5) == -4.5
+
+
+def _epi_problem(act, seed=13, bias=True):
+    g = torch.Generator().manual_seed(seed)
+    M, N, K = 6, 10, 24
+    a = W.cast(W.normal((M, K), g), "bf16")
+    b = W.cast(W.normal((K, N), g), "bf16")
+    c = W.uniform((M, N), g)
+    bv = W.normal((N,), g)  # drawn either way, so the scales below are the same draws
+    return _problem(W.row_major(a, "bf16"), W.row_major(b, "bf16"), W.row_major(c.contiguous(), "f32"),
+                    0.5, -1.5, torch.rand(M, generator=g) + 0.5, torch.rand(N, generator=g) + 0.5,
+                    bv if bias else None, act)
+
+
+def pin_bias_per_column_and_activation_last(orc):
+    # the bias is added once per output column, to every row
+    with_b = orc.gemm(_epi_problem("none"), want_bound=False)
+    without = orc.gemm(_epi_problem("none", bias=False), want_bound=False)
+    bias = _epi_problem("none").bias.double().numpy()
+    assert np.allclose(with_b - without, np.broadcast_to(bias, with_b.shape), rtol=0, atol=1e-13)
+    # the activation acts on the whole sum (product, beta*C and bias)
+    relu = orc.gemm(_epi_problem("relu"), want_bound=False)
+    assert np.array_equal(relu, np.where(with_b < 0, 0.0, with_b))
+    gelu = orc.gemm(_epi_problem("gelu_tanh"), want_bound=False)
+    exact = np.vectorize(lambda z: z * _phi(z))(with_b)
+    assert np.all(np.abs(gelu - exact) <= 5e-4)
+    # the one-by-one evaluation agrees, including the value before the activation
+    ms = np.repeat(np.arange(6), 10)
+    ns = np.tile(np.arange(10), 6)
+    pts, _, pre = orc.gemm_points(_epi_problem("gelu_tanh"), ms, ns, want_pre=True)
+    assert np.array_equal(pts, gelu.reshape(-1))
+    assert np.array_equal(pre, with_b.reshape(-1))
+
+
 PINS = [pin_hand_example, pin_hand_bound_signed, pin_view_address, pin_all_ones, pin_row_sums, pin_index_series,
         pin_rank_one, pin_identity_and_permutation, pin_brute_force, pin_f16_bf16_tables,
         pin_e4m3_table, pin_pages_strided_example, pin_strided_equals_contiguous,
-        pin_linearity_alpha_beta, pin_alpha_zero_beta_zero, pin_scales_once, pin_points_match_full]
+        pin_linearity_alpha_beta, pin_alpha_zero_beta_zero, pin_scales_once, pin_points_match_full,
+        pin_epilogue_hand, pin_gelu_closed_forms, pin_relu_closed_forms, pin_bias_per_column_and_activation_last]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[f.__name__ for f in PINS])
@@ -359,6 +439,20 @@ MUTANTS = {
     "mag_signed_products": ("acc += p;\n                    mag += fabs(p);", "acc += p;\n                    mag += p;"),
     "points_bound_is_mag": ("bound[i] = use_ab ? fabs(s) * mag : 0.0;", "bound[i] = use_ab ? mag : 0.0;"),
     "points_mag_signed": ("acc += p;\n                mag += fabs(p);", "acc += p;\n                mag += p;"),
+    # the fused epilogue: bias, activation and their order
+    "bias_per_row": ("if (bias) r += (double)bias[n];\n            out[m * N + n]",
+                     "if (bias) r += (double)bias[m % N];\n            out[m * N + n]"),
+    "activation_before_beta_c": (
+        "if (beta != 0.0) r += beta * elem(C, m, n);\n            if (bias) r += (double)bias[n];\n"
+        "            out[m * N + n] = dgo_activation(act, r);",
+        "if (bias) r += (double)bias[n];\n"
+        "            out[m * N + n] = dgo_activation(act, r) + (beta != 0.0 ? beta * elem(C, m, n) : 0.0);"),
+    "activation_dropped": ("out[m * N + n] = dgo_activation(act, r);", "out[m * N + n] = r;"),
+    "gelu_no_cubic": ("tanh(c * (z + 0.044715 * z * z * z))", "tanh(c * z)"),
+    "gelu_no_half": ("return 0.5 * z * (1.0 + tanh", "return z * (1.0 + tanh"),
+    "gelu_wrong_constant": ("sqrt(2.0 / acos(-1.0))", "sqrt(2.0 * acos(-1.0))"),
+    "relu_abs": ("case DGO_ACT_RELU: return z < 0.0 ? 0.0 : z;", "case DGO_ACT_RELU: return fabs(z);"),
+    "points_bias_dropped": ("if (bias) r += (double)bias[n];\n        out[i]", "out[i]"),
 }
 
 

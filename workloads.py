@@ -81,6 +81,8 @@ class Problem:
     scale_b: Optional[torch.Tensor] = None  # float32 [N] or None
     note: str = ""
     extra: dict = field(default_factory=dict)
+    bias: Optional[torch.Tensor] = None     # float32 [N] or None (fused epilogue)
+    act: str = "none"                       # "none", "relu" or "gelu_tanh" (fused epilogue)
 
     @property
     def M(self) -> int:
@@ -99,7 +101,8 @@ class Problem:
                        self.alpha, self.beta,
                        None if self.scale_a is None else self.scale_a.to(device),
                        None if self.scale_b is None else self.scale_b.to(device),
-                       self.note, dict(self.extra))
+                       self.note, dict(self.extra),
+                       None if self.bias is None else self.bias.to(device), self.act)
 
 
 def row_major(t: torch.Tensor, dtype: str, row_dims: int = 1) -> Operand:
