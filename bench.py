@@ -73,6 +73,8 @@ def flops_bytes(p: W.Problem):
         b += 4 * M
     if p.scale_b is not None:
         b += 4 * N
+    if p.bias is not None:
+        b += 4 * N
     return 2.0 * M * N * K, float(b)
 
 
@@ -230,11 +232,17 @@ def time_problem(p_gpu_list, dg, reps: int, warm: int):
     views = [dg_views(p, dg) for p in p_gpu_list]
     s = torch.cuda.Stream()
 
+    epis = [dg.epilogue(q.bias, q.act) if (q.bias is not None or q.act != "none") else None for q in p_gpu_list]
+
     def calls(n, stream):
         for i in range(n):
             q = p_gpu_list[i % len(views)]
             A, B, C = views[i % len(views)]
-            st = dg.dg_gemm(A, B, C, q.alpha, q.beta, q.scale_a, q.scale_b, stream)
+            e = epis[i % len(views)]
+            if e is None:
+                st = dg.dg_gemm(A, B, C, q.alpha, q.beta, q.scale_a, q.scale_b, stream)
+            else:
+                st = dg.dg_gemm_ex(A, B, C, q.alpha, q.beta, q.scale_a, q.scale_b, e, stream)
             assert st == dg.DG_OK, dg.status_string(st)
 
     with torch.cuda.stream(s):
@@ -275,7 +283,22 @@ SHAPES = [("small", "small_f16_128x128x256", W.cfg_small, 1),
           ("thin", "thin_f16_64x4096x4096_beta1", W.cfg_thin, 8),
           ("square_bf16", "square_bf16_4096^3", W.cfg_square_bf16, 2),
           ("square_e4m3", "square_e4m3_4096^3", W.cfg_square_e4m3, 2),
-          ("strided", "strided_nchw_bf16_3136x1024x256", W.cfg_strided, 17)]
+          ("strided", "strided_nchw_bf16_3136x1024x256", W.cfg_strided, 17),
+          # the fused epilogue (bias per output column + activation, one kernel)
+          ("square_bf16_gelu", "square_bf16_4096^3_bias_gelu",
+           lambda: W.with_epilogue(W.cfg_square_bf16(), "gelu_tanh"), 2),
+          ("thin_gelu", "thin_f16_64x4096x4096_beta1_bias_gelu",
+           lambda: W.with_epilogue(W.cfg_thin(), "gelu_tanh"), 8),
+          ("strided_nchw_out", "strided_nchw_bf16_3136x1024x256_to_nchw_bias_relu",
+           lambda: _strided_nchw_out(), 17)]
+
+
+def _strided_nchw_out() -> W.Problem:
+    """The strided workload with its output written as an NCHW tensor
+    [16, 1024, 14, 14] by the epilogue, with a bias and ReLU fused."""
+    p = W.with_epilogue(W.cfg_strided(), "relu")
+    return W.Problem(p.name + "_nchw_out", p.A, p.B, W.nchw_out(16, 1024, 14, 14), 1.0, 0.0,
+                     bias=p.bias, act="relu")
 
 
 def per_shape(dg, peaks, quick: bool, only=None):
@@ -694,7 +717,7 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true", help="no CPU baseline and no e2e leg (profiling runs)")
     ap.add_argument("--shape", default=None,
                     help="time only this per-shape workload (small, gemv, gemv_kt, thin, square_bf16, "
-                         "square_e4m3, strided) and print its line")
+                         "square_e4m3, strided, square_bf16_gelu, thin_gelu, strided_nchw_out) and print its line")
     ap.add_argument("--max-split", type=int, default=0, help="with --shape: cap the tensor-core split-K")
     ap.add_argument("--trace", action="store_true", help="with --shape: phase timestamps of CTA 0")
     ap.add_argument("--cpu-baseline-worker", type=int, default=0, help=argparse.SUPPRESS)

@@ -110,6 +110,51 @@ dg_status dg_gemm(const dg_view *A, const dg_view *B, const dg_view *C,
                   const float *scale_a, const float *scale_b,
                   void *stream);
 
+/* Activations of the fused epilogue. */
+typedef enum {
+    DG_ACT_NONE = 0,       /* identity                                              */
+    DG_ACT_RELU = 1,       /* z < 0 ? 0 : z (a NaN stays NaN)                        */
+    DG_ACT_GELU_TANH = 2   /* z/2 * (1 + tanh(sqrt(2/pi) * (z + 0.044715 z^3)))      */
+} dg_activation;
+
+/*
+ * The fused epilogue ("DeepGEMM is not a new model: the inner discipline of
+ * GPU matrix multiplication", §3.3: GEMM + BiasAdd + GeLU in one kernel, the
+ * bias broadcast in registers and GeLU in its tanh form before the store;
+ * "DeepGEMM deep dive", §5.1 epilogue fusion).  The GEMM result is turned
+ * into
+ *     C[m][n] = act( alpha * sa[m] * sb[n] * sum_k A[m][k] B[k][n]
+ *                    + beta * C[m][n] + bias[n] )
+ * before it is stored, so no intermediate output goes through memory.
+ *  bias        device float32[N] (one value per output column n, the same for
+ *              every row m), or NULL for no bias.  Read only; owned by the
+ *              caller.
+ *  activation  a dg_activation value; anything else is DG_ERR_VALUE.
+ *  reserved    set to 0 (anything else is DG_ERR_VALUE).
+ * The layout transform of the fusion (e.g. writing an NCHW output from an
+ * [N*H*W, C] product) needs no field: C is a strided view, and the
+ * tensor-core epilogue addresses a row of C through any number of dims.
+ */
+typedef struct {
+    const float *bias;
+    int32_t activation;
+    int32_t reserved;
+} dg_epilogue;
+
+/*
+ * dg_gemm_ex — dg_gemm with a fused epilogue (above).  `epilogue` NULL (or
+ * no bias with DG_ACT_NONE) is exactly dg_gemm.  The epilogue runs on every
+ * path: the tensor-core kernels (single CTA, CTA pairs, split-K clusters,
+ * gathered operands), the GEMVs, the CUDA-core kernel, and alpha == 0 or
+ * K == 0, where C = act(beta * C + bias).  Errors as dg_gemm, plus
+ * DG_ERR_VALUE for a bad activation or reserved field and DG_ERR_POINTER for
+ * a bias that is not device memory of the current device.
+ */
+dg_status dg_gemm_ex(const dg_view *A, const dg_view *B, const dg_view *C,
+                     float alpha, float beta,
+                     const float *scale_a, const float *scale_b,
+                     const dg_epilogue *epilogue, void *stream);
+
 /*
  * dg_gemv — y = alpha * x W + beta * y for a single row (or up to 8 rows) of
  * activations: the decode-time thin GEMM of "DeepGEMM is not a new model: the

@@ -2,7 +2,7 @@
 
 Argument marshalling only: every step of the computation runs in the CUDA
 kernels behind the C ABI declared in include/dg.h.  The names mirror the C
-entry points (dg_gemm, dg_gemv, dg_sync_status, ...).  PyTorch is used by
+entry points (dg_gemm, dg_gemm_ex, dg_gemv, dg_sync_status, ...).  PyTorch is used by
 callers for device memory and streams; a torch tensor can be turned into a
 view with `view()`.
 
@@ -28,6 +28,9 @@ ELEM_SIZE = {DG_F32: 4, DG_F16: 2, DG_BF16: 2, DG_E4M3: 1}
  DG_KIND_UMMA) = range(6)
 KIND_NAME = {0: "none", 1: "scale_c", 2: "simt", 3: "gemv_n", 4: "gemv_k", 5: "umma"}
 
+DG_ACT_NONE, DG_ACT_RELU, DG_ACT_GELU_TANH = 0, 1, 2
+ACT = {"none": DG_ACT_NONE, "relu": DG_ACT_RELU, "gelu_tanh": DG_ACT_GELU_TANH}
+
 (DG_OPT_FORCE_KIND, DG_OPT_WAIT_TIMEOUT_MS, DG_OPT_TEST_STALL, DG_OPT_MAX_SPLIT_K, DG_OPT_CTA_PAIR,
  DG_OPT_EARLY_LAUNCH, DG_OPT_TRACE, DG_OPT_EPI_TMA, DG_OPT_GATHER_CLUSTER,
  DG_OPT_PAIR_TAIL) = 1, 2, 3, 4, 5, 6, 7, 8, 9, 10
@@ -41,6 +44,14 @@ class dg_view(ctypes.Structure):
         ("shape", ctypes.c_int64 * 4),
         ("stride", ctypes.c_int64 * 4),
         ("dtype", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+
+class dg_epilogue(ctypes.Structure):
+    _fields_ = [
+        ("bias", ctypes.c_void_p),
+        ("activation", ctypes.c_int32),
         ("reserved", ctypes.c_int32),
     ]
 
@@ -90,6 +101,9 @@ def _load():
     L.dg_gemm.argtypes = [V, V, V, ctypes.c_float, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                           ctypes.c_void_p]
     L.dg_gemm.restype = ctypes.c_int
+    L.dg_gemm_ex.argtypes = [V, V, V, ctypes.c_float, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                             P(dg_epilogue), ctypes.c_void_p]
+    L.dg_gemm_ex.restype = ctypes.c_int
     L.dg_gemv.argtypes = [V, V, V, ctypes.c_float, ctypes.c_float, ctypes.c_void_p]
     L.dg_gemv.restype = ctypes.c_int
     L.dg_status_string.argtypes = [ctypes.c_int]
@@ -192,6 +206,23 @@ def dg_gemm(A: dg_view, B: dg_view, C: dg_view, alpha: float, beta: float,
                        _ptr(scale_a), _ptr(scale_b), _stream_ptr(stream))
 
 
+def epilogue(bias=None, act="none") -> dg_epilogue:
+    """A dg_epilogue: bias (device float32[N] tensor, address or None) and activation."""
+    e = dg_epilogue()
+    e.bias = ctypes.c_void_p(_ptr(bias) or 0)
+    e.activation = ACT[act] if isinstance(act, str) else int(act)
+    e.reserved = 0
+    return e
+
+
+def dg_gemm_ex(A: dg_view, B: dg_view, C: dg_view, alpha: float, beta: float,
+               scale_a=None, scale_b=None, epi=None, stream=None) -> int:
+    """dg_gemm with a fused epilogue C = act(... + beta * C + bias); returns the status."""
+    return lib.dg_gemm_ex(ctypes.byref(A), ctypes.byref(B), ctypes.byref(C), float(alpha), float(beta),
+                          _ptr(scale_a), _ptr(scale_b), None if epi is None else ctypes.byref(epi),
+                          _stream_ptr(stream))
+
+
 def dg_gemv(x: dg_view, W: dg_view, y: dg_view, alpha: float, beta: float, stream=None) -> int:
     return lib.dg_gemv(ctypes.byref(x), ctypes.byref(W), ctypes.byref(y), float(alpha), float(beta),
                        _stream_ptr(stream))
@@ -236,10 +267,16 @@ def dg_version() -> int:
 # ----------------------------------------------------------- conveniences
 
 def gemm(A, B, C, alpha: float = 1.0, beta: float = 0.0, scale_a=None, scale_b=None,
-         stream=None, a_row_dims: int = 1, b_row_dims: int = 1, c_row_dims: int = 1):
-    """dg_gemm on torch tensors (or dg_view objects); raises DgError on a bad status."""
-    st = dg_gemm(_as_view(A, a_row_dims), _as_view(B, b_row_dims), _as_view(C, c_row_dims),
-                 alpha, beta, scale_a, scale_b, stream)
+         stream=None, a_row_dims: int = 1, b_row_dims: int = 1, c_row_dims: int = 1,
+         bias=None, act="none"):
+    """dg_gemm (dg_gemm_ex when a bias or activation is given) on torch tensors
+    or dg_view objects; raises DgError on a bad status."""
+    if bias is None and act in ("none", DG_ACT_NONE):
+        st = dg_gemm(_as_view(A, a_row_dims), _as_view(B, b_row_dims), _as_view(C, c_row_dims),
+                     alpha, beta, scale_a, scale_b, stream)
+    else:
+        st = dg_gemm_ex(_as_view(A, a_row_dims), _as_view(B, b_row_dims), _as_view(C, c_row_dims),
+                        alpha, beta, scale_a, scale_b, epilogue(bias, act), stream)
     if st != DG_OK:
         raise DgError(st, "dg_gemm")
     return C

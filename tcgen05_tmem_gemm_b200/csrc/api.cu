@@ -219,7 +219,6 @@ void gemv_n_split(int64_t M, int64_t N, int64_t K, int num_sms, dg_plan_info *in
 bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int num_sms, Plan *pl) {
     const int dt = v.A->dtype;
     if (dt != DG_F16 && dt != DG_BF16 && dt != DG_E4M3) return false;
-    if (v.c.row.n > 1 || v.c.col.n > 1) return false;
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return false;
     const bool a_tma = v.a.tma_ok, b_tma = v.b.tma_ok;
     if (!a_tma && !b_tma) return false;
@@ -228,6 +227,10 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     if (!a_tma) swap = false;       // A is loaded by threads as the M-side operand
     else if (!b_tma) swap = true;   // B is, after the swap
     else swap = thin;
+    // C: the epilogue addresses a row (i) through any number of merged dims,
+    // computed once per row (a layout transform such as writing an NCHW
+    // output from an [N*H*W, C] product), and walks j with one stride
+    if ((swap ? v.c.row.n : v.c.col.n) > 1) return false;
     const ViewInfo &pvi = swap ? v.b : v.a;
     const bool p_tma = swap ? b_tma : a_tma;
     // unit-stride direction of P(i, k) and Q(k, j)
@@ -488,19 +491,29 @@ bool encode_2d(CUtensorMap *m, int dt, const void *ptr, int64_t inner, int64_t o
     return encode_2d_box(m, dt, ptr, inner, outer, outer_stride, 128 / elem_size(dt), box_outer, true);
 }
 
-EpiParams epi_params(const Views &v, bool swap, float alpha, float beta, const float *sa, const float *sb) {
+EpiParams epi_params(const Views &v, bool swap, float alpha, float beta, const float *sa, const float *sb,
+                     const float *bias, int act) {
     EpiParams e{};
     e.c = static_cast<char *>(v.C->ptr);
     const int64_t crs = axis_stride(v.c.row), ccs = axis_stride(v.c.col);
     e.ci = swap ? ccs : crs;
     e.cj = swap ? crs : ccs;
     e.c_dtype = v.C->dtype;
+    const Axis &ia = swap ? v.c.col : v.c.row;
+    e.ci_multi = ia.n > 1;
+    e.ci_axis = ia;
+    bool rows16 = true;  // every row starts 16-byte aligned
+    for (int d = 0; d < ia.n; ++d) rows16 = rows16 && ia.stride[d] % 16 == 0;
     const int ces = elem_size(v.C->dtype);
-    e.vec_ok = (e.cj == ces) && (reinterpret_cast<uintptr_t>(e.c) % 16 == 0) && (e.ci % 16 == 0);
+    e.vec_ok = (e.cj == ces) && (reinterpret_cast<uintptr_t>(e.c) % 16 == 0) && rows16;
     e.alpha = alpha;
     e.beta = beta;
     e.scale_i = swap ? sb : sa;
     e.scale_j = swap ? sa : sb;
+    // the bias belongs to the output column n: j, or i when the kernel computes C^T
+    e.bias_i = swap ? bias : nullptr;
+    e.bias_j = swap ? nullptr : bias;
+    e.act = act;
     return e;
 }
 
@@ -511,6 +524,8 @@ struct LaunchRec {
     DevView c{};
     int64_t M = 0, N = 0;
     float beta = 0.f;
+    const float *bias = nullptr;  // scale_c: the fused epilogue
+    int act = DG_ACT_NONE;
     int pdl = 0;
     SimtParams simt{};
     GemvParams gemv{};
@@ -522,7 +537,7 @@ struct LaunchRec {
 };
 
 dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const float *sa, const float *sb,
-                  DeviceState *ds, LaunchRec *rec) {
+                  const float *bias, int act, DeviceState *ds, LaunchRec *rec) {
     const dg_plan_info &in = pl.info;
     rec->kind = in.kind;
     // early launch, mode 3: the launch-bound K-contiguous GEMV (64 blocks: the
@@ -538,6 +553,8 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         rec->M = in.M;
         rec->N = in.N;
         rec->beta = beta;
+        rec->bias = bias;
+        rec->act = act;
         break;
     }
     case DG_KIND_SIMT: {
@@ -548,7 +565,7 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         p.M = (int32_t)in.M;
         p.N = (int32_t)in.N;
         p.K = (int32_t)in.K;
-        p.epi = epi_params(v, false, alpha, beta, sa, sb);
+        p.epi = epi_params(v, false, alpha, beta, sa, sb, bias, act);
         p.pdl = rec->pdl;
         rec->simt = p;
         break;
@@ -563,7 +580,7 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         p.K = (int32_t)in.K;
         p.N = (int32_t)in.N;
         p.in_dtype = v.A->dtype;
-        p.epi = epi_params(v, false, alpha, beta, sa, sb);
+        p.epi = epi_params(v, false, alpha, beta, sa, sb, bias, act);
         p.err_word = ds->err_word;
         p.timeout_ns = (uint64_t)g_timeout_ms.load() * 1000000ull;
         p.pdl = rec->pdl;
@@ -639,7 +656,7 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         int tc = 32;
         while (tc < 2 * bn) tc *= 2;
         p.tmem_cols = tc;
-        p.epi = epi_params(v, swap, alpha, beta, sa, sb);
+        p.epi = epi_params(v, swap, alpha, beta, sa, sb, bias, act);
         if (in.p_gather) {
             DevView d{};
             d.ptr = static_cast<const char *>(Pv->ptr);
@@ -675,7 +692,7 @@ dg_status fire(const LaunchRec &r, cudaStream_t stream) {
     int grid = 0;
     switch (r.kind) {
     case DG_KIND_NONE: return DG_OK;
-    case DG_KIND_SCALE_C: err = launch_scale_c(r.c, r.M, r.N, r.beta, r.pdl, stream); break;
+    case DG_KIND_SCALE_C: err = launch_scale_c(r.c, r.M, r.N, r.beta, r.bias, r.act, r.pdl, stream); break;
     case DG_KIND_SIMT: err = launch_simt(r.simt, stream); break;
     case DG_KIND_GEMV_N: err = launch_gemv_n(r.gemv, &r.t0, stream, &grid); break;
     case DG_KIND_GEMV_K: err = launch_gemv_k(r.gemv, stream, &grid); break;
@@ -696,6 +713,8 @@ struct CallKey {
     dg_view A, B, C;
     float alpha, beta;
     const float *sa, *sb;
+    const float *bias;
+    int act;
     int dev;
     uint32_t epoch;
 };
@@ -717,9 +736,17 @@ using namespace dg;
 
 extern "C" {
 
-dg_status dg_gemm(const dg_view *A, const dg_view *B, const dg_view *C, float alpha, float beta,
-                  const float *scale_a, const float *scale_b, void *stream) {
+dg_status dg_gemm_ex(const dg_view *A, const dg_view *B, const dg_view *C, float alpha, float beta,
+                     const float *scale_a, const float *scale_b, const dg_epilogue *epilogue, void *stream) {
     if (!A || !B || !C) return DG_ERR_NULL;
+    const float *bias = nullptr;
+    int act = DG_ACT_NONE;
+    if (epilogue) {
+        if (epilogue->activation < DG_ACT_NONE || epilogue->activation > DG_ACT_GELU_TANH || epilogue->reserved != 0)
+            return DG_ERR_VALUE;
+        bias = epilogue->bias;
+        act = epilogue->activation;
+    }
     // a call identical to a recent one on this thread and device reuses its
     // validated plan, parameters and tensor maps
     CallKey key;
@@ -731,6 +758,8 @@ dg_status dg_gemm(const dg_view *A, const dg_view *B, const dg_view *C, float al
     key.beta = beta;
     key.sa = scale_a;
     key.sb = scale_b;
+    key.bias = bias;
+    key.act = act;
     key.epoch = g_epoch.load();
     if (cudaGetDevice(&key.dev) != cudaSuccess) {
         cudaGetLastError();
@@ -761,14 +790,21 @@ dg_status dg_gemm(const dg_view *A, const dg_view *B, const dg_view *C, float al
     if (!device_accessible(C->ptr)) return DG_ERR_POINTER;
     if (use_ab && scale_a && !device_accessible(scale_a)) return DG_ERR_POINTER;
     if (use_ab && scale_b && !device_accessible(scale_b)) return DG_ERR_POINTER;
+    if (bias && !device_accessible(bias)) return DG_ERR_POINTER;
     const int slot = t_calls.next;
     t_calls.used[slot] = false;
-    st = prepare(v, pl, alpha, beta, use_ab ? scale_a : nullptr, use_ab ? scale_b : nullptr, ds, &t_calls.rec[slot]);
+    st = prepare(v, pl, alpha, beta, use_ab ? scale_a : nullptr, use_ab ? scale_b : nullptr, bias, act, ds,
+                 &t_calls.rec[slot]);
     if (st != DG_OK) return st;
     t_calls.key[slot] = key;
     t_calls.used[slot] = true;
     t_calls.next = (slot + 1) % 8;
     return fire(t_calls.rec[slot], static_cast<cudaStream_t>(stream));
+}
+
+dg_status dg_gemm(const dg_view *A, const dg_view *B, const dg_view *C, float alpha, float beta,
+                  const float *scale_a, const float *scale_b, void *stream) {
+    return dg_gemm_ex(A, B, C, alpha, beta, scale_a, scale_b, nullptr, stream);
 }
 
 dg_status dg_gemv(const dg_view *x, const dg_view *W, const dg_view *y, float alpha, float beta, void *stream) {

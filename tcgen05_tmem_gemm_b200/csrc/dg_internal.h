@@ -61,16 +61,29 @@ int elem_size(int dtype);
 // ------------------------------------------------------------- kernel params
 
 // Epilogue target: C viewed as (i, j) with byte strides, i on the tensor-core
-// M side, j on the N side (swapped when the kernel computes C^T).
+// M side, j on the N side (swapped when the kernel computes C^T).  The
+// epilogue computes  out = act(alpha * s_i * s_j * acc + beta * C + bias)
+// with the bias indexed by the output column n, which is j, or i when the
+// operands are swapped.
 struct EpiParams {
     char *c;
-    int64_t ci, cj;          // byte strides of C along i and j
+    int64_t ci, cj;          // byte strides of C along i and j (ci: when ci_multi == 0)
     int32_t c_dtype;
     int32_t vec_ok;          // C contiguous along j with 16-byte aligned rows
     float alpha, beta;
     const float *scale_i;    // per-i scale or null
     const float *scale_j;    // per-j scale or null
+    const float *bias_i;     // fused bias along i (swapped operands) or null
+    const float *bias_j;     // fused bias along j or null
+    int32_t act;             // fused activation (dg_activation)
+    int32_t ci_multi;        // C's i index spans several dims (e.g. an NCHW output): row offsets from ci_axis
+    Axis ci_axis;            // C's i group, outermost dim first
 };
+
+// Byte offset of C's row i.
+__host__ __device__ inline int64_t epi_row_offset(const EpiParams &e, int64_t i) {
+    return e.ci_multi ? axis_offset(e.ci_axis, i) : i * e.ci;
+}
 
 struct UmmaParams {
     int32_t Mi, Nj, K;       // tensor-core problem: D[Mi x Nj] = P[Mi x K] Q[K x Nj]
@@ -144,6 +157,7 @@ cudaError_t launch_gemv_n(const GemvParams &p, const CUtensorMap *tmap_w, cudaSt
 size_t gemv_n_smem_bytes(int r_inst, int kper);
 cudaError_t launch_gemv_k(const GemvParams &p, cudaStream_t s, int *grid_out);
 cudaError_t launch_simt(const SimtParams &p, cudaStream_t s);
-cudaError_t launch_scale_c(const DevView &c, int64_t M, int64_t N, float beta, int pdl, cudaStream_t s);
+cudaError_t launch_scale_c(const DevView &c, int64_t M, int64_t N, float beta, const float *bias, int act, int pdl,
+                           cudaStream_t s);
 
 }  // namespace dg

@@ -3,9 +3,10 @@
 //    reading every operand through the view addressing, FP32 accumulation.
 //    It is the bisection baseline (DG_OPT_FORCE_KIND = DG_KIND_SIMT) and the
 //    path for layouts the tensor-core kernel does not take.
-//  - scale_c: C = beta * C (or 0 when beta == 0) for alpha == 0 or K == 0,
-//    where the product is not formed ("DeepGEMM: a recalibration of the
-//    compute paradigm", §4.3: beta must still be applied when A is skipped).
+//  - scale_c: C = beta * C (or 0 when beta == 0), then the fused bias and
+//    activation, for alpha == 0 or K == 0, where the product is not formed
+//    ("DeepGEMM: a recalibration of the compute paradigm", §4.3: beta must
+//    still be applied when A is skipped).
 #include "common.cuh"
 
 namespace dg {
@@ -86,19 +87,24 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtParams p) {
             const float sj = e.scale_j ? e.scale_j[n] : 1.f;
             float v = (asi * sj) * acc[i][j];
             if (e.beta != 0.f) v = fmaf(e.beta, cin[j], v);
+            if (e.bias_j != nullptr || e.act != DG_ACT_NONE) v = epi_fuse(v, e.bias_j, n, e.act);
             store_elem(cp[j], p.c.dtype, v);
         }
     }
 }
 
-__global__ void scale_c_kernel(const DevView c, int64_t M, int64_t N, float beta) {
+// C = act(beta * C + bias[n]) (the product term is zero).
+__global__ void scale_c_kernel(const DevView c, int64_t M, int64_t N, float beta, const float *bias, int act) {
     pdl_wait_then_release();
     const int64_t total = M * N;
+    const bool fused = bias != nullptr || act != DG_ACT_NONE;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t m = e / N, n = e - (e / N) * N;
         char *cp = const_cast<char *>(c.ptr) + axis_offset(c.row, m) + axis_offset(c.col, n);
-        store_elem(cp, c.dtype, beta != 0.f ? beta * load_elem(cp, c.dtype) : 0.f);
+        float v = beta != 0.f ? beta * load_elem(cp, c.dtype) : 0.f;
+        if (fused) v = epi_fuse(v, bias, n, act);
+        store_elem(cp, c.dtype, v);
     }
 }
 
@@ -110,11 +116,12 @@ cudaError_t launch_simt(const SimtParams &p, cudaStream_t s) {
     return launch_ex(simt_gemm_kernel, grid, dim3(NT), 0, s, dim3(1, 1, 1), p.pdl, p);
 }
 
-cudaError_t launch_scale_c(const DevView &c, int64_t M, int64_t N, float beta, int pdl, cudaStream_t s) {
+cudaError_t launch_scale_c(const DevView &c, int64_t M, int64_t N, float beta, const float *bias, int act, int pdl,
+                           cudaStream_t s) {
     const int64_t total = M * N;
     int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 16);
     if (blocks < 1) blocks = 1;
-    return launch_ex(scale_c_kernel, dim3(blocks), dim3(256), 0, s, dim3(1, 1, 1), pdl, c, M, N, beta);
+    return launch_ex(scale_c_kernel, dim3(blocks), dim3(256), 0, s, dim3(1, 1, 1), pdl, c, M, N, beta, bias, act);
 }
 
 }  // namespace dg

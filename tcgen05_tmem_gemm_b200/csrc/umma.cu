@@ -673,7 +673,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         const EpiParams e = p.epi;  // a local copy: its fields stay in registers
         int local = 0;
         uint32_t nblk = 0;  // tensor-store blocks this warp has issued
-        if (p.split_k > 1 && e.beta != 0.f) {
+        if (p.split_k > 1 && e.beta != 0.f && !e.ci_multi) {
             // the rows this CTA will reduce: pull their C lines into L2 while
             // the main loops run
             const TileCoord tc = unit_coord(blockIdx.x, p);
@@ -733,14 +733,14 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             } else {
                 const bool row_ok = i < p.Mi;
                 const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
-                char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
+                char *crow = e.c + epi_row_offset(e, row_ok ? i : 0);
                 for (int c0 = 0; c0 < p.bn; c0 += 16) {
                     uint32_t r[16];
                     __syncwarp();
                     tmem_ld16(t_row + c0, r);
                     tmem_ld_wait();
                     if (!row_ok) continue;
-                    epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
+                    epilogue_chunk16(e, crow, asi, i, j0 + c0, p.Nj, r);
                 }
             }
             tc_fence_before();
@@ -869,11 +869,15 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             const int i0 = tc.ti * kBM + r0, jt = tc.tj * bn;
             const float alpha = e.alpha, beta = e.beta;
             const float *const scale_i = e.scale_i, *const scale_j = e.scale_j;
+            const float *const bias_i = e.bias_i, *const bias_j = e.bias_j;
+            const int act = e.act;
+            const bool fused = bias_i != nullptr || bias_j != nullptr || act != DG_ACT_NONE;
             char *const cbase = e.c;
             const int64_t ci = e.ci, cj = e.cj;
+            const bool ci_multi = e.ci_multi != 0;
             const int cdt = e.c_dtype;
-            const bool vec4 = cdt == DG_F32 && ci == 4 && rs_max % 4 == 0 && rs % 4 == 0 && i0 % 4 == 0 &&
-                              cj % 16 == 0 && (reinterpret_cast<uintptr_t>(cbase) & 15) == 0;
+            const bool vec4 = cdt == DG_F32 && !ci_multi && ci == 4 && rs_max % 4 == 0 && rs % 4 == 0 &&
+                              i0 % 4 == 0 && cj % 16 == 0 && (reinterpret_cast<uintptr_t>(cbase) & 15) == 0;
             constexpr int kB4 = 4;  // four-row groups per thread per batch (vector path)
             const int g_rows = vec4 ? rs / 4 : 1;
             // vector path: C of the first batch is loaded while the slices travel
@@ -961,6 +965,11 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                                 const float asi = alpha * (scale_i && i + k < Mi ? scale_i[i + k] : 1.f);
                                 o[k] = (asi * sj) * a4[k];
                                 if (beta != 0.f) o[k] = fmaf(beta, c4[k], o[k]);
+                                if (fused) {
+                                    if (bias_i && i + k < Mi) o[k] += bias_i[i + k];
+                                    if (bias_j) o[k] += bias_j[j];
+                                    o[k] = act_apply(act, o[k]);
+                                }
                             }
                             char *dstc = cbase + (int64_t)i * 4 + (int64_t)j * cj;
                             if (i + 3 < Mi) {
@@ -978,6 +987,11 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                                     const float asi = alpha * (scale_i ? scale_i[i + k] : 1.f);
                                     float val = (asi * sj) * a;
                                     if (beta != 0.f) val = fmaf(beta, load_elem(dstc + k * 4, cdt), val);
+                                    if (fused) {
+                                        if (bias_i) val += bias_i[i + k];
+                                        if (bias_j) val += bias_j[j];
+                                        val = act_apply(act, val);
+                                    }
                                     store_elem(dstc + k * 4, cdt, val);
                                 }
                             }
@@ -1008,8 +1022,8 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                                     if (q < S) a += ld_shared_f32(src[q] + off);
                             }
                             acc[b] = a;
-                            cin[b] = (ok && beta != 0.f) ? load_elem(cbase + (int64_t)i * ci + (int64_t)j * cj, cdt)
-                                                         : 0.f;
+                            const int64_t ro = ci_multi ? axis_offset(e.ci_axis, ok ? i : 0) : (int64_t)i * ci;
+                            cin[b] = (ok && beta != 0.f) ? load_elem(cbase + ro + (int64_t)j * cj, cdt) : 0.f;
                             // advance by 128 elements
                             if (along_i) {
                                 r += dr;
@@ -1029,7 +1043,13 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                             const float sj = scale_j ? scale_j[j] : 1.f;
                             float val = (asi * sj) * acc[b];
                             if (beta != 0.f) val = fmaf(beta, cin[b], val);
-                            store_elem(cbase + (int64_t)i * ci + (int64_t)j * cj, cdt, val);
+                            if (fused) {
+                                if (bias_i) val += bias_i[i];
+                                if (bias_j) val += bias_j[j];
+                                val = act_apply(act, val);
+                            }
+                            const int64_t ro = ci_multi ? axis_offset(e.ci_axis, i) : (int64_t)i * ci;
+                            store_elem(cbase + ro + (int64_t)j * cj, cdt, val);
                         }
                     }
                 }

@@ -6,13 +6,15 @@
 
 namespace dg {
 
-// Apply  out = alpha * s_i * s_j * acc + beta * C  to the 16 consecutive
-// columns jb .. jb+15 of one output row (row pointer `crow`, per-row factor
-// asi = alpha * s_i) and store them: 16-byte vector stores when C is
-// contiguous along j and the chunk is whole, otherwise element stores for any
-// strides, with every C load of the chunk issued before the first store.
-__device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow, float asi, int jb, int Nj,
+// Apply  out = act(alpha * s_i * s_j * acc + beta * C + bias)  to the 16
+// consecutive columns jb .. jb+15 of output row i (row pointer `crow`,
+// per-row factor asi = alpha * s_i) and store them: 16-byte vector stores
+// when C is contiguous along j and the chunk is whole, otherwise element
+// stores for any strides, with every C load of the chunk issued before the
+// first store.  The bias add and activation run only when the call has them.
+__device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow, float asi, int i, int jb, int Nj,
                                                  const uint32_t (&r)[16]) {
+    const bool fused = e.bias_i != nullptr || e.bias_j != nullptr || e.act != DG_ACT_NONE;
     if (e.vec_ok && jb + 16 <= Nj) {
         float v[16];
 #pragma unroll
@@ -20,6 +22,17 @@ __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow,
             const float sj = e.scale_j ? e.scale_j[jb + c] : 1.f;
             v[c] = (asi * sj) * __uint_as_float(r[c]);
         }
+        // C is loaded first (beta != 0), so the fused step sees the whole sum
+        auto fuse = [&]() {
+            if (!fused) return;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                float z = v[c];
+                if (e.bias_i) z += e.bias_i[i];
+                if (e.bias_j) z += e.bias_j[jb + c];
+                v[c] = act_apply(e.act, z);
+            }
+        };
         if (e.c_dtype == DG_F32) {
             float4 *dst = reinterpret_cast<float4 *>(crow + (int64_t)jb * 4);
             if (e.beta != 0.f) {
@@ -32,6 +45,7 @@ __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow,
                     v[4 * q + 3] = fmaf(e.beta, o.w, v[4 * q + 3]);
                 }
             }
+            fuse();
 #pragma unroll
             for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         } else {
@@ -56,6 +70,7 @@ __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow,
                     v[2 * q + 1] = fmaf(e.beta, hi, v[2 * q + 1]);
                 }
             }
+            fuse();
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 if (e.c_dtype == DG_BF16) {
@@ -83,6 +98,11 @@ __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow,
                 const float sj = e.scale_j ? e.scale_j[j] : 1.f;
                 float val = (asi * sj) * __uint_as_float(r[c]);
                 if (e.beta != 0.f) val = fmaf(e.beta, cin[c], val);
+                if (fused) {
+                    if (e.bias_i) val += e.bias_i[i];
+                    if (e.bias_j) val += e.bias_j[j];
+                    val = act_apply(e.act, val);
+                }
                 store_elem(crow + (int64_t)j * e.cj, e.c_dtype, val);
             }
         }
@@ -95,7 +115,8 @@ constexpr uint32_t kEpiBlockBytes = 32 * 128;
 constexpr uint32_t kEpiStoreBytes = 4 * 2 * kEpiBlockBytes;
 
 // Epilogue of one warp's 32 accumulator rows (TMEM lanes) x bn columns through
-// tensor stores, for beta == 0 and C unit-stride along j.  After tcgen05.ld a
+// tensor stores, for beta == 0 and C unit-stride along j (with the fused bias
+// and activation when the call has them).  After tcgen05.ld a
 // thread holds one row, so direct stores would touch 32 rows per instruction.
 // Instead the warp writes 32 rows x 128 bytes of output at a time into a
 // shared-memory block in the 128-byte-swizzle layout (row r's 16-byte unit u
@@ -114,9 +135,14 @@ __device__ __forceinline__ void epilogue_rows_tma(const EpiParams &e, const CUte
     if (i_base >= Mi) return;    // the whole warp is below C (warp-uniform)
     // parameters in registers: nothing below re-reads the parameter block
     const float *const scale_j = e.scale_j;
+    const float *const bias_j = e.bias_j;
+    const int act = e.act;
+    const bool fused = e.bias_i != nullptr || bias_j != nullptr || act != DG_ACT_NONE;
     const bool bf16_out = e.c_dtype == DG_BF16;
     const int i = i_base + lane;
     const float asi = i < Mi ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
+    const bool has_bi = e.bias_i != nullptr;
+    const float bi = (i < Mi && has_bi) ? e.bias_i[i] : 0.f;
     // blocks blk_first, blk_first + blk_step, ... of the row strip (warps that
     // share TMEM lanes split a strip this way)
     for (int c0 = blk_first * W; c0 < bn && j0 + c0 < Nj; c0 += blk_step * W) {
@@ -136,6 +162,16 @@ __device__ __forceinline__ void epilogue_rows_tma(const EpiParams &e, const CUte
         } else {
 #pragma unroll
             for (int c = 0; c < W; ++c) v[c] = asi * __uint_as_float(r[c]);
+        }
+        if (fused) {  // bias (per row or per column, clamped at the edge) and activation
+            const int jb = j0 + c0;
+#pragma unroll
+            for (int c = 0; c < W; ++c) {
+                float z = v[c];
+                if (has_bi) z += bi;
+                if (bias_j) z += bias_j[jb + c < Nj ? jb + c : Nj - 1];
+                v[c] = act_apply(act, z);
+            }
         }
         uint32_t w[32];
         if (ES == 4) {

@@ -262,14 +262,14 @@ __global__ void __launch_bounds__(192, 1)
             } else {
                 const bool row_ok = i < p.Mi;
                 const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
-                char *crow = e.c + (int64_t)(row_ok ? i : 0) * e.ci;
+                char *crow = e.c + epi_row_offset(e, row_ok ? i : 0);
                 for (int c0 = 0; c0 < pu.w; c0 += 16) {
                     uint32_t r[16];
                     __syncwarp();
                     tmem_ld16(t_row + c0, r);
                     tmem_ld_wait();
                     if (!row_ok) continue;
-                    epilogue_chunk16(e, crow, asi, j0 + c0, p.Nj, r);
+                    epilogue_chunk16(e, crow, asi, i, j0 + c0, p.Nj, r);
                 }
             }
             tc_fence_before();

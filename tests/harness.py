@@ -14,6 +14,12 @@ for FP16, so 4e-3 and 2e-3 leave a factor of two), and the FP32 accumulation
 error is relative to S, with the same 5e-4 as for FP32 output.  A wrong value
 on one entry is then held to the result's own size, not to S (which is about
 sqrt(K) times larger for random data).
+With the fused epilogue out = act(z), z = alpha*s*acc + beta*c + bias, the
+FP32 error of z is 5e-4 * S + 2^-22 * (|z| + |beta c| + |bias|); the
+activation passes it on multiplied by at most its largest slope (1 for ReLU,
+1.129 for GeLU in its tanh form) and GeLU's FP32 evaluation adds at most
+2^-20 |z| (tanh near -1 loses the low bits of 1 + tanh); 16-bit outputs then
+add their rounding relative to the result as above.
 NaN positions must agree exactly; infinities must agree in sign and place.
 """
 from __future__ import annotations
@@ -30,10 +36,19 @@ def dg_view_of(op: W.Operand) -> dg.dg_view:
     return dg.make_view(op.base.data_ptr() + op.offset, op.shape, op.stride, op.row_dims, op.dtype)
 
 
+def fused(problem: W.Problem) -> bool:
+    return problem.bias is not None or problem.act != "none"
+
+
 def run(problem: W.Problem, stream=None, check_status=True) -> W.Problem:
-    """Enqueue dg_gemm for a device-resident problem and wait for it."""
+    """Enqueue dg_gemm (dg_gemm_ex for a fused epilogue) for a
+    device-resident problem and wait for it."""
     A, B, C = dg_view_of(problem.A), dg_view_of(problem.B), dg_view_of(problem.C)
-    st = dg.dg_gemm(A, B, C, problem.alpha, problem.beta, problem.scale_a, problem.scale_b, stream)
+    if fused(problem):
+        st = dg.dg_gemm_ex(A, B, C, problem.alpha, problem.beta, problem.scale_a, problem.scale_b,
+                           dg.epilogue(problem.bias, problem.act), stream)
+    else:
+        st = dg.dg_gemm(A, B, C, problem.alpha, problem.beta, problem.scale_a, problem.scale_b, stream)
     if check_status:
         assert st == dg.DG_OK, dg.status_string(st)
     sst = dg.dg_sync_status(stream)
@@ -64,18 +79,35 @@ def c_matrix(problem: W.Problem) -> np.ndarray:
     return out
 
 
-def tolerance(out_dtype: str, ref, bound, beta_c):
+ACT_SLOPE = {"none": 1.0, "relu": 1.0, "gelu_tanh": 1.13}
+
+
+def tolerance(out_dtype: str, ref, bound, beta_c, pre=None, bias_abs=None, act="none"):
     ref = np.abs(ref)
+    if pre is None and bias_abs is None and act == "none":
+        # plain GEMM: out = z
+        if out_dtype == "f32":
+            return 5e-4 * bound + 2.0 ** -22 * (ref + np.abs(beta_c))
+        if out_dtype == "bf16":
+            return 4e-3 * ref + 5e-4 * bound
+        if out_dtype == "f16":
+            return 2e-3 * ref + 5e-4 * bound + 2.0 ** -24
+        raise ValueError(out_dtype)
+    z = np.abs(pre) if pre is not None else ref
+    b = bias_abs if bias_abs is not None else 0.0
+    tz = ACT_SLOPE[act] * (5e-4 * bound + 2.0 ** -22 * (z + np.abs(beta_c) + b))
+    if act == "gelu_tanh":
+        tz = tz + 2.0 ** -20 * z
     if out_dtype == "f32":
-        return 5e-4 * bound + 2.0 ** -22 * (ref + np.abs(beta_c))
+        return tz
     if out_dtype == "bf16":
-        return 4e-3 * ref + 5e-4 * bound
+        return 4e-3 * ref + tz
     if out_dtype == "f16":
-        return 2e-3 * ref + 5e-4 * bound + 2.0 ** -24
+        return 2e-3 * ref + tz + 2.0 ** -24
     raise ValueError(out_dtype)
 
 
-def compare(problem: W.Problem, got, ref, bound, beta_c=None, where=""):
+def compare(problem: W.Problem, got, ref, bound, beta_c=None, where="", pre=None, bias_abs=None):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     if beta_c is None:
@@ -87,7 +119,9 @@ def compare(problem: W.Problem, got, ref, bound, beta_c=None, where=""):
     assert np.array_equal(got[inf_r], ref[inf_r]), f"{where}: Inf signs differ"
     fin = ~(nan_r | inf_r)
     err = np.abs(got[fin] - ref[fin])
-    tol = tolerance(problem.C.dtype, ref[fin], bound[fin], beta_c[fin])
+    tol = tolerance(problem.C.dtype, ref[fin], bound[fin], beta_c[fin],
+                    None if pre is None else np.asarray(pre)[fin],
+                    None if bias_abs is None else np.broadcast_to(bias_abs, ref.shape)[fin], problem.act)
     bad = err > tol
     if bad.any():
         idx = np.argmax(err - tol)
@@ -105,14 +139,24 @@ def beta_c_of(problem: W.Problem) -> np.ndarray:
     return problem.beta * c_matrix(problem)
 
 
+def _bias_abs(problem: W.Problem, ns=None):
+    if problem.bias is None:
+        return None
+    b = np.abs(problem.bias.detach().cpu().double().numpy())
+    return b if ns is None else b[ns]
+
+
 def check_full(problem_cpu: W.Problem, stream=None) -> dict:
     """Run on the GPU and compare every output with the full oracle."""
-    ref, bound = oracle.gemm(problem_cpu)
+    if fused(problem_cpu):
+        ref, bound, pre = oracle.gemm(problem_cpu, want_pre=True)
+    else:
+        (ref, bound), pre = oracle.gemm(problem_cpu), None
     bc = beta_c_of(problem_cpu)
     gpu = problem_cpu.to("cuda")
     run(gpu, stream)
     got = c_matrix(gpu)
-    return compare(problem_cpu, got, ref, bound, bc, problem_cpu.name)
+    return compare(problem_cpu, got, ref, bound, bc, problem_cpu.name, pre, _bias_abs(problem_cpu))
 
 
 def tile_corners(M: int, N: int, bm: int, bn: int):
@@ -138,10 +182,11 @@ def check_sampled(problem_cpu: W.Problem, npts=2048, seed=0, gpu=None, extra=Non
         ms += list(extra[0])
         ns += list(extra[1])
     ms, ns = np.array(ms), np.array(ns)
-    ref, bound = oracle.gemm_points(problem_cpu, ms, ns)
+    ref, bound, pre = oracle.gemm_points(problem_cpu, ms, ns, want_pre=True)
     bc = problem_cpu.beta * c_matrix(problem_cpu)[ms, ns] if problem_cpu.beta != 0 else np.zeros(len(ms))
     if gpu is None:
         gpu = problem_cpu.to("cuda")
         run(gpu)
     got = c_matrix(gpu)[ms, ns]
-    return compare(problem_cpu, got, ref, bound, bc, problem_cpu.name)
+    return compare(problem_cpu, got, ref, bound, bc, problem_cpu.name,
+                   pre if fused(problem_cpu) else None, _bias_abs(problem_cpu, ns))

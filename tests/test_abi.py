@@ -213,6 +213,37 @@ def test_gemm_argument_errors_need_no_device():
                           None) == dg.DG_ERR_UNSUPPORTED
 
 
+def test_gemm_ex_epilogue_errors_need_no_device():
+    p = meta_problem("small", M=16, N=16, K=16)
+    A, B, C = views(p)
+    for act, reserved in ((3, 0), (-1, 0), (0, 1)):
+        e = dg.dg_epilogue()
+        e.bias = None
+        e.activation = act
+        e.reserved = reserved
+        assert dg.lib.dg_gemm_ex(ctypes.byref(A), ctypes.byref(B), ctypes.byref(C), 1.0, 0.0, None, None,
+                                 ctypes.byref(e), None) == dg.DG_ERR_VALUE
+    assert dg.lib.dg_gemm_ex(None, ctypes.byref(B), ctypes.byref(C), 1.0, 0.0, None, None, None,
+                             None) == dg.DG_ERR_NULL
+
+
+def test_plan_nchw_output_stays_on_tensor_cores():
+    # C written as an NCHW tensor [n, N, h, w] from the [n*h*w, N] product: the
+    # row index of C spans two dims (n and h*w), which the tensor-core epilogue
+    # addresses per row; the column walks one stride (h*w elements)
+    n, c, h, w, N = 4, 64, 7, 7, 128
+    A = dg.make_view(FAKE, (n, h, w, c), (c * h * w * 2, w * 2, 2, h * w * 2), 3, "bf16")
+    B = dg.make_view(FAKE, (c, N), (N * 2, 2), 1, "bf16")
+    C = dg.make_view(FAKE, (n, h, w, N), (N * h * w * 4, w * 4, 4, h * w * 4), 3, "f32")
+    info = dg.dg_analyse_view(C)
+    assert info.n_row == 2 and info.n_col == 1
+    assert dg.dg_plan(A, B, C, 1.0, 0.0, False, 148).as_dict()["kind_name"] == "umma"
+    # two dims along the other index of C (j) still go to the CUDA-core kernel
+    Ct = dg.make_view(FAKE, (n * h * w, 2, N // 2), (4, n * h * w * 4 * (N // 2) + 64, n * h * w * 4), 1, "f32")
+    assert dg.dg_analyse_view(Ct).n_col == 2
+    assert dg.dg_plan(A, B, Ct, 1.0, 0.0, False, 148).as_dict()["kind_name"] == "simt"
+
+
 def test_options():
     with pytest.raises(dg.DgError):
         dg.dg_set_option(dg.DG_OPT_FORCE_KIND, 99)

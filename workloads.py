@@ -235,6 +235,23 @@ def cfg_strided(seed: int = 1006, n=16, c=256, h=14, w=14, N=1024) -> Problem:
                    row_major(B, "bf16"), empty_out(n * h * w, N, "f32"), 1.0, 0.0)
 
 
+def with_epilogue(p: Problem, act: str = "gelu_tanh", seed: int = 2001, bias: bool = True) -> Problem:
+    """The same problem with a fused epilogue: a bias per output column drawn
+    from N(0, 1) (seeded) and an activation ("none", "relu", "gelu_tanh")."""
+    g = _gen(seed)
+    b = normal((p.N,), g).contiguous() if bias else None
+    return Problem(f"{p.name}_{'bias_' if bias else ''}{act}", p.A, p.B, p.C, p.alpha, p.beta,
+                   p.scale_a, p.scale_b, p.note, dict(p.extra), b, act)
+
+
+def nchw_out(n: int, c: int, h: int, w: int, dtype: str = "f32") -> Operand:
+    """An output written as an NCHW tensor [n, c, h, w] (NaN-filled) and
+    addressed as the [n*h*w, c] product it receives: the epilogue's layout
+    transform from rows of (n, h, w) to channel planes."""
+    t = torch.full((n, c, h, w), float("nan"), dtype=torch.float32).to(TORCH_DTYPE[dtype])
+    return nchw_as_rows(t, dtype)
+
+
 WORKLOADS = {
     "small": cfg_small,
     "gemv": cfg_gemv,
