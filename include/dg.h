@@ -231,6 +231,10 @@ typedef struct {
                               copying it to the others (1 = no sharing)             */
     int32_t pair_half_tiles;/* UMMA, CTA pairs: tiles of the last, partial wave that run
                               as two half-width tiles each                          */
+    int32_t stream_k_tiles; /* UMMA, CTA pairs: tiles of the last, partial wave whose k
+                              blocks are shared out over all pairs (Stream-K); their
+                              owners add the other pairs' partials                   */
+    int32_t reserved;
 } dg_plan_info;
 
 /* The dispatch decision dg_gemm would take for these views (pointers are only
@@ -276,8 +280,13 @@ typedef enum {
     DG_OPT_GATHER_CLUSTER = 9,    /* 1 (default): CTAs that need the same gathered
                                      operand tile share the loads through distributed
                                      shared memory; 0: each gathers the whole tile      */
-    DG_OPT_PAIR_TAIL = 10         /* 1 (default): CTA pairs run the last, partial wave
+    DG_OPT_PAIR_TAIL = 10,        /* 1 (default): CTA pairs run the last, partial wave
                                      of tiles as half-width tiles; 0: whole tiles only  */
+    DG_OPT_STREAM_K = 11          /* 1 (default): CTA pairs share the k blocks of the
+                                     last, partial wave of tiles out over all pairs
+                                     (Stream-K, "DeepGEMM deep dive" §5.2) when a
+                                     workspace for the stream is available; 0: off
+                                     (the half-width tail above applies instead)        */
 } dg_option;
 
 dg_status dg_set_option(int option, int64_t value);

@@ -37,15 +37,30 @@ std::atomic<uint64_t> g_trace{0};
 std::atomic<int> g_epi_tma{1};
 std::atomic<int> g_gather_cluster{1};
 std::atomic<int> g_pair_tail{1};
+std::atomic<int> g_stream_k{1};
 std::atomic<uint32_t> g_epoch{1};  // bumped by every option change: cached launches go stale
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxCluster = 8;    // portable thread-block cluster size: the most k splits
 
+// Stream-K workspace of one stream: partial accumulators, flags and the
+// sequence header (see UmmaParams).  Kernels of one stream run one after the
+// other, so a stream's launches can share it; launches on different streams
+// may overlap and get their own.
+struct SkWorkspace {
+    cudaStream_t stream = nullptr;
+    void *ptr = nullptr;
+    size_t bytes = 0;
+};
+constexpr int kMaxSkStreams = 16;  // further streams run without Stream-K
+constexpr size_t kSkHeaderBytes = 256;
+
 struct DeviceState {
     bool ready = false;
     int num_sms = 0;
     int *err_word = nullptr;       // device: DG_ERR_TIMEOUT when a bounded wait gave up
+    SkWorkspace sk[kMaxSkStreams];
+    int n_sk = 0;
 };
 
 std::mutex g_mu;
@@ -79,6 +94,65 @@ dg_status device_state(DeviceState **out) {
     }
     *out = &d;
     return DG_OK;
+}
+
+// Bytes of a Stream-K workspace for `pairs` CTA pairs and tiles bn wide: the
+// header, one flag per (pair, CTA, epilogue warp), one 128 x bn FP32 slot per
+// (pair, CTA).
+size_t sk_workspace_bytes(int pairs, int bn, size_t *flag_off, size_t *part_off) {
+    const size_t flags = ((size_t)pairs * 2 * 4 * sizeof(uint32_t) + 255) / 256 * 256;
+    *flag_off = kSkHeaderBytes;
+    *part_off = kSkHeaderBytes + flags;
+    return *part_off + (size_t)pairs * 2 * 128 * (size_t)bn * sizeof(float);
+}
+
+// The Stream-K workspace of `stream` on this device, at least `need` bytes,
+// or null when none can be had now: the stream is being captured into a
+// graph (nothing is allocated then; calls run without Stream-K until a call
+// outside the capture has allocated it) or every slot is taken.  A new or
+// larger workspace is allocated with its header and flags zeroed on the
+// stream; a smaller one it replaces is freed after the stream has drained,
+// and cached launches that pointed at it are invalidated.
+void *sk_workspace(DeviceState *ds, cudaStream_t stream, size_t need, size_t zero_bytes) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    SkWorkspace *w = nullptr;
+    for (int i = 0; i < ds->n_sk; ++i)
+        if (ds->sk[i].stream == stream) w = &ds->sk[i];
+    if (w && w->bytes >= need) return w->ptr;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (cap != cudaStreamCaptureStatusNone) return nullptr;
+    if (!w) {
+        if (ds->n_sk == kMaxSkStreams) return nullptr;
+        w = &ds->sk[ds->n_sk++];
+        w->stream = stream;
+    } else {
+        if (cudaStreamSynchronize(stream) != cudaSuccess || cudaFree(w->ptr) != cudaSuccess) {
+            cudaGetLastError();
+            w->ptr = nullptr;
+            w->bytes = 0;
+            return nullptr;
+        }
+        w->ptr = nullptr;
+        w->bytes = 0;
+        g_epoch.fetch_add(1);  // cached launches held the old pointer
+    }
+    void *ptr = nullptr;
+    if (cudaMalloc(&ptr, need) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (cudaMemsetAsync(ptr, 0, zero_bytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(ptr);
+        return nullptr;
+    }
+    w->ptr = ptr;
+    w->bytes = need;
+    return ptr;
 }
 
 bool device_accessible_uncached(const void *p) {
@@ -216,7 +290,7 @@ void gemv_n_split(int64_t M, int64_t N, int64_t K, int num_sms, dg_plan_info *in
 }
 
 // Which UMMA configuration serves these views (false: none).
-bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int num_sms, Plan *pl) {
+bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int num_sms, bool allow_sk, Plan *pl) {
     const int dt = v.A->dtype;
     if (dt != DG_F16 && dt != DG_BF16 && dt != DG_E4M3) return false;
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return false;
@@ -367,7 +441,15 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
         const int per = 128 / es;
         const bool quarter_ok = q_mn ? ((bn / 4) % per == 0) : ((bn / 4) % 8 == 0);
         const int64_t tail = pair_units % ncl;
-        if (g_pair_tail.load() != 0 && quarter_ok && pair_units > ncl && tail > 0 && 2 * tail <= ncl)
+        // Stream-K: the tiles of the last, partial wave share their k blocks
+        // out over every pair ("DeepGEMM deep dive", §5.2), when each of those
+        // tiles is split among at most kMaxFix + 1 pairs and every pair gets
+        // at least one k block
+        const int64_t kb_all = tail * kb_total;
+        if (allow_sk && g_stream_k.load() != 0 && pair_units > ncl && tail > 0 && 7 * tail >= ncl &&
+            kb_all >= ncl)
+            in.stream_k_tiles = (int32_t)tail;
+        else if (g_pair_tail.load() != 0 && quarter_ok && pair_units > ncl && tail > 0 && 2 * tail <= ncl)
             in.pair_half_tiles = (int32_t)tail;
     }
     pl->fp8 = (dt == DG_E4M3);
@@ -376,7 +458,7 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     return true;
 }
 
-dg_status make_plan(Views &v, float alpha, float beta, int num_sms, Plan *pl) {
+dg_status make_plan(Views &v, float alpha, float beta, int num_sms, Plan *pl, bool allow_sk = true) {
     (void)beta;
     dg_status st;
     if ((st = analyse(v.A, false, &v.a)) != DG_OK) return st;
@@ -405,7 +487,7 @@ dg_status make_plan(Views &v, float alpha, float beta, int num_sms, Plan *pl) {
                 return DG_OK;
             }
         } else if (force == DG_KIND_UMMA) {
-            if (umma_plan(v, M, N, K, beta, num_sms, pl)) return DG_OK;
+            if (umma_plan(v, M, N, K, beta, num_sms, allow_sk, pl)) return DG_OK;
         } else {
             if (M <= 8) {
                 if (gemv_applicable(v, M, N, K, DG_KIND_GEMV_N)) {
@@ -415,7 +497,7 @@ dg_status make_plan(Views &v, float alpha, float beta, int num_sms, Plan *pl) {
                 }
                 if (gemv_applicable(v, M, N, K, DG_KIND_GEMV_K)) { in.kind = DG_KIND_GEMV_K; return DG_OK; }
             }
-            if (umma_plan(v, M, N, K, beta, num_sms, pl)) return DG_OK;
+            if (umma_plan(v, M, N, K, beta, num_sms, allow_sk, pl)) return DG_OK;
         }
     }
     if (M > int64_t(65535) * 64 || N > INT32_MAX || K > INT32_MAX) return DG_ERR_UNSUPPORTED;
@@ -537,7 +619,7 @@ struct LaunchRec {
 };
 
 dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const float *sa, const float *sb,
-                  const float *bias, int act, DeviceState *ds, LaunchRec *rec) {
+                  const float *bias, int act, DeviceState *ds, void *sk_ws, LaunchRec *rec) {
     const dg_plan_info &in = pl.info;
     rec->kind = in.kind;
     // early launch, mode 3: the launch-bound K-contiguous GEMV (64 blocks: the
@@ -652,6 +734,17 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
             p.full_units = tiles - in.pair_half_tiles;
             p.num_units = p.full_units + 2 * in.pair_half_tiles;
             p.idesc_half = make_idesc(dt, in.p_mn_major, in.q_mn_major, bn / 2, 256);
+            if (in.stream_k_tiles > 0) {
+                // the workspace of the stream: header, flags, partial slots
+                if (!sk_ws) return DG_ERR_UNSUPPORTED;
+                size_t flag_off = 0, part_off = 0;
+                sk_workspace_bytes(in.grid / 2, bn, &flag_off, &part_off);
+                p.sk_tiles = in.stream_k_tiles;
+                p.dp_tiles = tiles - in.stream_k_tiles;
+                p.sk_hdr = static_cast<uint32_t *>(sk_ws);
+                p.sk_flag = reinterpret_cast<uint32_t *>(static_cast<char *>(sk_ws) + flag_off);
+                p.sk_part = reinterpret_cast<float *>(static_cast<char *>(sk_ws) + part_off);
+            }
         }
         int tc = 32;
         while (tc < 2 * bn) tc *= 2;
@@ -717,6 +810,7 @@ struct CallKey {
     int act;
     int dev;
     uint32_t epoch;
+    void *stream;  // a Stream-K launch uses its stream's workspace
 };
 
 bool key_equal(const CallKey &x, const CallKey &y) { return std::memcmp(&x, &y, sizeof(CallKey)) == 0; }
@@ -761,6 +855,7 @@ dg_status dg_gemm_ex(const dg_view *A, const dg_view *B, const dg_view *C, float
     key.bias = bias;
     key.act = act;
     key.epoch = g_epoch.load();
+    key.stream = stream;
     if (cudaGetDevice(&key.dev) != cudaSuccess) {
         cudaGetLastError();
         key.dev = -1;
@@ -791,9 +886,21 @@ dg_status dg_gemm_ex(const dg_view *A, const dg_view *B, const dg_view *C, float
     if (use_ab && scale_a && !device_accessible(scale_a)) return DG_ERR_POINTER;
     if (use_ab && scale_b && !device_accessible(scale_b)) return DG_ERR_POINTER;
     if (bias && !device_accessible(bias)) return DG_ERR_POINTER;
+    void *sk_ws = nullptr;
+    if (in.stream_k_tiles > 0) {
+        size_t flag_off = 0, part_off = 0;
+        const size_t need = sk_workspace_bytes(in.grid / 2, in.block_n, &flag_off, &part_off);
+        sk_ws = sk_workspace(ds, static_cast<cudaStream_t>(stream), need, part_off);
+        if (!sk_ws) {
+            // no workspace on this stream now (e.g. inside a graph capture): plan without Stream-K
+            st = make_plan(v, alpha, beta, ds->num_sms, &pl, false);
+            if (st != DG_OK) return st;
+        }
+        key.epoch = g_epoch.load();  // a replaced workspace invalidated the cache
+    }
     const int slot = t_calls.next;
     t_calls.used[slot] = false;
-    st = prepare(v, pl, alpha, beta, use_ab ? scale_a : nullptr, use_ab ? scale_b : nullptr, bias, act, ds,
+    st = prepare(v, pl, alpha, beta, use_ab ? scale_a : nullptr, use_ab ? scale_b : nullptr, bias, act, ds, sk_ws,
                  &t_calls.rec[slot]);
     if (st != DG_OK) return st;
     t_calls.key[slot] = key;
@@ -915,6 +1022,10 @@ dg_status dg_set_option(int option, int64_t value) {
     case DG_OPT_PAIR_TAIL:
         if (value < 0 || value > 1) return DG_ERR_VALUE;
         g_pair_tail.store((int)value);
+        return DG_OK;
+    case DG_OPT_STREAM_K:
+        if (value < 0 || value > 1) return DG_ERR_VALUE;
+        g_stream_k.store((int)value);
         return DG_OK;
     default: return DG_ERR_VALUE;
     }

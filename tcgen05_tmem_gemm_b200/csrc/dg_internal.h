@@ -107,6 +107,15 @@ struct UmmaParams {
     // instruction descriptor idesc_half
     int32_t full_units;
     uint32_t idesc_half;
+    // Stream-K (CTA pairs): the first dp_tiles tiles run whole, one pair
+    // each; the last sk_tiles tiles form one run of k blocks shared out evenly
+    // over all pairs.  A tile's owner (the pair holding its last k blocks)
+    // adds the partials the other pairs left in the workspace, in pair order.
+    int32_t sk_tiles;
+    int32_t dp_tiles;
+    float *sk_part;          // per (pair, CTA): 128 rows x bn FP32, column by column
+    uint32_t *sk_flag;       // per (pair, CTA, epilogue warp): sequence tag of the partial rows last written
+    uint32_t *sk_hdr;        // [0] sequence number of the last completed launch, [1] CTAs done
     // control
     int *err_word;
     uint64_t timeout_ns;

@@ -109,6 +109,27 @@ __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow,
     }
 }
 
+// Partial accumulators another CTA left in global memory for this tile
+// (Stream-K): `src[q]` holds a 128-row x bn FP32 tile column by column
+// (element (row, col) at src[q][col * 128 + row]); the epilogue adds them to
+// the accumulator in q order before anything else.
+constexpr int kMaxFix = 8;
+struct Fixup {
+    const float *src[kMaxFix];
+    int n;
+};
+
+__device__ __forceinline__ void add_fixups(const Fixup *fx, int row, int col0, uint32_t *r, int ncols) {
+    if (fx == nullptr) return;
+#pragma unroll
+    for (int q = 0; q < kMaxFix; ++q) {
+        if (q >= fx->n) break;
+        const float *src = fx->src[q] + (int64_t)col0 * 128 + row;
+#pragma unroll 16
+        for (int c = 0; c < ncols; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) + src[c * 128]);
+    }
+}
+
 // Shared memory of the TMA-store epilogue: two blocks of 32 rows x 128 bytes
 // for each of the four epilogue warps.
 constexpr uint32_t kEpiBlockBytes = 32 * 128;
@@ -130,7 +151,8 @@ constexpr uint32_t kEpiStoreBytes = 4 * 2 * kEpiBlockBytes;
 template <int ES>
 __device__ __forceinline__ void epilogue_rows_tma(const EpiParams &e, const CUtensorMap *cmap, uint32_t stage,
                                                   uint32_t t_row, int i_base, int Mi, int j0, int bn, int Nj,
-                                                  int lane, uint32_t &nblk, int blk_first = 0, int blk_step = 1) {
+                                                  int lane, uint32_t &nblk, int blk_first = 0, int blk_step = 1,
+                                                  const Fixup *fx = nullptr, int fx_row = 0) {
     constexpr int W = 128 / ES;  // output columns per block
     if (i_base >= Mi) return;    // the whole warp is below C (warp-uniform)
     // parameters in registers: nothing below re-reads the parameter block
@@ -151,6 +173,7 @@ __device__ __forceinline__ void epilogue_rows_tma(const EpiParams &e, const CUte
         for (int q = 0; q < W / 16; ++q)
             tmem_ld16(t_row + (uint32_t)(c0 + 16 * q), *reinterpret_cast<uint32_t(*)[16]>(&r[16 * q]));
         tmem_ld_wait();
+        add_fixups(fx, fx_row, c0, r, W);
         float v[W];
         if (scale_j != nullptr) {  // per-column scales (FP8): read once per block, clamped at the edge
             const int jb = j0 + c0;

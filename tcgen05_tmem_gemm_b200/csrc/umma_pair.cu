@@ -68,6 +68,106 @@ __device__ __forceinline__ PairUnit pair_unit(int u, const UmmaParams &p) {
     return r;
 }
 
+// One unit of a pair's schedule: a tile (or half of one) and a range of its
+// k blocks, with what the epilogue does with the accumulator.
+enum : int {
+    kWhole = 0,      // the whole k range: store C
+    kSkPartial = 1,  // Stream-K, a range that ends inside the tile: leave the partial in this pair's slot
+    kSkOwner = 2     // Stream-K, the range that ends the tile: add the other pairs' partials, store C
+};
+struct PairWork {
+    int ti, j0, w;   // tile row, first column, columns
+    int kb0, kb1;    // k blocks [kb0, kb1)
+    int role;
+    int sk_first;    // kSkOwner: the tile's first k block in the Stream-K run
+};
+
+// Pair c's share [lo, hi) of the Stream-K run of `total` k blocks.
+__device__ __forceinline__ void sk_range(int64_t total, int c, int P, int64_t &lo, int64_t &hi) {
+    lo = total * c / P;
+    hi = total * (c + 1) / P;
+}
+
+// Unit idx of pair c of P (false past its last unit).  Without Stream-K:
+// pair_unit's whole and half tiles.  With it: first the Stream-K units (the
+// range that ends inside a tile, whose partial other pairs wait for, then
+// the ranges that end tiles this pair owns), then the whole tiles
+// c, c + P, ... below dp_tiles.  A tile's owner holds its last k blocks and
+// so has the highest pair index of the tile: owners wait only on pairs with
+// lower indices, which are launched no later than they are.
+__device__ __forceinline__ bool pair_work(const UmmaParams &p, int c, int P, int idx, PairWork &w) {
+    const int KB = p.kb_total;
+    if (p.sk_tiles == 0) {
+        const int u = c + idx * P;
+        if (u >= p.num_units) return false;
+        const PairUnit pu = pair_unit(u, p);
+        w.ti = pu.ti;
+        w.j0 = pu.j0;
+        w.w = pu.w;
+        w.kb0 = 0;
+        w.kb1 = KB;
+        w.role = kWhole;
+        w.sk_first = 0;
+        return true;
+    }
+    int64_t lo, hi;
+    sk_range((int64_t)p.sk_tiles * KB, c, P, lo, hi);
+    const int64_t ta = lo / KB, tb = hi / KB;
+    const bool partial = hi > lo && hi % KB != 0;
+    const int n_sk = hi > lo ? (int)(tb - ta) + (partial ? 1 : 0) : 0;
+    int t;
+    if (idx < n_sk) {
+        int64_t ts, k0, k1;
+        if (partial && idx == 0) {
+            ts = tb;
+            k0 = lo > tb * KB ? lo : tb * KB;
+            k1 = hi;
+            w.role = kSkPartial;
+        } else {
+            ts = ta + idx - (partial ? 1 : 0);
+            k0 = lo > ts * KB ? lo : ts * KB;
+            k1 = (ts + 1) * KB;
+            w.role = kSkOwner;
+        }
+        w.kb0 = (int)(k0 - ts * KB);
+        w.kb1 = (int)(k1 - ts * KB);
+        w.sk_first = (int)(ts * KB);
+        t = p.dp_tiles + (int)ts;
+    } else {
+        t = c + (idx - n_sk) * P;
+        if (t >= p.dp_tiles) return false;
+        w.kb0 = 0;
+        w.kb1 = KB;
+        w.role = kWhole;
+        w.sk_first = 0;
+    }
+    w.ti = t % p.tiles_i;
+    w.j0 = (t / p.tiles_i) * p.bn;
+    w.w = p.bn;
+    return true;
+}
+
+// The pairs whose partials the owner c of the Stream-K tile starting at k
+// block `first` adds: q in [q0, c) with a non-empty range (every such range
+// ends inside the tile).
+__device__ __forceinline__ int sk_first_contributor(const UmmaParams &p, int c, int P, int first) {
+    const int64_t total = (int64_t)p.sk_tiles * p.kb_total;
+    int64_t lo, hi;
+    sk_range(total, c, P, lo, hi);
+    if (lo <= first) return c;  // this pair starts the tile: nothing to add
+    int q = c;
+    while (q > 0) {
+        --q;
+        if (total * q / P <= first) break;
+    }
+    return q;
+}
+
+// This CTA's slot of pair q: 128 rows x bn FP32, column by column.
+__device__ __forceinline__ float *sk_slot(const UmmaParams &p, int q, uint32_t rank) {
+    return p.sk_part + (size_t)(q * 2 + (int)rank) * (size_t)(kHalfM * p.bn);
+}
+
 template <bool FP8>
 __global__ void __launch_bounds__(192, 1)
     umma_pair_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
@@ -122,6 +222,11 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
+    // Stream-K: the tag of this launch's partials is one more than the
+    // sequence number the previous launch left (it completed before this
+    // launch passed its dependency wait), so flags of earlier launches, or of
+    // a launch that gave up on a wait, never match
+    const uint32_t sk_tag = p.sk_tiles > 0 ? ld_acquire_gpu(p.sk_hdr) + 1u : 0u;
     const int es = FP8 ? 1 : 2;
     const int bk = p.bk;
     const int half_bn = p.bn / 2;
@@ -137,16 +242,18 @@ __global__ void __launch_bounds__(192, 1)
             const int stages = p.stages, kb_total = p.kb_total, num_units = p.num_units;
             const bool stall = p.stall_loader != 0, p_mn = p.p_mn_major != 0, q_mn = p.q_mn_major != 0;
             const uint32_t stage_bytes = L.stage_bytes, a_bytes = L.a_bytes;
+            (void)num_units;
+            (void)kb_total;
             int it = 0, s = 0;
             uint32_t ph = 0;
-            for (int u = cluster_id; u < num_units && !*abort_flag; u += nclusters) {
-                const PairUnit pu = pair_unit(u, p);
-                const int i0 = pu.ti * 2 * kHalfM + (int)rank * kHalfM;
-                const int cw = pu.w / 2;  // this CTA's columns of the unit
-                const int j0 = pu.j0 + (int)rank * cw;
+            PairWork pw;
+            for (int idx = 0; !*abort_flag && pair_work(p, cluster_id, nclusters, idx, pw); ++idx) {
+                const int i0 = pw.ti * 2 * kHalfM + (int)rank * kHalfM;
+                const int cw = pw.w / 2;  // this CTA's columns of the unit
+                const int j0 = pw.j0 + (int)rank * cw;
                 const uint32_t tx = 2u * (a_bytes + (uint32_t)cw * kRowBytes);  // both CTAs' bytes
                 bool ok = true;
-                for (int kb = 0; kb < kb_total; ++kb, ++it) {
+                for (int kb = pw.kb0; kb < pw.kb1; ++kb, ++it) {
                     if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) { ok = false; break; }
                     if (!stall) {
                         const uint32_t full_c = dsmem_map(bar_full + 8 * s, 0);
@@ -200,17 +307,22 @@ __global__ void __launch_bounds__(192, 1)
             // field (address >> 4, below 2^14 for any shared-memory address)
             const uint64_t da0 = make_sw128_desc(sbase, p_lbo, 1024);
             const uint64_t db0 = make_sw128_desc(sbase + L.a_bytes, q_lbo, 1024);
+            (void)num_units;
+            (void)kb_total;
+            (void)full_units;
             int local = 0, s = 0;
             uint32_t ph = 0;
             bool ok = true;
-            for (int u = cluster_id; u < num_units && ok; u += nclusters, ++local) {
-                const uint32_t idesc = u < full_units ? idesc_full : idesc_half;
+            PairWork pw;
+            for (int idx = 0; ok && pair_work(p, cluster_id, nclusters, idx, pw); ++idx, ++local) {
+                const uint32_t idesc = pw.w == bn ? idesc_full : idesc_half;
                 const int b = local & 1;
                 const uint32_t tph = (uint32_t)(local >> 1) & 1u;
                 if (!mbar_wait(bar_tempty + 8 * b, tph ^ 1u, wc)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(b * bn);
-                for (int kb = 0; kb < kb_total; ++kb) {
+                const int kb0 = pw.kb0;
+                for (int kb = kb0; kb < pw.kb1; ++kb) {
                     if (!mbar_wait(bar_full + 8 * s, ph, wc)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t soff = (uint64_t)((s * stage_bytes) >> 4);
@@ -218,7 +330,7 @@ __global__ void __launch_bounds__(192, 1)
                     for (int kk = 0; kk < kRowBytes / (kUmmaK * es); ++kk) {
                         const uint64_t da = da0 + soff + (uint64_t)((kk * p_kstep) >> 4);
                         const uint64_t db = db0 + soff + (uint64_t)((kk * q_kstep) >> 4);
-                        const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+                        const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
                         if (FP8) umma_f8_pair(d_tmem, da, db, idesc, acc);
                         else umma_f16_pair(d_tmem, da, db, idesc, acc);
                     }
@@ -242,33 +354,84 @@ __global__ void __launch_bounds__(192, 1)
         const EpiParams e = p.epi;  // a local copy: its fields stay in registers
         int local = 0;
         uint32_t nblk = 0;  // tensor-store blocks this warp has issued
-        for (int u = cluster_id; u < p.num_units; u += nclusters, ++local) {
-            const PairUnit pu = pair_unit(u, p);
+        PairWork pw;
+        for (int idx = 0; pair_work(p, cluster_id, nclusters, idx, pw); ++idx, ++local) {
             const int b = local & 1;
             const uint32_t tph = (uint32_t)(local >> 1) & 1u;
             if (!mbar_wait(bar_tfull + 8 * b, tph, wc)) break;
             tc_fence_after();
-            const int i = pu.ti * 2 * kHalfM + (int)rank * kHalfM + row;
+            const int i = pw.ti * 2 * kHalfM + (int)rank * kHalfM + row;
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * p.bn);
-            const int j0 = pu.j0;
+            const int j0 = pw.j0;
+            if (pw.role == kSkPartial) {
+                // ------------------------- Stream-K: leave the partial for the tile's owner
+                float *slot = sk_slot(p, cluster_id, rank) + row;
+                for (int c0 = 0; c0 < pw.w; c0 += 16) {
+                    uint32_t r[16];
+                    __syncwarp();
+                    tmem_ld16(t_row + c0, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) slot[(c0 + c) * kHalfM] = __uint_as_float(r[c]);  // coalesced
+                }
+                tc_fence_before();
+                __syncwarp();  // orders the warp's stores before lane 0's release below
+                if (lane == 0) {
+                    mbar_arrive_cluster(dsmem_map(bar_tempty + 8 * b, 0));
+                    // one flag per warp (32 rows): the owner's warp of the same quarter waits on it
+                    st_release_gpu(p.sk_flag + (cluster_id * 2 + (int)rank) * 4 + quarter, sk_tag);
+                }
+                continue;
+            }
+            Fixup fx;
+            fx.n = 0;
+            if (pw.role == kSkOwner) {
+                // ------------------------- Stream-K: wait for the other pairs' partials
+                const int q0 = sk_first_contributor(p, cluster_id, nclusters, pw.sk_first);
+                const int64_t total = (int64_t)p.sk_tiles * p.kb_total;
+                for (int q = cluster_id - 1; q >= q0 && fx.n < kMaxFix; --q) {  // pair order: q = c-1, c-2, ...
+                    if (total * q / nclusters == total * (q + 1) / nclusters) continue;  // empty range
+                    const uint32_t *flag = p.sk_flag + (q * 2 + (int)rank) * 4 + quarter;
+                    if (ld_acquire_gpu(flag) != sk_tag) {
+                        const uint64_t t0 = globaltimer_ns();
+                        bool ok = true;
+                        while (ld_acquire_gpu(flag) != sk_tag) {
+                            if (*abort_flag || globaltimer_ns() - t0 > p.timeout_ns) {
+                                ok = false;
+                                break;
+                            }
+                        }
+                        if (!ok) {
+                            *abort_flag = 1;
+                            if (p.err_word) atomicExch(p.err_word, kErrTimeout);
+                            break;
+                        }
+                    }
+                    fx.src[fx.n++] = sk_slot(p, q, rank);
+                }
+            }
+            const Fixup *fxp = fx.n > 0 ? &fx : nullptr;
             if (p.epi_tma) {
                 const uint32_t blocks = sbase + L.epi_off + (uint32_t)quarter * 2u * kEpiBlockBytes;
                 const int i_base = i - lane;
                 __syncwarp();
                 if (e.c_dtype == DG_F32)
-                    epilogue_rows_tma<4>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, pu.w, p.Nj, lane, nblk);
+                    epilogue_rows_tma<4>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, pw.w, p.Nj, lane, nblk, 0, 1,
+                                         fxp, row);
                 else
-                    epilogue_rows_tma<2>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, pu.w, p.Nj, lane, nblk);
+                    epilogue_rows_tma<2>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, pw.w, p.Nj, lane, nblk, 0, 1,
+                                         fxp, row);
             } else {
                 const bool row_ok = i < p.Mi;
                 const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
                 char *crow = e.c + epi_row_offset(e, row_ok ? i : 0);
-                for (int c0 = 0; c0 < pu.w; c0 += 16) {
+                for (int c0 = 0; c0 < pw.w; c0 += 16) {
                     uint32_t r[16];
                     __syncwarp();
                     tmem_ld16(t_row + c0, r);
                     tmem_ld_wait();
                     if (!row_ok) continue;
+                    add_fixups(fxp, row, c0, r, 16);
                     epilogue_chunk16(e, crow, asi, i, j0 + c0, p.Nj, r);
                 }
             }
@@ -288,6 +451,15 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, (uint32_t)p.tmem_cols);
+    }
+    if (p.sk_tiles > 0 && threadIdx.x == 0) {
+        // the last CTA out publishes this launch's tag as the sequence number
+        __threadfence();
+        if (atomicAdd(p.sk_hdr + 1, 1u) == gridDim.x - 1) {
+            p.sk_hdr[1] = 0;
+            __threadfence();
+            st_release_gpu(p.sk_hdr, sk_tag);
+        }
     }
 }
 

@@ -149,6 +149,22 @@ def test_plan_square_bf16_and_fp8():
     assert pl["kind_name"] == "umma" and pl["block_k"] == 128 and pl["q_mn_major"] == 1
 
 
+def test_plan_square_stream_k_tail():
+    # 256 tiles of 256 x 256 on 74 CTA pairs: 222 whole, the last 34 shared
+    # out along k over every pair (Stream-K); without it, half-width tail tiles
+    p = meta_problem("square_bf16")
+    pl = dg.dg_plan(*views(p), 1.0, 0.0, False, 148).as_dict()
+    assert pl["cta_pair"] == 1 and pl["stream_k_tiles"] == 34 and pl["pair_half_tiles"] == 0
+    dg.dg_set_option(dg.DG_OPT_STREAM_K, 0)
+    try:
+        pl = dg.dg_plan(*views(p), 1.0, 0.0, False, 148).as_dict()
+        assert pl["stream_k_tiles"] == 0 and pl["pair_half_tiles"] == 34
+    finally:
+        dg.dg_set_option(dg.DG_OPT_STREAM_K, 1)
+    with pytest.raises(dg.DgError):
+        dg.dg_set_option(dg.DG_OPT_STREAM_K, 2)
+
+
 def test_plan_strided_gathers_a():
     pl = plan_of("strided")
     assert pl["kind_name"] == "umma" and pl["p_gather"] == 1 and pl["swap_ab"] == 0
@@ -372,8 +388,16 @@ def _check_plan(p, dt, M, N, K, alpha):
         if p["cta_pair"]:
             assert p["block_m"] == 256 and grid % 2 == 0 and bn >= 128 and split == 1
             assert 0 <= 2 * p["pair_half_tiles"] <= grid // 2
+            sk, pairs = p["stream_k_tiles"], grid // 2
+            assert not (sk and p["pair_half_tiles"])      # one tail treatment at a time
+            if sk:
+                pair_tiles = -(-Mi // 256) * tiles_j
+                kb_total = -(-K // p["block_k"])
+                assert sk == pair_tiles % pairs and pair_tiles > pairs   # the last, partial wave
+                assert 7 * sk >= pairs                   # a tile is split among at most 8 pairs
+                assert sk * kb_total >= pairs            # every pair gets at least one k block
         else:
-            assert p["block_m"] == 128 and p["pair_half_tiles"] == 0
+            assert p["block_m"] == 128 and p["pair_half_tiles"] == 0 and p["stream_k_tiles"] == 0
         assert p["vec_bytes"] in (1, 2, 4, 8, 16)
         if not p["p_gather"]:
             assert p["vec_bytes"] == 16
@@ -396,12 +420,13 @@ def test_plan_invariants_random_views():
         tags = [p["kind_name"]]
         if p["kind_name"] == "umma":
             tags += ["umma/pair"] * p["cta_pair"] + ["umma/split"] * (p["split_k"] > 1)
+            tags += ["umma/stream_k"] * (p["stream_k_tiles"] > 0)
             tags += ["umma/gather_cluster"] * (p["gather_cluster"] > 1)
         for t in tags:
             kinds[t] = kinds.get(t, 0) + 1
         _check_plan(p, dt, M, N, K, alpha)
     # the draw reaches every kernel family and the tensor-core variants
-    for k in ("gemv_n", "gemv_k", "umma", "simt", "umma/pair", "umma/split", "umma/gather_cluster"):
+    for k in ("gemv_n", "gemv_k", "umma", "simt", "umma/pair", "umma/split", "umma/gather_cluster", "umma/stream_k"):
         assert kinds.get(k, 0) >= 5, kinds
 
 
