@@ -301,7 +301,7 @@ def _strided_nchw_out() -> W.Problem:
                      bias=p.bias, act="relu")
 
 
-def per_shape(dg, peaks, quick: bool, only=None):
+def per_shape(dg, peaks, quick: bool, only=None, tune: bool = False):
     """Every workload of the benchmark definition: time, TFLOPS, GB/s and
     fraction of roofline, with the dispatcher's kernel choice."""
     out = {}
@@ -318,6 +318,21 @@ def per_shape(dg, peaks, quick: bool, only=None):
         fl, by = flops_bytes(base)
         t_roof, bound = roofline_time_s(base, peaks)
         med = t_graph
+        tuned = None
+        if tune:
+            # the library's autotuner on the same operands: the variant it keeps,
+            # then the same graph-replay timing with that variant in force
+            q = gpus[0]
+            epi = dg.epilogue(q.bias, q.act) if (q.bias is not None or q.act != "none") else None
+            st, res = dg.dg_autotune(A, B, C, q.alpha, q.beta, q.scale_a, q.scale_b, epi, None, 5)
+            assert st == dg.DG_OK, dg.status_string(st)
+            t_tuned, _, _ = time_problem(gpus, dg, reps, warm=5)
+            chosen = res.plan.as_dict()
+            tuned = {"us": t_tuned * 1e6, "frac_of_roofline": t_roof / t_tuned, "candidates": res.candidates,
+                     "trial_us_rule": res.default_us, "trial_us_best": res.best_us,
+                     "plan": {k: chosen[k] for k in ("kind_name", "block_n", "split_k", "cta_pair", "stream_k_tiles",
+                                                     "gather_cluster", "epi_tma_store", "stages", "grid")}}
+            dg.dg_tune_clear()
         out[name] = {"kernel": pl["kind_name"], "us": med * 1e6, "us_stream": t_stream * 1e6,
                      "host_us_per_call": host * 1e6,
                      "tflops": fl / med / 1e12, "gbs": by / med / 1e9, "bound": bound,
@@ -326,6 +341,8 @@ def per_shape(dg, peaks, quick: bool, only=None):
                      "timing": "CUDA-graph replay of the calls (device time); us_stream: back-to-back stream calls",
                      "l2": (f"{copies} rotating input copies, {copies * by / 1e6:.0f} MB"
                             if copies > 1 else "single copy (L2-resident)")}
+        if tuned is not None:
+            out[name]["autotuned"] = tuned
         del gpus
         torch.cuda.empty_cache()
     return out
@@ -340,7 +357,7 @@ def run_one_shape(args):
     if args.early_launch >= 0:
         dg.dg_set_option(dg.DG_OPT_EARLY_LAUNCH, args.early_launch)
 
-    res = per_shape(dg, load_peaks(), True, only=args.shape)
+    res = per_shape(dg, load_peaks(), True, only=args.shape, tune=args.autotune)
     out = {"shape": args.shape, **res}
     if args.trace:
         # one more call with CTA 0's phase timestamps (ns from kernel entry)
@@ -538,7 +555,7 @@ def run_dg(args):
         if not args.skip_cpu:
             result["e2e"] = e2e(dg, gv, gk, dev, stream, max(3, min(args.steps, 20)))
         if not args.no_per_shape:
-            result["per_shape"] = per_shape(dg, peaks, args.quick)
+            result["per_shape"] = per_shape(dg, peaks, args.quick, tune=args.autotune)
         if not args.skip_cpu:
             result["cpu_baseline"] = cpu_baseline(args.quick)
         print(json.dumps(result), flush=True)
@@ -721,6 +738,8 @@ def main():
     ap.add_argument("--max-split", type=int, default=0, help="with --shape: cap the tensor-core split-K")
     ap.add_argument("--trace", action="store_true", help="with --shape: phase timestamps of CTA 0")
     ap.add_argument("--cpu-baseline-worker", type=int, default=0, help=argparse.SUPPRESS)
+    ap.add_argument("--autotune", action="store_true",
+                    help="per-shape rows also report dg_autotune's chosen variant and its time")
     ap.add_argument("--early-launch", type=int, default=-1,
                     help="programmatic dependent launch policy (0 off, 1 at kernel start, 2 near the end, "
                          "3 the library's per-kernel default)")

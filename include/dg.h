@@ -244,6 +244,46 @@ dg_status dg_plan(const dg_view *A, const dg_view *B, const dg_view *C,
                   float alpha, float beta, int has_scales, int num_sms,
                   dg_plan_info *out);
 
+/*
+ * dg_autotune — the call of dg_gemm_ex, after timing the kernel variants that
+ * can serve it on these very operands ("DeepGEMM deep dive", §5.3: the best
+ * tile and pipeline settings depend on the shape and are found by measuring;
+ * "DeepGEMM: a recalibration of the compute paradigm", §6.1: the chosen
+ * configuration is cached per problem).  The variants are the tensor-core
+ * tile width (32..256 columns), k splits (1..8, on-chip cluster reduction),
+ * CTA pairs with or without the Stream-K tail, the gather-cluster size and
+ * the tensor-store epilogue; for the memory-bound GEMV, its k splits.  Each
+ * is run `reps` times (1..1000) after a warm-up and timed with CUDA events;
+ * the fastest is kept in a process-wide table keyed by the views (shapes,
+ * strides, types, pointer alignment), beta == 0, alpha == 0, the device and
+ * its SM count, and every later dg_gemm / dg_gemm_ex with the same key uses
+ * it.  Calls whose plan has no variants (CUDA-core kernel, K-contiguous GEMV,
+ * alpha == 0) just run.
+ *  On return C holds the product, as after dg_gemm_ex: the trials overwrite
+ *  C, and when beta != 0 its bytes are saved first (a temporary device
+ *  buffer of C's span) and put back before the final call.  The function
+ *  synchronises `stream`; it is DG_ERR_UNSUPPORTED while the stream is being
+ *  captured into a graph.  `out` (may be NULL) receives the number of
+ *  variants timed, the time per call of the rule's plan and of the chosen
+ *  one, and the chosen plan.
+ */
+typedef struct {
+    int32_t candidates;   /* variants timed                                  */
+    int32_t reserved;
+    float default_us;     /* time per call of the dispatcher's own plan       */
+    float best_us;        /* time per call of the chosen variant              */
+    dg_plan_info plan;    /* the chosen plan                                  */
+} dg_tune_result;
+
+dg_status dg_autotune(const dg_view *A, const dg_view *B, const dg_view *C,
+                      float alpha, float beta,
+                      const float *scale_a, const float *scale_b,
+                      const dg_epilogue *epilogue, void *stream, int reps,
+                      dg_tune_result *out);
+
+/* Forget every tuned variant (later calls plan by the rules again). */
+dg_status dg_tune_clear(void);
+
 /* Number of kernels this library has launched in this process. */
 uint64_t dg_launch_count(void);
 

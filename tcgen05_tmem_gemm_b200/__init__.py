@@ -87,6 +87,14 @@ class dg_plan_info(ctypes.Structure):
         return d
 
 
+class dg_tune_result(ctypes.Structure):
+    _fields_ = [
+        ("candidates", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("default_us", ctypes.c_float), ("best_us", ctypes.c_float),
+        ("plan", dg_plan_info),
+    ]
+
+
 class DgError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -116,6 +124,11 @@ def _load():
     L.dg_plan.argtypes = [V, V, V, ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int,
                           P(dg_plan_info)]
     L.dg_plan.restype = ctypes.c_int
+    L.dg_autotune.argtypes = [V, V, V, ctypes.c_float, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                              P(dg_epilogue), ctypes.c_void_p, ctypes.c_int, P(dg_tune_result)]
+    L.dg_autotune.restype = ctypes.c_int
+    L.dg_tune_clear.argtypes = []
+    L.dg_tune_clear.restype = ctypes.c_int
     L.dg_launch_count.argtypes = []
     L.dg_launch_count.restype = ctypes.c_uint64
     L.dg_set_option.argtypes = [ctypes.c_int, ctypes.c_int64]
@@ -249,6 +262,21 @@ def dg_plan(A: dg_view, B: dg_view, C: dg_view, alpha=1.0, beta=0.0, has_scales=
     if st != DG_OK:
         raise DgError(st, "dg_plan")
     return out
+
+
+def dg_autotune(A: dg_view, B: dg_view, C: dg_view, alpha: float, beta: float, scale_a=None, scale_b=None,
+                epi=None, stream=None, reps: int = 5):
+    """Time the kernel variants for this call, keep the fastest for its shape
+    key, and run the call: returns (status, dg_tune_result)."""
+    out = dg_tune_result()
+    st = lib.dg_autotune(ctypes.byref(A), ctypes.byref(B), ctypes.byref(C), float(alpha), float(beta),
+                         _ptr(scale_a), _ptr(scale_b), None if epi is None else ctypes.byref(epi),
+                         _stream_ptr(stream), int(reps), ctypes.byref(out))
+    return st, out
+
+
+def dg_tune_clear() -> None:
+    lib.dg_tune_clear()
 
 
 def dg_launch_count() -> int:

@@ -18,6 +18,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include <cudaTypedefs.h>
 
@@ -266,31 +267,59 @@ bool gemv_applicable(const Views &v, int64_t M, int64_t N, int64_t K, int kind) 
     return false;
 }
 
+// A plan variant: each field replaces the dispatcher's rule for one choice
+// (0 or -1: keep the rule).  dg_autotune times the variants a call admits
+// and keeps the fastest per shape key; a variant the operands do not admit
+// makes the planner fail, and the autotuner skips it.
+struct Override {
+    int bn = 0;          // tensor-core tile width
+    int split = 0;       // tensor-core k splits (1 = none)
+    int pair = -1;       // CTA pairs: 0 / 1
+    int sk = -1;         // Stream-K tail of a CTA-pair schedule: 0 / 1
+    int gcl = 0;         // gather-cluster size: 1, 2 or 4
+    int epi_tma = -1;    // tensor-store epilogue: 0 / 1
+    int stages = 0;      // pipeline depth (at most what shared memory holds)
+    int gemv_split = 0;  // GEMV_N k splits
+    bool any() const {
+        return bn || split || pair >= 0 || sk >= 0 || gcl || epi_tma >= 0 || stages || gemv_split;
+    }
+};
+
 // GEMV_N grid: 256-column strips times k splits (one cluster per strip, at
 // most 8), about two blocks per SM, k ranges in whole 64-row TMA stages (so
 // one split's last stage never reads the next split's rows) and each block's
 // slice of x within 64 KB of shared memory.
-void gemv_n_split(int64_t M, int64_t N, int64_t K, int num_sms, dg_plan_info *in) {
+bool gemv_n_split(int64_t M, int64_t N, int64_t K, int num_sms, dg_plan_info *in, int force_s = 0) {
     const int64_t r_inst = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
     const int64_t gx = (N + 255) / 256;
     int64_t S = (2 * num_sms + gx / 2) / gx;
     S = std::max<int64_t>(1, std::min<int64_t>(S, kMaxCluster));
     S = std::min<int64_t>(S, std::max<int64_t>(1, K / 64));
+    if (force_s > 0) {
+        if (force_s > kMaxCluster) return false;
+        S = force_s;
+    }
     int64_t kper = ((K + S - 1) / S + 63) / 64 * 64;
     while (kper * r_inst > 16384 && S < kMaxCluster) {
+        if (force_s > 0) return false;
         ++S;
         kper = ((K + S - 1) / S + 63) / 64 * 64;
     }
     S = (K + kper - 1) / kper;
+    if (force_s > 0 && S != force_s) return false;  // the k range does not split that many ways
     in->block_n = 256;
     in->block_k = (int32_t)kper;
     in->split_k = (int32_t)std::max<int64_t>(S, 1);
     in->grid = (int32_t)(gx * in->split_k);
     in->vec_bytes = 16;
+    return true;
 }
 
 // Which UMMA configuration serves these views (false: none).
-bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int num_sms, bool allow_sk, Plan *pl) {
+bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int num_sms, bool allow_sk, Plan *pl,
+               const Override *ov = nullptr) {
+    static const Override kNone;
+    if (!ov) ov = &kNone;
     const int dt = v.A->dtype;
     if (dt != DG_F16 && dt != DG_BF16 && dt != DG_E4M3) return false;
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return false;
@@ -352,7 +381,7 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
         bn = (int)(((bn + per - 1) / per) * per);
         if (bn > 256) return false;
     }
-    if (g_pair.load() != 2) {
+    if (g_pair.load() != 2 && !ov->bn) {
         // very few tiles: narrower ones put more SMs to work, each loading
         // less of Q and storing less of C (not when CTA pairs are forced:
         // they need tiles of 128 columns or more)
@@ -360,12 +389,20 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
         while (bn / 2 >= bn_min && bn % 2 == 0 && tiles_i * ((Nj + bn / 2 - 1) / (bn / 2)) <= num_sms / 8)
             bn /= 2;
     }
+    if (ov->bn) {
+        bn = ov->bn;
+        if (bn < 16 || bn > 256 || bn % 16 || (q_mn && bn % (128 / es))) return false;
+    }
     const int64_t tiles_j = (Nj + bn - 1) / bn;
     const int64_t tiles = tiles_i * tiles_j;
     const int64_t kb_total = (K + bk - 1) / bk;
     int64_t split = 1;
     const int max_split = g_max_split.load();
-    if (tiles * 2 <= num_sms && kb_total >= 8 && max_split > 1) {
+    if (ov->split) {
+        // every split is one CTA of a cluster and all of them resident at once
+        split = ov->split;
+        if (split > kMaxCluster || split > kb_total || (split > 1 && tiles * split > num_sms)) return false;
+    } else if (tiles * 2 <= num_sms && kb_total >= 8 && max_split > 1) {
         // k splits of a tile form one cluster and reduce on chip
         split = std::min<int64_t>(num_sms / tiles, kb_total / 4);
         split = std::min<int64_t>(split, std::min(max_split, kMaxCluster));
@@ -373,31 +410,49 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     }
     int64_t kb_per = (kb_total + split - 1) / split;
     split = (kb_total + kb_per - 1) / kb_per;
+    if (ov->split && split != ov->split) return false;  // k does not split that many ways
     const int64_t units = tiles * split;
     if (units > INT32_MAX) return false;
     // a CTA pair shares each 256 x bn tile when there are enough tiles to fill
     // the machine (or when forced); TMA operands only, no split
     const int pair_mode = g_pair.load();
     bool pair = false;
-    if (pair_mode > 0 && p_tma && split == 1 && bn >= 128 && num_sms >= 2) {
+    bool pair_ok = false;  // the operands admit CTA pairs
+    if (p_tma && split == 1 && bn >= 128 && num_sms >= 2) {
         const int per = 128 / es;
         // a CTA loads bn/2 columns of Q: whole 128-byte boxes (MN-major) or
         // two boxes of bn/4 rows (K-major)
-        const bool halves_ok = q_mn ? ((bn / 2) % per == 0) : ((bn / 4) % 8 == 0);
-        if (halves_ok) pair = (pair_mode == 2) || (Mi >= 256 && tiles >= num_sms);
+        pair_ok = q_mn ? ((bn / 2) % per == 0) : ((bn / 4) % 8 == 0);
+        if (pair_ok && pair_mode > 0) pair = (pair_mode == 2) || (Mi >= 256 && tiles >= num_sms);
+    }
+    if (ov->pair >= 0) {
+        if (ov->pair && !pair_ok) return false;
+        pair = ov->pair != 0;
     }
     // the epilogue stores C through tensor copies when C is row-major along j
     // with 16-byte aligned rows, is not read (beta == 0) and each tile is a
     // whole number of 128-byte blocks; split tiles use the cluster reduction
     const int ces = elem_size(v.C->dtype);
     const int blk = 128 / ces;  // columns per 128-byte block
-    const bool epi_tma = g_epi_tma.load() != 0 && !swap && split == 1 && beta == 0.f && v.c.tma_ok &&
-                         v.c.unit_dim == 1 && bn % blk == 0 && Nj >= blk && Mi >= 32;
-    int stages = pair ? umma_pair_max_stages(bn, epi_tma) : umma_max_stages(bn, !p_tma, epi_tma, (int)split);
+    const bool epi_ok = !swap && split == 1 && beta == 0.f && v.c.tma_ok && v.c.unit_dim == 1 && bn % blk == 0 &&
+                        Nj >= blk && Mi >= 32;
+    bool epi_tma = g_epi_tma.load() != 0 && epi_ok;
+    if (ov->epi_tma >= 0) {
+        if (ov->epi_tma && !epi_ok) return false;
+        epi_tma = ov->epi_tma != 0;
+    }
+    const int max_stages =
+        pair ? umma_pair_max_stages(bn, epi_tma) : umma_max_stages(bn, !p_tma, epi_tma, (int)split);
+    int stages = max_stages;
+    if (ov->stages) {
+        if (ov->stages < 2 || ov->stages > max_stages) return false;
+        stages = ov->stages;
+    }
     if (split > 1) {
         // the split-K reduction stages a CTA's partial in its operand ring
         const int64_t ring = (int64_t)stages * (128 * 128 + bn * 128);
         if (stages < 3 || (int64_t)umma_split_out_bytes(bn, (int)split) > ring) {
+            if (ov->split > 1) return false;
             stages = umma_max_stages(bn, !p_tma, epi_tma, 1);
             split = 1;
             kb_per = kb_total;
@@ -407,12 +462,18 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     // a gathered P tile is shared by the CTAs of its row of tiles: 2 or 4 of
     // them form a cluster and each gathers its share of every stage
     int gcl = 1;
-    if (!p_tma && split == 1 && !pair && gather_vec * pvi.es >= 4 && g_gather_cluster.load() != 0) {
+    const bool gcl_ok = !p_tma && split == 1 && !pair && gather_vec * pvi.es >= 4;
+    if (gcl_ok && g_gather_cluster.load() != 0) {
         for (int c : {4, 2})
             if (tiles_j % c == 0 && num_sms >= c) {
                 gcl = c;
                 break;
             }
+    }
+    if (ov->gcl) {
+        if (ov->gcl != 1 && (!gcl_ok || (ov->gcl != 2 && ov->gcl != 4) || tiles_j % ov->gcl || num_sms < ov->gcl))
+            return false;
+        gcl = ov->gcl;
     }
     dg_plan_info &in = pl->info;
     in.kind = DG_KIND_UMMA;
@@ -446,11 +507,15 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
         // tiles is split among at most kMaxFix + 1 pairs and every pair gets
         // at least one k block
         const int64_t kb_all = tail * kb_total;
-        if (allow_sk && g_stream_k.load() != 0 && pair_units > ncl && tail > 0 && 7 * tail >= ncl &&
-            kb_all >= ncl)
+        const bool sk_ok = pair_units > ncl && tail > 0 && 7 * tail >= ncl && kb_all >= ncl;
+        const bool sk = allow_sk && sk_ok && (ov->sk >= 0 ? ov->sk != 0 : g_stream_k.load() != 0);
+        if (ov->sk == 1 && allow_sk && !sk_ok) return false;
+        if (sk)
             in.stream_k_tiles = (int32_t)tail;
         else if (g_pair_tail.load() != 0 && quarter_ok && pair_units > ncl && tail > 0 && 2 * tail <= ncl)
             in.pair_half_tiles = (int32_t)tail;
+    } else if (ov->sk == 1) {
+        return false;
     }
     pl->fp8 = (dt == DG_E4M3);
     pl->smem = pair ? umma_pair_smem_bytes(bn, stages, epi_tma)
@@ -458,7 +523,64 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     return true;
 }
 
-dg_status make_plan(Views &v, float alpha, float beta, int num_sms, Plan *pl, bool allow_sk = true) {
+// ---------------------------------------------------------------- autotune
+// Tuned plan variants, keyed by everything a plan depends on except the
+// addresses themselves: the three views with their pointers reduced to the
+// 128-byte alignment class the planner looks at, beta == 0, alpha == 0, the
+// device and its SM count.
+struct TuneKey {
+    dg_view A, B, C;
+    int32_t beta_zero, alpha_zero, num_sms, dev;
+};
+
+TuneKey tune_key(const dg_view *A, const dg_view *B, const dg_view *C, float alpha, float beta, int num_sms) {
+    TuneKey k;
+    std::memset(&k, 0, sizeof(k));
+    k.A = *A;
+    k.B = *B;
+    k.C = *C;
+    for (dg_view *v : {&k.A, &k.B, &k.C}) v->ptr = reinterpret_cast<void *>(reinterpret_cast<uintptr_t>(v->ptr) & 127u);
+    k.beta_zero = beta == 0.f;
+    k.alpha_zero = alpha == 0.f;
+    k.num_sms = num_sms;
+    if (cudaGetDevice(&k.dev) != cudaSuccess) {
+        cudaGetLastError();
+        k.dev = -1;
+    }
+    return k;
+}
+
+struct TuneEntry {
+    TuneKey key;
+    Override ov;
+};
+std::mutex g_tune_mu;
+std::vector<TuneEntry> g_tuned;
+
+bool tuned_override(const TuneKey &k, Override *ov) {
+    std::lock_guard<std::mutex> lk(g_tune_mu);
+    for (const TuneEntry &e : g_tuned)
+        if (std::memcmp(&e.key, &k, sizeof(k)) == 0) {
+            *ov = e.ov;
+            return true;
+        }
+    return false;
+}
+
+void store_tuned(const TuneKey &k, const Override &ov) {
+    std::lock_guard<std::mutex> lk(g_tune_mu);
+    for (TuneEntry &e : g_tuned)
+        if (std::memcmp(&e.key, &k, sizeof(k)) == 0) {
+            e.ov = ov;
+            return;
+        }
+    g_tuned.push_back(TuneEntry{k, ov});
+}
+
+// `force`: plan with exactly this variant (an empty one: the rules, not the
+// tuned table); null: the tuned variant for these views if there is one.
+dg_status make_plan(Views &v, float alpha, float beta, int num_sms, Plan *pl, bool allow_sk = true,
+                    const Override *force = nullptr) {
     (void)beta;
     dg_status st;
     if ((st = analyse(v.A, false, &v.a)) != DG_OK) return st;
@@ -477,27 +599,41 @@ dg_status make_plan(Views &v, float alpha, float beta, int num_sms, Plan *pl, bo
     in.split_k = 1;
     if (M == 0 || N == 0) { in.kind = DG_KIND_NONE; return DG_OK; }
     if (alpha == 0.f || K == 0) { in.kind = DG_KIND_SCALE_C; return DG_OK; }
-    const int force = g_force_kind.load();
-    const bool simt_only = (v.A->dtype == DG_F32) || force == DG_KIND_SIMT;
+    Override tuned;
+    const Override *ov = force;
+    if (!ov && tuned_override(tune_key(v.A, v.B, v.C, alpha, beta, num_sms), &tuned)) ov = &tuned;
+    const bool forced = force != nullptr && force->any();
+    const int force_kind = g_force_kind.load();
+    const bool simt_only = (v.A->dtype == DG_F32) || force_kind == DG_KIND_SIMT;
     if (!simt_only) {
-        if (force == DG_KIND_GEMV_N || force == DG_KIND_GEMV_K) {
-            if (gemv_applicable(v, M, N, K, force)) {
-                in.kind = force;
-                if (force == DG_KIND_GEMV_N) gemv_n_split(M, N, K, num_sms, &in);
+        if (force_kind == DG_KIND_GEMV_N || force_kind == DG_KIND_GEMV_K) {
+            if (gemv_applicable(v, M, N, K, force_kind)) {
+                in.kind = force_kind;
+                if (force_kind == DG_KIND_GEMV_N && !gemv_n_split(M, N, K, num_sms, &in, ov ? ov->gemv_split : 0)) {
+                    if (forced) return DG_ERR_UNSUPPORTED;
+                    gemv_n_split(M, N, K, num_sms, &in);
+                }
                 return DG_OK;
             }
-        } else if (force == DG_KIND_UMMA) {
-            if (umma_plan(v, M, N, K, beta, num_sms, allow_sk, pl)) return DG_OK;
+        } else if (force_kind == DG_KIND_UMMA) {
+            if (umma_plan(v, M, N, K, beta, num_sms, allow_sk, pl, ov)) return DG_OK;
+            if (forced) return DG_ERR_UNSUPPORTED;
+            if (ov && umma_plan(v, M, N, K, beta, num_sms, allow_sk, pl)) return DG_OK;
         } else {
             if (M <= 8) {
                 if (gemv_applicable(v, M, N, K, DG_KIND_GEMV_N)) {
                     in.kind = DG_KIND_GEMV_N;
-                    gemv_n_split(M, N, K, num_sms, &in);
+                    if (!gemv_n_split(M, N, K, num_sms, &in, ov ? ov->gemv_split : 0)) {
+                        if (forced) return DG_ERR_UNSUPPORTED;
+                        gemv_n_split(M, N, K, num_sms, &in);
+                    }
                     return DG_OK;
                 }
                 if (gemv_applicable(v, M, N, K, DG_KIND_GEMV_K)) { in.kind = DG_KIND_GEMV_K; return DG_OK; }
             }
-            if (umma_plan(v, M, N, K, beta, num_sms, allow_sk, pl)) return DG_OK;
+            if (umma_plan(v, M, N, K, beta, num_sms, allow_sk, pl, ov)) return DG_OK;
+            if (forced) return DG_ERR_UNSUPPORTED;
+            if (ov && umma_plan(v, M, N, K, beta, num_sms, allow_sk, pl)) return DG_OK;  // a stale variant
         }
     }
     if (M > int64_t(65535) * 64 || N > INT32_MAX || K > INT32_MAX) return DG_ERR_UNSUPPORTED;
@@ -823,6 +959,74 @@ struct CallCache {
 };
 thread_local CallCache t_calls;
 
+// Check the buffers of a planned call, fetch the Stream-K workspace it needs
+// and prepare its launch.  Without a workspace on this stream (e.g. during a
+// graph capture) the call is planned again without Stream-K; with a forced
+// variant that needs one, it is DG_ERR_UNSUPPORTED.
+dg_status build_launch(Views &v, Plan &pl, float alpha, float beta, const float *scale_a, const float *scale_b,
+                       const float *bias, int act, DeviceState *ds, cudaStream_t stream, const Override *force,
+                       LaunchRec *rec) {
+    const dg_plan_info &in = pl.info;
+    // every buffer the launch touches must live on this device
+    const bool use_ab = in.kind != DG_KIND_SCALE_C;
+    if (use_ab && (!device_accessible(v.A->ptr) || !device_accessible(v.B->ptr))) return DG_ERR_POINTER;
+    if (!device_accessible(v.C->ptr)) return DG_ERR_POINTER;
+    if (use_ab && scale_a && !device_accessible(scale_a)) return DG_ERR_POINTER;
+    if (use_ab && scale_b && !device_accessible(scale_b)) return DG_ERR_POINTER;
+    if (bias && !device_accessible(bias)) return DG_ERR_POINTER;
+    void *sk_ws = nullptr;
+    if (in.stream_k_tiles > 0) {
+        size_t flag_off = 0, part_off = 0;
+        const size_t need = sk_workspace_bytes(in.grid / 2, in.block_n, &flag_off, &part_off);
+        sk_ws = sk_workspace(ds, stream, need, part_off);
+        if (!sk_ws) {
+            if (force && force->any()) return DG_ERR_UNSUPPORTED;
+            const dg_status st = make_plan(v, alpha, beta, ds->num_sms, &pl, false, force);
+            if (st != DG_OK) return st;
+        }
+    }
+    return prepare(v, pl, alpha, beta, use_ab ? scale_a : nullptr, use_ab ? scale_b : nullptr, bias, act, ds, sk_ws,
+                   rec);
+}
+
+// The variants dg_autotune times for a call whose rule-based plan is `base`.
+std::vector<Override> tune_candidates(const dg_plan_info &base) {
+    std::vector<Override> c;
+    c.push_back(Override{});  // the dispatcher's own rule first
+    if (base.kind == DG_KIND_GEMV_N) {
+        for (int s = 1; s <= kMaxCluster; ++s) {
+            Override o;
+            o.gemv_split = s;
+            c.push_back(o);
+        }
+        return c;
+    }
+    for (int bn : {32, 64, 128, 256}) {
+        for (int split : {1, 2, 3, 4, 6, 8}) {
+            for (int pair : {0, 1}) {
+                if (pair && split > 1) continue;
+                for (int sk : {0, 1}) {
+                    if (sk && !pair) continue;
+                    for (int gcl : {1, 2, 4}) {
+                        if (gcl > 1 && (!base.p_gather || split > 1 || pair)) continue;
+                        for (int epi : {0, 1}) {
+                            Override o;
+                            o.bn = bn;
+                            o.split = split;
+                            o.pair = pair;
+                            o.sk = pair ? sk : -1;
+                            o.gcl = base.p_gather ? gcl : 0;
+                            o.epi_tma = epi;
+                            c.push_back(o);
+                        }
+                    }
+                }
+            }
+        }
+    }
+    return c;
+}
+
 }  // namespace
 }  // namespace dg
 
@@ -878,31 +1082,12 @@ dg_status dg_gemm_ex(const dg_view *A, const dg_view *B, const dg_view *C, float
         st = make_plan(v, alpha, beta, ds->num_sms, &pl);
         if (st != DG_OK) return st;
     }
-    const dg_plan_info &in = pl.info;
-    // every buffer the launch touches must live on this device
-    const bool use_ab = in.kind != DG_KIND_SCALE_C;
-    if (use_ab && (!device_accessible(A->ptr) || !device_accessible(B->ptr))) return DG_ERR_POINTER;
-    if (!device_accessible(C->ptr)) return DG_ERR_POINTER;
-    if (use_ab && scale_a && !device_accessible(scale_a)) return DG_ERR_POINTER;
-    if (use_ab && scale_b && !device_accessible(scale_b)) return DG_ERR_POINTER;
-    if (bias && !device_accessible(bias)) return DG_ERR_POINTER;
-    void *sk_ws = nullptr;
-    if (in.stream_k_tiles > 0) {
-        size_t flag_off = 0, part_off = 0;
-        const size_t need = sk_workspace_bytes(in.grid / 2, in.block_n, &flag_off, &part_off);
-        sk_ws = sk_workspace(ds, static_cast<cudaStream_t>(stream), need, part_off);
-        if (!sk_ws) {
-            // no workspace on this stream now (e.g. inside a graph capture): plan without Stream-K
-            st = make_plan(v, alpha, beta, ds->num_sms, &pl, false);
-            if (st != DG_OK) return st;
-        }
-        key.epoch = g_epoch.load();  // a replaced workspace invalidated the cache
-    }
     const int slot = t_calls.next;
     t_calls.used[slot] = false;
-    st = prepare(v, pl, alpha, beta, use_ab ? scale_a : nullptr, use_ab ? scale_b : nullptr, bias, act, ds, sk_ws,
-                 &t_calls.rec[slot]);
+    st = build_launch(v, pl, alpha, beta, scale_a, scale_b, bias, act, ds, static_cast<cudaStream_t>(stream), nullptr,
+                      &t_calls.rec[slot]);
     if (st != DG_OK) return st;
+    key.epoch = g_epoch.load();  // a replaced Stream-K workspace invalidated the cache
     t_calls.key[slot] = key;
     t_calls.used[slot] = true;
     t_calls.next = (slot + 1) % 8;
@@ -912,6 +1097,119 @@ dg_status dg_gemm_ex(const dg_view *A, const dg_view *B, const dg_view *C, float
 dg_status dg_gemm(const dg_view *A, const dg_view *B, const dg_view *C, float alpha, float beta,
                   const float *scale_a, const float *scale_b, void *stream) {
     return dg_gemm_ex(A, B, C, alpha, beta, scale_a, scale_b, nullptr, stream);
+}
+
+dg_status dg_autotune(const dg_view *A, const dg_view *B, const dg_view *C, float alpha, float beta,
+                      const float *scale_a, const float *scale_b, const dg_epilogue *epilogue, void *stream,
+                      int reps, dg_tune_result *out) {
+    if (!A || !B || !C) return DG_ERR_NULL;
+    const float *bias = nullptr;
+    int act = DG_ACT_NONE;
+    if (epilogue) {
+        if (epilogue->activation < DG_ACT_NONE || epilogue->activation > DG_ACT_GELU_TANH || epilogue->reserved != 0)
+            return DG_ERR_VALUE;
+        bias = epilogue->bias;
+        act = epilogue->activation;
+    }
+    if (reps < 1 || reps > 1000) return DG_ERR_VALUE;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Views v{A, B, C, {}, {}, {}};
+    Plan base;
+    const Override rule;  // the dispatcher's rules, not an earlier tuning
+    dg_status st = make_plan(v, alpha, beta, 148, &base, true, &rule);
+    if (st != DG_OK) return st;
+    dg_tune_result res;
+    std::memset(&res, 0, sizeof(res));
+    if (base.info.kind == DG_KIND_NONE) {
+        if (out) *out = res;
+        return DG_OK;
+    }
+    DeviceState *ds = nullptr;
+    if ((st = device_state(&ds)) != DG_OK) return st;
+    if ((st = make_plan(v, alpha, beta, ds->num_sms, &base, true, &rule)) != DG_OK) return st;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return DG_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) return DG_ERR_UNSUPPORTED;  // it synchronises and may allocate
+    const TuneKey key = tune_key(A, B, C, alpha, beta, ds->num_sms);
+    const bool tunable = base.info.kind == DG_KIND_UMMA || base.info.kind == DG_KIND_GEMV_N;
+    if (tunable) {
+        // with beta != 0 every trial reads and rewrites C: keep its bytes and put them back
+        void *saved = nullptr;
+        size_t span = 0;
+        if (beta != 0.f) {
+            span = (size_t)v.c.span;
+            if (cudaMalloc(&saved, span) != cudaSuccess ||
+                cudaMemcpyAsync(saved, C->ptr, span, cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
+                cudaGetLastError();
+                if (saved) cudaFree(saved);
+                return DG_ERR_CUDA;
+            }
+        }
+        cudaEvent_t e0, e1;
+        if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) return DG_ERR_CUDA;
+        std::vector<dg_plan_info> seen;
+        float best = 0.f;
+        Override best_ov;
+        bool have = false;
+        for (const Override &o : tune_candidates(base.info)) {
+            Plan pl;
+            if (make_plan(v, alpha, beta, ds->num_sms, &pl, true, &o) != DG_OK || pl.info.kind != base.info.kind)
+                continue;  // a variant these operands do not admit
+            bool dup = false;
+            for (const dg_plan_info &q : seen) dup = dup || std::memcmp(&q, &pl.info, sizeof(q)) == 0;
+            if (dup) continue;
+            LaunchRec rec;
+            if (build_launch(v, pl, alpha, beta, scale_a, scale_b, bias, act, ds, s, &o, &rec) != DG_OK) continue;
+            seen.push_back(pl.info);
+            bool ok = fire(rec, s) == DG_OK;  // warm-up (tensor maps, instruction cache)
+            ok = ok && cudaEventRecord(e0, s) == cudaSuccess;
+            for (int r = 0; ok && r < reps; ++r) ok = fire(rec, s) == DG_OK;
+            ok = ok && cudaEventRecord(e1, s) == cudaSuccess && cudaEventSynchronize(e1) == cudaSuccess;
+            float ms = 0.f;
+            ok = ok && cudaEventElapsedTime(&ms, e0, e1) == cudaSuccess;
+            if (!ok) {
+                cudaGetLastError();
+                continue;
+            }
+            const float us = ms * 1000.f / (float)reps;
+            if (seen.size() == 1) res.default_us = us;
+            if (!have || us < best) {
+                best = us;
+                best_ov = o;
+                have = true;
+            }
+            ++res.candidates;
+        }
+        cudaEventDestroy(e0);
+        cudaEventDestroy(e1);
+        if (saved) {
+            const bool ok = cudaMemcpyAsync(C->ptr, saved, span, cudaMemcpyDeviceToDevice, s) == cudaSuccess &&
+                            cudaStreamSynchronize(s) == cudaSuccess;
+            cudaFree(saved);
+            if (!ok) return DG_ERR_CUDA;
+        }
+        if (have) {
+            store_tuned(key, best_ov);
+            g_epoch.fetch_add(1);  // cached launches of these views take the tuned plan from now on
+            res.best_us = best;
+        }
+    }
+    // the call itself, with the chosen variant
+    st = dg_gemm_ex(A, B, C, alpha, beta, scale_a, scale_b, epilogue, stream);
+    if (st != DG_OK) return st;
+    Plan chosen;
+    if (make_plan(v, alpha, beta, ds->num_sms, &chosen) == DG_OK) res.plan = chosen.info;
+    if (out) *out = res;
+    return DG_OK;
+}
+
+dg_status dg_tune_clear(void) {
+    {
+        std::lock_guard<std::mutex> lk(g_tune_mu);
+        g_tuned.clear();
+    }
+    g_epoch.fetch_add(1);
+    return DG_OK;
 }
 
 dg_status dg_gemv(const dg_view *x, const dg_view *W, const dg_view *y, float alpha, float beta, void *stream) {

@@ -243,6 +243,21 @@ def test_gemm_ex_epilogue_errors_need_no_device():
                              None) == dg.DG_ERR_NULL
 
 
+def test_autotune_argument_errors_need_no_device():
+    p = meta_problem("small", M=16, N=16, K=16)
+    A, B, C = views(p)
+    out = dg.dg_tune_result()
+    assert dg.lib.dg_autotune(None, ctypes.byref(B), ctypes.byref(C), 1.0, 0.0, None, None, None, None, 3,
+                              ctypes.byref(out)) == dg.DG_ERR_NULL
+    for reps in (0, 1001):
+        assert dg.lib.dg_autotune(ctypes.byref(A), ctypes.byref(B), ctypes.byref(C), 1.0, 0.0, None, None, None,
+                                  None, reps, ctypes.byref(out)) == dg.DG_ERR_VALUE
+    bad_k = dg.make_view(FAKE, (17, 16), (32, 2), 1, "f16")
+    assert dg.lib.dg_autotune(ctypes.byref(A), ctypes.byref(bad_k), ctypes.byref(C), 1.0, 0.0, None, None, None,
+                              None, 3, ctypes.byref(out)) == dg.DG_ERR_SHAPE
+    assert dg.lib.dg_tune_clear() == dg.DG_OK
+
+
 def test_plan_nchw_output_stays_on_tensor_cores():
     # C written as an NCHW tensor [n, N, h, w] from the [n*h*w, N] product: the
     # row index of C spans two dims (n and h*w), which the tensor-core epilogue
