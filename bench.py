@@ -566,6 +566,86 @@ def run_dg(args):
         dist.destroy_process_group()
 
 
+def run_shard(args):
+    """The decode step split over the ranks by columns (strong scaling): x is
+    replicated, rank r holds its column block of W and of K^T (rows of K),
+    computes its blocks of y = x W and z = x K^T with dg_gemm on its own GPU,
+    and one NCCL all-gather per output assembles the whole y and z on every
+    rank.  The job is one decode step's bytes per step, whatever the number of
+    ranks; the time is the slowest rank's."""
+    import datetime
+
+    import torch.distributed as dist
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    if "MASTER_PORT" not in os.environ:
+        import socket
+
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            os.environ["MASTER_PORT"] = str(sk.getsockname()[1])
+    dist.init_process_group("nccl", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    import tcgen05_tmem_gemm_b200 as dg
+    from tcgen05_tmem_gemm_b200 import shard
+
+    dev = torch.device("cuda", local)
+    gv, gk = W.cfg_gemv(), W.cfg_gemv_kt()
+    step_bytes = flops_bytes(gv)[1] + flops_bytes(gk)[1]
+    N, NK = gv.N, gk.N
+    x = gv.A.base.to(dev)
+    kmat = gk.B.base  # [128, 4096] row-major; K^T's columns are its rows
+    blocks = []
+    for _ in range(ROTATE):
+        wb = shard.local_block(gv.B.base, rank, world, dev)
+        kb = shard.local_block(kmat.t(), rank, world, dev)     # [4096, width] block of K^T
+        blocks.append((wb, kb))
+    yb = torch.zeros(1, shard.shard_width(N, world), dtype=torch.bfloat16, device=dev)
+    zb = torch.zeros(1, shard.shard_width(NK, world), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    n_launch = [0]
+
+    def step(i):
+        wb, kb = blocks[i % ROTATE]
+        n0 = dg.dg_launch_count()
+        shard.gemm_block(x, wb, yb, N, rank, world, stream=stream)
+        shard.gemm_block(x, kb, zb, NK, rank, world, stream=stream)
+        n_launch[0] += dg.dg_launch_count() - n0
+        return shard.assemble(yb, N), shard.assemble(zb, NK)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    n_launch[0] = 0
+    a.record()
+    for i in range(args.steps):
+        y, z = step(i)
+    b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    assert dg.dg_sync_status() == dg.DG_OK
+    elapsed_max = max_over_ranks(a.elapsed_time(b) * 1e-3, world, dev)
+    # the assembled outputs are the single-GPU products (same kernels per column block)
+    ref_y = torch.empty(1, N, dtype=torch.bfloat16, device=dev)
+    dg.gemm(x, gv.B.base.to(dev), ref_y)
+    ok = bool(torch.allclose(y.float(), ref_y.float(), rtol=2e-2, atol=1e-3))
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": step_bytes * args.steps / elapsed_max / 1e9, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": elapsed_max / args.steps * 1e3, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD + "; split by columns of W and K^T over the ranks",
+                       "parallelism": f"column shards x{world}, NCCL all-gather of y and z",
+                       "launch": "eager dg_gemm calls and all-gathers on the current stream"},
+            "gpu_launches": int(n_launch[0]), "assembled_matches_single_gpu": ok}), flush=True)
+    dist.destroy_process_group()
+
+
 def e2e(dg, gv, gk, dev, stream, steps):
     """Same step through dg_gemm with host buffers: pinned host -> device copies
     of x, W and K, both products, device -> host copies of both outputs, every
@@ -738,6 +818,8 @@ def main():
     ap.add_argument("--max-split", type=int, default=0, help="with --shape: cap the tensor-core split-K")
     ap.add_argument("--trace", action="store_true", help="with --shape: phase timestamps of CTA 0")
     ap.add_argument("--cpu-baseline-worker", type=int, default=0, help=argparse.SUPPRESS)
+    ap.add_argument("--shard", action="store_true",
+                    help="the decode step split over the ranks by columns, with NCCL all-gathers (strong scaling)")
     ap.add_argument("--autotune", action="store_true",
                     help="per-shape rows also report dg_autotune's chosen variant and its time")
     ap.add_argument("--early-launch", type=int, default=-1,
@@ -752,6 +834,8 @@ def main():
         run_reference(args)
     elif args.shape:
         run_one_shape(args)
+    elif args.shard:
+        run_shard(args)
     else:
         run_dg(args)
 
