@@ -354,6 +354,8 @@ def run_one_shape(args):
 
     if args.max_split:
         dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, args.max_split)
+    if args.stream_k >= 0:
+        dg.dg_set_option(dg.DG_OPT_STREAM_K, args.stream_k)
     if args.early_launch >= 0:
         dg.dg_set_option(dg.DG_OPT_EARLY_LAUNCH, args.early_launch)
 
@@ -816,6 +818,7 @@ def main():
                     help="time only this per-shape workload (small, gemv, gemv_kt, thin, square_bf16, "
                          "square_e4m3, strided, square_bf16_gelu, thin_gelu, strided_nchw_out) and print its line")
     ap.add_argument("--max-split", type=int, default=0, help="with --shape: cap the tensor-core split-K")
+    ap.add_argument("--stream-k", type=int, default=-1, help="with --shape: 0 or 1 turns the Stream-K tail off or on")
     ap.add_argument("--trace", action="store_true", help="with --shape: phase timestamps of CTA 0")
     ap.add_argument("--cpu-baseline-worker", type=int, default=0, help=argparse.SUPPRESS)
     ap.add_argument("--shard", action="store_true",

@@ -16,8 +16,11 @@
  *    (cudaMalloc / torch CUDA tensors / managed memory) on the current device.
  *    The library keeps no pointer after a call returns.  It owns one
  *    4-byte device status word per device, allocated on the first call on
- *    that device; that first call should therefore come before any CUDA
- *    stream capture.
+ *    that device (that first call should therefore come before any CUDA
+ *    stream capture), and one Stream-K workspace per stream that runs a
+ *    Stream-K plan (see DG_OPT_STREAM_K; about 19 MB for a 4096^3 product),
+ *    allocated on that stream's first such call outside a capture; a call
+ *    captured on a stream that has none runs without Stream-K.
  *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *    default stream).  Calls are asynchronous on that stream.
  *  - Errors: argument errors are returned synchronously, before anything is
@@ -25,9 +28,10 @@
  *    dg_sync_status) is reported by dg_sync_status.
  *  - Thread safety: calls may be made from several host threads and their
  *    kernels may run concurrently on different streams: split-K partial
- *    sums stay in on-chip (cluster) shared memory, so calls share no scratch
- *    buffers.  dg_set_option is process-global and should not race with
- *    running calls.
+ *    sums stay in on-chip (cluster) shared memory, and Stream-K partials go
+ *    through the workspace of the call's own stream, so calls on different
+ *    streams share no scratch buffers.  dg_set_option is process-global and
+ *    should not race with running calls.
  */
 #ifndef DG_H_
 #define DG_H_
