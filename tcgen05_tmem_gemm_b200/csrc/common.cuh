@@ -20,15 +20,32 @@ namespace dg {
 struct SmemLimit {
     static constexpr int kDevices = 64;
     std::atomic<int> bytes[kDevices] = {};
+    std::atomic<int> carve[kDevices] = {};
     std::mutex mu;
 
+    // prefer_max_shared: also ask that an SM running this kernel keep its
+    // whole unified L1/shared memory as shared memory, so that blocks of a
+    // shared-memory-hungry kernel on another stream (two 104 KB blocks of
+    // the N-contiguous GEMV per SM) still fit beside it.  A kernel with a
+    // small footprint otherwise gets an L1-heavy split, and an SM configured
+    // that way takes no large blocks until it drains.
     template <typename Kern>
-    cudaError_t ensure(Kern kern, size_t need) {
-        if (need <= 48 * 1024) return cudaSuccess;  // the default limit
+    cudaError_t ensure(Kern kern, size_t need, bool prefer_max_shared = false) {
+        if (need <= 48 * 1024 && !prefer_max_shared) return cudaSuccess;  // the default limit
         int dev = 0;
         cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;
         if (dev < 0 || dev >= kDevices) return cudaErrorInvalidDevice;
+        if (prefer_max_shared && carve[dev].load(std::memory_order_acquire) == 0) {
+            std::lock_guard<std::mutex> lk(mu);
+            if (carve[dev].load(std::memory_order_relaxed) == 0) {
+                e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+                if (e != cudaSuccess) return e;
+                carve[dev].store(1, std::memory_order_release);
+            }
+        }
+        if (need <= 48 * 1024) return cudaSuccess;
         if (bytes[dev].load(std::memory_order_acquire) >= (int)need) return cudaSuccess;
         std::lock_guard<std::mutex> lk(mu);
         if (bytes[dev].load(std::memory_order_relaxed) >= (int)need) return cudaSuccess;

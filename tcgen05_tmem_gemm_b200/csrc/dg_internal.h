@@ -80,9 +80,21 @@ struct EpiParams {
     Axis ci_axis;            // C's i group, outermost dim first
 };
 
-// Byte offset of C's row i.
+// Byte offset of C's row i.  Every loop over the axis is unrolled with
+// constant indices, so the epilogue's copy of EpiParams stays in registers.
 __host__ __device__ inline int64_t epi_row_offset(const EpiParams &e, int64_t i) {
-    return e.ci_multi ? axis_offset(e.ci_axis, i) : i * e.ci;
+    if (!e.ci_multi) return i * e.ci;
+    int64_t off = 0;
+#pragma unroll
+    for (int d = kMaxDims - 1; d >= 0; --d) {
+        if (d < e.ci_axis.n) {
+            const int64_t s = e.ci_axis.size[d];
+            const int64_t q = i / s;
+            off += (i - q * s) * e.ci_axis.stride[d];
+            i = q;
+        }
+    }
+    return off;
 }
 
 struct UmmaParams {

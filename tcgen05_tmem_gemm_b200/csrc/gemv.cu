@@ -367,9 +367,9 @@ __global__ void __launch_bounds__(256) gemv_k_kernel(const GemvParams p) {
 // Raise a kernel's dynamic shared-memory limit once per device and size, not
 // per call (`Tag` gives each kernel instantiation its own record).
 template <typename Tag, typename K>
-cudaError_t ensure_smem(K kern, size_t smem) {
+cudaError_t ensure_smem(K kern, size_t smem, bool prefer_max_shared = false) {
     static SmemLimit limit;
-    return limit.ensure(kern, smem);
+    return limit.ensure(kern, smem, prefer_max_shared);
 }
 
 template <typename T, int R, int Kind>
@@ -402,7 +402,8 @@ cudaError_t run_k(const GemvParams &p, cudaStream_t s, int *grid_out) {
     const int grid = (p.N + 1) / 2;
     const size_t smem = sizeof(float) * ((size_t)R * p.K + 8 * R);
     auto kern = gemv_k_kernel<T, R>;
-    cudaError_t e = ensure_smem<KernelTag<T, R, 1>>(kern, smem);
+    // it often runs beside the N-contiguous GEMV (decode steps): keep SMs shared-memory heavy
+    cudaError_t e = ensure_smem<KernelTag<T, R, 1>>(kern, smem, true);
     if (e != cudaSuccess) return e;
     *grid_out = grid;
     return launch_ex(kern, dim3(grid), dim3(256), smem, s, dim3(1, 1, 1), p.pdl, p);

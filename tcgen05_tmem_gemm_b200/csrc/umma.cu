@@ -1022,7 +1022,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                                     if (q < S) a += ld_shared_f32(src[q] + off);
                             }
                             acc[b] = a;
-                            const int64_t ro = ci_multi ? axis_offset(e.ci_axis, ok ? i : 0) : (int64_t)i * ci;
+                            const int64_t ro = ci_multi ? epi_row_offset(e, ok ? i : 0) : (int64_t)i * ci;
                             cin[b] = (ok && beta != 0.f) ? load_elem(cbase + ro + (int64_t)j * cj, cdt) : 0.f;
                             // advance by 128 elements
                             if (along_i) {
@@ -1048,7 +1048,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                                 if (bias_j) val += bias_j[j];
                                 val = act_apply(act, val);
                             }
-                            const int64_t ro = ci_multi ? axis_offset(e.ci_axis, i) : (int64_t)i * ci;
+                            const int64_t ro = ci_multi ? epi_row_offset(e, i) : (int64_t)i * ci;
                             store_elem(cbase + ro + (int64_t)j * cj, cdt, val);
                         }
                     }

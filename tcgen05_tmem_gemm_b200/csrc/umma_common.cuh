@@ -12,6 +12,17 @@ namespace dg {
 // when C is contiguous along j and the chunk is whole, otherwise element
 // stores for any strides, with every C load of the chunk issued before the
 // first store.  The bias add and activation run only when the call has them.
+// The bias and activation of 16 whole columns jb.. of row i (after beta * C).
+__device__ __forceinline__ void fuse16(const EpiParams &e, float (&v)[16], int i, int jb) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        float z = v[c];
+        if (e.bias_i) z += e.bias_i[i];
+        if (e.bias_j) z += e.bias_j[jb + c];
+        v[c] = act_apply(e.act, z);
+    }
+}
+
 __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow, float asi, int i, int jb, int Nj,
                                                  const uint32_t (&r)[16]) {
     const bool fused = e.bias_i != nullptr || e.bias_j != nullptr || e.act != DG_ACT_NONE;
@@ -22,17 +33,6 @@ __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow,
             const float sj = e.scale_j ? e.scale_j[jb + c] : 1.f;
             v[c] = (asi * sj) * __uint_as_float(r[c]);
         }
-        // C is loaded first (beta != 0), so the fused step sees the whole sum
-        auto fuse = [&]() {
-            if (!fused) return;
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                float z = v[c];
-                if (e.bias_i) z += e.bias_i[i];
-                if (e.bias_j) z += e.bias_j[jb + c];
-                v[c] = act_apply(e.act, z);
-            }
-        };
         if (e.c_dtype == DG_F32) {
             float4 *dst = reinterpret_cast<float4 *>(crow + (int64_t)jb * 4);
             if (e.beta != 0.f) {
@@ -45,7 +45,7 @@ __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow,
                     v[4 * q + 3] = fmaf(e.beta, o.w, v[4 * q + 3]);
                 }
             }
-            fuse();
+            if (fused) fuse16(e, v, i, jb);  // C was loaded first: the whole sum
 #pragma unroll
             for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         } else {
@@ -70,7 +70,7 @@ __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow,
                     v[2 * q + 1] = fmaf(e.beta, hi, v[2 * q + 1]);
                 }
             }
-            fuse();
+            if (fused) fuse16(e, v, i, jb);  // C was loaded first: the whole sum
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 if (e.c_dtype == DG_BF16) {
@@ -109,27 +109,6 @@ __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow,
     }
 }
 
-// Partial accumulators another CTA left in global memory for this tile
-// (Stream-K): `src[q]` holds a 128-row x bn FP32 tile column by column
-// (element (row, col) at src[q][col * 128 + row]); the epilogue adds them to
-// the accumulator in q order before anything else.
-constexpr int kMaxFix = 8;
-struct Fixup {
-    const float *src[kMaxFix];
-    int n;
-};
-
-__device__ __forceinline__ void add_fixups(const Fixup *fx, int row, int col0, uint32_t *r, int ncols) {
-    if (fx == nullptr) return;
-#pragma unroll
-    for (int q = 0; q < kMaxFix; ++q) {
-        if (q >= fx->n) break;
-        const float *src = fx->src[q] + (int64_t)col0 * 128 + row;
-#pragma unroll 16
-        for (int c = 0; c < ncols; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) + src[c * 128]);
-    }
-}
-
 // Shared memory of the TMA-store epilogue: two blocks of 32 rows x 128 bytes
 // for each of the four epilogue warps.
 constexpr uint32_t kEpiBlockBytes = 32 * 128;
@@ -151,8 +130,7 @@ constexpr uint32_t kEpiStoreBytes = 4 * 2 * kEpiBlockBytes;
 template <int ES>
 __device__ __forceinline__ void epilogue_rows_tma(const EpiParams &e, const CUtensorMap *cmap, uint32_t stage,
                                                   uint32_t t_row, int i_base, int Mi, int j0, int bn, int Nj,
-                                                  int lane, uint32_t &nblk, int blk_first = 0, int blk_step = 1,
-                                                  const Fixup *fx = nullptr, int fx_row = 0) {
+                                                  int lane, uint32_t &nblk, int blk_first = 0, int blk_step = 1) {
     constexpr int W = 128 / ES;  // output columns per block
     if (i_base >= Mi) return;    // the whole warp is below C (warp-uniform)
     // parameters in registers: nothing below re-reads the parameter block
@@ -173,7 +151,6 @@ __device__ __forceinline__ void epilogue_rows_tma(const EpiParams &e, const CUte
         for (int q = 0; q < W / 16; ++q)
             tmem_ld16(t_row + (uint32_t)(c0 + 16 * q), *reinterpret_cast<uint32_t(*)[16]>(&r[16 * q]));
         tmem_ld_wait();
-        add_fixups(fx, fx_row, c0, r, W);
         float v[W];
         if (scale_j != nullptr) {  // per-column scales (FP8): read once per block, clamped at the edge
             const int jb = j0 + c0;

@@ -383,18 +383,20 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 continue;
             }
-            Fixup fx;
-            fx.n = 0;
             if (pw.role == kSkOwner) {
-                // ------------------------- Stream-K: wait for the other pairs' partials
+                // ------------------------- Stream-K: add the other pairs' partials into TMEM
+                // Wait (bounded) for each lower pair's flag of this warp's rows, then
+                // add its partial to the accumulator in place (tcgen05.ld, add,
+                // tcgen05.st), in pair order q = c-1, c-2, ...; the epilogue below
+                // then reads the finished sum like any other tile.
                 const int q0 = sk_first_contributor(p, cluster_id, nclusters, pw.sk_first);
                 const int64_t total = (int64_t)p.sk_tiles * p.kb_total;
-                for (int q = cluster_id - 1; q >= q0 && fx.n < kMaxFix; --q) {  // pair order: q = c-1, c-2, ...
-                    if (total * q / nclusters == total * (q + 1) / nclusters) continue;  // empty range
+                bool ok = true;
+                for (int q = cluster_id - 1; q >= q0 && ok; --q) {
+                    if (total * q / nclusters == total * (q + 1) / nclusters) continue;  // empty range: no partial
                     const uint32_t *flag = p.sk_flag + (q * 2 + (int)rank) * 4 + quarter;
                     if (ld_acquire_gpu(flag) != sk_tag) {
                         const uint64_t t0 = globaltimer_ns();
-                        bool ok = true;
                         while (ld_acquire_gpu(flag) != sk_tag) {
                             if (*abort_flag || globaltimer_ns() - t0 > p.timeout_ns) {
                                 ok = false;
@@ -407,20 +409,28 @@ __global__ void __launch_bounds__(192, 1)
                             break;
                         }
                     }
-                    fx.src[fx.n++] = sk_slot(p, q, rank);
+                    const float *src = sk_slot(p, q, rank) + row;
+                    for (int c0 = 0; c0 < pw.w; c0 += 16) {
+                        uint32_t r[16];
+                        __syncwarp();
+                        tmem_ld16(t_row + c0, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            r[c] = __float_as_uint(__uint_as_float(r[c]) + src[(c0 + c) * kHalfM]);
+                        tmem_st16(t_row + c0, r);
+                    }
+                    tmem_st_wait();
                 }
             }
-            const Fixup *fxp = fx.n > 0 ? &fx : nullptr;
             if (p.epi_tma) {
                 const uint32_t blocks = sbase + L.epi_off + (uint32_t)quarter * 2u * kEpiBlockBytes;
                 const int i_base = i - lane;
                 __syncwarp();
                 if (e.c_dtype == DG_F32)
-                    epilogue_rows_tma<4>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, pw.w, p.Nj, lane, nblk, 0, 1,
-                                         fxp, row);
+                    epilogue_rows_tma<4>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, pw.w, p.Nj, lane, nblk);
                 else
-                    epilogue_rows_tma<2>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, pw.w, p.Nj, lane, nblk, 0, 1,
-                                         fxp, row);
+                    epilogue_rows_tma<2>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, pw.w, p.Nj, lane, nblk);
             } else {
                 const bool row_ok = i < p.Mi;
                 const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
@@ -431,7 +441,6 @@ __global__ void __launch_bounds__(192, 1)
                     tmem_ld16(t_row + c0, r);
                     tmem_ld_wait();
                     if (!row_ok) continue;
-                    add_fixups(fxp, row, c0, r, 16);
                     epilogue_chunk16(e, crow, asi, i, j0 + c0, p.Nj, r);
                 }
             }
