@@ -296,9 +296,11 @@ typedef enum {
     DG_OPT_FORCE_KIND = 1,        /* 0 = automatic, else a dg_kind to use when it is
                                      applicable (DG_KIND_SIMT always is)              */
     DG_OPT_WAIT_TIMEOUT_MS = 2,   /* bound on every device-side wait (default 2000)   */
-    DG_OPT_TEST_STALL = 3,        /* 1: the tensor-core kernel's loader issues no
-                                     copies, so its waits run out and the call
-                                     reports DG_ERR_TIMEOUT (tests of the bound)      */
+    DG_OPT_TEST_STALL = 3,        /* tests of the bounds: 1 the tensor-core kernel's
+                                     loader issues no copies; 2 the split-K CTAs send
+                                     no partial slices to their owners.  Either way
+                                     waits run out and the call reports
+                                     DG_ERR_TIMEOUT                                     */
     DG_OPT_MAX_SPLIT_K = 4,       /* upper bound on the tensor-core kernel's split-K
                                      (default and cluster limit 8; 1 disables)         */
     DG_OPT_CTA_PAIR = 5,          /* paired-CTA (256-row) tensor-core tiles: 0 never,

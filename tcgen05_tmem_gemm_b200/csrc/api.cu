@@ -1292,7 +1292,8 @@ dg_status dg_set_option(int option, int64_t value) {
         g_timeout_ms.store(value);
         return DG_OK;
     case DG_OPT_TEST_STALL:
-        g_stall.store(value ? 1 : 0);
+        if (value < 0 || value > 2) return DG_ERR_VALUE;
+        g_stall.store((int)value);
         return DG_OK;
     case DG_OPT_TRACE:
         g_trace.store((uint64_t)value);

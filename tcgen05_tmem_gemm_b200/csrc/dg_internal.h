@@ -85,7 +85,9 @@ struct EpiParams {
 __host__ __device__ inline int64_t epi_row_offset(const EpiParams &e, int64_t i) {
     if (!e.ci_multi) return i * e.ci;
     int64_t off = 0;
+#if defined(__CUDA_ARCH__)
 #pragma unroll
+#endif
     for (int d = kMaxDims - 1; d >= 0; --d) {
         if (d < e.ci_axis.n) {
             const int64_t s = e.ci_axis.size[d];
@@ -131,7 +133,7 @@ struct UmmaParams {
     // control
     int *err_word;
     uint64_t timeout_ns;
-    int32_t stall_loader;
+    int32_t stall_loader;    // test hooks: 1 loaders issue nothing, 2 split-K sends no slices
     int32_t pdl;             // 0 off, 1 release dependents at start, 2 near the end
     uint64_t *trace;         // optional phase timestamps of CTA 0 (%globaltimer, ns)
 };

@@ -340,7 +340,7 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
     const GatherGeom g = gather_geom(p, VB, bk, es);
     const GatherSrc src = gather_src(p);
     const int stages = p.stages;
-    const bool stall = p.stall_loader != 0;
+    const bool stall = p.stall_loader == 1;
     const int nthreads = kGatherWarps * 32;
     const bool one_batch = VB < 4 && g.total <= nthreads * kGatherUnroll;  // register path look-ahead
     // a gather cluster splits every stage's copies among its CTAs (cp.async
@@ -508,7 +508,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             // and phase advance without division
             const int stages = p.stages, num_units = p.num_units, kb_total = p.kb_total;
             const int kb_per_split = p.kb_per_split, bn = p.bn;
-            const bool stall = p.stall_loader != 0, p_mn = p.p_mn_major != 0, q_mn = p.q_mn_major != 0;
+            const bool stall = p.stall_loader == 1, p_mn = p.p_mn_major != 0, q_mn = p.q_mn_major != 0;
             const uint32_t stage_bytes = L.stage_bytes, p_bytes = L.p_bytes;
             int it = 0, s = 0;  // global k-block counter across tiles, its stage
             uint32_t ph = 0;
@@ -556,7 +556,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             const int last = it;
             for (int d = 1; d <= p.stages && last - d >= 0; ++d) {
                 const int j = last - d;
-                if (p.stall_loader) break;
+                if (p.stall_loader == 1) break;
                 mbar_wait_drain(bar_full + 8 * (j % p.stages), (uint32_t)(j / p.stages) & 1u, p.timeout_ns);
             }
         }
@@ -850,7 +850,9 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             if (threadIdx.x == kEpiWarp0 * 32) trace_at(p, 57);
             fence_proxy_async_smem();  // the slices are read by the bulk copies
             asm volatile("bar.sync 2, 128;" ::: "memory");
-            if (threadIdx.x == kEpiWarp0 * 32 && !*abort_flag) {
+            // (test hook, stall mode 2: no slice is sent, so every owner's
+            // receive wait runs out and reports the timeout)
+            if (threadIdx.x == kEpiWarp0 * 32 && !*abort_flag && p.stall_loader != 2) {
                 trace_at(p, 58);
                 for (int q = 1; q < S; ++q) {
                     const uint32_t dr = (rank + (uint32_t)q) % (uint32_t)S;

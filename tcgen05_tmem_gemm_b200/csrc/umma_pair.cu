@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(192, 1)
             // (memory clobbers) would otherwise make it re-read the parameters,
             // and stage and phase advance without division
             const int stages = p.stages, kb_total = p.kb_total, num_units = p.num_units;
-            const bool stall = p.stall_loader != 0, p_mn = p.p_mn_major != 0, q_mn = p.q_mn_major != 0;
+            const bool stall = p.stall_loader == 1, p_mn = p.p_mn_major != 0, q_mn = p.q_mn_major != 0;
             const uint32_t stage_bytes = L.stage_bytes, a_bytes = L.a_bytes;
             (void)num_units;
             (void)kb_total;
@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(192, 1)
             if (!leader) pdl_release();
             // full[] of the even CTA counts both CTAs' bytes: once its last
             // phases complete, every copy of the pair has landed
-            if (leader && !p.stall_loader)
+            if (leader && p.stall_loader != 1)
                 for (int d = 1; d <= p.stages && it - d >= 0; ++d) {
                     const int j = it - d;
                     mbar_wait_drain(bar_full + 8 * (j % p.stages), (uint32_t)(j / p.stages) & 1u, p.timeout_ns);

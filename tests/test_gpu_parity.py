@@ -470,6 +470,24 @@ def test_bounded_wait_reports_timeout_and_recovers():
     check_full(W.cfg_small())
 
 
+def test_split_k_exchange_wait_reports_timeout_and_recovers():
+    # stall mode 2: the main loops run, but no CTA of a split-K cluster sends
+    # its slices, so every owner's wait for them runs out; the kernel records
+    # the timeout and every CTA still reaches the end of the kernel (no slice
+    # copy is in flight), and the next call is correct
+    p = W.cfg_thin(M=40, N=1000, K=784)
+    pl = expect_kind(p, "umma", swap_ab=1)
+    assert pl["split_k"] > 1
+    g = p.to("cuda")
+    dg.dg_set_option(dg.DG_OPT_WAIT_TIMEOUT_MS, 300)
+    dg.dg_set_option(dg.DG_OPT_TEST_STALL, 2)
+    A, B, C = dg_view_of(g.A), dg_view_of(g.B), dg_view_of(g.C)
+    assert dg.dg_gemm(A, B, C, g.alpha, g.beta) == dg.DG_OK
+    assert dg.dg_sync_status() == dg.DG_ERR_TIMEOUT
+    dg.dg_set_option(dg.DG_OPT_TEST_STALL, 0)
+    check_full(p)
+
+
 @pytest.mark.parametrize("mode", [0, 1, 2, 3])
 def test_early_launch_modes_back_to_back(mode):
     # Programmatic dependent launch lets a kernel start before the previous one
