@@ -288,6 +288,41 @@ dg_status dg_autotune(const dg_view *A, const dg_view *B, const dg_view *C,
 /* Forget every tuned variant (later calls plan by the rules again). */
 dg_status dg_tune_clear(void);
 
+/*
+ * dg_gemm_static — dg_gemm for callers that cannot let a library allocate
+ * device memory: work captured into a CUDA graph (an allocation there fails
+ * or ends the capture), frameworks whose own pool owns and accounts for every
+ * byte of device memory, and serving loops where an allocation's implicit
+ * device synchronisation is not allowed.  The paper has no counterpart; this
+ * is an interface for such callers.
+ *
+ * Same arguments and result as dg_gemm.  It calls no cudaMalloc, cudaFree or
+ * other allocating routine: the status word and the Stream-K workspace (the
+ * scratch memory of the CTA-pair kernel's Stream-K tail) live in one
+ * file-scope device array of 24 MiB, which the CUDA runtime places on every
+ * device that loads the library and which stays there until the process
+ * exits.  The caller still passes A, B, C and the scales.
+ *  - A problem whose Stream-K workspace would exceed the array (more than
+ *    about 24 MiB of FP32 partial tiles; a 4096^3 product on 148 SMs needs
+ *    19.4 MB) returns DG_ERR_UNSUPPORTED before anything is launched; with
+ *    DG_OPT_STREAM_K set to 0 such a problem runs without scratch.
+ *  - The first call on a device does a set-up: it looks up the array's
+ *    device address with the device current and clears the words that must
+ *    start at zero (the status word, the Stream-K sequence header and flags)
+ *    with cudaMemsetAsync on `stream`.  Make that first call before any stream
+ *    capture.
+ *  - Every call on a device shares the array, which keeps the last call's
+ *    contents (the Stream-K flags carry sequence tags, so a later call never
+ *    reads an earlier call's partials).  Calls whose kernels overlap on the
+ *    GPU (concurrent streams, host threads) race on it: serialise them.
+ *  - A device-side wait that gives up leaves C undefined and is recorded in
+ *    the array's status word, which dg_sync_status does not read.
+ */
+dg_status dg_gemm_static(const dg_view *A, const dg_view *B, const dg_view *C,
+                         float alpha, float beta,
+                         const float *scale_a, const float *scale_b,
+                         void *stream);
+
 /* Number of kernels this library has launched in this process. */
 uint64_t dg_launch_count(void);
 

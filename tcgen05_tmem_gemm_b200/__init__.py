@@ -127,6 +127,9 @@ def _load():
     L.dg_autotune.argtypes = [V, V, V, ctypes.c_float, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                               P(dg_epilogue), ctypes.c_void_p, ctypes.c_int, P(dg_tune_result)]
     L.dg_autotune.restype = ctypes.c_int
+    L.dg_gemm_static.argtypes = [V, V, V, ctypes.c_float, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                 ctypes.c_void_p]
+    L.dg_gemm_static.restype = ctypes.c_int
     L.dg_tune_clear.argtypes = []
     L.dg_tune_clear.restype = ctypes.c_int
     L.dg_launch_count.argtypes = []

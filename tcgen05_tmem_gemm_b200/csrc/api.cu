@@ -1203,6 +1203,112 @@ dg_status dg_autotune(const dg_view *A, const dg_view *B, const dg_view *C, floa
     return DG_OK;
 }
 
+}  // extern "C"
+
+// ------------------------------------------------ the allocation-free entry
+// Some callers cannot let a library call cudaMalloc: code running inside a
+// CUDA graph capture (an allocation there fails or would end the capture),
+// frameworks that own every byte of device memory through their own pool and
+// account for it, and real-time serving loops where an allocation's implicit
+// device synchronisation is not allowed.  dg_gemm allocates twice on first use
+// (the status word of the device, the Stream-K workspace of a stream); the
+// entry point below allocates nothing: both live in this file-scope array,
+// which the CUDA runtime places in device memory when it loads the library's
+// module on a device, and which stays there until the process exits.
+namespace dg {
+namespace {
+constexpr size_t kStaticScratchBytes = size_t(24) << 20;  // 24 MiB per device
+constexpr size_t kStaticStatusBytes = 256;                 // the status word, then the Stream-K workspace
+constexpr size_t kStaticZeroBytes = kStaticStatusBytes + kSkHeaderBytes + 8192;  // status, header, flags of 256 pairs
+}  // namespace
+}  // namespace dg
+
+static __device__ __align__(256) unsigned char g_static_scratch[dg::kStaticScratchBytes];
+
+namespace dg {
+namespace {
+struct StaticState {
+    bool ready = false;
+    void *scratch = nullptr;  // device address of g_static_scratch on this device
+    int num_sms = 0;
+};
+StaticState g_static[kMaxDevices];
+
+// Once per device, with the device current: the array's device address (in
+// host code its name is only a host-side stand-in), the SM count, the tensor
+// map encoder, and the words that must start at zero cleared on the stream.
+dg_status static_setup(int dev, cudaStream_t stream, StaticState **out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    StaticState &st = g_static[dev];
+    if (!st.ready) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) {
+            cudaGetLastError();
+            return DG_ERR_CUDA;
+        }
+        if (cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return DG_ERR_CUDA;
+        if (!g_encode) {
+            cudaDriverEntryPointQueryResult q;
+            void *fn = nullptr;
+            if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+                    cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || !fn)
+                return DG_ERR_CUDA;
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        if (cudaMemsetAsync(ptr, 0, kStaticZeroBytes, stream) != cudaSuccess) return DG_ERR_CUDA;
+        st.scratch = ptr;
+        st.ready = true;
+    }
+    *out = &st;
+    return DG_OK;
+}
+}  // namespace
+}  // namespace dg
+
+extern "C" {
+
+dg_status dg_gemm_static(const dg_view *A, const dg_view *B, const dg_view *C, float alpha, float beta,
+                         const float *scale_a, const float *scale_b, void *stream) {
+    if (!A || !B || !C) return DG_ERR_NULL;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Views v{A, B, C, {}, {}, {}};
+    Plan pl;
+    dg_status st = make_plan(v, alpha, beta, 148, &pl);
+    if (st != DG_OK) return st;
+    if (pl.info.kind == DG_KIND_NONE) return DG_OK;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DG_ERR_CUDA;
+    StaticState *ss = nullptr;
+    if ((st = static_setup(dev, s, &ss)) != DG_OK) return st;
+    if (ss->num_sms != 148 && (st = make_plan(v, alpha, beta, ss->num_sms, &pl)) != DG_OK) return st;
+    const dg_plan_info &in = pl.info;
+    const bool use_ab = in.kind != DG_KIND_SCALE_C;
+    if (use_ab && (!device_accessible(A->ptr) || !device_accessible(B->ptr))) return DG_ERR_POINTER;
+    if (!device_accessible(C->ptr)) return DG_ERR_POINTER;
+    if (use_ab && scale_a && !device_accessible(scale_a)) return DG_ERR_POINTER;
+    if (use_ab && scale_b && !device_accessible(scale_b)) return DG_ERR_POINTER;
+    char *scratch = static_cast<char *>(ss->scratch);
+    void *sk_ws = nullptr;
+    if (in.stream_k_tiles > 0) {
+        size_t flag_off = 0, part_off = 0;
+        const size_t need = sk_workspace_bytes(in.grid / 2, in.block_n, &flag_off, &part_off);
+        if (kStaticStatusBytes + need > kStaticScratchBytes || part_off > kStaticZeroBytes - kStaticStatusBytes)
+            return DG_ERR_UNSUPPORTED;  // the problem's Stream-K workspace does not fit the static array
+        sk_ws = scratch + kStaticStatusBytes;
+    }
+    DeviceState ds;  // no allocation: the status word is the array's first word
+    ds.ready = true;
+    ds.num_sms = ss->num_sms;
+    ds.err_word = reinterpret_cast<int *>(scratch);
+    LaunchRec rec;
+    st = prepare(v, pl, alpha, beta, use_ab ? scale_a : nullptr, use_ab ? scale_b : nullptr, nullptr, DG_ACT_NONE,
+                 &ds, sk_ws, &rec);
+    if (st != DG_OK) return st;
+    return fire(rec, s);
+}
+
 dg_status dg_tune_clear(void) {
     {
         std::lock_guard<std::mutex> lk(g_tune_mu);
