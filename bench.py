@@ -455,21 +455,24 @@ def run_dg(args):
     assert dg.dg_sync_status(stream) == dg.DG_OK
 
     def run_units(evs):
+        # the unit's x*W graph is submitted first, so the GPU starts on it at
+        # once while the host submits the x*K^T graph; the side stream waits
+        # only for the unit's start (the fork event), not for x*W
         launches = 0
         for u, n in enumerate(units):
             (gw, nw), (gk, nk) = graphs[n]
             fork = torch.cuda.Event()
             join = torch.cuda.Event()
             fork.record(stream)
-            side.wait_event(fork)
-            with torch.cuda.stream(side):
-                gk.replay()
-            join.record(side)
             if evs is not None:
                 evs[u][0].record(stream)
             gw.replay()
             if evs is not None:
                 evs[u][1].record(stream)
+            side.wait_event(fork)
+            with torch.cuda.stream(side):
+                gk.replay()
+            join.record(side)
             stream.wait_event(join)
             launches += nw + nk
         return launches

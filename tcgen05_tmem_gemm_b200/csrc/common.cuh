@@ -125,23 +125,34 @@ __host__ __device__ __forceinline__ int elem_bytes(int dtype) {
     return dtype == DG_F32 ? 4 : dtype == DG_E4M3 ? 1 : 2;
 }
 
+// The hardware's tanh approximation (one instruction; the PTX ISA gives its
+// largest relative error as about 2^-11).
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // The fused activation ("DeepGEMM is not a new model: the inner discipline of
-// GPU matrix multiplication", §3.3: GeLU in its tanh form after the bias add).
-// ReLU keeps NaN; GeLU is z/2 (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))) with
-// the accurate tanhf, so FP32 outputs keep FP32 accuracy.
-__device__ __forceinline__ float act_apply(int act, float z) {
+// GPU matrix multiplication", §3.3: GeLU in its tanh form after the bias add,
+// with a fast tanh).  ReLU keeps NaN; GeLU is
+// z/2 (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))).  For a 16-bit output
+// (`fast`) the tanh is the hardware approximation, whose error (2^-11 of the
+// tanh) stays below the output's own rounding (2^-9 for BF16, 2^-11 for FP16);
+// an FP32 output takes the accurate tanhf, so it keeps FP32 accuracy.
+__device__ __forceinline__ float act_apply(int act, float z, bool fast = false) {
     if (act == DG_ACT_RELU) return z < 0.f ? 0.f : z;
     if (act == DG_ACT_GELU_TANH) {
         const float u = 0.7978845608028654f * fmaf(0.044715f * z, z * z, z);  // sqrt(2/pi) (z + 0.044715 z^3)
-        return 0.5f * z * (1.f + tanhf(u));
+        return 0.5f * z * (1.f + (fast ? tanh_approx(u) : tanhf(u)));
     }
     return z;
 }
 
 // The bias add and activation of the epilogue, for an epilogue that has them.
-__device__ __forceinline__ float epi_fuse(float z, const float *bias, int64_t idx, int act) {
+__device__ __forceinline__ float epi_fuse(float z, const float *bias, int64_t idx, int act, bool fast) {
     if (bias != nullptr) z += bias[idx];
-    return act_apply(act, z);
+    return act_apply(act, z, fast);
 }
 
 // out = act(alpha * s_i * s_j * acc + beta * c_in + bias)   (c_in read only when beta != 0)

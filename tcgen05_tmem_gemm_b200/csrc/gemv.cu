@@ -108,7 +108,8 @@ __device__ __forceinline__ void store_out(const EpiParams &e, int r, int n, floa
     const float asi = e.alpha * (e.scale_i ? e.scale_i[r] : 1.f);
     const float sj = e.scale_j ? e.scale_j[n] : 1.f;
     float v = epi_value(acc, asi, sj, e.beta, cp, e.c_dtype);
-    if (e.bias_j != nullptr || e.act != DG_ACT_NONE) v = epi_fuse(v, e.bias_j, n, e.act);  // bias per column n
+    if (e.bias_j != nullptr || e.act != DG_ACT_NONE)
+        v = epi_fuse(v, e.bias_j, n, e.act, e.c_dtype != DG_F32);  // bias per column n
     store_elem(cp, e.c_dtype, v);
 }
 

@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtParams p) {
             const float sj = e.scale_j ? e.scale_j[n] : 1.f;
             float v = (asi * sj) * acc[i][j];
             if (e.beta != 0.f) v = fmaf(e.beta, cin[j], v);
-            if (e.bias_j != nullptr || e.act != DG_ACT_NONE) v = epi_fuse(v, e.bias_j, n, e.act);
+            if (e.bias_j != nullptr || e.act != DG_ACT_NONE) v = epi_fuse(v, e.bias_j, n, e.act, p.c.dtype != DG_F32);
             store_elem(cp[j], p.c.dtype, v);
         }
     }
@@ -103,7 +103,7 @@ __global__ void scale_c_kernel(const DevView c, int64_t M, int64_t N, float beta
         const int64_t m = e / N, n = e - (e / N) * N;
         char *cp = const_cast<char *>(c.ptr) + axis_offset(c.row, m) + axis_offset(c.col, n);
         float v = beta != 0.f ? beta * load_elem(cp, c.dtype) : 0.f;
-        if (fused) v = epi_fuse(v, bias, n, act);
+        if (fused) v = epi_fuse(v, bias, n, act, c.dtype != DG_F32);
         store_elem(cp, c.dtype, v);
     }
 }

@@ -970,7 +970,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                                 if (fused) {
                                     if (bias_i && i + k < Mi) o[k] += bias_i[i + k];
                                     if (bias_j) o[k] += bias_j[j];
-                                    o[k] = act_apply(act, o[k]);
+                                    o[k] = act_apply(act, o[k], cdt != DG_F32);
                                 }
                             }
                             char *dstc = cbase + (int64_t)i * 4 + (int64_t)j * cj;
@@ -992,7 +992,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                                     if (fused) {
                                         if (bias_i) val += bias_i[i + k];
                                         if (bias_j) val += bias_j[j];
-                                        val = act_apply(act, val);
+                                        val = act_apply(act, val, cdt != DG_F32);
                                     }
                                     store_elem(dstc + k * 4, cdt, val);
                                 }
@@ -1048,7 +1048,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                             if (fused) {
                                 if (bias_i) val += bias_i[i];
                                 if (bias_j) val += bias_j[j];
-                                val = act_apply(act, val);
+                                val = act_apply(act, val, cdt != DG_F32);
                             }
                             const int64_t ro = ci_multi ? epi_row_offset(e, i) : (int64_t)i * ci;
                             store_elem(cbase + ro + (int64_t)j * cj, cdt, val);

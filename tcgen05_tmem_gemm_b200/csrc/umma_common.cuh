@@ -19,7 +19,7 @@ __device__ __forceinline__ void fuse16(const EpiParams &e, float (&v)[16], int i
         float z = v[c];
         if (e.bias_i) z += e.bias_i[i];
         if (e.bias_j) z += e.bias_j[jb + c];
-        v[c] = act_apply(e.act, z);
+        v[c] = act_apply(e.act, z, e.c_dtype != DG_F32);
     }
 }
 
@@ -101,7 +101,7 @@ __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow,
                 if (fused) {
                     if (e.bias_i) val += e.bias_i[i];
                     if (e.bias_j) val += e.bias_j[j];
-                    val = act_apply(e.act, val);
+                    val = act_apply(e.act, val, e.c_dtype != DG_F32);
                 }
                 store_elem(crow + (int64_t)j * e.cj, e.c_dtype, val);
             }
@@ -170,7 +170,7 @@ __device__ __forceinline__ void epilogue_rows_tma(const EpiParams &e, const CUte
                 float z = v[c];
                 if (has_bi) z += bi;
                 if (bias_j) z += bias_j[jb + c < Nj ? jb + c : Nj - 1];
-                v[c] = act_apply(act, z);
+                v[c] = act_apply(act, z, ES == 2);  // 16-bit output: the hardware tanh
             }
         }
         uint32_t w[32];

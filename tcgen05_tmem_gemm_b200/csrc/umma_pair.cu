@@ -163,7 +163,9 @@ __device__ __forceinline__ int sk_first_contributor(const UmmaParams &p, int c, 
     return q;
 }
 
-// This CTA's slot of pair q: 128 rows x bn FP32, column by column.
+// This CTA's slot of pair q: 128 rows x bn FP32 in groups of four columns,
+// element (row, col) at [(col / 4) * 128 + row] * 4 + col % 4, so that a
+// warp's 16-byte stores and loads of one column group are 512 contiguous bytes.
 __device__ __forceinline__ float *sk_slot(const UmmaParams &p, int q, uint32_t rank) {
     return p.sk_part + (size_t)(q * 2 + (int)rank) * (size_t)(kHalfM * p.bn);
 }
@@ -365,14 +367,17 @@ __global__ void __launch_bounds__(192, 1)
             const int j0 = pw.j0;
             if (pw.role == kSkPartial) {
                 // ------------------------- Stream-K: leave the partial for the tile's owner
-                float *slot = sk_slot(p, cluster_id, rank) + row;
+                float4 *slot = reinterpret_cast<float4 *>(sk_slot(p, cluster_id, rank)) + row;
                 for (int c0 = 0; c0 < pw.w; c0 += 16) {
                     uint32_t r[16];
                     __syncwarp();
                     tmem_ld16(t_row + c0, r);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) slot[(c0 + c) * kHalfM] = __uint_as_float(r[c]);  // coalesced
+                    for (int g = 0; g < 4; ++g)  // column group (c0 + 4g) / 4
+                        slot[((c0 >> 2) + g) * kHalfM] =
+                            make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
+                                        __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
                 }
                 tc_fence_before();
                 __syncwarp();  // orders the warp's stores before lane 0's release below
@@ -409,16 +414,29 @@ __global__ void __launch_bounds__(192, 1)
                             break;
                         }
                     }
-                    const float *src = sk_slot(p, q, rank) + row;
-                    for (int c0 = 0; c0 < pw.w; c0 += 16) {
-                        uint32_t r[16];
-                        __syncwarp();
-                        tmem_ld16(t_row + c0, r);
-                        tmem_ld_wait();
+                    // 64 columns at a time: their 16 loads are in flight together, so the
+                    // partial costs a few round trips to L2, not one per 16 columns
+                    const float4 *src = reinterpret_cast<const float4 *>(sk_slot(p, q, rank)) + row;
+                    for (int c0 = 0; c0 < pw.w; c0 += 64) {
+                        float4 pv[16];
 #pragma unroll
-                        for (int c = 0; c < 16; ++c)
-                            r[c] = __float_as_uint(__uint_as_float(r[c]) + src[(c0 + c) * kHalfM]);
-                        tmem_st16(t_row + c0, r);
+                        for (int g = 0; g < 16; ++g) pv[g] = src[((c0 >> 2) + g) * kHalfM];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            uint32_t r[16];
+                            __syncwarp();
+                            tmem_ld16(t_row + c0 + 16 * k, r);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int g = 0; g < 4; ++g) {
+                                const float4 a = pv[4 * k + g];
+                                r[4 * g] = __float_as_uint(__uint_as_float(r[4 * g]) + a.x);
+                                r[4 * g + 1] = __float_as_uint(__uint_as_float(r[4 * g + 1]) + a.y);
+                                r[4 * g + 2] = __float_as_uint(__uint_as_float(r[4 * g + 2]) + a.z);
+                                r[4 * g + 3] = __float_as_uint(__uint_as_float(r[4 * g + 3]) + a.w);
+                            }
+                            tmem_st16(t_row + c0 + 16 * k, r);
+                        }
                     }
                     tmem_st_wait();
                 }

@@ -17,9 +17,10 @@ sqrt(K) times larger for random data).
 With the fused epilogue out = act(z), z = alpha*s*acc + beta*c + bias, the
 FP32 error of z is 5e-4 * S + 2^-22 * (|z| + |beta c| + |bias|); the
 activation passes it on multiplied by at most its largest slope (1 for ReLU,
-1.129 for GeLU in its tanh form) and GeLU's FP32 evaluation adds at most
-2^-20 |z| (tanh near -1 loses the low bits of 1 + tanh); 16-bit outputs then
-add their rounding relative to the result as above.
+1.129 for GeLU in its tanh form) and GeLU's evaluation adds at most 2^-20 |z|
+for FP32 outputs (accurate tanh; near -1, 1 + tanh loses low bits) or 2^-11 |z|
+for 16-bit outputs (the hardware tanh approximation); 16-bit outputs then add
+their rounding relative to the result as above.
 NaN positions must agree exactly; infinities must agree in sign and place.
 """
 from __future__ import annotations
@@ -97,7 +98,10 @@ def tolerance(out_dtype: str, ref, bound, beta_c, pre=None, bias_abs=None, act="
     b = bias_abs if bias_abs is not None else 0.0
     tz = ACT_SLOPE[act] * (5e-4 * bound + 2.0 ** -22 * (z + np.abs(beta_c) + b))
     if act == "gelu_tanh":
-        tz = tz + 2.0 ** -20 * z
+        # FP32 outputs evaluate tanh accurately; 16-bit outputs with the
+        # hardware approximation (relative error about 2^-11 of the tanh, so at
+        # most 2^-12 |z| in the output), below their own rounding
+        tz = tz + (2.0 ** -20 if out_dtype == "f32" else 2.0 ** -11) * z
     if out_dtype == "f32":
         return tz
     if out_dtype == "bf16":
