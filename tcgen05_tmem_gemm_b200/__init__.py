@@ -33,7 +33,7 @@ ACT = {"none": DG_ACT_NONE, "relu": DG_ACT_RELU, "gelu_tanh": DG_ACT_GELU_TANH}
 
 (DG_OPT_FORCE_KIND, DG_OPT_WAIT_TIMEOUT_MS, DG_OPT_TEST_STALL, DG_OPT_MAX_SPLIT_K, DG_OPT_CTA_PAIR,
  DG_OPT_EARLY_LAUNCH, DG_OPT_TRACE, DG_OPT_EPI_TMA, DG_OPT_GATHER_CLUSTER,
- DG_OPT_PAIR_TAIL, DG_OPT_STREAM_K) = 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11
+ DG_OPT_PAIR_TAIL, DG_OPT_STREAM_K, DG_OPT_DETERMINISTIC) = 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12
 
 
 class dg_view(ctypes.Structure):
@@ -78,7 +78,7 @@ class dg_plan_info(ctypes.Structure):
         ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
         ("cta_pair", ctypes.c_int32), ("epi_tma_store", ctypes.c_int32),
         ("gather_cluster", ctypes.c_int32), ("pair_half_tiles", ctypes.c_int32),
-        ("stream_k_tiles", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("stream_k_tiles", ctypes.c_int32), ("split_reduce_add", ctypes.c_int32),
     ]
 
     def as_dict(self) -> dict:

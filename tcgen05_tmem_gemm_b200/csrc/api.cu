@@ -38,7 +38,8 @@ std::atomic<uint64_t> g_trace{0};
 std::atomic<int> g_epi_tma{1};
 std::atomic<int> g_gather_cluster{1};
 std::atomic<int> g_pair_tail{1};
-std::atomic<int> g_stream_k{1};
+std::atomic<int> g_stream_k{0};
+std::atomic<int> g_deterministic{0};
 std::atomic<uint32_t> g_epoch{1};  // bumped by every option change: cached launches go stale
 
 constexpr int kMaxDevices = 64;
@@ -492,6 +493,10 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     in.epi_tma_store = epi_tma && split == 1;
     in.gather_cluster = gcl;
     if (gcl > 1) in.grid = (int32_t)std::min<int64_t>(units2, (num_sms / gcl) * gcl);
+    // split-K with beta == 1 and FP32 C: the splits can add their partials
+    // straight into C through one 2-D tensor map of C (its i group one dim)
+    if (split > 1 && beta == 1.f && v.C->dtype == DG_F32 && v.c.tma_ok && g_deterministic.load() == 0)
+        in.split_reduce_add = 1;
     if (pair) {
         const int64_t pair_units = ((Mi + 255) / 256) * tiles_j;
         in.block_m = 256;
@@ -886,6 +891,17 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         while (tc < 2 * bn) tc *= 2;
         p.tmem_cols = tc;
         p.epi = epi_params(v, swap, alpha, beta, sa, sb, bias, act);
+        if (in.split_reduce_add && act == DG_ACT_NONE) {
+            // C as a 2-D FP32 map along its unit-stride dim, 32 x 32 boxes: i is
+            // unit-stride when C's rows are (no swap) or its columns are (swap)
+            const bool inner_i = swap ? v.c.unit_dim == 1 : v.c.unit_dim == 2;
+            const Axis &ia = swap ? v.c.col : v.c.row, &ja = swap ? v.c.row : v.c.col;
+            const bool ok = inner_i ? encode_2d_box(&rec->t2, DG_F32, v.C->ptr, Mi, Nj, axis_stride(ja), 32, 32, false)
+                                    : encode_2d_box(&rec->t2, DG_F32, v.C->ptr, Nj, Mi, axis_stride(ia), 32, 32, true);
+            if (!ok) return DG_ERR_UNSUPPORTED;
+            p.red_add = 1;
+            p.red_inner_i = inner_i;
+        }
         if (in.p_gather) {
             DevView d{};
             d.ptr = static_cast<const char *>(Pv->ptr);
@@ -1431,6 +1447,10 @@ dg_status dg_set_option(int option, int64_t value) {
     case DG_OPT_STREAM_K:
         if (value < 0 || value > 1) return DG_ERR_VALUE;
         g_stream_k.store((int)value);
+        return DG_OK;
+    case DG_OPT_DETERMINISTIC:
+        if (value < 0 || value > 1) return DG_ERR_VALUE;
+        g_deterministic.store((int)value);
         return DG_OK;
     default: return DG_ERR_VALUE;
     }

@@ -121,6 +121,12 @@ struct UmmaParams {
     // instruction descriptor idesc_half
     int32_t full_units;
     uint32_t idesc_half;
+    // split-K with beta = 1 and FP32 C: every split adds its scaled partial
+    // straight into C with tensor reduce-adds (third map: C, 32 x 32 FP32
+    // boxes), instead of the cluster exchange; red_inner_i: C is unit-stride
+    // along i (the map's inner dim is i), else along j
+    int32_t red_add;
+    int32_t red_inner_i;
     // Stream-K (CTA pairs): the first dp_tiles tiles run whole, one pair
     // each; the last sk_tiles tiles form one run of k blocks shared out evenly
     // over all pairs.  A tile's owner (the pair holding its last k blocks)

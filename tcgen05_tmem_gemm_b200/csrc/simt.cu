@@ -73,21 +73,21 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtParams p) {
         const float asi = e.alpha * (e.scale_i ? e.scale_i[m] : 1.f);
         const int64_t cro = axis_offset(p.c.row, m);
         char *cp[4];
-        float cin[4];
+        float cin[4], sj[4], bj[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 4; ++j) {  // every load before the first store
             const int n = n0 + tx * 4 + j;
             cp[j] = n < p.N ? const_cast<char *>(p.c.ptr) + cro + axis_offset(p.c.col, n) : nullptr;
             cin[j] = (cp[j] && e.beta != 0.f) ? load_elem(cp[j], p.c.dtype) : 0.f;
+            sj[j] = (cp[j] && e.scale_j) ? e.scale_j[n] : 1.f;
+            bj[j] = (cp[j] && e.bias_j) ? e.bias_j[n] : 0.f;
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             if (!cp[j]) continue;
-            const int n = n0 + tx * 4 + j;
-            const float sj = e.scale_j ? e.scale_j[n] : 1.f;
-            float v = (asi * sj) * acc[i][j];
+            float v = (asi * sj[j]) * acc[i][j];
             if (e.beta != 0.f) v = fmaf(e.beta, cin[j], v);
-            if (e.bias_j != nullptr || e.act != DG_ACT_NONE) v = epi_fuse(v, e.bias_j, n, e.act, p.c.dtype != DG_F32);
+            if (e.bias_j != nullptr || e.act != DG_ACT_NONE) v = act_apply(e.act, v + bj[j], p.c.dtype != DG_F32);
             store_elem(cp[j], p.c.dtype, v);
         }
     }

@@ -145,6 +145,18 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, uint32_t src,
                  : "memory");
 }
 
+// 2-D tiled reduce-add of a shared-memory box into global memory at (c0 =
+// innermost, c1): each element of the box is added to the tensor's element
+// by the memory system (FP32 adds for an FP32 map); elements outside the
+// tensor are skipped.  Completion is tracked with bulk groups like
+// tma_store_2d.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *m, uint32_t src, int32_t c0, int32_t c1) {
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(m)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 template <int N>

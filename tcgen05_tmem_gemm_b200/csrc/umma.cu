@@ -419,7 +419,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         // descriptor fetches start at once, while thread 0 sets up the barriers
         tma_prefetch_desc(&tmap_q);
         if (!GATHER) tma_prefetch_desc(&tmap_p);
-        if (p.epi_tma) tma_prefetch_desc(&tmap_c);
+        if (p.epi_tma || p.red_add) tma_prefetch_desc(&tmap_c);
     }
     pdl_wait();
     if (p.pdl == 1) pdl_release();
@@ -673,7 +673,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         const EpiParams e = p.epi;  // a local copy: its fields stay in registers
         int local = 0;
         uint32_t nblk = 0;  // tensor-store blocks this warp has issued
-        if (p.split_k > 1 && e.beta != 0.f && !e.ci_multi) {
+        if (p.split_k > 1 && !p.red_add && e.beta != 0.f && !e.ci_multi) {
             // the rows this CTA will reduce: pull their C lines into L2 while
             // the main loops run
             const TileCoord tc = unit_coord(blockIdx.x, p);
@@ -796,7 +796,77 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         }
     }
 
-    if (p.split_k > 1) {
+    if (p.split_k > 1 && p.red_add) {
+        // ------------------------------------- split-K partials added into C
+        // beta = 1 and FP32 C: C += alpha * s_i * s_j * partial (+ bias, by the
+        // first split only) is linear in the splits, so each CTA adds its own
+        // scaled partial into C with tensor reduce-adds, which the memory
+        // system applies element by element.  No slices travel between the
+        // CTAs and no CTA waits for another; the order of the adds, and so the
+        // last bits of C, can vary from run to run.  The blocks are staged in
+        // the idle operand ring: 32 x 32 FP32, laid out along C's unit-stride
+        // dim (i: rows of 32 i, no swizzle; j: rows of 32 j, 128-byte swizzle).
+        __syncwarp();
+        if (!cluster_ready) {
+            cluster_wait();  // the start-up barrier every thread arrived on
+            cluster_ready = true;
+        }
+        if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4 && !*abort_flag) {
+            tc_fence_after();
+            const int quarter = warp & 3;
+            const EpiParams e = p.epi;  // a local copy: its fields stay in registers
+            const TileCoord tc = unit_coord(blockIdx.x, p);
+            const int i_base = tc.ti * kBM + quarter * 32, i = i_base + lane;
+            const int j0 = tc.tj * p.bn, Nj = p.Nj;
+            const bool row_ok = i < p.Mi;
+            const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
+            const bool first = tc.split == 0;  // the bias enters C once
+            const float *const bias_j = first ? e.bias_j : nullptr;
+            const float bi = (first && e.bias_i && row_ok) ? e.bias_i[i] : 0.f;
+            const float *const scale_j = e.scale_j;
+            const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16);
+            const uint32_t blocks = sbase + (uint32_t)quarter * 2u * kEpiBlockBytes;
+            const bool inner_i = p.red_inner_i != 0;
+            uint32_t nblk = 0;
+            for (int c0 = 0; c0 < p.bn && j0 + c0 < Nj; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld16(t_row + (uint32_t)c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                tmem_ld16(t_row + (uint32_t)(c0 + 16), *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+                tmem_ld_wait();
+                float v[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const int j = min(j0 + c0 + c, Nj - 1);  // columns past C are clipped by the copy
+                    float x = (asi * (scale_j ? scale_j[j] : 1.f)) * __uint_as_float(r[c]);
+                    if (bias_j) x += bias_j[j];
+                    v[c] = x + bi;
+                }
+                const uint32_t buf = blocks + (nblk & 1u) * kEpiBlockBytes;
+                if (lane == 0) bulk_wait_read<1>();  // the copy that last read this block is done with it
+                __syncwarp();
+                if (inner_i) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) st_shared_f32(buf + (uint32_t)c * 128u + (uint32_t)lane * 4u, v[c]);
+                } else {
+                    const uint32_t rowa = buf + (uint32_t)lane * 128u;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        st_shared_v4(rowa + ((uint32_t)(u ^ (lane & 7)) << 4), __float_as_uint(v[4 * u]),
+                                     __float_as_uint(v[4 * u + 1]), __float_as_uint(v[4 * u + 2]),
+                                     __float_as_uint(v[4 * u + 3]));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if (inner_i) tma_reduce_add_2d(&tmap_c, buf, i_base, j0 + c0);
+                    else tma_reduce_add_2d(&tmap_c, buf, j0 + c0, i_base);
+                    bulk_commit();
+                }
+                ++nblk;
+            }
+            if (lane == 0) bulk_wait_all();  // every add has reached C before the CTA ends
+        }
+    } else if (p.split_k > 1) {
         // ------------------------------------------ cluster reduction of k splits
         // CTA s of the cluster owns rows [128 s / S, 128 (s+1) / S) of the
         // tile.  Once its own main loop is done (its ring is then idle), each
@@ -1006,10 +1076,10 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                     const int total = rs * bn;
                     int r = along_i ? t % rs : t / bn, c = along_i ? t / rs : t % bn;
                     const int dr = along_i ? 128 % rs : 128 / bn, dc = along_i ? 128 / rs : 128 % bn;
-                    constexpr int kB = 8;  // outputs per thread per batch: their C loads are in flight together
+                    constexpr int kB = 8;  // outputs per thread per batch: their loads are in flight together
                     for (int base = t; base < total; base += 128 * kB) {
                         int ii[kB], jj[kB];
-                        float acc[kB], cin[kB];
+                        float acc[kB], cin[kB], sc[kB], bs[kB];
 #pragma unroll
                         for (int b = 0; b < kB; ++b) {
                             const int i = i0 + r, j = jt + c;
@@ -1026,6 +1096,9 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                             acc[b] = a;
                             const int64_t ro = ci_multi ? epi_row_offset(e, ok ? i : 0) : (int64_t)i * ci;
                             cin[b] = (ok && beta != 0.f) ? load_elem(cbase + ro + (int64_t)j * cj, cdt) : 0.f;
+                            // scales and bias loaded with the batch, before any store
+                            sc[b] = ok ? alpha * (scale_i ? scale_i[i] : 1.f) * (scale_j ? scale_j[j] : 1.f) : 0.f;
+                            bs[b] = ok ? (bias_i ? bias_i[i] : 0.f) + (bias_j ? bias_j[j] : 0.f) : 0.f;
                             // advance by 128 elements
                             if (along_i) {
                                 r += dr;
@@ -1041,13 +1114,10 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                         for (int b = 0; b < kB; ++b) {
                             if (ii[b] < 0) continue;
                             const int i = ii[b], j = jj[b];
-                            const float asi = alpha * (scale_i ? scale_i[i] : 1.f);
-                            const float sj = scale_j ? scale_j[j] : 1.f;
-                            float val = (asi * sj) * acc[b];
+                            float val = sc[b] * acc[b];
                             if (beta != 0.f) val = fmaf(beta, cin[b], val);
                             if (fused) {
-                                if (bias_i) val += bias_i[i];
-                                if (bias_j) val += bias_j[j];
+                                if (bias_i || bias_j) val += bs[b];
                                 val = act_apply(act, val, cdt != DG_F32);
                             }
                             const int64_t ro = ci_multi ? epi_row_offset(e, i) : (int64_t)i * ci;

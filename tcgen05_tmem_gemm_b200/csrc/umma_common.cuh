@@ -85,22 +85,29 @@ __device__ __forceinline__ void epilogue_chunk16(const EpiParams &e, char *crow,
             dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
         }
     } else {
-        float cin[16];
+        // Every load of the chunk (C, column scales, bias) is issued before
+        // the first store: the stores go through a plain pointer the compiler
+        // cannot tell apart from the scale and bias arrays, so a load placed
+        // after a store would wait for it, one element at a time.
+        float cin[16], sjv[16], bjv[16];
+        const float bi = e.bias_i ? e.bias_i[i] : 0.f;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
             const int j = jb + c;
-            cin[c] = (e.beta != 0.f && j < Nj) ? load_elem(crow + (int64_t)j * e.cj, e.c_dtype) : 0.f;
+            const bool ok = j < Nj;
+            cin[c] = (e.beta != 0.f && ok) ? load_elem(crow + (int64_t)j * e.cj, e.c_dtype) : 0.f;
+            sjv[c] = (e.scale_j && ok) ? e.scale_j[j] : 1.f;
+            bjv[c] = (e.bias_j && ok) ? e.bias_j[j] : 0.f;
         }
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
             const int j = jb + c;
             if (j < Nj) {
-                const float sj = e.scale_j ? e.scale_j[j] : 1.f;
-                float val = (asi * sj) * __uint_as_float(r[c]);
+                float val = (asi * sjv[c]) * __uint_as_float(r[c]);
                 if (e.beta != 0.f) val = fmaf(e.beta, cin[c], val);
                 if (fused) {
-                    if (e.bias_i) val += e.bias_i[i];
-                    if (e.bias_j) val += e.bias_j[j];
+                    if (e.bias_i) val += bi;
+                    if (e.bias_j) val += bjv[c];
                     val = act_apply(e.act, val, e.c_dtype != DG_F32);
                 }
                 store_elem(crow + (int64_t)j * e.cj, e.c_dtype, val);

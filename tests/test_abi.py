@@ -149,18 +149,32 @@ def test_plan_square_bf16_and_fp8():
     assert pl["kind_name"] == "umma" and pl["block_k"] == 128 and pl["q_mn_major"] == 1
 
 
+def test_plan_thin_split_reduce_add():
+    # beta = 1 with FP32 C: the k splits add into C unless deterministic
+    p = meta_problem("thin")
+    pl = dg.dg_plan(*views(p), 1.0, 1.0, False, 148).as_dict()
+    assert pl["split_k"] == 4 and pl["split_reduce_add"] == 1
+    assert dg.dg_plan(*views(p), 1.0, 0.5, False, 148).as_dict()["split_reduce_add"] == 0
+    dg.dg_set_option(dg.DG_OPT_DETERMINISTIC, 1)
+    try:
+        assert dg.dg_plan(*views(p), 1.0, 1.0, False, 148).as_dict()["split_reduce_add"] == 0
+    finally:
+        dg.dg_set_option(dg.DG_OPT_DETERMINISTIC, 0)
+
+
 def test_plan_square_stream_k_tail():
-    # 256 tiles of 256 x 256 on 74 CTA pairs: 222 whole, the last 34 shared
-    # out along k over every pair (Stream-K); without it, half-width tail tiles
+    # 256 tiles of 256 x 256 on 74 CTA pairs: 222 whole, the last 34 as
+    # half-width tiles (the default), or shared out along k over every pair
+    # (Stream-K, opt-in)
     p = meta_problem("square_bf16")
     pl = dg.dg_plan(*views(p), 1.0, 0.0, False, 148).as_dict()
-    assert pl["cta_pair"] == 1 and pl["stream_k_tiles"] == 34 and pl["pair_half_tiles"] == 0
-    dg.dg_set_option(dg.DG_OPT_STREAM_K, 0)
+    assert pl["cta_pair"] == 1 and pl["stream_k_tiles"] == 0 and pl["pair_half_tiles"] == 34
+    dg.dg_set_option(dg.DG_OPT_STREAM_K, 1)
     try:
         pl = dg.dg_plan(*views(p), 1.0, 0.0, False, 148).as_dict()
-        assert pl["stream_k_tiles"] == 0 and pl["pair_half_tiles"] == 34
+        assert pl["stream_k_tiles"] == 34 and pl["pair_half_tiles"] == 0
     finally:
-        dg.dg_set_option(dg.DG_OPT_STREAM_K, 1)
+        dg.dg_set_option(dg.DG_OPT_STREAM_K, 0)
     with pytest.raises(dg.DgError):
         dg.dg_set_option(dg.DG_OPT_STREAM_K, 2)
 
@@ -387,6 +401,8 @@ def _check_plan(p, dt, M, N, K, alpha):
         tiles_j = -(-Nj // bn)
         tiles = -(-Mi // 128) * tiles_j
         assert 1 <= grid <= SMS
+        if p["split_reduce_add"]:
+            assert split > 1
         if split > 1:
             assert p["stages"] >= 3 and not p["cta_pair"] and p["gather_cluster"] == 1
             assert not p["epi_tma_store"]
@@ -425,12 +441,15 @@ def test_plan_invariants_random_views():
 
     rng = random.Random(20261203)
     kinds = {}
-    for _ in range(3000):
+    for n in range(3000):
         dt, cdt, M, N, K, A, B, C, alpha, beta = _random_problem(rng)
+        dg.dg_set_option(dg.DG_OPT_STREAM_K, n % 2)      # half the draws with the opt-in Stream-K tail
         try:
             info = dg.dg_plan(A, B, C, alpha, beta, rng.random() < 0.3, SMS)
         except dg.DgError:
             continue                                     # a view the library rejects up front
+        finally:
+            dg.dg_set_option(dg.DG_OPT_STREAM_K, 0)
         p = info.as_dict()
         tags = [p["kind_name"]]
         if p["kind_name"] == "umma":

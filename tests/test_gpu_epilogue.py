@@ -30,6 +30,7 @@ def _reset_options():
     dg.dg_set_option(dg.DG_OPT_CTA_PAIR, 1)
     dg.dg_set_option(dg.DG_OPT_EPI_TMA, 1)
     dg.dg_set_option(dg.DG_OPT_GATHER_CLUSTER, 1)
+    dg.dg_set_option(dg.DG_OPT_DETERMINISTIC, 0)
 
 
 def expect(p, kind, **fields):
@@ -94,6 +95,15 @@ def test_split_k_swapped_bias_along_i(act):
     p = W.with_epilogue(W.cfg_thin(M=40, N=1000, K=784), act)
     pl = expect(p, "umma", swap_ab=1)
     assert pl["split_k"] > 1
+    check_full(p)
+
+
+def test_split_k_reduce_add_bias_once():
+    # beta = 1, FP32 C, a bias and no activation: the splits add their partials
+    # into C and only the first adds the bias
+    p = W.with_epilogue(W.cfg_thin(M=48, N=1024, K=2048), "none")
+    pl = expect(p, "umma", swap_ab=1)
+    assert pl["split_k"] > 1 and pl["split_reduce_add"] == 1, pl
     check_full(p)
 
 

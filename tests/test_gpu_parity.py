@@ -33,6 +33,7 @@ def _reset_options():
     dg.dg_set_option(dg.DG_OPT_EPI_TMA, 1)
     dg.dg_set_option(dg.DG_OPT_GATHER_CLUSTER, 1)
     dg.dg_set_option(dg.DG_OPT_PAIR_TAIL, 1)
+    dg.dg_set_option(dg.DG_OPT_DETERMINISTIC, 0)
 
 
 def expect_kind(p, kind, **fields):
@@ -178,12 +179,17 @@ def test_thin_beta_one_split_k():
     check_full(p)
 
 
+@pytest.mark.parametrize("deterministic", [1, 0])
 @pytest.mark.parametrize("case", ["s8_ragged_rows", "s3_rows_not_multiple_of_4", "s2_bf16_out", "fp8_scales",
                                   "no_swap_row_major_c"])
-def test_split_k_cluster_reduction(case):
+def test_split_k_cluster_reduction(case, deterministic):
     # Every path of the on-chip split-K reduction: four-row vector steps with
     # a ragged last row group, the element-wise path (S = 3, BF16 output, C
-    # row-major along j) and per-row / per-column scales.
+    # row-major along j) and per-row / per-column scales.  With beta = 1 and
+    # FP32 C the default adds the splits' partials straight into C instead
+    # (tensor reduce-adds along i when swapped, along j otherwise);
+    # deterministic = 1 keeps the cluster reduction for those cases too.
+    dg.dg_set_option(dg.DG_OPT_DETERMINISTIC, deterministic)
     g = torch.Generator().manual_seed(len(case) * 31)
     ms, out, beta = 8, "f32", 1.0
     if case == "s8_ragged_rows":
@@ -210,11 +216,28 @@ def test_split_k_cluster_reduction(case):
         p = W.Problem(case, A, B, C, 1.0, beta)
     pl = expect_kind(p, "umma")
     assert pl["split_k"] > 1 and pl["epi_tma_store"] == 0, pl
+    assert pl["split_reduce_add"] == int(beta == 1.0 and out == "f32" and not deterministic), pl
     if case == "s3_rows_not_multiple_of_4":
         assert pl["split_k"] == 3
     if case == "no_swap_row_major_c":
         assert pl["swap_ab"] == 0
     check_full(p)
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 4096, 2048), (40, 1000, 784), (7, 300, 4096)])
+def test_split_k_reduce_add_into_c(M, N, K):
+    # beta = 1, FP32 C: every split adds alpha * partial into C in the memory
+    # system; against the oracle, and against the fixed-order cluster
+    # reduction within the tolerance (the order of the adds differs)
+    p = W.cfg_thin(M=M, N=N, K=K)
+    pl = expect_kind(p, "umma", swap_ab=1)
+    assert pl["split_k"] > 1 and pl["split_reduce_add"] == 1, pl
+    check_full(p)
+    a = c_matrix(run(p.to("cuda")))
+    dg.dg_set_option(dg.DG_OPT_DETERMINISTIC, 1)
+    assert expect_kind(p, "umma")["split_reduce_add"] == 0
+    b = c_matrix(run(p.to("cuda")))
+    assert np.allclose(a, b, rtol=1e-5, atol=1e-4)
 
 
 def test_thin_without_split_k_matches():
@@ -478,6 +501,8 @@ def test_split_k_exchange_wait_reports_timeout_and_recovers():
     p = W.cfg_thin(M=40, N=1000, K=784)
     pl = expect_kind(p, "umma", swap_ab=1)
     assert pl["split_k"] > 1
+    dg.dg_set_option(dg.DG_OPT_DETERMINISTIC, 1)  # the cluster exchange (beta = 1 would add into C)
+    assert expect_kind(p, "umma")["split_reduce_add"] == 0
     g = p.to("cuda")
     dg.dg_set_option(dg.DG_OPT_WAIT_TIMEOUT_MS, 300)
     dg.dg_set_option(dg.DG_OPT_TEST_STALL, 2)

@@ -22,8 +22,9 @@ pytestmark = pytest.mark.gpu
 
 @pytest.fixture(autouse=True)
 def _reset_options():
+    dg.dg_set_option(dg.DG_OPT_STREAM_K, 1)  # opt-in: the half-width tail is the default
     yield
-    dg.dg_set_option(dg.DG_OPT_STREAM_K, 1)
+    dg.dg_set_option(dg.DG_OPT_STREAM_K, 0)
     dg.dg_set_option(dg.DG_OPT_TEST_STALL, 0)
     dg.dg_set_option(dg.DG_OPT_WAIT_TIMEOUT_MS, 2000)
     dg.dg_set_option(dg.DG_OPT_PAIR_TAIL, 1)

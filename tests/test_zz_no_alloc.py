@@ -46,13 +46,17 @@ def test_static_scratch_entry_matches_dg_gemm_twice(M, N, K, stream_k):
     b = W.cast(W.normal((K, N), g), "bf16")
     ref_p = W.Problem("dg_gemm", W.row_major(a, "bf16"), W.row_major(b, "bf16"), W.empty_out(M, N, "bf16"))
     gp = ref_p.to("cuda")
-    if stream_k and torch.cuda.get_device_properties(0).multi_processor_count == 148:
-        assert plan(gp)["stream_k_tiles"] > 0  # the Stream-K workspace is in use
-    ref = c_matrix(run(gp))
-    S = _scale(gp)
-    tol = tolerance("bf16", ref, S, np.zeros_like(ref))
-    for call in range(2):
-        q = W.Problem("static", gp.A, gp.B, W.empty_out(M, N, "bf16").to("cuda"))
-        got = _call_static(q)
-        err = np.abs(got - ref)
-        assert np.all(err <= tol), (call, float(err.max()))
+    dg.dg_set_option(dg.DG_OPT_STREAM_K, 1 if stream_k else 0)
+    try:
+        if stream_k and torch.cuda.get_device_properties(0).multi_processor_count == 148:
+            assert plan(gp)["stream_k_tiles"] > 0  # the Stream-K workspace is in use
+        ref = c_matrix(run(gp))
+        S = _scale(gp)
+        tol = tolerance("bf16", ref, S, np.zeros_like(ref))
+        for call in range(2):
+            q = W.Problem("static", gp.A, gp.B, W.empty_out(M, N, "bf16").to("cuda"))
+            got = _call_static(q)
+            err = np.abs(got - ref)
+            assert np.all(err <= tol), (call, float(err.max()))
+    finally:
+        dg.dg_set_option(dg.DG_OPT_STREAM_K, 0)
