@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         mbar_init(bar_drain, 1);
         mbar_init(bar_recv, 1);
         // split-K: the slices of this CTA's rows from the other CTAs of the cluster
-        if (p.split_k > 1)
+        if (p.split_k > 1 && !p.red_add)
             mbar_arrive_expect_tx(bar_recv, (uint32_t)(p.split_k - 1) * split_slice_bytes(p.bn, p.split_k));
         *abort_flag = 0;
         fence_barrier_init();
@@ -485,7 +485,8 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     // a thread waits for it before its first access to another CTA, and at the
     // latest before the next cluster barrier, so the start is not delayed.
     // Cluster barrier operations are always issued by whole, converged warps.
-    const bool clustered = p.split_k > 1 || G > 1;
+    // split-K CTAs that add into C (red_add) exchange nothing: no cluster
+    const bool clustered = (p.split_k > 1 && !p.red_add) || G > 1;
     bool cluster_ready = !clustered;  // warp-uniform
     if (clustered) {
         __syncwarp();
@@ -1172,7 +1173,8 @@ cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtens
     static SmemLimit s_limit[4];
     const cudaError_t e = s_limit[(fp8 ? 2 : 0) + (gather ? 1 : 0)].ensure(kern, smem);
     if (e != cudaSuccess) return e;
-    const int cluster = p.split_k > 1 ? p.split_k : (gather && p.gather_cluster > 1 ? p.gather_cluster : 1);
+    const int cluster = (p.split_k > 1 && !p.red_add) ? p.split_k
+                                                        : (gather && p.gather_cluster > 1 ? p.gather_cluster : 1);
     return launch_ex(kern, dim3(grid), dim3(gather ? 448 : 192), smem, s, dim3(cluster, 1, 1), p.pdl, *tp, *tq, *tc,
                      p);
 }
