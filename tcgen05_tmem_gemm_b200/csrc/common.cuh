@@ -136,16 +136,32 @@ __device__ __forceinline__ float tanh_approx(float x) {
 // The fused activation ("DeepGEMM is not a new model: the inner discipline of
 // GPU matrix multiplication", §3.3: GeLU in its tanh form after the bias add,
 // with a fast tanh).  ReLU keeps NaN; GeLU is
-// z/2 (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))).  For a 16-bit output
-// (`fast`) the tanh is the hardware approximation, whose error (2^-11 of the
-// tanh) stays below the output's own rounding (2^-9 for BF16, 2^-11 for FP16);
-// an FP32 output takes the accurate tanhf, so it keeps FP32 accuracy.
+// z/2 (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))), evaluated as h + h tanh(u)
+// with h = z/2 and u = z (sqrt(2/pi) + 0.044715 sqrt(2/pi) z^2): six
+// operations, one of them the tanh.  For a 16-bit output (`FAST`) the tanh is
+// the hardware approximation, whose error (2^-11 of the tanh) stays below the
+// output's own rounding (2^-9 for BF16, 2^-11 for FP16); an FP32 output takes
+// the accurate tanhf, so it keeps FP32 accuracy.
+template <bool FAST>
+__device__ __forceinline__ float gelu_tanh(float z) {
+    const float u = z * fmaf(0.035677408136300125f, z * z, 0.7978845608028654f);
+    const float t = FAST ? tanh_approx(u) : tanhf(u);
+    const float h = 0.5f * z;
+    return fmaf(h, t, h);
+}
+
+// The activation chosen at compile time (the epilogues pick the instance once
+// per tile, so no element pays for the choice).
+template <int ACT, bool FAST>
+__device__ __forceinline__ float act_fn(float z) {
+    if (ACT == DG_ACT_RELU) return z < 0.f ? 0.f : z;
+    if (ACT == DG_ACT_GELU_TANH) return gelu_tanh<FAST>(z);
+    return z;
+}
+
 __device__ __forceinline__ float act_apply(int act, float z, bool fast = false) {
-    if (act == DG_ACT_RELU) return z < 0.f ? 0.f : z;
-    if (act == DG_ACT_GELU_TANH) {
-        const float u = 0.7978845608028654f * fmaf(0.044715f * z, z * z, z);  // sqrt(2/pi) (z + 0.044715 z^3)
-        return 0.5f * z * (1.f + (fast ? tanh_approx(u) : tanhf(u)));
-    }
+    if (act == DG_ACT_RELU) return act_fn<DG_ACT_RELU, false>(z);
+    if (act == DG_ACT_GELU_TANH) return fast ? gelu_tanh<true>(z) : gelu_tanh<false>(z);
     return z;
 }
 

@@ -450,17 +450,7 @@ __global__ void __launch_bounds__(192, 1)
                 else
                     epilogue_rows_tma<2>(e, &tmap_c, blocks, t_row, i_base, p.Mi, j0, pw.w, p.Nj, lane, nblk);
             } else {
-                const bool row_ok = i < p.Mi;
-                const float asi = row_ok ? e.alpha * (e.scale_i ? e.scale_i[i] : 1.f) : 0.f;
-                char *crow = e.c + epi_row_offset(e, row_ok ? i : 0);
-                for (int c0 = 0; c0 < pw.w; c0 += 16) {
-                    uint32_t r[16];
-                    __syncwarp();
-                    tmem_ld16(t_row + c0, r);
-                    tmem_ld_wait();
-                    if (!row_ok) continue;
-                    epilogue_chunk16(e, crow, asi, i, j0 + c0, p.Nj, r);
-                }
+                epilogue_rows_thread(e, t_row, i, p.Mi, j0, pw.w, p.Nj);
             }
             tc_fence_before();
             __syncwarp();
