@@ -424,7 +424,6 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         if (!GATHER) tma_prefetch_desc(&tmap_p);
         if (p.epi_tma || p.red_add) tma_prefetch_desc(&tmap_c);
     }
-    pdl_wait();
     if (p.pdl == 1) pdl_release();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
@@ -499,6 +498,10 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     }
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // The set-up above touches only this CTA's shared memory and TMEM, so it
+    // runs while the previous kernel finishes; every global access below
+    // waits for that kernel (programmatic dependent launch).
+    pdl_wait();
     if (threadIdx.x == 0) trace_at(p, 1);
 
     const int es = FP8 ? 1 : 2;
@@ -679,11 +682,13 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         const EpiParams e = p.epi;  // a local copy: its fields stay in registers
         int local = 0;
         uint32_t nblk = 0;  // tensor-store blocks this warp has issued
-        if (p.split_k > 1 && !p.red_add && e.beta != 0.f && !e.ci_multi) {
-            // the rows this CTA will reduce: pull their C lines into L2 while
-            // the main loops run
+        if (p.split_k > 1 && e.beta != 0.f && !e.ci_multi && blockIdx.x < p.num_units) {
+            // the rows this CTA will reduce (cluster reduction), or a 1/split
+            // share of the tile it adds into (reduce-add): pull their C lines
+            // into L2 while the main loops run, so that the epilogue's reads
+            // or adds find them there
             const TileCoord tc = unit_coord(blockIdx.x, p);
-            const int S = p.split_k, rank = (int)cluster_ctarank();
+            const int S = p.split_k, rank = p.red_add ? tc.split : (int)cluster_ctarank();
             const int r0 = rank * kBM / S, rs = (rank + 1) * kBM / S - r0;
             const int ces = elem_bytes(e.c_dtype);
             const int t = threadIdx.x - kEpiWarp0 * 32;

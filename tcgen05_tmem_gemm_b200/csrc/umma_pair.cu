@@ -180,7 +180,6 @@ __global__ void __launch_bounds__(192, 1)
         tma_prefetch_desc(&tmap_q);
         if (p.epi_tma) tma_prefetch_desc(&tmap_c);
     }
-    pdl_wait();
     if (p.pdl == 1) pdl_release();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -223,6 +222,10 @@ __global__ void __launch_bounds__(192, 1)
     cluster_sync();  // both CTAs' barriers exist before either signals the other's
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // The set-up above touches only the pair's shared memory and TMEM, so it
+    // runs while the previous kernel finishes; every global access below
+    // waits for that kernel (programmatic dependent launch).
+    pdl_wait();
 
     // Stream-K: the tag of this launch's partials is one more than the
     // sequence number the previous launch left (it completed before this
