@@ -372,7 +372,7 @@ def run_one_shape(args):
     res = per_shape(dg, load_peaks(), True, only=args.shape, tune=args.autotune)
     out = {"shape": args.shape, **res}
     if args.trace:
-        # one more call with CTA 0's phase timestamps (ns from kernel entry)
+        # one more call with CTA 0's phase timestamps (SM cycles from kernel entry)
         buf = torch.zeros(64, dtype=torch.int64, device="cuda")
         key = [k for k in SHAPES if k[0] == args.shape][0]
         prob = key[2]().to("cuda")
@@ -383,7 +383,7 @@ def run_one_shape(args):
         dg.dg_set_option(dg.DG_OPT_TRACE, 0)
         t = buf.cpu().tolist()
         t0 = t[0]
-        out["trace_ns"] = {i: (v - t0) for i, v in enumerate(t) if v}
+        out["trace_cycles"] = {i: (v - t0) for i, v in enumerate(t) if v}
     print(json.dumps(out), flush=True)
 
 

@@ -357,7 +357,8 @@ typedef enum {
                                      results.                                          */
     DG_OPT_TRACE = 7,             /* device address of 64 uint64 slots (0 = off): the
                                      single-CTA tensor-core kernel's CTA 0 writes
-                                     %globaltimer at its phase boundaries (analysis)   */
+                                     its SM cycle counter (%clock64) at its phase
+                                     boundaries (analysis)                             */
     DG_OPT_EPI_TMA = 8,           /* 1 (default): tensor-core epilogues store C through
                                      tensor copies where the plan allows; 0: thread
                                      stores only                                        */

@@ -163,14 +163,15 @@ __device__ __forceinline__ void st_shared_vec(uint32_t dst, const typename VecOf
     }
 }
 
-// Phase timestamps of CTA 0 for performance analysis (DG_OPT_TRACE): slot 0
+// Phase timestamps of CTA 0 for performance analysis (DG_OPT_TRACE), in SM
+// cycles (the cycle counter costs a few cycles to read): slot 0
 // entry, 1 set-up done, 2+kb first-unit loads issued (k block kb < 16),
 // 18+kb MMAs of k block kb issued, 34 first accumulator complete (seen by the
 // epilogue), 35 first epilogue done, 36 teardown, 37..52 gather k block kb
 // written (first unit); split-K: 53 accumulator complete, 54 first cluster
 // barrier passed, 55 partials pushed and second barrier passed, 56 reduced.
 __device__ __forceinline__ void trace_at(const UmmaParams &p, int slot) {
-    if (p.trace != nullptr && blockIdx.x == 0) p.trace[slot] = globaltimer_ns();
+    if (p.trace != nullptr && blockIdx.x == 0) p.trace[slot] = (uint64_t)clock64();
 }
 
 // OR of `pred` over the gather warps (named barrier 1), returned to all of them.
