@@ -141,7 +141,7 @@ struct UmmaParams {
     uint64_t timeout_ns;
     int32_t stall_loader;    // test hooks: 1 loaders issue nothing, 2 split-K sends no slices
     int32_t pdl;             // 0 off, 1 release dependents at start, 2 near the end
-    uint64_t *trace;         // optional phase timestamps of CTA 0 (%globaltimer, ns)
+    uint64_t *trace;         // optional phase timestamps of CTA 0 (SM cycles, %clock64)
 };
 
 struct GemvParams {

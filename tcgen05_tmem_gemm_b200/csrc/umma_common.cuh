@@ -219,7 +219,8 @@ constexpr uint32_t kEpiStoreBytes = 4 * 2 * kEpiBlockBytes;
 // writes whole lines and skips everything outside C.  Two blocks alternate,
 // so packing one overlaps the copy of the other.  `stage` is this warp's
 // 2 x kEpiBlockBytes (1024-byte aligned), `nblk` counts the blocks the warp
-// has issued; the caller waits for its copies (bulk_wait_all) before exit.
+// has issued; before exit the caller waits until its copies have read shared
+// memory (bulk_wait_read<0>); their writes land before the grid completes.
 // The warp stores 128-byte column blocks blk_first, blk_first + blk_step, ...
 template <int ES>
 __device__ __forceinline__ void epilogue_rows_tma(const EpiParams &e, const CUtensorMap *cmap, uint32_t stage,

@@ -174,6 +174,29 @@ __device__ __forceinline__ void trace_at(const UmmaParams &p, int slot) {
     if (p.trace != nullptr && blockIdx.x == 0) p.trace[slot] = (uint64_t)clock64();
 }
 
+// The tensor copies of k block k0.. of tile (ti, tj) into the stage at `ps`
+// (P, unless it is gathered) and `qs` (Q), completing on barrier `full`.
+// MN-major operands come as boxes of 128 bytes along i or j.
+template <bool GATHER>
+__device__ __forceinline__ void load_kblock(const CUtensorMap *tp, const CUtensorMap *tq, uint32_t full, uint32_t ps,
+                                            uint32_t qs, int ti, int tj, int k0, int bn, int bk, int es, bool p_mn,
+                                            bool q_mn, uint32_t q_box_bytes) {
+    if (!GATHER) {
+        if (p_mn) {
+            const int per = 128 / es;  // i per box
+            for (int c = 0; c < kBM / per; ++c) tma_load_2d(ps + c * bk * 128, tp, full, ti * kBM + c * per, k0);
+        } else {
+            tma_load_2d(ps, tp, full, k0, ti * kBM);
+        }
+    }
+    if (q_mn) {
+        const int per = 128 / es;
+        for (int c = 0; c < bn / per; ++c) tma_load_2d(qs + c * q_box_bytes, tq, full, tj * bn + c * per, k0);
+    } else {
+        tma_load_2d(qs, tq, full, k0, tj * bn);
+    }
+}
+
 // OR of `pred` over the gather warps (named barrier 1), returned to all of them.
 __device__ __forceinline__ bool named_bar_or(bool pred) {
     uint32_t r;
@@ -453,6 +476,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     const bool helpers = GATHER && p.split_k == 1 && p.num_units == (int)gridDim.x &&
                          (!p.epi_tma ||
                           L.stage_bytes * (uint32_t)p.stages >= (uint32_t)kGatherWarps * 2u * kEpiBlockBytes);
+    int pre_issued = 0;  // k blocks of the first unit copied during the set-up (thread 0)
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             // gather stages: one arrival per gather thread when its cp.async
@@ -477,6 +501,30 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
+        // Every stage is free: for a unit that streams more k blocks than the
+        // ring holds, this thread, the producer lane, puts the first round of
+        // copies in flight now, while the other warps finish the set-up
+        // (their first global access waits for the previous kernel, and so
+        // does this one).  Not in a cluster (a gather cluster, or split-K
+        // reduced on chip), whose start would wait for these copies; and not
+        // for short units, whose set-up measured faster without it.
+        const bool no_cluster = !GATHER && !(p.split_k > 1 && !p.red_add);
+        if (no_cluster && p.stall_loader != 1 && (int)blockIdx.x < p.num_units) {
+            const TileCoord tc = unit_coord(blockIdx.x, p);
+            const int kb0 = tc.split * p.kb_per_split;
+            const int nkb = min(p.kb_total, kb0 + p.kb_per_split) - kb0;
+            pre_issued = nkb > p.stages ? p.stages : 0;
+            const uint32_t tx0 = (GATHER ? (uint32_t)(G - 1) * (L.p_bytes / G) : L.p_bytes) + L.q_bytes;
+            const uint32_t qbb = (uint32_t)(p.q_mn_major ? p.bk * 128 : p.bn * 128);
+            if (pre_issued > 0) pdl_wait();
+            for (int q = 0; q < pre_issued; ++q) {
+                const uint32_t full = bar_full + 8 * q;
+                const uint32_t ps = sbase + q * L.stage_bytes;
+                mbar_arrive_expect_tx(full, tx0);
+                load_kblock<GATHER>(&tmap_p, &tmap_q, full, ps, ps + L.p_bytes, tc.ti, tc.tj, (kb0 + q) * p.bk, p.bn,
+                                    p.bk, FP8 ? 1 : 2, p.p_mn_major != 0, p.q_mn_major != 0, qbb);
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), (uint32_t)p.tmem_cols);
@@ -520,8 +568,10 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             const int kb_per_split = p.kb_per_split, bn = p.bn;
             const bool stall = p.stall_loader == 1, p_mn = p.p_mn_major != 0, q_mn = p.q_mn_major != 0;
             const uint32_t stage_bytes = L.stage_bytes, p_bytes = L.p_bytes;
-            int it = 0, s = 0;  // global k-block counter across tiles, its stage
-            uint32_t ph = 0;
+            // the set-up issued stages 0 .. pre_issued-1 of the first unit
+            int it = pre_issued, s = pre_issued == stages ? 0 : pre_issued;  // k-block counter, its stage
+            uint32_t ph = pre_issued == stages ? 1u : 0u;
+            int skip = pre_issued;
             // gathered P: the parts of the other CTAs of a gather cluster arrive as bytes
             const uint32_t tx = (GATHER ? (uint32_t)(G - 1) * (p_bytes / G) : p_bytes) + L.q_bytes;
             for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
@@ -529,30 +579,14 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                 const int kb0 = tc.split * kb_per_split;
                 const int kb1 = min(kb_total, kb0 + kb_per_split);
                 bool ok = true;
-                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                for (int kb = kb0 + skip; kb < kb1; ++kb, ++it) {
                     if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) { ok = false; break; }
                     if (!stall) {  // test hook: with stall nothing arrives, consumers time out
                         const uint32_t full = bar_full + 8 * s;
                         mbar_arrive_expect_tx(full, tx);
                         const uint32_t ps = sbase + s * stage_bytes;
-                        const uint32_t qs = ps + p_bytes;
-                        const int k0 = kb * bk;
-                        if (!GATHER) {
-                            if (p_mn) {
-                                const int per = 128 / es;  // i per box
-                                for (int c = 0; c < kBM / per; ++c)
-                                    tma_load_2d(ps + c * bk * 128, &tmap_p, full, tc.ti * kBM + c * per, k0);
-                            } else {
-                                tma_load_2d(ps, &tmap_p, full, k0, tc.ti * kBM);
-                            }
-                        }
-                        if (q_mn) {
-                            const int per = 128 / es;
-                            for (int c = 0; c < bn / per; ++c)
-                                tma_load_2d(qs + c * q_box_bytes, &tmap_q, full, tc.tj * bn + c * per, k0);
-                        } else {
-                            tma_load_2d(qs, &tmap_q, full, k0, tc.tj * bn);
-                        }
+                        load_kblock<GATHER>(&tmap_p, &tmap_q, full, ps, ps + p_bytes, tc.ti, tc.tj, kb * bk, bn, bk,
+                                            es, p_mn, q_mn, q_box_bytes);
                         if (it < 16) trace_at(p, 2 + it);
                     }
                     if (++s == stages) {
@@ -560,6 +594,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                         ph ^= 1u;
                     }
                 }
+                skip = 0;
                 if (!ok) break;
             }
             // let the copies already issued land before the CTA can exit
@@ -752,7 +787,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             if (local == 0 && threadIdx.x == kEpiWarp0 * 32) trace_at(p, 35);
         }
         // the tensor stores read this warp's blocks and write C after the loop
-        if (p.epi_tma && lane == 0) bulk_wait_all();
+        if (p.epi_tma && lane == 0) bulk_wait_read<0>();  // writes land before the grid completes
     } else if (GATHER) {
         // ------------------------------------------------ gather producers
         const int gtid = threadIdx.x - (kEpiWarp0 + 4) * 32;
@@ -798,7 +833,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                                          1 + hw / 4, 3);
                 tc_fence_before();
             }
-            if (p.epi_tma && lane == 0) bulk_wait_all();
+            if (p.epi_tma && lane == 0) bulk_wait_read<0>();  // writes land before the grid completes
         }
     }
 
@@ -870,7 +905,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                 }
                 ++nblk;
             }
-            if (lane == 0) bulk_wait_all();  // every add has reached C before the CTA ends
+            if (lane == 0) bulk_wait_read<0>();  // the adds land before the grid completes
         }
     } else if (p.split_k > 1) {
         // ------------------------------------------ cluster reduction of k splits

@@ -460,7 +460,7 @@ __global__ void __launch_bounds__(192, 1)
             if (lane == 0) mbar_arrive_cluster(dsmem_map(bar_tempty + 8 * b, 0));
         }
         // the tensor stores read this warp's blocks and write C after the loop
-        if (p.epi_tma && lane == 0) bulk_wait_all();
+        if (p.epi_tma && lane == 0) bulk_wait_read<0>();  // writes land before the grid completes
     }
 
     // --------------------------------------------------------------- teardown
