@@ -90,6 +90,17 @@ def roofline_time_s(p: W.Problem, peaks):
     return max(t_tc, t_mem), ("tensor" if t_tc >= t_mem else "hbm")
 
 
+def gpu_smi_id(dev: int) -> str:
+    """The GPU's UUID as nvidia-smi and NVML name it ("GPU-..."), so that the
+    clock samples come from the GPU this process runs on even when
+    CUDA_VISIBLE_DEVICES renumbers the devices; the index as a fallback."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev)
+
+
 class ClockSampler:
     """nvidia-smi samples (every 100 ms) of SM clock and throttle reasons."""
 
@@ -100,7 +111,7 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.samples = []
         self.proc = None
-        self.dev = device_index
+        self.dev = gpu_smi_id(device_index)
         self.thread = None
 
     def start(self):
@@ -311,6 +322,58 @@ def _strided_nchw_out() -> W.Problem:
                      bias=p.bias, act="relu")
 
 
+class NvmlClockPoller:
+    """SM clock and power-cap state polled through NVML every half millisecond
+    in a thread, for timed regions far shorter than nvidia-smi's interval
+    (a per-shape timing lasts a few milliseconds).  Reads only."""
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.ok = False
+        self.stop_flag = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            gid = gpu_smi_id(device_index)
+            self.h = (pynvml.nvmlDeviceGetHandleByUUID(gid) if gid.startswith("GPU-")
+                      else pynvml.nvmlDeviceGetHandleByIndex(device_index))
+            self.ok = True
+        except Exception:  # no NVML: the rows go without a clock
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        cap = getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4)
+        while not self.stop_flag.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, bool(reasons & cap)))
+            except Exception:
+                return
+            time.sleep(0.0005)
+
+    def __enter__(self):
+        if self.ok:
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self.stop_flag.set()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.samples:
+            return None
+        return {"sm_mhz_median": statistics.median(m for m, _ in self.samples),
+                "sm_mhz_min": min(m for m, _ in self.samples),
+                "sw_power_cap_share": sum(1 for _, c in self.samples if c) / len(self.samples),
+                "samples": len(self.samples)}
+
+
 def per_shape(dg, peaks, quick: bool, only=None, tune: bool = False):
     """Every workload of the benchmark definition: time, TFLOPS, GB/s and
     fraction of roofline, with the dispatcher's kernel choice."""
@@ -324,7 +387,8 @@ def per_shape(dg, peaks, quick: bool, only=None, tune: bool = False):
         gpus = [base.to("cuda") for _ in range(copies)]
         A, B, C = dg_views(gpus[0], dg)
         pl = dg.dg_plan(A, B, C, base.alpha, base.beta, base.scale_a is not None).as_dict()
-        t_graph, t_stream, host = time_problem(gpus, dg, reps, warm=5)
+        with NvmlClockPoller(torch.cuda.current_device()) as clk:
+            t_graph, t_stream, host = time_problem(gpus, dg, reps, warm=5)
         fl, by = flops_bytes(base)
         t_roof, bound = roofline_time_s(base, peaks)
         med = t_graph
@@ -350,7 +414,8 @@ def per_shape(dg, peaks, quick: bool, only=None, tune: bool = False):
                      "tiles": {k: pl[k] for k in ("block_n", "block_k", "split_k", "swap_ab", "p_gather", "grid")},
                      "timing": "CUDA-graph replay of the calls (device time); us_stream: back-to-back stream calls",
                      "l2": (f"{copies} rotating input copies, {copies * by / 1e6:.0f} MB"
-                            if copies > 1 else "single copy (L2-resident)")}
+                            if copies > 1 else "single copy (L2-resident)"),
+                     "clocks": clk.summary()}
         if tuned is not None:
             out[name]["autotuned"] = tuned
         del gpus
