@@ -226,6 +226,7 @@ struct Plan {
 struct Views {
     const dg_view *A, *B, *C;
     ViewInfo a, b, c;
+    int act = DG_ACT_NONE;  // the call's activation: split-K partials add into C only without one
 };
 
 uint32_t make_idesc(int in_dtype, bool p_mn, bool q_mn, int bn, int m = 128) {
@@ -495,8 +496,10 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     if (gcl > 1) in.grid = (int32_t)std::min<int64_t>(units2, (num_sms / gcl) * gcl);
     // split-K with beta == 1 and FP32 C: the splits can add their partials
     // straight into C through one 2-D tensor map of C (its i group one dim)
-    if (split > 1 && beta == 1.f && v.C->dtype == DG_F32 && v.c.tma_ok && g_deterministic.load() == 0)
+    if (split > 1 && beta == 1.f && v.C->dtype == DG_F32 && v.c.tma_ok && g_deterministic.load() == 0 &&
+        v.act == DG_ACT_NONE) {
         in.split_reduce_add = 1;
+    }
     if (pair) {
         const int64_t pair_units = ((Mi + 255) / 256) * tiles_j;
         in.block_m = 256;
@@ -524,7 +527,7 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     }
     pl->fp8 = (dt == DG_E4M3);
     pl->smem = pair ? umma_pair_smem_bytes(bn, stages, epi_tma)
-                    : umma_smem_bytes(bn, stages, !p_tma, epi_tma, (int)split);
+                    : umma_smem_bytes(bn, stages, !p_tma, epi_tma, in.split_reduce_add ? 1 : (int)split);
     return true;
 }
 
@@ -923,7 +926,9 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         rec->fp8 = pl.fp8;
         rec->gather = in.p_gather != 0;
         rec->grid = in.grid;
-        rec->smem = pl.smem;
+        // the kernel lays out its shared memory from these parameters
+        rec->smem = rec->pair ? pl.smem
+                              : umma_smem_bytes(p.bn, p.stages, rec->gather, p.epi_tma != 0, p.red_add ? 1 : p.split_k);
         break;
     }
     default: return DG_ERR_UNSUPPORTED;
@@ -1086,6 +1091,7 @@ dg_status dg_gemm_ex(const dg_view *A, const dg_view *B, const dg_view *C, float
                 return fire(t_calls.rec[i], static_cast<cudaStream_t>(stream));
 
     Views v{A, B, C, {}, {}, {}};
+    v.act = act;
     Plan pl;
     // argument errors are reported before any CUDA call
     dg_status st = make_plan(v, alpha, beta, 148, &pl);
@@ -1130,6 +1136,7 @@ dg_status dg_autotune(const dg_view *A, const dg_view *B, const dg_view *C, floa
     if (reps < 1 || reps > 1000) return DG_ERR_VALUE;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     Views v{A, B, C, {}, {}, {}};
+    v.act = act;
     Plan base;
     const Override rule;  // the dispatcher's rules, not an earlier tuning
     dg_status st = make_plan(v, alpha, beta, 148, &base, true, &rule);

@@ -452,7 +452,8 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const SmemLayout L = smem_layout(p.bn, p.stages, GATHER, p.epi_tma != 0, p.split_k);
+    // split-K partials added into C (red_add) need no receive region
+    const SmemLayout L = smem_layout(p.bn, p.stages, GATHER, p.epi_tma != 0, p.red_add ? 1 : p.split_k);
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_full = sbase + L.bar_off;
     const uint32_t bar_empty = bar_full + 8 * p.stages;
