@@ -244,8 +244,9 @@ def dg_views(p: W.Problem, dg):
 def time_problem(p_gpu_list, dg, reps: int, warm: int):
     """Per-call times over `reps` calls that rotate through the given
     device-resident copies:
-      graph  - the calls captured in one CUDA graph and replayed (device time,
-               no host launch cost between kernels),
+      graph  - the calls captured in one CUDA graph and replayed ten times
+               (device time, no host launch cost between kernels): the median
+               per call over the replays, and (p10, p90) as the fourth value,
       stream - the same calls enqueued back to back on a stream (includes the
                host cost of each call when the GPU outruns the host),
       host   - host seconds per dg_gemm call while enqueuing."""
@@ -281,16 +282,22 @@ def time_problem(p_gpu_list, dg, reps: int, warm: int):
             calls(reps, s)
         g.replay()
         torch.cuda.synchronize()
+        # ten replays back to back, each bracketed by its own events: the
+        # per-call time is the median over replays, with p10 and p90
+        n_rep = 10
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_rep)]
         hold_gpu()
-        a.record(s)
-        for _ in range(3):
+        for ea, eb in evs:
+            ea.record(s)
             g.replay()
-        b.record(s)
+            eb.record(s)
         torch.cuda.synchronize()
-        t_graph = a.elapsed_time(b) * 1e-3 / (3 * reps)
+        per_call = sorted(ea.elapsed_time(eb) * 1e-3 / reps for ea, eb in evs)
+        t_graph = statistics.median(per_call)
+        spread = (per_call[1], per_call[-2])  # p10, p90 of ten
         del g
     assert dg.dg_sync_status(s) == dg.DG_OK
-    return t_graph, t_stream, host
+    return t_graph, t_stream, host, spread
 
 
 # (key, name, workload, rotating copies).  The HBM-bound workloads rotate
@@ -381,14 +388,17 @@ def per_shape(dg, peaks, quick: bool, only=None, tune: bool = False):
     for key, name, fn, copies in SHAPES:
         if only is not None and key != only:
             continue
-        # every copy is used at least once per graph, so the rotation is real
-        reps = max(20 if quick else 100, copies)
+        # every copy is used at least once per graph, so the rotation is real;
+        # ten replays of 20 calls keep a 4096^3 GEMM's window near 20 ms, short
+        # of the power cap that a longer run settles into (the burst peak is
+        # the reference)
+        reps = max(20, copies)
         base = fn()
         gpus = [base.to("cuda") for _ in range(copies)]
         A, B, C = dg_views(gpus[0], dg)
         pl = dg.dg_plan(A, B, C, base.alpha, base.beta, base.scale_a is not None).as_dict()
         with NvmlClockPoller(torch.cuda.current_device()) as clk:
-            t_graph, t_stream, host = time_problem(gpus, dg, reps, warm=5)
+            t_graph, t_stream, host, spread = time_problem(gpus, dg, reps, warm=5)
         fl, by = flops_bytes(base)
         t_roof, bound = roofline_time_s(base, peaks)
         med = t_graph
@@ -400,19 +410,22 @@ def per_shape(dg, peaks, quick: bool, only=None, tune: bool = False):
             epi = dg.epilogue(q.bias, q.act) if (q.bias is not None or q.act != "none") else None
             st, res = dg.dg_autotune(A, B, C, q.alpha, q.beta, q.scale_a, q.scale_b, epi, None, 5)
             assert st == dg.DG_OK, dg.status_string(st)
-            t_tuned, _, _ = time_problem(gpus, dg, reps, warm=5)
+            t_tuned, _, _, _ = time_problem(gpus, dg, reps, warm=5)
             chosen = res.plan.as_dict()
             tuned = {"us": t_tuned * 1e6, "frac_of_roofline": t_roof / t_tuned, "candidates": res.candidates,
                      "trial_us_rule": res.default_us, "trial_us_best": res.best_us,
                      "plan": {k: chosen[k] for k in ("kind_name", "block_n", "split_k", "cta_pair", "stream_k_tiles",
                                                      "gather_cluster", "epi_tma_store", "stages", "grid")}}
             dg.dg_tune_clear()
-        out[name] = {"kernel": pl["kind_name"], "us": med * 1e6, "us_stream": t_stream * 1e6,
+        p10, p90 = spread
+        out[name] = {"kernel": pl["kind_name"], "us": med * 1e6, "us_p10": p10 * 1e6, "us_p90": p90 * 1e6,
+                     "calls_timed": 10 * reps, "us_stream": t_stream * 1e6,
                      "host_us_per_call": host * 1e6,
                      "tflops": fl / med / 1e12, "gbs": by / med / 1e9, "bound": bound,
                      "roofline_us": t_roof * 1e6, "frac_of_roofline": t_roof / med,
                      "tiles": {k: pl[k] for k in ("block_n", "block_k", "split_k", "swap_ab", "p_gather", "grid")},
-                     "timing": "CUDA-graph replay of the calls (device time); us_stream: back-to-back stream calls",
+                     "timing": ("CUDA-graph replay of the calls, median per call over ten replays (device "
+                                "time); us_stream: back-to-back stream calls"),
                      "l2": (f"{copies} rotating input copies, {copies * by / 1e6:.0f} MB"
                             if copies > 1 else "single copy (L2-resident)"),
                      "clocks": clk.summary()}
