@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libdg.so")
-SOURCES = ["api.cu", "view.cpp", "simt.cu", "gemv.cu", "umma.cu", "umma_gather.cu", "umma_pair.cu"]
+SOURCES = ["api.cu", "view.cpp", "simt.cu", "gemv.cu", "umma.cu", "umma_gather.cu", "umma_gather_split.cu", "umma_pair.cu"]
 HEADERS = ["dg_internal.h", "sm100.cuh", "common.cuh", "umma_common.cuh", "umma_kernel.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -173,7 +173,8 @@ struct SimtParams {
 
 // tc: C's tensor map when p.epi_tma (otherwise not read)
 using UmmaKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const UmmaParams);
-UmmaKernelFn umma_gather_kernel(bool fp8);  // the gather instances (umma_gather.cu)
+UmmaKernelFn umma_gather_kernel(bool fp8, bool split);  // the gather instances (umma_gather.cu)
+UmmaKernelFn umma_gather_kernel_split(bool fp8);        // those for split-K plans (umma_gather_split.cu)
 cudaError_t launch_umma(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq, const CUtensorMap *tc,
                         bool fp8, bool gather, int grid, size_t smem, cudaStream_t s);
 size_t umma_smem_bytes(int bn, int stages, bool gather, bool epi_tma, int split);

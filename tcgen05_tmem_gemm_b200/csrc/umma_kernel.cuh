@@ -437,10 +437,14 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-template <bool FP8, bool GATHER>
+template <bool FP8, bool GATHER, bool SPLIT>
 __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_c, const UmmaParams p) {
+    // instances for unsplit plans carry no split-K paths (a smaller
+    // instruction footprint: every phase of a one-tile CTA is a first pass
+    // through its code)
+    constexpr bool kSplit = SPLIT;
     if (threadIdx.x == 0) trace_at(p, 0);
     if (threadIdx.x == 64) {
         // descriptor fetches start at once, while thread 0 sets up the barriers
@@ -497,7 +501,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         mbar_init(bar_drain, 1);
         mbar_init(bar_recv, 1);
         // split-K: the slices of this CTA's rows from the other CTAs of the cluster
-        if (p.split_k > 1 && !p.red_add)
+        if (kSplit && p.split_k > 1 && !p.red_add)
             mbar_arrive_expect_tx(bar_recv, (uint32_t)(p.split_k - 1) * split_slice_bytes(p.bn, p.split_k));
         *abort_flag = 0;
         fence_barrier_init();
@@ -509,7 +513,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         // does this one).  Not in a cluster (a gather cluster, or split-K
         // reduced on chip), whose start would wait for these copies; and not
         // for short units, whose set-up measured faster without it.
-        const bool no_cluster = !GATHER && !(p.split_k > 1 && !p.red_add);
+        const bool no_cluster = !GATHER && !(kSplit && p.split_k > 1 && !p.red_add);
         if (no_cluster && p.stall_loader != 1 && (int)blockIdx.x < p.num_units) {
             const TileCoord tc = unit_coord(blockIdx.x, p);
             const int kb0 = tc.split * p.kb_per_split;
@@ -540,7 +544,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     // latest before the next cluster barrier, so the start is not delayed.
     // Cluster barrier operations are always issued by whole, converged warps.
     // split-K CTAs that add into C (red_add) exchange nothing: no cluster
-    const bool clustered = (p.split_k > 1 && !p.red_add) || G > 1;
+    const bool clustered = (kSplit && p.split_k > 1 && !p.red_add) || G > 1;
     bool cluster_ready = !clustered;  // warp-uniform
     if (clustered) {
         __syncwarp();
@@ -719,7 +723,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         const EpiParams e = p.epi;  // a local copy: its fields stay in registers
         int local = 0;
         uint32_t nblk = 0;  // tensor-store blocks this warp has issued
-        if (p.split_k > 1 && e.beta != 0.f && !e.ci_multi && blockIdx.x < p.num_units) {
+        if (kSplit && p.split_k > 1 && e.beta != 0.f && !e.ci_multi && blockIdx.x < p.num_units) {
             // the rows this CTA will reduce (cluster reduction), or a 1/split
             // share of the tile it adds into (reduce-add): pull their C lines
             // into L2 while the main loops run, so that the epilogue's reads
@@ -760,7 +764,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * p.bn);
             const int j0 = tc.tj * p.bn;
 
-            if (p.split_k > 1) {
+            if (kSplit && p.split_k > 1) {
                 // one unit per CTA: the partial stays in TMEM until the cluster
                 // has finished its main loops (see the reduction below)
                 tc_fence_before();
@@ -838,7 +842,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         }
     }
 
-    if (p.split_k > 1 && p.red_add) {
+    if (kSplit && p.split_k > 1 && p.red_add) {
         // ------------------------------------- split-K partials added into C
         // beta = 1 and FP32 C: C += alpha * s_i * s_j * partial (+ bias, by the
         // first split only) is linear in the splits, so each CTA adds its own
@@ -908,7 +912,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             }
             if (lane == 0) bulk_wait_read<0>();  // the adds land before the grid completes
         }
-    } else if (p.split_k > 1) {
+    } else if (kSplit && p.split_k > 1) {
         // ------------------------------------------ cluster reduction of k splits
         // CTA s of the cluster owns rows [128 s / S, 128 (s+1) / S) of the
         // tile.  Once its own main loop is done (its ring is then idle), each
