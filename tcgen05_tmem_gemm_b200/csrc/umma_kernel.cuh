@@ -1,5 +1,5 @@
 // Tensor-core GEMM for sm_100a: tcgen05.mma with TMEM accumulators.
-// (The kernel template; umma.cu and umma_gather.cu each instantiate part of it.)
+// (The kernel template; umma.cu, umma_gather.cu and umma_gather_split.cu each instantiate part of it.)
 //
 // Computes D[i][j] = sum_k P[i][k] Q[k][j] tile by tile and applies the
 // epilogue  out = alpha * s_i * s_j * D + beta * C_in  on the way out.  P is A
@@ -30,12 +30,16 @@
 //    same rows of P form a cluster and each gathers one k-slice of every stage,
 //    copied to the others through distributed shared memory.  With one tile
 //    per CTA these warps then take part of the epilogue;
-//  - split-K: the splits of a tile form a cluster; each CTA sends the rows
-//    other CTAs own from its partial into their shared memory, and each owner
-//    adds the slices in split order (deterministic) and runs the epilogue
-//    ("DeepGEMM deep dive", §5.2).  No global workspace.
-// Every wait is bounded (WaitCtl); on expiry the CTA records DG_ERR_TIMEOUT,
-// drains what it has in flight, frees TMEM and exits.
+//  - split-K ("DeepGEMM deep dive", §5.2), no global workspace either way:
+//    with beta = 1 and FP32 C (and no activation) each split adds its scaled
+//    partial into C with tensor reduce-adds, with no cluster; otherwise the
+//    splits of a tile form a cluster, each CTA sends the rows other CTAs own
+//    from its partial into their shared memory, and each owner adds the
+//    slices in split order (deterministic) and runs the epilogue.
+// The template's SPLIT parameter leaves the split-K paths out of instances
+// that only run unsplit plans.  Every wait is bounded (WaitCtl); on expiry the
+// CTA records DG_ERR_TIMEOUT, drains what it has in flight, frees TMEM and
+// exits.
 #pragma once
 
 #include <atomic>
