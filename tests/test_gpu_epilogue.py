@@ -237,3 +237,65 @@ def test_full_size_fused(name):
     else:
         assert pl["cta_pair"] == 1
         check_sampled(p, npts=3000, extra=tile_corners(p.M, p.N, 128, 128))
+
+
+def _off_16(t: torch.Tensor) -> torch.Tensor:
+    """A device copy of 1-D t whose first element sits 4 bytes past a 16-byte
+    boundary, so that no 16-byte vector load of it is legal."""
+    big = torch.empty(t.numel() + 4, dtype=t.dtype, device="cuda")
+    v = big[1:1 + t.numel()]
+    v.copy_(t.to("cuda"))
+    assert v.data_ptr() % 16 == 4
+    return v
+
+
+def _fp8_problem(M, N, K, seed, k_major_b=False):
+    g = torch.Generator().manual_seed(seed)
+    qa, sa = W.quantise_e4m3(W.normal((M, K), g), dim=1)
+    if k_major_b:  # B read K-major from an [N, K] tensor (CTA pairs need it for FP8)
+        qbt, sb = W.quantise_e4m3(W.normal((N, K), g), dim=1)
+        B = W.transposed(qbt, "e4m3")
+    else:
+        qb, sb = W.quantise_e4m3(W.normal((K, N), g), dim=0)
+        B = W.row_major(qb, "e4m3")
+    return W.Problem("fp8_off16", W.row_major(qa, "e4m3"), B, W.empty_out(M, N, "bf16"), 1.0, 0.0, sa, sb)
+
+
+@pytest.mark.parametrize("case", ["tensor_store_bf16", "tensor_store_f32", "thread_store_beta", "pair_fp8",
+                                  "umma_fp8", "gemv"])
+def test_bias_and_scales_off_16_byte_boundaries(case):
+    # The epilogues read the bias and the column scales as 16-byte vectors only
+    # when the array allows it; arrays 4 bytes past a 16-byte boundary take the
+    # element loads, with the same results.
+    from harness import _bias_abs, beta_c_of, compare
+    import oracle
+
+    if case == "tensor_store_bf16":
+        p, kind = W.with_epilogue(_rm(300, 520, 200, "bf16", "bf16", 21), "gelu_tanh"), dict(epi_tma_store=1)
+    elif case == "tensor_store_f32":
+        p, kind = W.with_epilogue(_rm(300, 520, 200, "bf16", "f32", 22), "relu"), dict(epi_tma_store=1)
+    elif case == "thread_store_beta":
+        p, kind = W.with_epilogue(_rm(300, 520, 200, "bf16", "f32", 23, beta=0.5), "gelu_tanh"), \
+            dict(epi_tma_store=0)
+    elif case == "pair_fp8":
+        dg.dg_set_option(dg.DG_OPT_CTA_PAIR, 2)
+        dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, 1)
+        p, kind = W.with_epilogue(_fp8_problem(512, 512, 512, 24, k_major_b=True), "gelu_tanh"), dict(cta_pair=1)
+    elif case == "umma_fp8":
+        p, kind = W.with_epilogue(_fp8_problem(300, 400, 256, 25), "relu"), dict(cta_pair=0)
+    else:
+        g = torch.Generator().manual_seed(26)
+        x = W.cast(W.normal((1, 1024), g, 0.02), "bf16")
+        Wt = W.cast(W.normal((1024, 2056), g, 0.02), "bf16")
+        p = W.with_epilogue(W.Problem("gemv_off16", W.row_major(x, "bf16"), W.row_major(Wt, "bf16"),
+                                      W.empty_out(1, 2056, "bf16")), "gelu_tanh")
+        kind = {}
+    pl = expect(p, "gemv_n" if case == "gemv" else "umma", **kind)
+    ref, bound, pre = oracle.gemm(p, want_pre=True)
+    gp = p.to("cuda")
+    gp.bias = _off_16(p.bias)
+    if p.scale_a is not None:
+        gp.scale_a = _off_16(p.scale_a)
+        gp.scale_b = _off_16(p.scale_b)
+    run(gp)
+    compare(p, c_matrix(gp), ref, bound, beta_c_of(p), f"{case} {pl['kind_name']}", pre, _bias_abs(p))
