@@ -634,3 +634,37 @@ def test_full_size_square_tile_corners(name):
     pl = expect_kind(p, "umma")
     _assert_bench_plan(name, pl)
     check_sampled(p, npts=3000, extra=tile_corners(p.M, p.N, 128, 128))
+
+
+@pytest.mark.parametrize("tma", [1, 0])
+def test_output_past_4_gib(tma):
+    # C of 8 GiB (65536 x 32768 FP32): the byte offsets of its last rows pass
+    # 2^32, through the tensor-store and the thread-store epilogues.  The
+    # oracle evaluates the sampled outputs on the sub-problem of their rows of
+    # A and columns of B (the same data, the same definition).
+    dg.dg_set_option(dg.DG_OPT_EPI_TMA, tma)
+    M, N, K = 65536, 32768, 16
+    g = torch.Generator().manual_seed(65536)
+    a = W.cast(W.normal((M, K), g), "bf16")
+    b = W.cast(W.normal((K, N), g), "bf16")
+    c = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    p = W.Problem("past_4gib", W.row_major(a, "bf16"), W.row_major(b, "bf16"), W.row_major(c, "f32"))
+    pl = plan(p)
+    assert pl["kind_name"] == "umma" and pl["epi_tma_store"] == tma, pl
+    ga, gb = a.to("cuda"), b.to("cuda")
+    A = dg.make_view(ga.data_ptr(), (M, K), (2 * K, 2), 1, "bf16")
+    B = dg.make_view(gb.data_ptr(), (K, N), (2 * N, 2), 1, "bf16")
+    C = dg.make_view(c.data_ptr(), (M, N), (4 * N, 4), 1, "f32")
+    assert dg.dg_gemm(A, B, C, 1.0, 0.0) == dg.DG_OK
+    assert dg.dg_sync_status() == dg.DG_OK
+    rng = np.random.default_rng(7)
+    ms = np.concatenate([rng.integers(0, M, 200), np.full(40, M - 1), rng.integers(M - 128, M, 40), [0, M - 1]])
+    ns = np.concatenate([rng.integers(0, N, 200), rng.integers(0, N, 40), np.full(40, N - 1), [N - 1, 0]])
+    got = c[torch.as_tensor(ms, device="cuda"), torch.as_tensor(ns, device="cuda")].double().cpu().numpy()
+    n = len(ms)
+    sub = W.Problem("past_4gib_rows_cols", W.row_major(a[torch.as_tensor(ms)].contiguous(), "bf16"),
+                    W.row_major(b[:, torch.as_tensor(ns)].contiguous(), "bf16"), W.empty_out(n, n, "f32"))
+    ref, bound = oracle.gemm_points(sub, np.arange(n), np.arange(n))
+    compare(sub, got, ref, bound, np.zeros(n), "past_4gib")
+    del c
+    torch.cuda.empty_cache()
