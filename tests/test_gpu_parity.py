@@ -668,3 +668,37 @@ def test_output_past_4_gib(tma):
     compare(sub, got, ref, bound, np.zeros(n), "past_4gib")
     del c
     torch.cuda.empty_cache()
+
+
+def test_gathered_operand_past_2_gib():
+    # An NCHW feature map of 2.5 GB (x[48, 256, 320, 320] BF16) read in place
+    # as [n*h*w, c]: the gather's byte offsets pass 2^31.  Sampled outputs,
+    # the last rows among them, against the oracle on their sub-problem.
+    n, c, h, w, N = 48, 256, 320, 320, 32
+    x = W.pattern((n, c, h, w), "bf16", device="cuda")
+    g = torch.Generator().manual_seed(2 ** 31 % 1000)
+    b = W.cast(W.uniform((c, N), g), "bf16")
+    M = n * h * w
+    cmat = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    A = W.nchw_as_rows(x, "bf16")
+    p = W.Problem("nchw_past_2gib", A, W.row_major(b, "bf16"), W.row_major(cmat, "f32"))
+    assert plan(p)["p_gather"] == 1
+    gb = b.to("cuda")
+    Av = dg.make_view(x.data_ptr(), A.shape, A.stride, A.row_dims, "bf16")
+    Bv = dg.make_view(gb.data_ptr(), (c, N), (2 * N, 2), 1, "bf16")
+    Cv = dg.make_view(cmat.data_ptr(), (M, N), (4 * N, 4), 1, "f32")
+    assert dg.dg_gemm(Av, Bv, Cv, 1.0, 0.0) == dg.DG_OK
+    assert dg.dg_sync_status() == dg.DG_OK
+    rng = np.random.default_rng(31)
+    ms = np.concatenate([rng.integers(0, M, 200), rng.integers(M - 4096, M, 60), [0, M - 1]])
+    ns = np.concatenate([rng.integers(0, N, 200), rng.integers(0, N, 60), [N - 1, 0]])
+    got = cmat[torch.as_tensor(ms, device="cuda"), torch.as_tensor(ns, device="cuda")].double().cpu().numpy()
+    mi = torch.as_tensor(ms, device="cuda")
+    rows = x.view(n, c, h * w)[mi // (h * w), :, mi % (h * w)].cpu().contiguous()  # [len(ms), c]
+    k = len(ms)
+    sub = W.Problem("nchw_past_2gib_rows_cols", W.row_major(rows, "bf16"),
+                    W.row_major(b[:, torch.as_tensor(ns)].contiguous(), "bf16"), W.empty_out(k, k, "f32"))
+    ref, bound = oracle.gemm_points(sub, np.arange(k), np.arange(k))
+    compare(sub, got, ref, bound, np.zeros(k), "nchw_past_2gib")
+    del x, cmat
+    torch.cuda.empty_cache()

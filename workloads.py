@@ -150,6 +150,19 @@ def quantise_e4m3(x: torch.Tensor, dim: int):
     return q, scale.contiguous()
 
 
+def pattern(shape, dtype: str = "bf16", device="cpu") -> torch.Tensor:
+    """A deterministic tensor ((i mod 251) - 125) / 128 over the flat index i,
+    made where it will live (on the device for operands too large to draw on
+    the host).  Every value is a multiple of 1/128 below 1 in magnitude, exact
+    in F16 and BF16."""
+    numel = 1
+    for s in shape:
+        numel *= int(s)
+    i = torch.arange(numel, device=device, dtype=torch.int64)
+    v = ((i % 251) - 125).to(torch.float32) / 128.0
+    return v.to(TORCH_DTYPE[dtype]).reshape(tuple(shape))
+
+
 def empty_out(M: int, N: int, dtype: str, fill=float("nan")) -> Operand:
     t = torch.full((M, N), fill, dtype=torch.float32).to(TORCH_DTYPE[dtype])
     return row_major(t, dtype)
