@@ -702,3 +702,70 @@ def test_gathered_operand_past_2_gib():
     compare(sub, got, ref, bound, np.zeros(k), "nchw_past_2gib")
     del x, cmat
     torch.cuda.empty_cache()
+
+
+def _sampled_against_subproblem(a_rows, b_cols, got, name, out, alpha=1.0):
+    """The oracle on the sub-problem made of the sampled outputs' rows of A
+    ([k, K]) and columns of B ([K, k]): output i is (i, i); `out` is the real
+    output's dtype, which sets the tolerance."""
+    k = a_rows.shape[0]
+    dt = {torch.bfloat16: "bf16", torch.float16: "f16"}[a_rows.dtype]
+    sub = W.Problem(name, W.row_major(a_rows.contiguous(), dt), W.row_major(b_cols.contiguous(), dt),
+                    W.empty_out(k, k, out), alpha)
+    ref, bound = oracle.gemm_points(sub, np.arange(k), np.arange(k))
+    compare(sub, got, ref, bound, np.zeros(k), name)
+
+
+def test_gemv_weight_past_4_gib():
+    # Decode GEMV on W[65536 x 40960] BF16 (5.4 GB, 2.7e9 elements, made on
+    # the device): TMA coordinates and k splits far past the benchmark's.
+    K, N = 65536, 40960
+    Wt = W.pattern((K, N), "bf16", device="cuda")
+    g = torch.Generator().manual_seed(40960)
+    x = W.cast(W.normal((1, K), g, 0.02), "bf16")
+    y = torch.full((1, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    p = W.Problem("gemv_past_4gib", W.row_major(x, "bf16"), W.row_major(Wt, "bf16"), W.row_major(y, "bf16"))
+    assert plan(p)["kind_name"] == "gemv_n"
+    gx = x.to("cuda")
+    X = dg.make_view(gx.data_ptr(), (1, K), (2 * K, 2), 1, "bf16")
+    Wv = dg.make_view(Wt.data_ptr(), (K, N), (2 * N, 2), 1, "bf16")
+    Y = dg.make_view(y.data_ptr(), (1, N), (2 * N, 2), 1, "bf16")
+    assert dg.dg_gemm(X, Wv, Y, 1.0, 0.0) == dg.DG_OK
+    assert dg.dg_sync_status() == dg.DG_OK
+    ns = np.concatenate([np.random.default_rng(5).integers(0, N, 96), [0, N - 1, N - 2]])
+    ni = torch.as_tensor(ns, device="cuda")
+    got = y[0, ni].double().cpu().numpy()
+    cols = Wt[:, ni].cpu()  # [K, k]
+    _sampled_against_subproblem(x.expand(len(ns), K), cols, got, "gemv_past_4gib", "bf16")
+    del Wt
+    torch.cuda.empty_cache()
+
+
+def test_square_16384_many_pair_tiles():
+    # 16384 x 16384 x 1024 BF16 on CTA pairs: 4096 tiles on 74 pairs, the
+    # persistent schedule's later waves and last half-width tiles; the tile
+    # corners of a band of tiles and random outputs against the oracle.
+    M = N = 16384
+    K = 1024
+    g = torch.Generator().manual_seed(16384)
+    a = W.cast(W.normal((M, K), g), "bf16")
+    b = W.cast(W.normal((K, N), g), "bf16")
+    cmat = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    p = W.Problem("square_16384", W.row_major(a, "bf16"), W.row_major(b, "bf16"), W.row_major(cmat, "bf16"))
+    pl = plan(p)
+    assert pl["kind_name"] == "umma" and pl["cta_pair"] == 1, pl
+    ga, gb = a.to("cuda"), b.to("cuda")
+    A = dg.make_view(ga.data_ptr(), (M, K), (2 * K, 2), 1, "bf16")
+    B = dg.make_view(gb.data_ptr(), (K, N), (2 * N, 2), 1, "bf16")
+    C = dg.make_view(cmat.data_ptr(), (M, N), (2 * N, 2), 1, "bf16")
+    assert dg.dg_gemm(A, B, C, 1.0, 0.0) == dg.DG_OK
+    assert dg.dg_sync_status() == dg.DG_OK
+    cm, cn = tile_corners(M, N, 256, pl["block_n"])
+    band = [(m, n) for m, n in zip(cm, cn) if m >= M - 1024]  # the last rows of tiles
+    rng = np.random.default_rng(3)
+    ms = np.array([m for m, _ in band] + list(rng.integers(0, M, 300)))
+    ns = np.array([n for _, n in band] + list(rng.integers(0, N, 300)))
+    got = cmat[torch.as_tensor(ms, device="cuda"), torch.as_tensor(ns, device="cuda")].double().cpu().numpy()
+    _sampled_against_subproblem(a[torch.as_tensor(ms)], b[:, torch.as_tensor(ns)], got, "square_16384", "bf16")
+    del cmat
+    torch.cuda.empty_cache()
