@@ -138,6 +138,9 @@ typedef enum {
  * The layout transform of the fusion (e.g. writing an NCHW output from an
  * [N*H*W, C] product) needs no field: C is a strided view, and the
  * tensor-core epilogue addresses a row of C through any number of dims.
+ * Accuracy: everything before the store is FP32; GeLU's tanh is the hardware
+ * approximation for F16/BF16 outputs (relative error about 2^-11, below their
+ * rounding) and the accurate tanhf for FP32 outputs.
  */
 typedef struct {
     const float *bias;
