@@ -392,6 +392,7 @@ __device__ __forceinline__ void gather_role(const UmmaParams &p, const SmemLayou
             g_row_off[r] = i < p.Mi ? axis_offset(p.pv.row, i) : -1;
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kGatherWarps * 32) : "memory");
+        pdl_wait();  // before the first copy (returns at once after the first unit)
         bool ok = true;
         V cur[kGatherUnroll], nxt[kGatherUnroll];
         if (one_batch && kb0 < kb1) gather_load<VB>(src, g, g_row_off, kb0 * bk, gtid, cur);
@@ -557,9 +558,11 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // The set-up above touches only this CTA's shared memory and TMEM, so it
-    // runs while the previous kernel finishes; every global access below
-    // waits for that kernel (programmatic dependent launch).
-    pdl_wait();
+    // runs while the previous kernel finishes (programmatic dependent launch).
+    // Each role waits for that kernel right before its first global access,
+    // after the work it can do from the parameters alone (the gather's row
+    // offsets, the producer's unit coordinates); the MMA issuer and the
+    // gather-cluster forwarder touch no global memory and do not wait.
     if (threadIdx.x == 0) trace_at(p, 1);
 
     const int es = FP8 ? 1 : 2;
@@ -583,6 +586,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
             int skip = pre_issued;
             // gathered P: the parts of the other CTAs of a gather cluster arrive as bytes
             const uint32_t tx = (GATHER ? (uint32_t)(G - 1) * (p_bytes / G) : p_bytes) + L.q_bytes;
+            pdl_wait();
             for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
                 const TileCoord tc = unit_coord(u, p);
                 const int kb0 = tc.split * kb_per_split;
@@ -722,6 +726,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
         }
     } else if (warp < kEpiWarp0 + 4) {
         // ---------------------------------------------------------- epilogue
+        pdl_wait();
         const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
         const int row = quarter * 32 + lane;         // row inside the tile
         const EpiParams e = p.epi;  // a local copy: its fields stay in registers
