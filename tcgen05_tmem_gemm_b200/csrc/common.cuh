@@ -95,8 +95,13 @@ cudaError_t launch_ex(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_
     }
     cfg.attrs = attr;
     cfg.numAttrs = n;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
-    return e != cudaSuccess ? e : cudaGetLastError();
+    // The launch's own result is the return value.  A failed launch also
+    // leaves its error as the thread's last error: consume it, so that it is
+    // not reported again by a later call (the library's or the caller's); an
+    // error someone else left pending is not this launch's and is left alone.
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e != cudaSuccess) cudaGetLastError();
+    return e;
 }
 
 __device__ __forceinline__ float load_elem(const char *p, int dtype) {
