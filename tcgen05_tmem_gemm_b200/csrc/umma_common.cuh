@@ -270,17 +270,12 @@ __device__ __forceinline__ void epilogue_rows_tma(const EpiParams &e, const CUte
         if (ES == 4) {
 #pragma unroll
             for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(v[c]);
+        } else if (bf16_out) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) w[c] = pack2<true>(v[2 * c], v[2 * c + 1]);
         } else {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                if (bf16_out) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * c], v[2 * c + 1]);
-                    w[c] = *reinterpret_cast<uint32_t *>(&h);
-                } else {
-                    __half2 h = __floats2half2_rn(v[2 * c], v[2 * c + 1]);
-                    w[c] = *reinterpret_cast<uint32_t *>(&h);
-                }
-            }
+            for (int c = 0; c < 32; ++c) w[c] = pack2<false>(v[2 * c], v[2 * c + 1]);
         }
         const uint32_t buf = stage + (nblk & 1u) * kEpiBlockBytes;
         if (lane == 0) bulk_wait_read<1>();  // the copy that last read this block is done with it
