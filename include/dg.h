@@ -224,7 +224,7 @@ typedef struct {
     int32_t p_gather;      /* UMMA: the M-side operand is loaded by threads, not TMA */
     int32_t p_mn_major;    /* UMMA: operand layouts in smem (0 K-major, 1 MN-major)  */
     int32_t q_mn_major;
-    int32_t block_m, block_n, block_k;
+    int32_t block_m, block_n, block_k;  /* tile rows, columns, and k per pipeline stage */
     int32_t stages;
     int32_t split_k;
     int32_t grid;          /* CTAs launched                                          */
@@ -261,8 +261,9 @@ dg_status dg_plan(const dg_view *A, const dg_view *B, const dg_view *C,
  * "DeepGEMM: a recalibration of the compute paradigm", §6.1: the chosen
  * configuration is cached per problem).  The variants are the tensor-core
  * tile width (32..256 columns), k splits (1..8, on-chip cluster reduction),
- * CTA pairs with or without the Stream-K tail, the gather-cluster size and
- * the tensor-store epilogue; for the memory-bound GEMV, its k splits.  Each
+ * CTA pairs with or without the Stream-K tail and with one or two 128-byte
+ * k sub-blocks per stage, the gather-cluster size and the tensor-store
+ * epilogue; for the memory-bound GEMV, its k splits.  Each
  * is run `reps` times (1..1000) after a warm-up and timed with CUDA events;
  * the fastest is kept in a process-wide table keyed by the views (shapes,
  * strides, types, pointer alignment), beta == 0, alpha == 0, the device and
@@ -375,13 +376,19 @@ typedef enum {
                                      (their order, and so the last bits, can vary from
                                      run to run); 1: always the cluster reduction in a
                                      fixed order (bit-identical runs)                    */
-    DG_OPT_STREAM_K = 11          /* 1: CTA pairs share the k blocks of the last,
+    DG_OPT_STREAM_K = 11,         /* 1: CTA pairs share the k blocks of the last,
                                      partial wave of tiles out over all pairs (Stream-K,
                                      "DeepGEMM deep dive" §5.2) when a workspace for the
                                      stream is available; 0 (default): the half-width
                                      tail above.  On 4096^3 the tail measured faster on
                                      B200 (BF16 104 against 106 us, E4M3 58 against
                                      63 us); dg_autotune times both per shape           */
+    DG_OPT_PAIR_DEEP_STAGES = 13  /* 1 (default): CTA-pair stages two 128-byte k
+                                     sub-blocks deep (block_k = 256 bytes of K) when an
+                                     operand is MN-major and K is a whole number of such
+                                     stages, so MN-major tiles arrive in half as many,
+                                     twice as tall copies (4096^3 on B200: BF16 103.6 ->
+                                     96.4 us, E4M3 57.7 -> 56.8 us); 0: one sub-block  */
 } dg_option;
 
 dg_status dg_set_option(int option, int64_t value);

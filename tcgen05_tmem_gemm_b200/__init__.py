@@ -33,7 +33,8 @@ ACT = {"none": DG_ACT_NONE, "relu": DG_ACT_RELU, "gelu_tanh": DG_ACT_GELU_TANH}
 
 (DG_OPT_FORCE_KIND, DG_OPT_WAIT_TIMEOUT_MS, DG_OPT_TEST_STALL, DG_OPT_MAX_SPLIT_K, DG_OPT_CTA_PAIR,
  DG_OPT_EARLY_LAUNCH, DG_OPT_TRACE, DG_OPT_EPI_TMA, DG_OPT_GATHER_CLUSTER,
- DG_OPT_PAIR_TAIL, DG_OPT_STREAM_K, DG_OPT_DETERMINISTIC) = 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12
+ DG_OPT_PAIR_TAIL, DG_OPT_STREAM_K, DG_OPT_DETERMINISTIC,
+ DG_OPT_PAIR_DEEP_STAGES) = 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13
 
 
 class dg_view(ctypes.Structure):

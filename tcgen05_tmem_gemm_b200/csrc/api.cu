@@ -38,6 +38,7 @@ std::atomic<uint64_t> g_trace{0};
 std::atomic<int> g_epi_tma{1};
 std::atomic<int> g_gather_cluster{1};
 std::atomic<int> g_pair_tail{1};
+std::atomic<int> g_pair_deep{1};  // CTA-pair stages two k sub-blocks deep where they apply
 std::atomic<int> g_stream_k{0};
 std::atomic<int> g_deterministic{0};
 std::atomic<uint32_t> g_epoch{1};  // bumped by every option change: cached launches go stale
@@ -282,8 +283,9 @@ struct Override {
     int epi_tma = -1;    // tensor-store epilogue: 0 / 1
     int stages = 0;      // pipeline depth (at most what shared memory holds)
     int gemv_split = 0;  // GEMV_N k splits
+    int ksub = 0;        // CTA-pair stage depth in 128-byte k sub-blocks: 1 or 2
     bool any() const {
-        return bn || split || pair >= 0 || sk >= 0 || gcl || epi_tma >= 0 || stages || gemv_split;
+        return bn || split || pair >= 0 || sk >= 0 || gcl || epi_tma >= 0 || stages || gemv_split || ksub;
     }
 };
 
@@ -443,8 +445,21 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
         if (ov->epi_tma && !epi_ok) return false;
         epi_tma = ov->epi_tma != 0;
     }
+    // CTA pairs: stages two 128-byte k sub-blocks deep when an operand is
+    // MN-major (its copies come in half as many boxes, each twice as tall;
+    // the copy engine has a fixed cost per box) and K is a whole number of
+    // such stages; at least three of them must fit.  With B MN-major, a
+    // 16-bit tile pair needs six boxes per two 128-byte k sub-blocks in
+    // one-deep stages and four in two-deep ones, an E4M3 pair four and three
+    // (4096^3 on B200: BF16 103.6 -> 96.4 us, E4M3 57.7 -> 56.8 us)
+    const bool deep_ok = pair && (p_mn || q_mn) && K % (2 * bk) == 0 && umma_pair_max_stages(bn, epi_tma, 2) >= 3;
+    int ksub = (deep_ok && g_pair_deep.load() != 0) ? 2 : 1;
+    if (ov->ksub) {
+        if (ov->ksub != 1 && (ov->ksub != 2 || !deep_ok)) return false;
+        ksub = ov->ksub;
+    }
     const int max_stages =
-        pair ? umma_pair_max_stages(bn, epi_tma) : umma_max_stages(bn, !p_tma, epi_tma, (int)split);
+        pair ? umma_pair_max_stages(bn, epi_tma, ksub) : umma_max_stages(bn, !p_tma, epi_tma, (int)split);
     int stages = max_stages;
     if (ov->stages) {
         if (ov->stages < 2 || ov->stages > max_stages) return false;
@@ -485,7 +500,7 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
     in.q_mn_major = q_mn;
     in.block_m = 128;
     in.block_n = bn;
-    in.block_k = bk;
+    in.block_k = bk * ksub;  // k per stage
     in.stages = stages;
     in.split_k = (int32_t)split;
     in.grid = (int32_t)(split > 1 ? units2 : std::min<int64_t>(units2, num_sms));  // split: one unit per CTA
@@ -514,7 +529,7 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
         // out over every pair ("DeepGEMM deep dive", §5.2), when each of those
         // tiles is split among at most kMaxFix + 1 pairs and every pair gets
         // at least one k block
-        const int64_t kb_all = tail * kb_total;
+        const int64_t kb_all = tail * ((K + bk * ksub - 1) / (bk * ksub));  // stages of the tail's tiles
         const bool sk_ok = pair_units > ncl && tail > 0 && 7 * tail >= ncl && kb_all >= ncl;
         const bool sk = allow_sk && sk_ok && (ov->sk >= 0 ? ov->sk != 0 : g_stream_k.load() != 0);
         if (ov->sk == 1 && allow_sk && !sk_ok) return false;
@@ -526,7 +541,7 @@ bool umma_plan(const Views &v, int64_t M, int64_t N, int64_t K, float beta, int 
         return false;
     }
     pl->fp8 = (dt == DG_E4M3);
-    pl->smem = pair ? umma_pair_smem_bytes(bn, stages, epi_tma)
+    pl->smem = pair ? umma_pair_smem_bytes(bn, stages, epi_tma, ksub)
                     : umma_smem_bytes(bn, stages, !p_tma, epi_tma, in.split_reduce_add ? 1 : (int)split);
     return true;
 }
@@ -827,7 +842,11 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         const bool swap = in.swap_ab != 0;
         const int dt = v.A->dtype;
         const int es = elem_size(dt);
-        const int bk = in.block_k, bn = in.block_n;
+        const int bk = 128 / es, bn = in.block_n;
+        // a CTA-pair stage may be two 128-byte k sub-blocks deep (block_k = 2 * bk)
+        const int ksub = in.cta_pair ? in.block_k / bk : 1;
+        if (ksub < 1 || ksub > 2 || ksub * bk != in.block_k) return DG_ERR_UNSUPPORTED;
+        const int mn_rows = ksub * bk;  // rows of k in an MN-major box
         const int64_t Mi = swap ? in.N : in.M, Nj = swap ? in.M : in.N;
         CUtensorMap &tp = rec->t0, &tq = rec->t1;
         // P(i, k): A (no swap) or B^T; Q(k, j): B (no swap) or A^T
@@ -838,14 +857,14 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         const Axis &p_i = swap ? pi.col : pi.row, &p_k = swap ? pi.row : pi.col;
         const Axis &q_k = swap ? qi.col : qi.row, &q_j = swap ? qi.row : qi.col;
         if (!in.p_gather) {
-            const bool ok = in.p_mn_major ? encode_2d(&tp, dt, Pv->ptr, Mi, in.K, axis_stride(p_k), bk)
+            const bool ok = in.p_mn_major ? encode_2d(&tp, dt, Pv->ptr, Mi, in.K, axis_stride(p_k), mn_rows)
                                           : encode_2d(&tp, dt, Pv->ptr, in.K, Mi, axis_stride(p_i), 128);
             if (!ok) return DG_ERR_UNSUPPORTED;
         }
         {
             // a CTA of a pair loads half of a tile's columns, as boxes of bn/4 rows when K-major
             const int q_rows = in.cta_pair ? bn / 4 : bn;
-            const bool ok = in.q_mn_major ? encode_2d(&tq, dt, Qv->ptr, Nj, in.K, axis_stride(q_k), bk)
+            const bool ok = in.q_mn_major ? encode_2d(&tq, dt, Qv->ptr, Nj, in.K, axis_stride(q_k), mn_rows)
                                           : encode_2d(&tq, dt, Qv->ptr, in.K, Nj, axis_stride(q_j), q_rows);
             if (!ok) return DG_ERR_UNSUPPORTED;
         }
@@ -865,7 +884,8 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
         p.tiles_i = (int32_t)((Mi + in.block_m - 1) / in.block_m);
         p.tiles_j = (int32_t)((Nj + bn - 1) / bn);
         p.split_k = in.split_k;
-        p.kb_total = (int32_t)((in.K + bk - 1) / bk);
+        p.ksub = ksub;
+        p.kb_total = (int32_t)((in.K + ksub * bk - 1) / (ksub * bk));  // stages along k
         p.kb_per_split = (p.kb_total + p.split_k - 1) / p.split_k;
         p.num_units = p.tiles_i * p.tiles_j * p.split_k;
         p.p_mn_major = in.p_mn_major;
@@ -1031,14 +1051,18 @@ std::vector<Override> tune_candidates(const dg_plan_info &base) {
                     for (int gcl : {1, 2, 4}) {
                         if (gcl > 1 && (!base.p_gather || split > 1 || pair)) continue;
                         for (int epi : {0, 1}) {
-                            Override o;
-                            o.bn = bn;
-                            o.split = split;
-                            o.pair = pair;
-                            o.sk = pair ? sk : -1;
-                            o.gcl = base.p_gather ? gcl : 0;
-                            o.epi_tma = epi;
-                            c.push_back(o);
+                            for (int ks : {1, 2}) {
+                                if (ks == 2 && !pair) continue;
+                                Override o;
+                                o.bn = bn;
+                                o.split = split;
+                                o.pair = pair;
+                                o.sk = pair ? sk : -1;
+                                o.gcl = base.p_gather ? gcl : 0;
+                                o.epi_tma = epi;
+                                o.ksub = pair ? ks : 0;
+                                c.push_back(o);
+                            }
                         }
                     }
                 }
@@ -1458,6 +1482,10 @@ dg_status dg_set_option(int option, int64_t value) {
     case DG_OPT_DETERMINISTIC:
         if (value < 0 || value > 1) return DG_ERR_VALUE;
         g_deterministic.store((int)value);
+        return DG_OK;
+    case DG_OPT_PAIR_DEEP_STAGES:
+        if (value < 0 || value > 1) return DG_ERR_VALUE;
+        g_pair_deep.store((int)value);
         return DG_OK;
     default: return DG_ERR_VALUE;
     }

@@ -103,6 +103,7 @@ struct UmmaParams {
     int32_t Mi, Nj, K;       // tensor-core problem: D[Mi x Nj] = P[Mi x K] Q[K x Nj]
     int32_t bn;              // tile width along j (64, 128 or 256)
     int32_t bk;              // tile depth (128 bytes of K)
+    int32_t ksub;            // CTA pairs: k sub-blocks of bk per stage (1 or 2); a stage is ksub * bk deep
     int32_t stages;
     int32_t tiles_i, tiles_j, split_k, kb_per_split, kb_total;
     int32_t num_units;       // tiles_i * tiles_j * split_k
@@ -182,8 +183,8 @@ int umma_max_stages(int bn, bool gather, bool epi_tma, int split);
 uint32_t umma_split_out_bytes(int bn, int split);  // ring bytes a split-K partial is staged in
 cudaError_t launch_umma_pair(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq,
                              const CUtensorMap *tc, bool fp8, int grid, size_t smem, cudaStream_t s);
-size_t umma_pair_smem_bytes(int bn, int stages, bool epi_tma);
-int umma_pair_max_stages(int bn, bool epi_tma);
+size_t umma_pair_smem_bytes(int bn, int stages, bool epi_tma, int ksub);
+int umma_pair_max_stages(int bn, bool epi_tma, int ksub);
 
 cudaError_t launch_gemv_n(const GemvParams &p, const CUtensorMap *tmap_w, cudaStream_t s, int *grid_out);
 size_t gemv_n_smem_bytes(int r_inst, int kper);

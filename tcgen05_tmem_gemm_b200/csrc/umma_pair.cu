@@ -30,14 +30,24 @@ namespace {
 constexpr int kHalfM = 128;   // rows of P (and TMEM lanes) per CTA
 constexpr int kRowBytes = 128;
 
+// A stage holds ksub k sub-blocks of 128 bytes per row (ksub = 1 or 2).  Its
+// P part (128 rows) and Q part (bn/2 columns) are each laid out as whole
+// 128-byte-swizzled boxes: K-major, one box of 128 rows (P) or bn/2 rows in
+// boxes of bn/4 (Q) per sub-block, the sub-blocks one after the other;
+// MN-major, one box of ksub * bk rows of k per 128-byte column group, the
+// groups one after the other.  A deeper stage loads the same bytes in half as
+// many boxes when Q is MN-major (the copy engine has a fixed cost per box).
 struct PairLayout {
+    uint32_t a_sub, b_sub;  // bytes of one k sub-block of P and of Q
     uint32_t a_bytes, b_bytes, stage_bytes, epi_off, bar_off, aux_off, total;
 };
 
-__host__ __device__ inline PairLayout pair_layout(int bn, int stages, bool epi_tma) {
+__host__ __device__ inline PairLayout pair_layout(int bn, int stages, bool epi_tma, int ksub) {
     PairLayout L;
-    L.a_bytes = kHalfM * kRowBytes;
-    L.b_bytes = (uint32_t)(bn / 2) * kRowBytes;
+    L.a_sub = kHalfM * kRowBytes;
+    L.b_sub = (uint32_t)(bn / 2) * kRowBytes;
+    L.a_bytes = (uint32_t)ksub * L.a_sub;
+    L.b_bytes = (uint32_t)ksub * L.b_sub;
     L.stage_bytes = L.a_bytes + L.b_bytes;  // a multiple of 1024: bn is a multiple of 16
     L.epi_off = L.stage_bytes * stages;
     L.bar_off = L.epi_off + (epi_tma ? kEpiStoreBytes : 0u);
@@ -170,7 +180,7 @@ __device__ __forceinline__ float *sk_slot(const UmmaParams &p, int q, uint32_t r
     return p.sk_part + (size_t)(q * 2 + (int)rank) * (size_t)(kHalfM * p.bn);
 }
 
-template <bool FP8>
+template <bool FP8, int KSUB>
 __global__ void __launch_bounds__(192, 1)
     umma_pair_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_c, const UmmaParams p) {
@@ -183,7 +193,7 @@ __global__ void __launch_bounds__(192, 1)
     if (p.pdl == 1) pdl_release();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const PairLayout L = pair_layout(p.bn, p.stages, p.epi_tma != 0);
+    const PairLayout L = pair_layout(p.bn, p.stages, p.epi_tma != 0, KSUB);
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_full = sbase + L.bar_off;
     const uint32_t bar_empty = bar_full + 8 * p.stages;
@@ -246,7 +256,9 @@ __global__ void __launch_bounds__(192, 1)
             // and stage and phase advance without division
             const int stages = p.stages, kb_total = p.kb_total, num_units = p.num_units;
             const bool stall = p.stall_loader == 1, p_mn = p.p_mn_major != 0, q_mn = p.q_mn_major != 0;
-            const uint32_t stage_bytes = L.stage_bytes, a_bytes = L.a_bytes;
+            const uint32_t stage_bytes = L.stage_bytes, a_bytes = L.a_bytes, a_sub = L.a_sub, b_sub = L.b_sub;
+            constexpr int ksub = KSUB;
+            const uint32_t mn_box_bytes = (uint32_t)(ksub * bk) * kRowBytes;  // an MN-major box: ksub * bk rows
             (void)num_units;
             (void)kb_total;
             int it = 0, s = 0;
@@ -256,7 +268,7 @@ __global__ void __launch_bounds__(192, 1)
                 const int i0 = pw.ti * 2 * kHalfM + (int)rank * kHalfM;
                 const int cw = pw.w / 2;  // this CTA's columns of the unit
                 const int j0 = pw.j0 + (int)rank * cw;
-                const uint32_t tx = 2u * (a_bytes + (uint32_t)cw * kRowBytes);  // both CTAs' bytes
+                const uint32_t tx = 2u * (a_bytes + (uint32_t)(ksub * cw) * kRowBytes);  // both CTAs' bytes
                 bool ok = true;
                 for (int kb = pw.kb0; kb < pw.kb1; ++kb, ++it) {
                     if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) { ok = false; break; }
@@ -265,21 +277,23 @@ __global__ void __launch_bounds__(192, 1)
                         if (leader) mbar_arrive_expect_tx(bar_full + 8 * s, tx);
                         const uint32_t as = sbase + s * stage_bytes;
                         const uint32_t bs = as + a_bytes;
-                        const int k0 = kb * bk;
+                        const int k0 = kb * ksub * bk;
                         if (p_mn) {
                             for (int c = 0; c < kHalfM / per; ++c)
-                                tma_load_2d_pair(as + c * bk * 128, &tmap_p, full_c, i0 + c * per, k0);
+                                tma_load_2d_pair(as + c * mn_box_bytes, &tmap_p, full_c, i0 + c * per, k0);
                         } else {
-                            tma_load_2d_pair(as, &tmap_p, full_c, k0, i0);
+                            for (int j = 0; j < ksub; ++j)
+                                tma_load_2d_pair(as + j * a_sub, &tmap_p, full_c, k0 + j * bk, i0);
                         }
                         if (q_mn) {
                             for (int c = 0; c < cw / per; ++c)
-                                tma_load_2d_pair(bs + c * bk * 128, &tmap_q, full_c, j0 + c * per, k0);
+                                tma_load_2d_pair(bs + c * mn_box_bytes, &tmap_q, full_c, j0 + c * per, k0);
                         } else {
                             // boxes of bn/4 rows: two per CTA for a whole tile, one for a half
-                            for (int c = 0; c < cw / (half_bn / 2); ++c)
-                                tma_load_2d_pair(bs + c * (half_bn / 2) * kRowBytes, &tmap_q, full_c, k0,
-                                                 j0 + c * (half_bn / 2));
+                            for (int j = 0; j < ksub; ++j)
+                                for (int c = 0; c < cw / (half_bn / 2); ++c)
+                                    tma_load_2d_pair(bs + j * b_sub + c * (half_bn / 2) * kRowBytes, &tmap_q, full_c,
+                                                     k0 + j * bk, j0 + c * (half_bn / 2));
                         }
                     }
                     if (++s == stages) {
@@ -304,10 +318,16 @@ __global__ void __launch_bounds__(192, 1)
             const int stages = p.stages, kb_total = p.kb_total, num_units = p.num_units;
             const int full_units = p.full_units, bn = p.bn;
             const uint32_t idesc_full = p.idesc, idesc_half = p.idesc_half, stage_bytes = L.stage_bytes;
-            const uint32_t p_lbo = p.p_mn_major ? (uint32_t)(bk * 128) : 16u;
-            const uint32_t q_lbo = p.q_mn_major ? (uint32_t)(bk * 128) : 16u;
+            constexpr int ksub = KSUB;
+            // MN-major: the next 128-byte column group is one box (ksub * bk rows) further, and
+            // k advances by rows of the box; K-major: k advances within the 128-byte rows of a
+            // sub-block, and the next sub-block follows the previous one
+            const uint32_t p_lbo = p.p_mn_major ? (uint32_t)(ksub * bk * 128) : 16u;
+            const uint32_t q_lbo = p.q_mn_major ? (uint32_t)(ksub * bk * 128) : 16u;
             const uint32_t p_kstep = p.p_mn_major ? kUmmaK * 128 : kUmmaK * es;
             const uint32_t q_kstep = p.q_mn_major ? kUmmaK * 128 : kUmmaK * es;
+            const uint32_t p_sstep = p.p_mn_major ? (uint32_t)(kRowBytes / (kUmmaK * es)) * p_kstep : L.a_sub;
+            const uint32_t q_sstep = p.q_mn_major ? (uint32_t)(kRowBytes / (kUmmaK * es)) * q_kstep : L.b_sub;
             // descriptors of stage 0; a stage's differ only in the start address
             // field (address >> 4, below 2^14 for any shared-memory address)
             const uint64_t da0 = make_sw128_desc(sbase, p_lbo, 1024);
@@ -332,12 +352,17 @@ __global__ void __launch_bounds__(192, 1)
                     tc_fence_after();
                     const uint64_t soff = (uint64_t)((s * stage_bytes) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < kRowBytes / (kUmmaK * es); ++kk) {
-                        const uint64_t da = da0 + soff + (uint64_t)((kk * p_kstep) >> 4);
-                        const uint64_t db = db0 + soff + (uint64_t)((kk * q_kstep) >> 4);
-                        const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
-                        if (FP8) umma_f8_pair(d_tmem, da, db, idesc, acc);
-                        else umma_f16_pair(d_tmem, da, db, idesc, acc);
+                    for (int sub = 0; sub < ksub; ++sub) {
+                        const uint64_t sa = soff + (uint64_t)((sub * p_sstep) >> 4);
+                        const uint64_t sb = soff + (uint64_t)((sub * q_sstep) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < kRowBytes / (kUmmaK * es); ++kk) {
+                            const uint64_t da = da0 + sa + (uint64_t)((kk * p_kstep) >> 4);
+                            const uint64_t db = db0 + sb + (uint64_t)((kk * q_kstep) >> 4);
+                            const uint32_t acc = (kb > kb0 || sub > 0 || kk > 0) ? 1u : 0u;
+                            if (FP8) umma_f8_pair(d_tmem, da, db, idesc, acc);
+                            else umma_f16_pair(d_tmem, da, db, idesc, acc);
+                        }
                     }
                     tc_commit_pair_mc(bar_empty + 8 * s, 0x3);  // the stage is free in both CTAs
                     if (++s == stages) {
@@ -485,20 +510,25 @@ __global__ void __launch_bounds__(192, 1)
 
 }  // namespace
 
-size_t umma_pair_smem_bytes(int bn, int stages, bool epi_tma) { return pair_layout(bn, stages, epi_tma).total; }
+size_t umma_pair_smem_bytes(int bn, int stages, bool epi_tma, int ksub) {
+    return pair_layout(bn, stages, epi_tma, ksub).total;
+}
 
-int umma_pair_max_stages(int bn, bool epi_tma) {
+int umma_pair_max_stages(int bn, bool epi_tma, int ksub) {
     int s = 2;
-    while (s < 12 && pair_layout(bn, s + 1, epi_tma).total <= 227 * 1024) ++s;
+    while (s < 12 && pair_layout(bn, s + 1, epi_tma, ksub).total <= 227 * 1024) ++s;
     return s;
 }
 
 cudaError_t launch_umma_pair(const UmmaParams &p, const CUtensorMap *tp, const CUtensorMap *tq,
                              const CUtensorMap *tc, bool fp8, int grid, size_t smem, cudaStream_t s) {
     void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const UmmaParams);
-    kern = fp8 ? umma_pair_kernel<true> : umma_pair_kernel<false>;
-    static SmemLimit s_limit[2];
-    const cudaError_t e = s_limit[fp8 ? 1 : 0].ensure(kern, smem);
+    if (p.ksub != 1 && p.ksub != 2) return cudaErrorInvalidValue;
+    const bool deep = p.ksub == 2;
+    kern = fp8 ? (deep ? umma_pair_kernel<true, 2> : umma_pair_kernel<true, 1>)
+               : (deep ? umma_pair_kernel<false, 2> : umma_pair_kernel<false, 1>);
+    static SmemLimit s_limit[4];
+    const cudaError_t e = s_limit[(fp8 ? 2 : 0) + (deep ? 1 : 0)].ensure(kern, smem);
     if (e != cudaSuccess) return e;
     return launch_ex(kern, dim3(grid), dim3(192), smem, s, dim3(2, 1, 1), p.pdl, *tp, *tq, *tc, p);
 }

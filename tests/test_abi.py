@@ -149,6 +149,27 @@ def test_plan_square_bf16_and_fp8():
     assert pl["kind_name"] == "umma" and pl["block_k"] == 128 and pl["q_mn_major"] == 1
 
 
+def test_plan_pair_deep_stages():
+    # CTA pairs with B MN-major (row-major [K, N]) and K a multiple of 128:
+    # stages two 64-deep k sub-blocks deep, three of them (64 KB each)
+    pl = plan_of("square_bf16", M=4096, N=4096, K=128)
+    assert pl["cta_pair"] == 1 and pl["q_mn_major"] == 1
+    assert pl["block_k"] == 128 and pl["stages"] == 3
+    dg.dg_set_option(dg.DG_OPT_PAIR_DEEP_STAGES, 0)
+    try:
+        pl = plan_of("square_bf16", M=4096, N=4096, K=128)
+        assert pl["block_k"] == 64 and pl["stages"] == 6
+    finally:
+        dg.dg_set_option(dg.DG_OPT_PAIR_DEEP_STAGES, 1)
+    # K not a whole number of deep stages: one sub-block per stage
+    pl = plan_of("square_bf16", M=4096, N=4096, K=192)
+    assert pl["cta_pair"] == 1 and pl["block_k"] == 64
+    pl = plan_of("square_e4m3", M=4096, N=4096, K=256)
+    assert pl["cta_pair"] == 1 and pl["block_k"] == 256 and pl["stages"] == 3
+    with pytest.raises(dg.DgError):
+        dg.dg_set_option(dg.DG_OPT_PAIR_DEEP_STAGES, 2)
+
+
 def test_plan_thin_split_reduce_add():
     # beta = 1 with FP32 C: the k splits add into C unless deterministic
     p = meta_problem("thin")
@@ -392,7 +413,11 @@ def _check_plan(p, dt, M, N, K, alpha):
         es = ES[dt]
         assert dt in ("f16", "bf16", "e4m3")
         bn, split, grid = p["block_n"], p["split_k"], p["grid"]
-        assert p["block_k"] == 128 // es
+        # k per stage: one 128-byte sub-block, or two for CTA pairs with an
+        # MN-major operand and K a whole number of such stages
+        if p["block_k"] != 128 // es:
+            assert p["cta_pair"] and p["block_k"] == 256 // es and K % p["block_k"] == 0
+            assert p["p_mn_major"] or p["q_mn_major"]
         assert 16 <= bn <= 256 and bn % 16 == 0         # N of a 128-row tcgen05.mma
         if p["q_mn_major"]:
             assert bn % (128 // es) == 0                 # whole 128-byte boxes

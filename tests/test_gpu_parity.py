@@ -34,6 +34,7 @@ def _reset_options():
     dg.dg_set_option(dg.DG_OPT_GATHER_CLUSTER, 1)
     dg.dg_set_option(dg.DG_OPT_PAIR_TAIL, 1)
     dg.dg_set_option(dg.DG_OPT_DETERMINISTIC, 0)
+    dg.dg_set_option(dg.DG_OPT_PAIR_DEEP_STAGES, 1)
 
 
 def expect_kind(p, kind, **fields):
@@ -170,6 +171,51 @@ def test_umma_cta_pair_fp8():
                   1.0, 0.0, sa, sb)
     expect_kind(p, "umma", cta_pair=1)
     check_full(p)
+
+
+def _pair_deep_problem(case):
+    g = torch.Generator().manual_seed(sum(map(ord, case)))
+    if case == "e4m3_b_mn":
+        # tiles 256 wide (a CTA's half of an MN-major E4M3 tile is one 128-byte box)
+        M, N, K = 2560, 1024, 512
+        qa, sa = W.quantise_e4m3(W.normal((M, K), g), dim=1)
+        qb, sb = W.quantise_e4m3(W.normal((K, N), g), dim=0)
+        return W.Problem(case, W.row_major(qa, "e4m3"), W.row_major(qb, "e4m3"), W.empty_out(M, N, "bf16"),
+                         1.0, 0.0, sa, sb), 1
+    ta = case in ("bf16_a_mn", "bf16_a_mn_b_k")
+    tb = case == "bf16_a_mn_b_k"
+    M, N, K = {"ragged": (300, 520, 256), "half_tail": (2560, 2048, 256)}.get(case, (512, 512, 384))
+    a = W.cast(W.normal((K, M) if ta else (M, K), g), "bf16")
+    b = W.cast(W.normal((N, K) if tb else (K, N), g), "bf16")
+    A = W.transposed(a, "bf16") if ta else W.row_major(a, "bf16")
+    B = W.transposed(b, "bf16") if tb else W.row_major(b, "bf16")
+    if case == "ragged":
+        c = W.uniform((M, N), g)
+        return W.Problem(case, A, B, W.row_major(c.to(torch.bfloat16).contiguous(), "bf16"), 0.75, 0.5), 2
+    return W.Problem(case, A, B, W.empty_out(M, N, "f32")), 2
+
+
+@pytest.mark.parametrize("case", ["bf16_b_mn", "bf16_a_mn", "bf16_a_mn_b_k", "e4m3_b_mn", "ragged", "half_tail"])
+def test_pair_deep_stages_match_shallow(case):
+    # CTA-pair stages two 128-byte k sub-blocks deep (taller MN-major boxes)
+    # issue the same MMAs in the same k order as stages one sub-block deep,
+    # so the results agree bit for bit; each is also checked against the oracle
+    p, es = _pair_deep_problem(case)
+    if case == "half_tail":
+        if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+            pytest.skip("the tail size is worked out for 148 SMs")
+    else:
+        dg.dg_set_option(dg.DG_OPT_CTA_PAIR, 2)
+        dg.dg_set_option(dg.DG_OPT_MAX_SPLIT_K, 1)
+    outs = []
+    for deep in (1, 0):
+        dg.dg_set_option(dg.DG_OPT_PAIR_DEEP_STAGES, deep)
+        pl = expect_kind(p, "umma", cta_pair=1, block_k=(2 if deep else 1) * 128 // es)
+        if case == "half_tail":
+            assert pl["pair_half_tiles"] == 6
+        check_full(p)
+        outs.append(c_matrix(run(p.to("cuda"))))
+    assert np.array_equal(outs[0], outs[1])
 
 
 def test_thin_beta_one_split_k():

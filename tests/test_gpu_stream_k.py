@@ -28,6 +28,7 @@ def _reset_options():
     dg.dg_set_option(dg.DG_OPT_TEST_STALL, 0)
     dg.dg_set_option(dg.DG_OPT_WAIT_TIMEOUT_MS, 2000)
     dg.dg_set_option(dg.DG_OPT_PAIR_TAIL, 1)
+    dg.dg_set_option(dg.DG_OPT_PAIR_DEEP_STAGES, 1)
 
 
 def _needs_148():
@@ -47,10 +48,12 @@ def _bf16(M, N, K, seed, tb=False, out="bf16", beta=0.0):
 @pytest.mark.parametrize("tb", [False, True])
 def test_stream_k_matches_oracle_and_is_deterministic(tb):
     _needs_148()
-    # 16 x 12 = 192 tiles on 74 pairs: 148 whole, 44 shared out (176 k blocks)
+    # 16 x 12 = 192 tiles on 74 pairs: 148 whole, 44 shared out (176 k blocks
+    # of 64, or 88 stages two k blocks deep when B is MN-major)
     p = _bf16(4096, 3072, 256, 31 + int(tb), tb)
     pl = plan(p.to("cuda"))
     assert pl["cta_pair"] == 1 and pl["stream_k_tiles"] == 44 and pl["pair_half_tiles"] == 0, pl
+    assert pl["block_k"] == (64 if tb else 128), pl
     check_full(p)
     a = c_matrix(run(p.to("cuda")))
     b = c_matrix(run(p.to("cuda")))
@@ -65,7 +68,9 @@ def test_stream_k_matches_oracle_and_is_deterministic(tb):
 def test_stream_k_many_pairs_per_tile():
     _needs_148()
     # 17 x 5 = 85 tiles: 11 shared out as 88 k blocks over 74 pairs, so a tile's
-    # 8 k blocks are split among up to 7 pairs (the owner adds up to 6 partials)
+    # 8 k blocks are split among up to 7 pairs (the owner adds up to 6 partials);
+    # stages one k block deep (two-deep stages would leave 44 for 74 pairs)
+    dg.dg_set_option(dg.DG_OPT_PAIR_DEEP_STAGES, 0)
     p = _bf16(4352, 1280, 512, 33, out="f32")
     pl = plan(p.to("cuda"))
     assert pl["stream_k_tiles"] == 11, pl
@@ -127,7 +132,9 @@ def test_stream_k_graph_replay_and_second_stream():
 def test_stream_k_timeout_then_correct():
     _needs_148()
     # a launch whose waits run out leaves flags of its own tag behind; the
-    # next launch's tag differs, so it is correct
+    # next launch's tag differs, so it is correct (stages one k block deep:
+    # K = 128 in two-deep stages would leave 44 stages for 74 pairs)
+    dg.dg_set_option(dg.DG_OPT_PAIR_DEEP_STAGES, 0)
     p = _bf16(4096, 3072, 128, 38)
     dg.dg_set_option(dg.DG_OPT_WAIT_TIMEOUT_MS, 300)
     dg.dg_set_option(dg.DG_OPT_TEST_STALL, 1)
