@@ -1007,6 +1007,20 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                               i0 % 4 == 0 && cj % 16 == 0 && (reinterpret_cast<uintptr_t>(cbase) & 15) == 0;
             constexpr int kB4 = 4;  // four-row groups per thread per batch (vector path)
             const int g_rows = vec4 ? rs / 4 : 1;
+            // vector path: the four outputs (i .. i+3, j) of a group are
+            // mul[k] * sum + beta * C + add[k]: mul = alpha * s_i * s_j, add = the
+            // bias.  Their factors are loaded with the group's C, before any
+            // store (a load after a store through C's pointer would wait for it).
+            auto load_factors = [&](int i, int j, float (&mul)[4], float (&add)[4]) {
+                const float sj = scale_j ? scale_j[j] : 1.f;
+                const float bj = (fused && bias_j) ? bias_j[j] : 0.f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const bool in = i + k < Mi;
+                    mul[k] = alpha * (scale_i && in ? scale_i[i + k] : 1.f) * sj;
+                    add[k] = ((fused && bias_i && in) ? bias_i[i + k] : 0.f) + bj;
+                }
+            };
             // vector path: C of the first batch is loaded while the slices travel
             float4 cfirst[kB4];
 #pragma unroll
@@ -1043,6 +1057,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                     int gr = t % g_rows, gc = t / g_rows;
                     for (int base = t; base < total; base += 128 * kB) {
                         float4 cin[kB], acc[kB];
+                        float mul[kB][4], add[kB][4];
                         int rr[kB], cc[kB];
 #pragma unroll
                         for (int b = 0; b < kB; ++b) {
@@ -1059,6 +1074,9 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                             const int i = i0 + r, j = jt + c;
                             acc[b] = make_float4(0.f, 0.f, 0.f, 0.f);
                             cin[b] = acc[b];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) mul[b][k] = add[b][k] = 0.f;
+                            if (g < total && j < Nj && i < Mi) load_factors(i, j, mul[b], add[b]);
                             if (g < total && j < Nj && i + 3 < Mi) {
                                 if (beta != 0.f)
                                     cin[b] = base == t ? cfirst[b]
@@ -1083,20 +1101,14 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                             const int r = rr[b], c = cc[b];
                             const int i = i0 + r, j = jt + c;
                             if (!(g < total && j < Nj && i < Mi)) continue;
-                            const float sj = scale_j ? scale_j[j] : 1.f;
                             const float a4[4] = {acc[b].x, acc[b].y, acc[b].z, acc[b].w};
                             const float c4[4] = {cin[b].x, cin[b].y, cin[b].z, cin[b].w};
                             float o[4];
 #pragma unroll
                             for (int k = 0; k < 4; ++k) {
-                                const float asi = alpha * (scale_i && i + k < Mi ? scale_i[i + k] : 1.f);
-                                o[k] = (asi * sj) * a4[k];
+                                o[k] = mul[b][k] * a4[k];
                                 if (beta != 0.f) o[k] = fmaf(beta, c4[k], o[k]);
-                                if (fused) {
-                                    if (bias_i && i + k < Mi) o[k] += bias_i[i + k];
-                                    if (bias_j) o[k] += bias_j[j];
-                                    o[k] = act_apply(act, o[k], cdt != DG_F32);
-                                }
+                                if (fused) o[k] = act_apply(act, o[k] + add[b][k], cdt != DG_F32);
                             }
                             char *dstc = cbase + (int64_t)i * 4 + (int64_t)j * cj;
                             if (i + 3 < Mi) {
@@ -1111,14 +1123,9 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
 #pragma unroll
                                     for (int q = 0; q < kMaxSplit; ++q)
                                         if (q < S) a += ld_shared_f32(src[q] + off);
-                                    const float asi = alpha * (scale_i ? scale_i[i + k] : 1.f);
-                                    float val = (asi * sj) * a;
+                                    float val = mul[b][k] * a;
                                     if (beta != 0.f) val = fmaf(beta, load_elem(dstc + k * 4, cdt), val);
-                                    if (fused) {
-                                        if (bias_i) val += bias_i[i + k];
-                                        if (bias_j) val += bias_j[j];
-                                        val = act_apply(act, val, cdt != DG_F32);
-                                    }
+                                    if (fused) val = act_apply(act, val + add[b][k], cdt != DG_F32);
                                     store_elem(dstc + k * 4, cdt, val);
                                 }
                             }
