@@ -43,6 +43,7 @@
 #pragma once
 
 #include <atomic>
+#include <type_traits>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -1095,6 +1096,11 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                                 }
                             }
                         }
+                        // the activation is picked once per batch: this code runs once per
+                        // CTA, so its instruction footprint, more than its arithmetic, sets
+                        // its time (C is FP32 here: the accurate tanh)
+                        auto finish = [&](auto act_c) {
+                            constexpr int kAct = decltype(act_c)::value;
 #pragma unroll
                         for (int b = 0; b < kB; ++b) {
                             const int g = base + b * 128;
@@ -1108,7 +1114,7 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                             for (int k = 0; k < 4; ++k) {
                                 o[k] = mul[b][k] * a4[k];
                                 if (beta != 0.f) o[k] = fmaf(beta, c4[k], o[k]);
-                                if (fused) o[k] = act_apply(act, o[k] + add[b][k], cdt != DG_F32);
+                                if (fused) o[k] = act_fn<kAct, false>(o[k] + add[b][k]);
                             }
                             char *dstc = cbase + (int64_t)i * 4 + (int64_t)j * cj;
                             if (i + 3 < Mi) {
@@ -1125,11 +1131,15 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                                         if (q < S) a += ld_shared_f32(src[q] + off);
                                     float val = mul[b][k] * a;
                                     if (beta != 0.f) val = fmaf(beta, load_elem(dstc + k * 4, cdt), val);
-                                    if (fused) val = act_apply(act, val + add[b][k], cdt != DG_F32);
+                                    if (fused) val = act_fn<kAct, false>(val + add[b][k]);
                                     store_elem(dstc + k * 4, cdt, val);
                                 }
                             }
                         }
+                        };
+                        if (act == DG_ACT_RELU) finish(std::integral_constant<int, DG_ACT_RELU>{});
+                        else if (act == DG_ACT_GELU_TANH) finish(std::integral_constant<int, DG_ACT_GELU_TANH>{});
+                        else finish(std::integral_constant<int, DG_ACT_NONE>{});
                     }
                 } else {
                     // any C layout: element by element; consecutive threads take
