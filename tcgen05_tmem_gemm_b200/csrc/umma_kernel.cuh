@@ -1182,19 +1182,32 @@ __global__ void __launch_bounds__(GATHER ? 448 : 192, 1)
                                 if (c >= bn) { c -= bn; ++r; }
                             }
                         }
+                        // the activation and C's type are picked once per batch (a smaller
+                        // instruction footprint for this once-per-CTA code; C is never E4M3)
+                        auto finish = [&](auto act_c, auto cd_c) {
+                            constexpr int kAct = decltype(act_c)::value, kCd = decltype(cd_c)::value;
 #pragma unroll
-                        for (int b = 0; b < kB; ++b) {
-                            if (ii[b] < 0) continue;
-                            const int i = ii[b], j = jj[b];
-                            float val = sc[b] * acc[b];
-                            if (beta != 0.f) val = fmaf(beta, cin[b], val);
-                            if (fused) {
-                                if (bias_i || bias_j) val += bs[b];
-                                val = act_apply(act, val, cdt != DG_F32);
+                            for (int b = 0; b < kB; ++b) {
+                                if (ii[b] < 0) continue;
+                                const int i = ii[b], j = jj[b];
+                                float val = sc[b] * acc[b];
+                                if (beta != 0.f) val = fmaf(beta, cin[b], val);
+                                if (fused) {
+                                    if (bias_i || bias_j) val += bs[b];
+                                    val = act_fn<kAct, kCd != DG_F32>(val);
+                                }
+                                const int64_t ro = ci_multi ? epi_row_offset(e, i) : (int64_t)i * ci;
+                                st_out<kCd>(cbase + ro + (int64_t)j * cj, val);
                             }
-                            const int64_t ro = ci_multi ? epi_row_offset(e, i) : (int64_t)i * ci;
-                            store_elem(cbase + ro + (int64_t)j * cj, cdt, val);
-                        }
+                        };
+                        auto finish_act = [&](auto act_c) {
+                            if (cdt == DG_F32) finish(act_c, std::integral_constant<int, DG_F32>{});
+                            else if (cdt == DG_BF16) finish(act_c, std::integral_constant<int, DG_BF16>{});
+                            else finish(act_c, std::integral_constant<int, DG_F16>{});
+                        };
+                        if (act == DG_ACT_RELU) finish_act(std::integral_constant<int, DG_ACT_RELU>{});
+                        else if (act == DG_ACT_GELU_TANH) finish_act(std::integral_constant<int, DG_ACT_GELU_TANH>{});
+                        else finish_act(std::integral_constant<int, DG_ACT_NONE>{});
                     }
                 }
             }
