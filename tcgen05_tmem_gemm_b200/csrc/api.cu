@@ -862,8 +862,8 @@ dg_status prepare(const Views &v, const Plan &pl, float alpha, float beta, const
             if (!ok) return DG_ERR_UNSUPPORTED;
         }
         {
-            // a CTA of a pair loads half of a tile's columns, as boxes of bn/4 rows when K-major
-            const int q_rows = in.cta_pair ? bn / 4 : bn;
+            // a CTA of a pair loads half of a tile's columns: one box of bn/2 rows when K-major
+            const int q_rows = in.cta_pair ? bn / 2 : bn;
             const bool ok = in.q_mn_major ? encode_2d(&tq, dt, Qv->ptr, Nj, in.K, axis_stride(q_k), mn_rows)
                                           : encode_2d(&tq, dt, Qv->ptr, in.K, Nj, axis_stride(q_j), q_rows);
             if (!ok) return DG_ERR_UNSUPPORTED;

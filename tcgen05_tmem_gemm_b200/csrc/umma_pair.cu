@@ -268,7 +268,11 @@ __global__ void __launch_bounds__(192, 1)
                 const int i0 = pw.ti * 2 * kHalfM + (int)rank * kHalfM;
                 const int cw = pw.w / 2;  // this CTA's columns of the unit
                 const int j0 = pw.j0 + (int)rank * cw;
-                const uint32_t tx = 2u * (a_bytes + (uint32_t)(ksub * cw) * kRowBytes);  // both CTAs' bytes
+                // both CTAs' bytes: MN-major Q in boxes of 128-byte column groups (cw
+                // columns), K-major Q in one box of the CTA's bn/2 rows per sub-block,
+                // for a half-width unit too (its second half is loaded and not used)
+                const uint32_t qrows = q_mn ? (uint32_t)cw : (uint32_t)half_bn;
+                const uint32_t tx = 2u * (a_bytes + (uint32_t)ksub * qrows * kRowBytes);
                 bool ok = true;
                 for (int kb = pw.kb0; kb < pw.kb1; ++kb, ++it) {
                     if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, wc)) { ok = false; break; }
@@ -289,11 +293,10 @@ __global__ void __launch_bounds__(192, 1)
                             for (int c = 0; c < cw / per; ++c)
                                 tma_load_2d_pair(bs + c * mn_box_bytes, &tmap_q, full_c, j0 + c * per, k0);
                         } else {
-                            // boxes of bn/4 rows: two per CTA for a whole tile, one for a half
+                            // one box of bn/2 rows per sub-block (a box's fixed cost is paid
+                            // once); a half-width unit's CTA uses the first bn/4 of them
                             for (int j = 0; j < ksub; ++j)
-                                for (int c = 0; c < cw / (half_bn / 2); ++c)
-                                    tma_load_2d_pair(bs + j * b_sub + c * (half_bn / 2) * kRowBytes, &tmap_q, full_c,
-                                                     k0 + j * bk, j0 + c * (half_bn / 2));
+                                tma_load_2d_pair(bs + j * b_sub, &tmap_q, full_c, k0 + j * bk, j0);
                         }
                     }
                     if (++s == stages) {
